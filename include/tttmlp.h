@@ -1,0 +1,170 @@
+/*
+ * tttmlp.h -- C ABI of the TTT-MLP layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (One-Minute Video Generation with Test-Time Training, paper notes
+ * page, sections "关键设计 / TTT-MLP 层" and "关键设计 / 门控 + 双向机制"):
+ *
+ *   per head h, hidden state W = (W1 [m x d], W2 [d x m]), m = 4 d,
+ *   f(u; W) = W2 GELU(W1 u) with erf-GELU and no biases;
+ *   per token t (in walking order), with q = theta_Q x_t, k = theta_K x_t,
+ *   v = theta_V x_t:
+ *       W_t = W_{t-1} - eta * grad_W || f(k; W_{t-1}) - v ||^2
+ *       z_t = f(q; W_t)                      (read AFTER the update)
+ *   mini-batch variant, chunk size b (b = 1 is the rule above): the gradients
+ *   of a chunk are taken at the chunk-start state and token t of the chunk is
+ *   read with the prefix state W^c - eta * sum_{s<=t in chunk} grad(s);
+ *   gate:  out = x + tanh(alpha) * z   (alpha a vector over channels);
+ *   bidirectional: X' = gate_f(X, fwd(X)), Y = gate_r(X', rev(X')), the two
+ *   directions sharing theta and W_0, the reverse one walking t = T-1 .. 0
+ *   with its chunks formed in that walking order.
+ *
+ * All functions are thread-safe, never throw, and allocate nothing: device
+ * memory (inputs, outputs, workspace) is owned by the caller.  Every pointer
+ * argument except the *_host ones of ttt_mlp_forward_host is a DEVICE pointer
+ * on the current CUDA device.  Work is enqueued on `stream` (0 = the legacy
+ * default stream) and the functions return once it is enqueued, except
+ * ttt_mlp_status and ttt_mlp_forward_host, which synchronise the stream.
+ */
+#ifndef TTTMLP_H_
+#define TTTMLP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TTT_API __attribute__((visibility("default")))
+#else
+#define TTT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* ttt_stream_t;
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_INVALID_ARG = 1,   /* a pointer, size or value violates the contract below */
+    TTT_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. a head dim other than 16/32/64) */
+    TTT_ERR_CUDA = 3,          /* a CUDA runtime call failed; ttt_last_error() has its message */
+    TTT_ERR_NONFINITE = 4,     /* (ttt_mlp_status) an output z was NaN/Inf: the scan diverged */
+    TTT_ERR_TIMEOUT = 5        /* (ttt_mlp_status) a bounded on-chip wait expired; outputs invalid */
+} ttt_status;
+
+typedef enum { TTT_FWD = 0, TTT_REV = 1, TTT_BIDIR = 2 } ttt_direction;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+/*
+ * Shapes and layouts.
+ *   T   tokens (>= 1);  H heads (>= 1);  d head dim (16, 32 or 64);  m = 4 d.
+ *   D   model dim = H * d (the gate needs TTT(X) in X's own shape; the heads'
+ *       outputs are concatenated, there is no output projection).
+ *   per_head_input = 1:  X, Y are [H, T, d]; theta_q/k/v are [H, d, d] with
+ *                        q = theta_q[h] x (row e of theta_q[h] gives q_e).
+ *   per_head_input = 0:  X, Y are [T, D]; theta_q/k/v are [H*d, D] (the
+ *                        nn.Linear weight layout: q_{h,e} = sum_c theta_q[h*d+e][c] x_c).
+ *   x_dtype: element type of X, theta_q/k/v and Y.  The hidden state, the
+ *   projections' outputs, the scan and all accumulations are fp32.
+ *   All arrays are dense row-major, 16-byte aligned.
+ */
+typedef struct {
+    int T;
+    int H;
+    int d;
+    int m;                 /* must be 4 * d */
+    int D;                 /* must be H * d */
+    int per_head_input;    /* 1 or 0, see above */
+    ttt_dtype x_dtype;
+} ttt_mlp_desc;
+
+/*
+ * Bytes of device workspace ttt_mlp_forward needs for (desc, b, dir).
+ * Returns 0 if the arguments are invalid (ttt_last_error() says why).
+ */
+TTT_API size_t ttt_mlp_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
+
+/*
+ * The gated TTT-MLP layer, one direction or both (see the top of this file).
+ *
+ *   X          input, layout/dtype per desc.
+ *   theta_q/k/v  projections, layout/dtype per desc (shared by both directions).
+ *   W1_0 [H, m, d], W2_0 [H, d, m]  fp32 initial hidden state (both directions).
+ *   eta        gradient step, used exactly as given (finite, >= 0).
+ *   b          chunk size, 1 <= b <= 256; a ragged last chunk is allowed.
+ *   dir        TTT_FWD: Y = gate(X, fwd(X); alpha_f)
+ *              TTT_REV: Y = gate(X, rev(X); alpha_r)
+ *              TTT_BIDIR: Y = gate(X', rev(X'); alpha_r), X' = gate(X, fwd(X); alpha_f)
+ *   alpha_f, alpha_r  [D] fp32 gate vectors; channel (h, e) is alpha[h*d + e].
+ *              alpha_f is required for FWD and BIDIR, alpha_r for REV and BIDIR.
+ *   Y          output, same layout/dtype as X.  Must not alias X.
+ *   Z_out      optional (may be NULL) fp32 [n_dir, <X layout>] pre-gate outputs z_t,
+ *              n_dir = 1 for FWD/REV, 2 for BIDIR (slot 0 forward, slot 1 reverse).
+ *   W1_T, W2_T optional (may be NULL) fp32 [n_dir, H, m, d] and [n_dir, H, d, m]
+ *              hidden state after each direction's last token.
+ *   workspace  device memory of at least ttt_mlp_workspace_size(desc, b, dir)
+ *              bytes, 256-byte aligned, not shared with a concurrent call.
+ *
+ * Returns TTT_OK once the work is enqueued; argument errors are reported
+ * before anything is enqueued.  Divergence and expired waits are recorded in
+ * the workspace and reported by ttt_mlp_status.
+ */
+TTT_API ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X,
+                           const void* theta_q, const void* theta_k, const void* theta_v,
+                           const float* W1_0, const float* W2_0, float eta, int b,
+                           ttt_direction dir, const float* alpha_f, const float* alpha_r,
+                           void* Y, float* Z_out, float* W1_T, float* W2_T,
+                           void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads and clears the status word a previous
+ * ttt_mlp_forward left in `workspace`: TTT_OK, TTT_ERR_NONFINITE (an output
+ * was NaN/Inf, e.g. eta too large for the squared-norm loss) or
+ * TTT_ERR_TIMEOUT (a bounded wait inside a kernel expired; outputs invalid).
+ */
+TTT_API ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream);
+
+/*
+ * Bytes of device workspace ttt_mlp_forward_host needs: the workspace of
+ * ttt_mlp_forward plus device staging for X and Y.  0 on invalid arguments.
+ */
+TTT_API size_t ttt_mlp_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
+
+/*
+ * End-to-end variant: X_host and Y_host are HOST buffers (pinned for full
+ * copy speed); everything else as in ttt_mlp_forward (device pointers).
+ * Copies X_host to the device, runs the layer, copies Y back to Y_host,
+ * synchronises `stream` and returns the status as ttt_mlp_status would.
+ */
+TTT_API ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host,
+                                const void* theta_q, const void* theta_k, const void* theta_v,
+                                const float* W1_0, const float* W2_0, float eta, int b,
+                                ttt_direction dir, const float* alpha_f, const float* alpha_r,
+                                void* Y_host, void* workspace, size_t workspace_bytes,
+                                ttt_stream_t stream);
+
+/*
+ * Kernel selection, process-wide (for tests and comparisons): 0 = automatic
+ * (the fastest kernel that takes the shape), 1 = the FP32 SIMT kernels,
+ * 2 = the tensor-core kernels (a later ttt_mlp_forward returns
+ * TTT_ERR_UNSUPPORTED if the shape is outside them).  scan_impl selects the
+ * scan kernel, proj_impl the full-mode projection kernel.
+ */
+TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);
+
+/* Message for the last non-OK status returned on the calling thread ("" if none). */
+TTT_API const char* ttt_last_error(void);
+
+/*
+ * Number of kernels the library has launched in this process (all entry
+ * points, all threads).  Used to count launches inside a timed region.
+ */
+TTT_API uint64_t ttt_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTTMLP_H_ */

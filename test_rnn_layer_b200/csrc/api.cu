@@ -1,0 +1,309 @@
+// C ABI of the TTT-MLP layer: argument checks, workspace carving and the
+// direction driver.  Every step of the computation runs in this library's
+// kernels; this file only sequences them on the caller's stream.
+//
+// Bidirectional composition (paper notes page, "关键设计 / 门控 + 双向机制"):
+// the forward scan runs on X and its gate writes X' = X + tanh(alpha_f) z_f;
+// the reverse scan runs on X' (same theta, same W_0) and its gate writes
+// Y = X' + tanh(alpha_r) z_r.
+#include <atomic>
+#include <cstdarg>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/tttmlp.h"
+#include "internal.h"
+
+namespace ttt {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
+
+}  // namespace ttt
+
+using namespace ttt;
+
+namespace {
+
+thread_local std::string t_err;
+
+ttt_status fail(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+ttt_status fail(ttt_status code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_err = buf;
+    return code;
+}
+
+#define CUDA_TRY(expr)                                                                           \
+    do {                                                                                         \
+        cudaError_t e_ = (expr);                                                                 \
+        if (e_ != cudaSuccess) return fail(TTT_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+    } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t elem_size(ttt_dtype t) { return t == TTT_BF16 ? 2 : 4; }
+
+ttt_status check_desc(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (!desc) return fail(TTT_ERR_INVALID_ARG, "desc is NULL");
+    const ttt_mlp_desc& q = *desc;
+    if (q.T < 1 || q.H < 1) return fail(TTT_ERR_INVALID_ARG, "T=%d and H=%d must be >= 1", q.T, q.H);
+    if (q.d < 1 || q.m != 4 * q.d)
+        return fail(TTT_ERR_INVALID_ARG, "m=%d must be 4*d (d=%d)", q.m, q.d);
+    if ((long long)q.D != (long long)q.H * q.d)
+        return fail(TTT_ERR_INVALID_ARG, "D=%d must equal H*d=%lld", q.D, (long long)q.H * q.d);
+    if (q.per_head_input != 0 && q.per_head_input != 1)
+        return fail(TTT_ERR_INVALID_ARG, "per_head_input must be 0 or 1");
+    if (q.x_dtype != TTT_F32 && q.x_dtype != TTT_BF16) return fail(TTT_ERR_INVALID_ARG, "bad x_dtype");
+    if (dir != TTT_FWD && dir != TTT_REV && dir != TTT_BIDIR) return fail(TTT_ERR_INVALID_ARG, "bad direction");
+    if (b < 1 || b > 256) return fail(TTT_ERR_INVALID_ARG, "b=%d outside [1, 256]", b);
+    if (q.d != 16 && q.d != 32 && q.d != 64)
+        return fail(TTT_ERR_UNSUPPORTED, "head dim d=%d not supported (16, 32, 64)", q.d);
+    if ((long long)q.T * q.D > (1LL << 40)) return fail(TTT_ERR_INVALID_ARG, "T*D too large");
+    return TTT_OK;
+}
+
+struct Layout {
+    size_t status, qkv[3], xp, delta, scratch, total;
+    long long scratch_per_head;
+    bool split_reverse;   // reverse projection as theta X + theta bf16(X' - X)
+};
+
+Layout plan(const ttt_mlp_desc& q, int b, ttt_direction dir) {
+    Layout L{};
+    const size_t n = (size_t)q.T * q.D;
+    size_t off = 0;
+    L.status = off; off += kAlign;
+    for (int w = 0; w < 3; ++w) { L.qkv[w] = off; off = align_up(off + n * sizeof(float)); }
+    L.split_reverse = (dir == TTT_BIDIR) && !q.per_head_input && q.x_dtype == TTT_BF16;
+    L.xp = off;
+    if (dir == TTT_BIDIR) off = align_up(off + n * sizeof(float));
+    L.delta = off;
+    if (L.split_reverse) off = align_up(off + n * 2);
+    L.scratch = off;
+    // the SIMT chunk kernel may run for any b (it is selectable for b = 1 too)
+    L.scratch_per_head = scan_chunk_simt_scratch_floats(q.d, q.m, b);
+    off = align_up(off + (size_t)q.H * L.scratch_per_head * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+struct Dir {
+    int reverse;
+    const void* xin;
+    int xin_bf16;
+    const float* alpha;
+    void* out;
+    int out_bf16;
+    __nv_bfloat16* delta;
+    float* zdbg;
+    float* w1t;
+    float* w2t;
+};
+
+ttt_status project(const ttt_mlp_desc& q, const void* src, int src_bf16, const void* const th[3],
+                   float* const out[3], int accumulate, cudaStream_t s) {
+    const int th_bf16 = q.x_dtype == TTT_BF16;
+    if (q.per_head_input) {
+        if (accumulate) return fail(TTT_ERR_UNSUPPORTED, "internal: accumulate in per-head projection");
+        CUDA_TRY(launch_proj_per_head(src, src_bf16, th, th_bf16, out, q.T, q.H, q.d, s));
+    } else {
+        CUDA_TRY(launch_proj_full_simt(src, src_bf16, th, th_bf16, out, q.T, q.D, q.D, accumulate, s));
+    }
+    return TTT_OK;
+}
+
+ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W1_0, const float* W2_0,
+                float eta, int b, const Dir& dd, cudaStream_t s) {
+    ScanArgs a{};
+    a.Q = reinterpret_cast<const float*>(ws + L.qkv[0]);
+    a.K = reinterpret_cast<const float*>(ws + L.qkv[1]);
+    a.V = reinterpret_cast<const float*>(ws + L.qkv[2]);
+    if (q.per_head_input) { a.qkv_hs = (long long)q.T * q.d; a.qkv_ts = q.d; }
+    else { a.qkv_hs = q.d; a.qkv_ts = q.D; }
+    a.x_hs = a.qkv_hs; a.x_ts = a.qkv_ts;
+    a.Xin = dd.xin; a.xin_bf16 = dd.xin_bf16;
+    a.alpha = dd.alpha;
+    a.Out = dd.out; a.out_bf16 = dd.out_bf16;
+    a.Delta = dd.delta; a.Zdbg = dd.zdbg;
+    a.W1_0 = W1_0; a.W2_0 = W2_0; a.W1_T = dd.w1t; a.W2_T = dd.w2t;
+    a.T = q.T; a.H = q.H; a.d = q.d; a.m = q.m; a.b = b; a.reverse = dd.reverse;
+    a.eta = eta;
+    a.status = reinterpret_cast<int*>(ws + L.status);
+    a.scratch = reinterpret_cast<float*>(ws + L.scratch);
+    a.scratch_per_head = L.scratch_per_head;
+    const int impl = g_scan_impl.load();
+    if (impl == 2) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan kernel not available for this shape");
+    if (b == 1 && impl != 1) {
+        CUDA_TRY(launch_scan_token(a, s));
+    } else {
+        CUDA_TRY(launch_scan_chunk_simt(a, s));
+    }
+    return TTT_OK;
+}
+
+ttt_status check_ptrs(const ttt_mlp_desc& q, const void* X, const void* tq, const void* tk, const void* tv,
+                      const float* W1_0, const float* W2_0, float eta, ttt_direction dir,
+                      const float* alpha_f, const float* alpha_r) {
+    if (!X || !tq || !tk || !tv || !W1_0 || !W2_0)
+        return fail(TTT_ERR_INVALID_ARG, "X, theta_q/k/v, W1_0 and W2_0 must be non-NULL");
+    if ((dir == TTT_FWD || dir == TTT_BIDIR) && !alpha_f)
+        return fail(TTT_ERR_INVALID_ARG, "alpha_f is required for this direction");
+    if ((dir == TTT_REV || dir == TTT_BIDIR) && !alpha_r)
+        return fail(TTT_ERR_INVALID_ARG, "alpha_r is required for this direction");
+    if (!std::isfinite(eta) || eta < 0.f) return fail(TTT_ERR_INVALID_ARG, "eta must be finite and >= 0");
+    const void* ps[] = {X, tq, tk, tv, W1_0, W2_0, alpha_f, alpha_r};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+    (void)q;
+    return TTT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttt_mlp_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc(desc, b, dir) != TTT_OK) return 0;
+    return plan(*desc, b, dir).total;
+}
+
+size_t ttt_mlp_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc(desc, b, dir) != TTT_OK) return 0;
+    const size_t io = align_up((size_t)desc->T * desc->D * elem_size(desc->x_dtype));
+    return plan(*desc, b, dir).total + 2 * io;
+}
+
+ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                           const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                           ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
+                           float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes,
+                           ttt_stream_t stream_) {
+    ttt_status st = check_desc(desc, b, dir);
+    if (st != TTT_OK) return st;
+    const ttt_mlp_desc& q = *desc;
+    st = check_ptrs(q, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, dir, alpha_f, alpha_r);
+    if (st != TTT_OK) return st;
+    if (!Y || !workspace) return fail(TTT_ERR_INVALID_ARG, "Y and workspace must be non-NULL");
+    const void* outs[] = {Y, Z_out, W1_T, W2_T};
+    for (const void* p : outs)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "output pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t xbytes = (size_t)q.T * q.D * elem_size(q.x_dtype);
+    {
+        const char* xs = static_cast<const char*>(X);
+        const char* ys = static_cast<const char*>(Y);
+        if (xs < ys + xbytes && ys < xs + xbytes) return fail(TTT_ERR_INVALID_ARG, "Y must not alias X");
+    }
+    const Layout L = plan(q, b, dir);
+    if (workspace_bytes < L.total)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, L.total);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    char* ws = static_cast<char*>(workspace);
+    CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16, s));
+    const int x_bf16 = q.x_dtype == TTT_BF16;
+    const void* th[3] = {theta_q, theta_k, theta_v};
+    float* qkv[3] = {reinterpret_cast<float*>(ws + L.qkv[0]), reinterpret_cast<float*>(ws + L.qkv[1]),
+                     reinterpret_cast<float*>(ws + L.qkv[2])};
+    const size_t n = (size_t)q.T * q.D;
+    const size_t nW = (size_t)q.H * q.m * q.d;
+    float* xp = reinterpret_cast<float*>(ws + L.xp);
+
+    // first (or only) direction
+    Dir d0{};
+    d0.reverse = dir == TTT_REV;
+    d0.xin = X; d0.xin_bf16 = x_bf16;
+    d0.alpha = (dir == TTT_REV) ? alpha_r : alpha_f;
+    if (dir == TTT_BIDIR) { d0.out = xp; d0.out_bf16 = 0; }
+    else { d0.out = Y; d0.out_bf16 = x_bf16; }
+    d0.delta = L.split_reverse ? reinterpret_cast<__nv_bfloat16*>(ws + L.delta) : nullptr;
+    d0.zdbg = Z_out; d0.w1t = W1_T; d0.w2t = W2_T;
+    st = project(q, X, x_bf16, th, qkv, 0, s);
+    if (st != TTT_OK) return st;
+    st = scan(q, L, ws, W1_0, W2_0, eta, b, d0, s);
+    if (st != TTT_OK) return st;
+    if (dir != TTT_BIDIR) return TTT_OK;
+
+    // reverse direction on X' = X + tanh(alpha_f) z_f
+    if (L.split_reverse) {
+        // theta X' = theta X + theta (X' - X): add the projection of the bf16
+        // gate increment onto the forward projections already in place.
+        st = project(q, ws + L.delta, 1, th, qkv, 1, s);
+    } else {
+        st = project(q, xp, 0, th, qkv, 0, s);
+    }
+    if (st != TTT_OK) return st;
+    Dir d1{};
+    d1.reverse = 1;
+    d1.xin = xp; d1.xin_bf16 = 0;
+    d1.alpha = alpha_r;
+    d1.out = Y; d1.out_bf16 = x_bf16;
+    d1.zdbg = Z_out ? Z_out + n : nullptr;
+    d1.w1t = W1_T ? W1_T + nW : nullptr;
+    d1.w2t = W2_T ? W2_T + nW : nullptr;
+    return scan(q, L, ws, W1_0, W2_0, eta, b, d1, s);
+}
+
+ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {
+    if (!workspace) return fail(TTT_ERR_INVALID_ARG, "workspace is NULL");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    CUDA_TRY(cudaStreamSynchronize(s));
+    int word = 0;
+    CUDA_TRY(cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost));
+    CUDA_TRY(cudaMemset(workspace, 0, sizeof(int)));
+    if (word & kStatusTimeout) return fail(TTT_ERR_TIMEOUT, "a bounded wait inside a scan kernel expired");
+    if (word & kStatusNonFinite) return fail(TTT_ERR_NONFINITE, "the scan produced non-finite outputs");
+    return TTT_OK;
+}
+
+ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, const void* theta_q,
+                                const void* theta_k, const void* theta_v, const float* W1_0, const float* W2_0,
+                                float eta, int b, ttt_direction dir, const float* alpha_f, const float* alpha_r,
+                                void* Y_host, void* workspace, size_t workspace_bytes, ttt_stream_t stream_) {
+    ttt_status st = check_desc(desc, b, dir);
+    if (st != TTT_OK) return st;
+    if (!X_host || !Y_host || !workspace) return fail(TTT_ERR_INVALID_ARG, "X_host, Y_host, workspace must be non-NULL");
+    const ttt_mlp_desc& q = *desc;
+    const size_t need = ttt_mlp_host_io_workspace_size(desc, b, dir);
+    if (workspace_bytes < need)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    const Layout L = plan(q, b, dir);
+    const size_t xbytes = (size_t)q.T * q.D * elem_size(q.x_dtype);
+    char* ws = static_cast<char*>(workspace);
+    void* Xd = ws + L.total;
+    void* Yd = ws + L.total + align_up(xbytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    CUDA_TRY(cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, s));
+    st = ttt_mlp_forward(desc, Xd, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Yd,
+                         nullptr, nullptr, nullptr, workspace, L.total, stream_);
+    if (st != TTT_OK) return st;
+    CUDA_TRY(cudaMemcpyAsync(Y_host, Yd, xbytes, cudaMemcpyDeviceToHost, s));
+    return ttt_mlp_status(workspace, stream_);
+}
+
+ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl) {
+    if (scan_impl < 0 || scan_impl > 2 || proj_impl < 0 || proj_impl > 2)
+        return fail(TTT_ERR_INVALID_ARG, "kernel selector must be 0 (auto), 1 (SIMT) or 2 (tensor core)");
+    g_scan_impl.store(scan_impl);
+    g_proj_impl.store(proj_impl);
+    return TTT_OK;
+}
+
+const char* ttt_last_error(void) { return t_err.c_str(); }
+
+uint64_t ttt_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

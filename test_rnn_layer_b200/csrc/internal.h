@@ -1,0 +1,58 @@
+// Internal launcher interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttt {
+
+// Status bits a kernel may set in the workspace status word.
+enum : int { kStatusNonFinite = 1, kStatusTimeout = 2 };
+
+// Token-stream and gate arguments of one direction's scan.  Element (h, t, j)
+// of a [H, T, d]-style stream lives at base + h * hs + t * ts + j; the same
+// (hs, ts) pair describes both the per-head layout [H, T, d] (hs = T d,
+// ts = d) and the concatenated-heads layout [T, H d] (hs = d, ts = H d).
+struct ScanArgs {
+    const float* Q;
+    const float* K;
+    const float* V;
+    long long qkv_hs, qkv_ts;
+    const void* Xin;        // gate residual input
+    int xin_bf16;
+    long long x_hs, x_ts;   // layout of Xin, Out, Delta and Zdbg
+    const float* alpha;     // [H d], channel (h, j) = alpha[h d + j]
+    void* Out;              // gate output: x + tanh(alpha) z
+    int out_bf16;
+    __nv_bfloat16* Delta;   // optional: bf16(tanh(alpha) z), same layout
+    float* Zdbg;            // optional: pre-gate z (fp32)
+    const float* W1_0;      // [H, m, d]
+    const float* W2_0;      // [H, d, m]
+    float* W1_T;            // optional [H, m, d]
+    float* W2_T;            // optional [H, d, m]
+    int T, H, d, m, b, reverse;
+    float eta;
+    int* status;            // OR-ed status bits
+    float* scratch;         // per-head scratch (chunk SIMT kernel)
+    long long scratch_per_head;  // floats
+};
+
+// Scan kernels.  Each returns a cudaError_t from the launch.
+cudaError_t launch_scan_token(const ScanArgs& a, cudaStream_t s);        // b == 1
+cudaError_t launch_scan_chunk_simt(const ScanArgs& a, cudaStream_t s);   // any b
+long long scan_chunk_simt_scratch_floats(int d, int m, int b);
+
+// Per-head projections: U[which][h, t, e] = sum_j theta_which[h][e][j] x[h, t, j].
+cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
+                                 float* const out[3], int T, int H, int d, cudaStream_t s);
+
+// Full-mode projections: C_which[t, n] (+)= sum_c A[t, c] Theta_which[n, c],
+// A [T, Dm] row-major, Theta [N, Dm] row-major, C [T, N] fp32.
+cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
+                                  float* const out[3], int T, int N, int Dm, int accumulate,
+                                  cudaStream_t s);
+
+void count_launch();
+
+}  // namespace ttt

@@ -1,0 +1,118 @@
+// theta_Q / theta_K / theta_V projections on the FP32 SIMT pipe.
+//
+// Per-head mode: q_t = theta_Q[h] x_t for every head and token (a d x d
+// matrix-vector product per token); full mode: U = X Theta^T with X [T, Dm]
+// and Theta [N, Dm] (the nn.Linear layout), fp32 accumulation and output.
+// Paper notes page, "关键设计 / TTT-MLP 层": theta_K, theta_V, theta_Q are the
+// outer-loop key/value/query projections.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+namespace {
+
+constexpr int kPhTok = 32;       // tokens per CTA, per-head projection
+constexpr int kPhThreads = 256;
+
+__global__ void __launch_bounds__(kPhThreads)
+proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk, const void* thv,
+                     int th_bf16, float* oq, float* ok, float* ov, int T, int d) {
+    extern __shared__ float sm[];
+    float* th = sm;                     // [3][d][d]
+    float* xs = sm + 3 * d * d;         // [kPhTok][d]
+    const int h = blockIdx.y;
+    const int t0 = blockIdx.x * kPhTok;
+    const int nt = min(kPhTok, T - t0);
+    const void* ths[3] = {thq, thk, thv};
+    for (int p = threadIdx.x; p < 3 * d * d; p += blockDim.x) {
+        const int w = p / (d * d), q = p % (d * d);
+        th[p] = load_elem(ths[w], (long long)h * d * d + q, th_bf16);
+    }
+    for (int p = threadIdx.x; p < nt * d; p += blockDim.x)
+        xs[p] = load_elem(X, ((long long)h * T + t0) * d + p, x_bf16);
+    __syncthreads();
+    float* outs[3] = {oq, ok, ov};
+    for (int p = threadIdx.x; p < 3 * nt * d; p += blockDim.x) {
+        const int w = p / (nt * d), q = p % (nt * d);
+        const int r = q / d, e = q % d;
+        const float* row = th + (w * d + e) * d;
+        const float* x = xs + r * d;
+        float acc = 0.f;
+        for (int j = 0; j < d; ++j) acc = fmaf(row[j], x[j], acc);
+        outs[w][((long long)h * T + t0 + r) * d + e] = acc;
+    }
+}
+
+// C[t, n] (+)= sum_c A[t, c] B[n, c]; 64 x 64 tile, 16-deep k steps, 4 x 4 per thread.
+constexpr int kGT = 64, kGK = 16;
+
+__global__ void __launch_bounds__(256)
+proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1, const void* B2, int b_bf16,
+                      float* C0, float* C1, float* C2, int T, int N, int Dm, int accumulate) {
+    __shared__ float As[kGK][kGT + 4];
+    __shared__ float Bs[kGK][kGT + 4];
+    const void* B = blockIdx.z == 0 ? B0 : (blockIdx.z == 1 ? B1 : B2);
+    float* C = blockIdx.z == 0 ? C0 : (blockIdx.z == 1 ? C1 : C2);
+    const int n0 = blockIdx.x * kGT, t0 = blockIdx.y * kGT;
+    const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+    float acc[4][4] = {};
+    for (int c0 = 0; c0 < Dm; c0 += kGK) {
+        for (int p = threadIdx.x; p < kGT * kGK; p += 256) {
+            const int r = p / kGK, c = p % kGK;
+            const int t = t0 + r, n = n0 + r, cc = c0 + c;
+            As[c][r] = (t < T && cc < Dm) ? load_elem(A, (long long)t * Dm + cc, a_bf16) : 0.f;
+            Bs[c][r] = (n < N && cc < Dm) ? load_elem(B, (long long)n * Dm + cc, b_bf16) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int c = 0; c < kGK; ++c) {
+            float av[4], bv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { av[u] = As[c][ty * 4 + u]; bv[u] = Bs[c][tx * 4 + u]; }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int t = t0 + ty * 4 + u;
+        if (t >= T) continue;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int n = n0 + tx * 4 + v;
+            if (n >= N) continue;
+            float* dst = C + (long long)t * N + n;
+            *dst = accumulate ? *dst + acc[u][v] : acc[u][v];
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
+                                 float* const out[3], int T, int H, int d, cudaStream_t s) {
+    const size_t smem = sizeof(float) * (3 * (size_t)d * d + (size_t)kPhTok * d);
+    cudaError_t e = cudaFuncSetAttribute(proj_per_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    dim3 grid((T + kPhTok - 1) / kPhTok, H);
+    proj_per_head_kernel<<<grid, kPhThreads, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16,
+                                                        out[0], out[1], out[2], T, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
+                                  float* const out[3], int T, int N, int Dm, int accumulate,
+                                  cudaStream_t s) {
+    count_launch();
+    dim3 grid((N + kGT - 1) / kGT, (T + kGT - 1) / kGT, 3);
+    proj_full_simt_kernel<<<grid, 256, 0, s>>>(A, a_bf16, theta[0], theta[1], theta[2], th_bf16, out[0], out[1],
+                                                out[2], T, N, Dm, accumulate);
+    return cudaGetLastError();
+}
+
+}  // namespace ttt

@@ -1,0 +1,174 @@
+"""Python binding of libtttmlp.so (the C ABI in include/tttmlp.h).
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name; all arithmetic runs in the library's CUDA kernels.  PyTorch
+is used for device memory and streams.  There is no fallback: if the
+library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtttmlp.so")
+_lib = None
+
+TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_CUDA, TTT_ERR_NONFINITE, TTT_ERR_TIMEOUT = range(6)
+STATUS_NAMES = {0: "TTT_OK", 1: "TTT_ERR_INVALID_ARG", 2: "TTT_ERR_UNSUPPORTED", 3: "TTT_ERR_CUDA",
+                4: "TTT_ERR_NONFINITE", 5: "TTT_ERR_TIMEOUT"}
+TTT_FWD, TTT_REV, TTT_BIDIR = 0, 1, 2
+TTT_F32, TTT_BF16 = 0, 1
+DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
+
+EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
+            "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count"]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {ttt_last_error()}")
+
+
+class ttt_mlp_desc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("m", ctypes.c_int),
+                ("D", ctypes.c_int), ("per_head_input", ctypes.c_int), ("x_dtype", ctypes.c_int)]
+
+
+def make_desc(T: int, H: int, d: int, per_head: bool, bf16: bool) -> ttt_mlp_desc:
+    return ttt_mlp_desc(T, H, d, 4 * d, H * d, 1 if per_head else 0, TTT_BF16 if bf16 else TTT_F32)
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libtttmlp.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with python -m test_rnn_layer_b200.build")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i, f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+        dp = ctypes.POINTER(ttt_mlp_desc)
+        L.ttt_mlp_workspace_size.restype = sz
+        L.ttt_mlp_workspace_size.argtypes = [dp, i, i]
+        L.ttt_mlp_host_io_workspace_size.restype = sz
+        L.ttt_mlp_host_io_workspace_size.argtypes = [dp, i, i]
+        L.ttt_mlp_forward.restype = i
+        L.ttt_mlp_forward.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.ttt_mlp_forward_host.restype = i
+        L.ttt_mlp_forward_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, sz, vp]
+        L.ttt_mlp_status.restype = i
+        L.ttt_mlp_status.argtypes = [vp, vp]
+        L.ttt_mlp_select_kernels.restype = i
+        L.ttt_mlp_select_kernels.argtypes = [i, i]
+        L.ttt_last_error.restype = ctypes.c_char_p
+        L.ttt_last_error.argtypes = []
+        L.ttt_launch_count.restype = ctypes.c_uint64
+        L.ttt_launch_count.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _p(x):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return ctypes.c_void_p(x.data_ptr())
+    return ctypes.c_void_p(int(x))
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+# ------------------------------------------------------------------ the C entry points
+def ttt_last_error() -> str:
+    return lib().ttt_last_error().decode()
+
+
+def ttt_launch_count() -> int:
+    return int(lib().ttt_launch_count())
+
+
+def ttt_mlp_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
+    return int(lib().ttt_mlp_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_mlp_host_io_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
+    return int(lib().ttt_mlp_host_io_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_mlp_select_kernels(scan_impl: int, proj_impl: int) -> int:
+    return int(lib().ttt_mlp_select_kernels(scan_impl, proj_impl))
+
+
+def ttt_mlp_forward(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r, Y,
+                    Z_out, W1_T, W2_T, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_mlp_forward(ctypes.byref(desc), _p(X), _p(theta_q), _p(theta_k), _p(theta_v), _p(W1_0),
+                                     _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f), _p(alpha_r), _p(Y),
+                                     _p(Z_out), _p(W1_T), _p(W2_T), _p(workspace), int(workspace_bytes),
+                                     _stream(stream)))
+
+
+def ttt_mlp_forward_host(desc, X_host, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r,
+                         Y_host, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_mlp_forward_host(ctypes.byref(desc), _p(X_host), _p(theta_q), _p(theta_k), _p(theta_v),
+                                          _p(W1_0), _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f),
+                                          _p(alpha_r), _p(Y_host), _p(workspace), int(workspace_bytes),
+                                          _stream(stream)))
+
+
+def ttt_mlp_status(workspace, stream=None) -> int:
+    return int(lib().ttt_mlp_status(_p(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------------------ tensor-level convenience
+def check(status: int, where: str) -> None:
+    if status != TTT_OK:
+        raise TTTError(status, where)
+
+
+def alloc_workspace(desc: ttt_mlp_desc, b: int, direction: int, device, host_io: bool = False) -> torch.Tensor:
+    n = (ttt_mlp_host_io_workspace_size if host_io else ttt_mlp_workspace_size)(desc, b, direction)
+    if n == 0:
+        raise TTTError(TTT_ERR_INVALID_ARG, "workspace size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def layer_forward(X, theta_q, theta_k, theta_v, W1_0, W2_0, eta: float, b: int, dirs: str, alpha_f=None,
+                  alpha_r=None, per_head: bool = True, want_z: bool = False, want_state: bool = False,
+                  workspace: torch.Tensor | None = None, check_status: bool = True, stream=None) -> dict:
+    """Allocate outputs (torch, on X's device) and call ttt_mlp_forward once."""
+    dev = X.device
+    if per_head:
+        H, T, d = X.shape
+    else:
+        T, D = X.shape
+        d = W1_0.shape[2]
+        H = W1_0.shape[0]
+    desc = make_desc(T, H, d, per_head, X.dtype == torch.bfloat16)
+    direction = DIRS[dirs]
+    nd = 2 if dirs == "bidir" else 1
+    ws = workspace if workspace is not None else alloc_workspace(desc, b, direction, dev)
+    Y = torch.empty_like(X)
+    Z = torch.empty((nd,) + tuple(X.shape), dtype=torch.float32, device=dev) if want_z else None
+    W1T = torch.empty((nd,) + tuple(W1_0.shape), dtype=torch.float32, device=dev) if want_state else None
+    W2T = torch.empty((nd,) + tuple(W2_0.shape), dtype=torch.float32, device=dev) if want_state else None
+    st = ttt_mlp_forward(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r, Y, Z,
+                         W1T, W2T, ws, ws.numel(), stream)
+    check(st, "ttt_mlp_forward")
+    out = {"Y": Y, "Z": Z, "W1_T": W1T, "W2_T": W2T, "workspace": ws}
+    if check_status:
+        st = ttt_mlp_status(ws, stream)
+        out["status"] = st
+        check(st, "ttt_mlp_status")
+    return out

@@ -1,0 +1,119 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/tttmlp.h declares, sizes workspaces, and rejects bad
+arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from test_rnn_layer_b200 import build as B
+from test_rnn_layer_b200 import tttmlp as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tttmlp.h")).read()
+    return sorted(set(re.findall(r"TTT_API\s+[\w\s\*]+?\b(ttt_\w+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported():
+    names = _declared()
+    assert "ttt_mlp_forward" in names and len(names) >= 8
+    out = subprocess.run(["nm", "-D", "--defined-only", L.library_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (ttt_\w+)", out))
+    assert set(names) <= exported, set(names) - exported
+    lib = L.lib()
+    for n in names:
+        assert getattr(lib, n) is not None
+    assert set(L.EXPORTED) == set(names)
+
+
+def test_library_needs_no_driver_at_load_time():
+    out = subprocess.run(["ldd", L.library_path()], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "not found" not in out
+
+
+def _desc(**kw):
+    base = dict(T=1024, H=4, d=64, per_head=True, bf16=False)
+    base.update(kw)
+    return L.make_desc(base["T"], base["H"], base["d"], base["per_head"], base["bf16"])
+
+
+def test_workspace_sizes():
+    d = _desc()
+    n1 = L.ttt_mlp_workspace_size(d, 1, L.TTT_FWD)
+    nb = L.ttt_mlp_workspace_size(d, 1, L.TTT_BIDIR)
+    assert n1 >= 3 * 1024 * 256 * 4 and nb >= n1 + 1024 * 256 * 4
+    assert L.ttt_mlp_host_io_workspace_size(d, 1, L.TTT_FWD) >= n1 + 2 * 1024 * 256 * 4
+    full = _desc(T=313344, H=48, per_head=False, bf16=True)
+    n = L.ttt_mlp_workspace_size(full, 64, L.TTT_BIDIR)
+    # Q, K, V and X' in fp32 plus the bf16 gate increment: at least 9.0 bytes per element
+    assert n >= 313344 * 3072 * 18
+    assert n % 256 == 0
+
+
+@pytest.mark.parametrize("bad", [dict(T=0), dict(H=0), dict(d=48), dict(d=0)])
+def test_bad_desc_rejected(bad):
+    d = _desc(**bad)
+    assert L.ttt_mlp_workspace_size(d, 1, L.TTT_FWD) == 0
+    assert L.ttt_last_error()
+
+
+def test_bad_m_and_D_rejected():
+    d = _desc()
+    d.m = 200
+    assert L.ttt_mlp_workspace_size(d, 1, L.TTT_FWD) == 0 and "m=" in L.ttt_last_error()
+    d = _desc()
+    d.D = 100
+    assert L.ttt_mlp_workspace_size(d, 1, L.TTT_FWD) == 0 and "D=" in L.ttt_last_error()
+
+
+@pytest.mark.parametrize("b", [0, -1, 257])
+def test_bad_chunk_rejected(b):
+    assert L.ttt_mlp_workspace_size(_desc(), b, L.TTT_FWD) == 0
+
+
+def _fwd(desc, **over):
+    args = dict(X=0x1000, tq=0x2000, tk=0x3000, tv=0x4000, W1=0x5000, W2=0x6000, eta=0.01, b=16,
+                dir=L.TTT_BIDIR, af=0x7000, ar=0x8000, Y=0x90000000, Z=None, W1T=None, W2T=None,
+                ws=0x100000000, wsb=1 << 40)
+    args.update(over)
+    return L.ttt_mlp_forward(desc, args["X"], args["tq"], args["tk"], args["tv"], args["W1"], args["W2"],
+                             args["eta"], args["b"], args["dir"], args["af"], args["ar"], args["Y"], args["Z"],
+                             args["W1T"], args["W2T"], args["ws"], args["wsb"], 0)
+
+
+def test_forward_argument_errors_before_any_cuda_call():
+    """Every call below is rejected by argument checks, so the fake addresses
+    never reach the device.  Still skipped where a GPU exists."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses are only used where no GPU exists")
+    d = _desc()
+    assert _fwd(d, X=None) == L.TTT_ERR_INVALID_ARG
+    assert _fwd(d, ar=None) == L.TTT_ERR_INVALID_ARG and "alpha_r" in L.ttt_last_error()
+    assert _fwd(d, eta=float("nan")) == L.TTT_ERR_INVALID_ARG
+    assert _fwd(d, eta=-1.0) == L.TTT_ERR_INVALID_ARG
+    assert _fwd(d, X=0x1004) == L.TTT_ERR_INVALID_ARG and "aligned" in L.ttt_last_error()
+    assert _fwd(d, ws=0x100000010) == L.TTT_ERR_INVALID_ARG and "256" in L.ttt_last_error()
+    assert _fwd(d, wsb=1024) == L.TTT_ERR_INVALID_ARG and "too small" in L.ttt_last_error()
+    assert _fwd(d, Y=0x1000) == L.TTT_ERR_INVALID_ARG and "alias" in L.ttt_last_error()
+    assert _fwd(d, b=0) == L.TTT_ERR_INVALID_ARG
+    assert _fwd(_desc(d=48)) == L.TTT_ERR_UNSUPPORTED
+
+
+def test_kernel_selector_validation():
+    assert L.ttt_mlp_select_kernels(3, 0) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_mlp_select_kernels(0, 0) == L.TTT_OK
+
+
+def test_status_null_workspace():
+    assert L.lib().ttt_mlp_status(None, None) == L.TTT_ERR_INVALID_ARG
