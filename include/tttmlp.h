@@ -163,6 +163,20 @@ TTT_API const char* ttt_last_error(void);
  */
 TTT_API uint64_t ttt_launch_count(void);
 
+/*
+ * Per-kernel timing, for benchmarks.  ttt_kernel_timing(1) clears the record
+ * and starts bracketing every kernel launch of this library with two CUDA
+ * events recorded on the launch's stream; ttt_kernel_timing(0) stops.
+ * ttt_kernel_times waits for the recorded events and reports, per kernel
+ * name (at most max_kernels), the summed device time in ms and the launch
+ * count; the names go to `names` as a '\n'-separated list (truncated to
+ * names_cap bytes).  Returns the number of distinct kernels, -1 on a CUDA
+ * error.  total_ms and launches may be NULL.
+ */
+TTT_API ttt_status ttt_kernel_timing(int enable);
+TTT_API int ttt_kernel_times(int max_kernels, char* names, size_t names_cap, double* total_ms,
+                             uint64_t* launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -11,7 +11,9 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/tttmlp.h"
 #include "internal.h"
@@ -19,7 +21,33 @@
 namespace ttt {
 
 static std::atomic<uint64_t> g_launches{0};
-void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// Per-kernel timing: while on, each launch is bracketed by two CUDA events on
+// its own stream; ttt_kernel_times sums the elapsed times per kernel name.
+struct TimedLaunch {
+    const char* name;
+    cudaEvent_t start, stop;
+};
+static std::mutex g_timing_mu;
+static std::atomic<bool> g_timing_on{false};
+static std::vector<TimedLaunch> g_timed;
+
+LaunchScope::LaunchScope(const char* name, cudaStream_t s) : name_(name), s_(s) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (g_timing_on.load(std::memory_order_relaxed)) {
+        if (cudaEventCreate(&start_) == cudaSuccess) cudaEventRecord(start_, s_);
+        else start_ = nullptr;
+    }
+}
+
+LaunchScope::~LaunchScope() {
+    if (!start_) return;
+    cudaEvent_t stop = nullptr;
+    if (cudaEventCreate(&stop) != cudaSuccess) { cudaEventDestroy(start_); return; }
+    cudaEventRecord(stop, s_);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timed.push_back({name_, start_, stop});
+}
 
 static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
 
@@ -300,6 +328,46 @@ ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl) {
     g_scan_impl.store(scan_impl);
     g_proj_impl.store(proj_impl);
     return TTT_OK;
+}
+
+ttt_status ttt_kernel_timing(int enable) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    if (enable) {
+        for (auto& r : g_timed) { cudaEventDestroy(r.start); cudaEventDestroy(r.stop); }
+        g_timed.clear();
+    }
+    g_timing_on.store(enable != 0);
+    return TTT_OK;
+}
+
+int ttt_kernel_times(int max_kernels, char* names, size_t names_cap, double* total_ms, uint64_t* launches) {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    std::vector<std::string> keys;
+    std::vector<double> ms;
+    std::vector<uint64_t> cnt;
+    for (auto& r : g_timed) {
+        if (cudaEventSynchronize(r.stop) != cudaSuccess) return -1;
+        float e = 0.f;
+        if (cudaEventElapsedTime(&e, r.start, r.stop) != cudaSuccess) return -1;
+        size_t k = 0;
+        while (k < keys.size() && keys[k] != r.name) ++k;
+        if (k == keys.size()) { keys.emplace_back(r.name); ms.push_back(0.0); cnt.push_back(0); }
+        ms[k] += e;
+        cnt[k] += 1;
+    }
+    std::string csv;
+    const int n = (int)keys.size() < max_kernels ? (int)keys.size() : max_kernels;
+    for (int k = 0; k < n; ++k) {
+        if (total_ms) total_ms[k] = ms[k];
+        if (launches) launches[k] = cnt[k];
+        csv += keys[k];
+        csv += '\n';
+    }
+    if (names && names_cap) {
+        std::strncpy(names, csv.c_str(), names_cap - 1);
+        names[names_cap - 1] = '\0';
+    }
+    return (int)keys.size();
 }
 
 const char* ttt_last_error(void) { return t_err.c_str(); }

@@ -53,6 +53,19 @@ cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const t
                                   float* const out[3], int T, int N, int Dm, int accumulate,
                                   cudaStream_t s);
 
-void count_launch();
+// Counts a kernel launch and, while kernel timing is on, brackets it with
+// CUDA events recorded on its stream.  Construct right before the launch.
+class LaunchScope {
+  public:
+    LaunchScope(const char* name, cudaStream_t s);
+    ~LaunchScope();
+    LaunchScope(const LaunchScope&) = delete;
+    LaunchScope& operator=(const LaunchScope&) = delete;
+
+  private:
+    const char* name_;
+    cudaStream_t s_;
+    cudaEvent_t start_ = nullptr;
+};
 
 }  // namespace ttt

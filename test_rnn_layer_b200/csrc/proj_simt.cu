@@ -98,7 +98,7 @@ cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const th
     cudaError_t e = cudaFuncSetAttribute(proj_per_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    count_launch();
+    LaunchScope scope("proj_per_head", s);
     dim3 grid((T + kPhTok - 1) / kPhTok, H);
     proj_per_head_kernel<<<grid, kPhThreads, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16,
                                                         out[0], out[1], out[2], T, d);
@@ -108,7 +108,7 @@ cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const th
 cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
                                   float* const out[3], int T, int N, int Dm, int accumulate,
                                   cudaStream_t s) {
-    count_launch();
+    LaunchScope scope("proj_full_simt", s);
     dim3 grid((N + kGT - 1) / kGT, (T + kGT - 1) / kGT, 3);
     proj_full_simt_kernel<<<grid, 256, 0, s>>>(A, a_bf16, theta[0], theta[1], theta[2], th_bf16, out[0], out[1],
                                                 out[2], T, N, Dm, accumulate);

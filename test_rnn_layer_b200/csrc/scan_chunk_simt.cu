@@ -157,7 +157,7 @@ cudaError_t launch_scan_chunk_simt(const ScanArgs& a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(scan_chunk_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    count_launch();
+    LaunchScope scope("scan_chunk_simt", s);
     scan_chunk_simt_kernel<<<a.H, kThreads, smem, s>>>(a);
     return cudaGetLastError();
 }

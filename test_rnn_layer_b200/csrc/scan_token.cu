@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(4 * D) scan_token_kernel(ScanArgs a) {
 }  // namespace
 
 cudaError_t launch_scan_token(const ScanArgs& a, cudaStream_t s) {
-    count_launch();
+    LaunchScope scope("scan_token", s);
     switch (a.d) {
         case 16: scan_token_kernel<16><<<a.H, 64, 0, s>>>(a); break;
         case 32: scan_token_kernel<32><<<a.H, 128, 0, s>>>(a); break;

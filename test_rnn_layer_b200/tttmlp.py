@@ -23,7 +23,8 @@ TTT_F32, TTT_BF16 = 0, 1
 DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
-            "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count"]
+            "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
+            "ttt_kernel_timing", "ttt_kernel_times"]
 
 
 class TTTError(RuntimeError):
@@ -70,6 +71,11 @@ def lib():
         L.ttt_last_error.argtypes = []
         L.ttt_launch_count.restype = ctypes.c_uint64
         L.ttt_launch_count.argtypes = []
+        L.ttt_kernel_timing.restype = i
+        L.ttt_kernel_timing.argtypes = [i]
+        L.ttt_kernel_times.restype = i
+        L.ttt_kernel_times.argtypes = [i, ctypes.c_char_p, sz, ctypes.POINTER(ctypes.c_double),
+                                       ctypes.POINTER(ctypes.c_uint64)]
         _lib = L
     return _lib
 
@@ -97,6 +103,22 @@ def ttt_last_error() -> str:
 
 def ttt_launch_count() -> int:
     return int(lib().ttt_launch_count())
+
+
+def ttt_kernel_timing(enable: bool) -> int:
+    return int(lib().ttt_kernel_timing(1 if enable else 0))
+
+
+def ttt_kernel_times(max_kernels: int = 32) -> dict:
+    """{kernel name: (total ms, launches)} recorded since ttt_kernel_timing(True)."""
+    names = ctypes.create_string_buffer(4096)
+    ms = (ctypes.c_double * max_kernels)()
+    cnt = (ctypes.c_uint64 * max_kernels)()
+    n = lib().ttt_kernel_times(max_kernels, names, 4096, ms, cnt)
+    if n < 0:
+        raise TTTError(TTT_ERR_CUDA, "ttt_kernel_times")
+    keys = names.value.decode().split("\n")[:min(n, max_kernels)]
+    return {k: (ms[i], int(cnt[i])) for i, k in enumerate(keys)}
 
 
 def ttt_mlp_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
