@@ -146,6 +146,36 @@ TTT_API ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_
                                 ttt_stream_t stream);
 
 /*
+ * ttt_mlp_forward for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart: this is a deployment aid.  Code embedded in a
+ * host framework that owns the allocator, plug-ins forbidden to call
+ * cudaMalloc, or services that must not allocate after start-up cannot obtain
+ * a workspace.  This entry point takes the same arguments as ttt_mlp_forward
+ * except the workspace and runs the same kernels; its scratch is a fixed
+ * 32 MiB array in the library's own device memory, held by every GPU that
+ * loads the library until the process exits.
+ *   - Shapes whose ttt_mlp_workspace_size exceeds 32 MiB are rejected with
+ *     TTT_ERR_UNSUPPORTED and a message saying so.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.  (If the
+ *     caller switched ttt_kernel_timing on, that hook still creates events.)
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     the status word is cleared at the start of each call.  Calls whose GPU
+ *     work overlaps (other streams, other host threads) race on it: order them.
+ *   - Divergence and expired waits are recorded in that array but not
+ *     reported: check the outputs for NaN/Inf where that matters.
+ */
+TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void* X,
+                                           const void* theta_q, const void* theta_k, const void* theta_v,
+                                           const float* W1_0, const float* W2_0, float eta, int b,
+                                           ttt_direction dir, const float* alpha_f, const float* alpha_r,
+                                           void* Y, float* Z_out, float* W1_T, float* W2_T,
+                                           ttt_stream_t stream);
+
+/*
  * Kernel selection, process-wide (for tests and comparisons): 0 = automatic
  * (the fastest kernel that takes the shape), 1 = the FP32 SIMT kernels,
  * 2 = the tensor-core kernels (a later ttt_mlp_forward returns

@@ -70,6 +70,20 @@ ttt_status fail(ttt_status code, const char* fmt, ...) {
     return code;
 }
 
+}  // namespace
+
+ttt_status ttt::set_error(ttt_status code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_err = buf;
+    return code;
+}
+
+namespace {
+
 #define CUDA_TRY(expr)                                                                           \
     do {                                                                                         \
         cudaError_t e_ = (expr);                                                                 \

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/tttmlp.h"
+
 namespace ttt {
 
 // Status bits a kernel may set in the workspace status word.
@@ -52,6 +54,9 @@ cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const th
 cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
                                   float* const out[3], int T, int N, int Dm, int accumulate,
                                   cudaStream_t s);
+
+// Records a message for ttt_last_error() on this thread and returns `code`.
+ttt_status set_error(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 
 // Counts a kernel launch and, while kernel timing is on, brackets it with
 // CUDA events recorded on its stream.  Construct right before the launch.

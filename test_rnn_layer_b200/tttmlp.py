@@ -24,7 +24,7 @@ DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
-            "ttt_kernel_timing", "ttt_kernel_times"]
+            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc"]
 
 
 class TTTError(RuntimeError):
@@ -63,6 +63,8 @@ def lib():
         L.ttt_mlp_forward.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_forward_host.restype = i
         L.ttt_mlp_forward_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, sz, vp]
+        L.ttt_mlp_forward_noalloc.restype = i
+        L.ttt_mlp_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp]
         L.ttt_mlp_status.restype = i
         L.ttt_mlp_status.argtypes = [vp, vp]
         L.ttt_mlp_select_kernels.restype = i
@@ -147,6 +149,15 @@ def ttt_mlp_forward_host(desc, X_host, theta_q, theta_k, theta_v, W1_0, W2_0, et
                                           _p(W1_0), _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f),
                                           _p(alpha_r), _p(Y_host), _p(workspace), int(workspace_bytes),
                                           _stream(stream)))
+
+
+def ttt_mlp_forward_noalloc(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r,
+                            Y, Z_out, W1_T, W2_T, stream=None) -> int:
+    """ttt_mlp_forward without a workspace argument: for callers that cannot
+    allocate device memory (the library uses its own fixed 32 MiB scratch)."""
+    return int(lib().ttt_mlp_forward_noalloc(ctypes.byref(desc), _p(X), _p(theta_q), _p(theta_k), _p(theta_v),
+                                             _p(W1_0), _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f),
+                                             _p(alpha_r), _p(Y), _p(Z_out), _p(W1_T), _p(W2_T), _stream(stream)))
 
 
 def ttt_mlp_status(workspace, stream=None) -> int:
