@@ -155,11 +155,19 @@ struct Dir {
 };
 
 ttt_status project(const ttt_mlp_desc& q, const void* src, int src_bf16, const void* const th[3],
-                   float* const out[3], int accumulate, cudaStream_t s) {
+                   float* const out[3], int accumulate, int* status, cudaStream_t s) {
     const int th_bf16 = q.x_dtype == TTT_BF16;
     if (q.per_head_input) {
         if (accumulate) return fail(TTT_ERR_UNSUPPORTED, "internal: accumulate in per-head projection");
         CUDA_TRY(launch_proj_per_head(src, src_bf16, th, th_bf16, out, q.T, q.H, q.d, s));
+        return TTT_OK;
+    }
+    const int impl = g_proj_impl.load();
+    const bool tc_ok = src_bf16 && th_bf16 && proj_full_tc_supported(q.D, q.D);
+    if (impl == 2 && !tc_ok)
+        return fail(TTT_ERR_UNSUPPORTED, "tensor-core projection needs bf16 inputs, D %% 256 == 0");
+    if (tc_ok && impl != 1) {
+        CUDA_TRY(launch_proj_full_tc(src, th, out, q.T, q.D, q.D, accumulate, status, s));
     } else {
         CUDA_TRY(launch_proj_full_simt(src, src_bf16, th, th_bf16, out, q.T, q.D, q.D, accumulate, s));
     }
@@ -263,6 +271,7 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     const size_t n = (size_t)q.T * q.D;
     const size_t nW = (size_t)q.H * q.m * q.d;
     float* xp = reinterpret_cast<float*>(ws + L.xp);
+    int* status = reinterpret_cast<int*>(ws + L.status);
 
     // first (or only) direction
     Dir d0{};
@@ -273,7 +282,7 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     else { d0.out = Y; d0.out_bf16 = x_bf16; }
     d0.delta = L.split_reverse ? reinterpret_cast<__nv_bfloat16*>(ws + L.delta) : nullptr;
     d0.zdbg = Z_out; d0.w1t = W1_T; d0.w2t = W2_T;
-    st = project(q, X, x_bf16, th, qkv, 0, s);
+    st = project(q, X, x_bf16, th, qkv, 0, status, s);
     if (st != TTT_OK) return st;
     st = scan(q, L, ws, W1_0, W2_0, eta, b, d0, s);
     if (st != TTT_OK) return st;
@@ -283,9 +292,9 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     if (L.split_reverse) {
         // theta X' = theta X + theta (X' - X): add the projection of the bf16
         // gate increment onto the forward projections already in place.
-        st = project(q, ws + L.delta, 1, th, qkv, 1, s);
+        st = project(q, ws + L.delta, 1, th, qkv, 1, status, s);
     } else {
-        st = project(q, xp, 0, th, qkv, 0, s);
+        st = project(q, xp, 0, th, qkv, 0, status, s);
     }
     if (st != TTT_OK) return st;
     Dir d1{};

@@ -55,6 +55,11 @@ cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const t
                                   float* const out[3], int T, int N, int Dm, int accumulate,
                                   cudaStream_t s);
 
+// tcgen05 projections (bf16 A and Theta, N % 256 == 0, K % 64 == 0), same contract.
+bool proj_full_tc_supported(int N, int K);
+cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
+                                int accumulate, int* status, cudaStream_t s);
+
 // Records a message for ttt_last_error() on this thread and returns `code`.
 ttt_status set_error(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
 

@@ -1,0 +1,244 @@
+// theta_Q / theta_K / theta_V projections of the full layer on the tcgen05
+// tensor cores: C_w[t, n] (+)= sum_c A[t, c] Theta_w[n, c], A and Theta bf16,
+// fp32 accumulation in TMEM, fp32 output (paper notes page, "关键设计 /
+// TTT-MLP 层": the outer-loop key/value/query projections).
+//
+// Persistent kernel, one CTA per SM, 128 x 256 output tiles (M = 128 tokens,
+// N = 256 features of one projection), K consumed in 64-wide blocks:
+//   warp 0      TMA producer: A and Theta tiles into a 4-stage ring (128-byte swizzle)
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M128 N256 K16) and commits
+//   warps 2..5  epilogue: TMEM -> registers -> swizzled shared staging -> TMA store
+//               (or TMA reduce-add when accumulating onto C)
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile overlap
+// the main loop of the next.  Every wait is bounded; on expiry the CTA records
+// kStatusTimeout, drains and exits.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_prims.cuh"
+
+namespace ttt {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int B_BYTES = BN * BK * 2;          // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BUF = 32 * 32 * 4;          // one 32 x 32 fp32 box
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_WARPS * 2 * EPI_BUF + 256;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct ProjTcArgs {
+    CUtensorMap mapA;
+    CUtensorMap mapB[3];
+    CUtensorMap mapC[3];
+    int K;                 // reduction length (model dim)
+    int m_tiles, n_tiles_per, tiles;
+    int accumulate;
+    int* status;
+};
+
+__global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_constant__ ProjTcArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage_base = smem;
+    uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(epi_base + EPI_WARPS * 2 * EPI_BUF);
+    uint64_t* empty = full + STAGES;
+    uint64_t* tmem_full = empty + STAGES;
+    uint64_t* tmem_empty = tmem_full + 2;
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { tc::mbar_init(&full[s], 1); tc::mbar_init(&empty[s], 1); }
+        for (int a = 0; a < 2; ++a) { tc::mbar_init(&tmem_full[a], 1); tc::mbar_init(&tmem_empty[a], EPI_WARPS); }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::tma_prefetch_desc(&p.mapA);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_base_slot, TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_slot;
+    const int KB = p.K / BK;
+    const int n_tiles = 3 * p.n_tiles_per;
+
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicOr(p.status, kStatusTimeout);
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer
+        if (tc::elect_one()) {
+            int s = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
+                const int mt = tile / n_tiles, nt = tile % n_tiles;
+                const int which = nt / p.n_tiles_per;
+                const int n0 = (nt % p.n_tiles_per) * BN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&empty[s], phase ^ 1, abort_flag)) { give_up(); break; }
+                    uint8_t* st = stage_base + s * STAGE_BYTES;
+                    tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                    tc::tma_load_2d(st, &p.mapA, kb * BK, mt * BM, &full[s]);
+                    tc::tma_load_2d(st + A_BYTES, &p.mapB[which], kb * BK, n0, &full[s]);
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (tc::elect_one()) {
+            constexpr uint32_t idesc = tc::instr_desc(1, BM, BN, 0, 0);
+            int s = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!tc::mbar_wait(&tmem_empty[acc], acc_phase ^ 1, abort_flag)) { give_up(); break; }
+                tc::tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * BN;
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!tc::mbar_wait(&full[s], phase, abort_flag)) { ok = false; break; }
+                    tc::tc_fence_after();
+                    const uint32_t a_addr = tc::smem_u32(stage_base + s * STAGE_BYTES);
+                    const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = tc::smem_desc(a_addr + k * 32, 16, 1024);
+                        const uint64_t bd = tc::smem_desc(b_addr + k * 32, 16, 1024);
+                        tc::mma_f16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
+                    }
+                    tc::mma_commit(&empty[s]);
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
+                }
+                if (!ok) { give_up(); break; }
+                tc::mma_commit(&tmem_full[acc]);
+            }
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5 -> TMEM lane quarters 2, 3, 0, 1)
+        const int q = warp % 4;
+        uint8_t* bufs = epi_base + (warp - 2) * 2 * EPI_BUF;
+        int it = 0, nbuf = 0;
+        for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            const int mt = tile / n_tiles, nt = tile % n_tiles;
+            const int which = nt / p.n_tiles_per;
+            const int n0 = (nt % p.n_tiles_per) * BN;
+            if (!tc::mbar_wait(&tmem_full[acc], acc_phase, abort_flag)) { give_up(); break; }
+            tc::tc_fence_after();
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + c * 32, r);
+                tc::tmem_wait_ld();
+                uint8_t* buf = bufs + nbuf * EPI_BUF;
+                if (lane == 0) tc::bulk_wait_group_read<1>();   // the store that last used `buf` has read it
+                __syncwarp();
+                // row `lane` of a 32 x 32 fp32 box, 128-byte swizzle: 16-byte chunk j at (j ^ (row & 7))
+                uint4* row = reinterpret_cast<uint4*>(buf + lane * 128);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    row[j ^ (lane & 7)] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    const int x = n0 + c * 32, y = mt * BM + 32 * q;
+                    if (p.accumulate) tc::tma_reduce_add_2d(&p.mapC[which], buf, x, y);
+                    else tc::tma_store_2d(&p.mapC[which], buf, x, y);
+                    tc::bulk_commit_group();
+                }
+                nbuf ^= 1;
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tmem_empty[acc]);
+        }
+        if (lane == 0) tc::bulk_wait_group<0>();
+    }
+
+    if (*abort_flag) {
+        // let copies and MMAs already in flight land before the CTA's memory goes away
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (tc::globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool proj_full_tc_supported(int N, int K) { return N % BN == 0 && K % BK == 0 && N > 0 && K > 0; }
+
+cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
+                                int accumulate, int* status, cudaStream_t s) {
+    ProjTcArgs p{};
+    bool ok = make_map(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, T, (uint64_t)K * 2, BK, BM);
+    for (int w = 0; w < 3 && ok; ++w) {
+        ok = make_map(&p.mapB[w], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, theta[w], K, N, (uint64_t)K * 2, BK, BN) &&
+             make_map(&p.mapC[w], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out[w], N, T, (uint64_t)N * 4, 32, 32);
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    p.K = K;
+    p.m_tiles = (T + BM - 1) / BM;
+    p.n_tiles_per = N / BN;
+    p.tiles = p.m_tiles * 3 * p.n_tiles_per;
+    p.accumulate = accumulate;
+    p.status = status;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    LaunchScope scope("proj_full_tc", s);
+    const int grid = p.tiles < sms ? p.tiles : sms;
+    proj_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace ttt

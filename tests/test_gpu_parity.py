@@ -157,3 +157,16 @@ def test_launches_are_counted():
     n0 = L.ttt_launch_count()
     run_gpu(w, inp)
     assert L.ttt_launch_count() - n0 >= 2
+
+
+@pytest.mark.parametrize("T", [1000, 128])
+def test_full_layer_eta_zero_isolates_projection(impl, T):
+    """eta = 0 freezes the state, so z = W2_0 GELU(W1_0 q) depends only on the
+    projections: a tight check of the full-layer projection kernels (forward
+    pass, and the reverse pass's accumulation onto the forward projections)."""
+    w = S.FULL63S.with_T(T)
+    inp = S.make_inputs(w)
+    g = run_gpu(w, inp, eta=0.0, want_z=True)
+    o = run_oracle(w, inp, eta=0.0)
+    assert maxrel(to_np(g["Z"][0]), o["Z_f"]) < 1e-5
+    assert maxrel(to_np(g["Z"][1]), o["Z_r"]) < 2e-4
