@@ -193,9 +193,15 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
     a.status = reinterpret_cast<int*>(ws + L.status);
     a.scratch = reinterpret_cast<float*>(ws + L.scratch);
     a.scratch_per_head = L.scratch_per_head;
+    // Kernel choice: the tf32 tensor-core scan serves bf16-input layers (whose
+    // tolerance is 2e-2); fp32-input layers keep the fp32 kernels unless the
+    // tensor-core kernel is requested explicitly.
     const int impl = g_scan_impl.load();
-    if (impl == 2) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan kernel not available for this shape");
-    if (b == 1 && impl != 1) {
+    const bool tc_ok = scan_chunk_tc_supported(q.d, b);
+    if (impl == 2 && !tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
+    if (impl == 2 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+        CUDA_TRY(launch_scan_chunk_tc(a, s));
+    } else if (b == 1 && impl != 1) {
         CUDA_TRY(launch_scan_token(a, s));
     } else {
         CUDA_TRY(launch_scan_chunk_simt(a, s));

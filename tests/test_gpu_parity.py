@@ -132,7 +132,9 @@ def test_reverse_equals_flipped_forward_on_gpu():
     flipped["X"] = inp["X"].flip(1).contiguous()
     flipped["alpha_f"] = inp["alpha_r"]
     g_fwd = run_gpu(w, flipped, dirs="fwd", want_z=True)
-    assert maxrel(to_np(g_rev["Z"][0]), to_np(g_fwd["Z"][0].flip(1))) < 1e-4
+    # Same arithmetic up to the order of the token sums inside the tf32 MMAs
+    # (the reverse pass holds its tokens in natural order): a few tf32 ulps.
+    assert maxrel(to_np(g_rev["Z"][0]), to_np(g_fwd["Z"][0].flip(1))) < 1e-3
 
 
 def test_host_io_entry_point_matches_device_entry_point():
@@ -163,7 +165,9 @@ def test_launches_are_counted():
 def test_full_layer_eta_zero_isolates_projection(impl, T):
     """eta = 0 freezes the state, so z = W2_0 GELU(W1_0 q) depends only on the
     projections: a tight check of the full-layer projection kernels (forward
-    pass, and the reverse pass's accumulation onto the forward projections)."""
+    pass, and the reverse pass's accumulation onto the forward projections).
+    The scan is pinned to the fp32 kernel so only the projection kernel varies."""
+    L.check(L.ttt_mlp_select_kernels(1, impl), "select")
     w = S.FULL63S.with_T(T)
     inp = S.make_inputs(w)
     g = run_gpu(w, inp, eta=0.0, want_z=True)
