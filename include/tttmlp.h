@@ -179,8 +179,10 @@ TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void*
  * Kernel selection, process-wide (for tests and comparisons): 0 = automatic
  * (the fastest kernel that takes the shape), 1 = the FP32 SIMT kernels,
  * 2 = the tensor-core kernels (a later ttt_mlp_forward returns
- * TTT_ERR_UNSUPPORTED if the shape is outside them).  scan_impl selects the
- * scan kernel, proj_impl the full-mode projection kernel.
+ * TTT_ERR_UNSUPPORTED if the shape is outside them), and for the scan only
+ * 3 = the tensor-core scan with one CTA per head instead of a two-CTA
+ * cluster.  scan_impl selects the scan kernel, proj_impl the full-mode
+ * projection kernel.
  */
 TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);
 

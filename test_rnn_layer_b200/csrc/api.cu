@@ -199,8 +199,11 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
     const int impl = g_scan_impl.load();
     const bool tc_ok = scan_chunk_tc_supported(q.d, b);
     if (impl == 2 && !tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
-    if (impl == 2 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+    if (impl == 3) {
+        if (!tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
         CUDA_TRY(launch_scan_chunk_tc(a, s));
+    } else if (impl == 2 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+        CUDA_TRY(launch_scan_chunk_tc2(a, s));
     } else if (b == 1 && impl != 1) {
         CUDA_TRY(launch_scan_token(a, s));
     } else {
@@ -352,8 +355,10 @@ ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, co
 }
 
 ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl) {
-    if (scan_impl < 0 || scan_impl > 2 || proj_impl < 0 || proj_impl > 2)
-        return fail(TTT_ERR_INVALID_ARG, "kernel selector must be 0 (auto), 1 (SIMT) or 2 (tensor core)");
+    if (scan_impl < 0 || scan_impl > 3 || proj_impl < 0 || proj_impl > 2)
+        return fail(TTT_ERR_INVALID_ARG,
+                    "kernel selector must be 0 (auto), 1 (SIMT), 2 (tensor core) or, for the scan, 3 (tensor core, "
+                    "one CTA per head)");
     g_scan_impl.store(scan_impl);
     g_proj_impl.store(proj_impl);
     return TTT_OK;

@@ -46,7 +46,8 @@ cudaError_t launch_scan_chunk_simt(const ScanArgs& a, cudaStream_t s);   // any 
 long long scan_chunk_simt_scratch_floats(int d, int m, int b);
 // tcgen05 chunk scan: d = 64, 2 <= b <= 64, tf32 contractions with fp32 accumulation.
 bool scan_chunk_tc_supported(int d, int b);
-cudaError_t launch_scan_chunk_tc(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan_chunk_tc(const ScanArgs& a, cudaStream_t s);    // one CTA per head
+cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s);   // a cluster of two CTAs per head
 
 // Per-head projections: U[which][h, t, e] = sum_j theta_which[h][e][j] x[h, t, j].
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,

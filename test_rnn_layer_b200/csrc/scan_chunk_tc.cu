@@ -27,6 +27,7 @@
 // Stages are bulk-synchronous: threads write operands, one thread issues the
 // MMAs and commits them to an mbarrier, all threads wait (bounded) and read
 // the results from tensor memory.
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -75,15 +76,24 @@ __device__ __forceinline__ uint32_t sw_off(int R, int c, int stride) {
                       ((c & 3) << 2));
 }
 
-#ifdef TTT_DEBUG_DUMP
-// Debug builds only: head 0, chunk 0 intermediates are copied to g_dbg
-// (regions of 16384 floats), row-major [row][col].
+#if defined(TTT_DEBUG_DUMP) || defined(TTT_DEBUG_STAGES)
+// Debug builds only: TTT_DEBUG_DUMP copies head 0, chunk 0 intermediates to
+// g_dbg (regions of 16384 floats, row-major); TTT_DEBUG_STAGES accumulates the
+// cycles thread 0 of CTA 0 spends between stage boundaries.
 __device__ float* g_dbg = nullptr;
+#endif
+#ifdef TTT_DEBUG_DUMP
 enum { DBG_AT = 0, DBG_S, DBG_YT, DBG_PT, DBG_W1, DBG_DW2T, DBG_AQT, DBG_ZN, DBG_Z, DBG_D2T, DBG_G, DBG_N };
 #define DBG(region, row, col, ncol, val)                                                                       \
     do {                                                                                                       \
         if (g_dbg && blockIdx.x == 0 && c == 0) g_dbg[(region) * 16384 + (row) * (ncol) + (col)] = (val);     \
     } while (0)
+#else
+#define DBG(region, row, col, ncol, val) \
+    do {                                 \
+    } while (0)
+#endif
+#ifdef TTT_DEBUG_STAGES
 #define STAMP(k)                                                      \
     do {                                                              \
         if (tid == 0 && blockIdx.x == 0) {                            \
@@ -95,9 +105,6 @@ enum { DBG_AT = 0, DBG_S, DBG_YT, DBG_PT, DBG_W1, DBG_DW2T, DBG_AQT, DBG_ZN, DBG
 #else
 #define STAMP(k) \
     do {         \
-    } while (0)
-#define DBG(region, row, col, ncol, val) \
-    do {                                 \
     } while (0)
 #endif
 
@@ -136,23 +143,37 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-// K-major operand descriptor at K-step kk (8 tf32 = 32 bytes per step).
-__device__ __forceinline__ uint64_t kdesc(uint32_t base, int kk, uint32_t stride) {
-    return tc::smem_desc(base + (kk >> 2) * stride + (kk & 3) * 32, 16, 1024);
+// A K-major operand descriptor advanced to K-step kk (8 tf32 = 32 bytes per step): only the start-address field (low
+// bits, 16-byte units) changes, and it cannot carry out of its 14 bits.
+__device__ __forceinline__ uint64_t kstep(uint64_t d0, int kk, uint32_t stride) {
+    return d0 + (uint64_t)(((kk >> 2) * stride + (kk & 3) * 32) >> 4);
+}
+
+// Swizzled addressing for a thread that owns one column c and walks down the
+// rows: element (R, c) sits at ph[R & 7] + (R >> 3) * 1024, so the eight row
+// phases are computed once instead of per element.
+__device__ __forceinline__ void col_phases(int c, int stride, uint32_t (&ph)[8]) {
+    const uint32_t base = (uint32_t)((c >> 5) * stride + (c & 3) * 4);
+    const uint32_t cq = (uint32_t)((c & 31) >> 2);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) ph[r] = base + r * 128 + ((cq ^ r) << 4);
+}
+
+// Byte offset of the 16-byte chunk holding columns c .. c+3 (c a multiple of 4) of row R.
+__device__ __forceinline__ uint32_t row4_off(int R, int c, int stride) {
+    return (uint32_t)((c >> 5) * stride + (R >> 3) * 1024 + (R & 7) * 128 + ((((c & 31) >> 2) ^ (R & 7)) << 4));
+}
+
+__device__ __forceinline__ void st4(uint8_t* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
 }
 
 __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_constant__ ScanTcArgs P) {
     const ScanArgs& a = P.a;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* fW2G = reinterpret_cast<float*>(sm + OFF_W2G);
-    float* fGQ = reinterpret_cast<float*>(sm + OFF_GQ);
-    const float* fV = reinterpret_cast<const float*>(sm + OFF_V);
     float* fK = reinterpret_cast<float*>(sm + OFF_K);
     float* fQ = reinterpret_cast<float*>(sm + OFF_Q);
-    float* fX1 = reinterpret_cast<float*>(sm + OFF_X1);
-    float* fX2 = reinterpret_cast<float*>(sm + OFF_X2);
-    float* fX3 = reinterpret_cast<float*>(sm + OFF_X3);
     uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
     uint64_t* bar_k = bar_mma + 1;
     uint64_t* bar_q = bar_mma + 2;
@@ -237,57 +258,98 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
     uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0;
 
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
+    const uint64_t dK = tc::smem_desc(sK, 16, 1024), dQ = tc::smem_desc(sQ, 16, 1024);
+    const uint64_t dW2 = tc::smem_desc(sW2G, 16, 1024), dG = tc::smem_desc(sW2G + 8192, 16, 1024);
+    const uint64_t dX1 = tc::smem_desc(sX1, 16, 1024), dX2 = tc::smem_desc(sX2, 16, 1024);
+    const uint64_t dX3 = tc::smem_desc(sX3, 16, 1024), dGQ = tc::smem_desc(sGQ, 16, 1024);
     constexpr uint32_t ID32 = tc::instr_desc(2, 128, 32, 0, 0);
 
     // W2 [j][i] (tf32 copy, K-major) from the W2^T master in tensor memory.
     auto refresh_w2 = [&]() {
         const int j0 = 32 * (g & 1);
-        uint32_t r[32];
-        tc::tmem_ld_32x32b_x32(tm + lane_base + TM_W2T + hh * 64 + j0, r);
-        tc::tmem_wait_ld();
+        uint32_t ph[8];
+        col_phases(i_row, 16384, ph);
+        uint8_t* p = sm + OFF_W2G + (j0 >> 3) * 1024;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) fW2G[sw_off(j0 + k, i_row, 16384) / 4] = tf32r(__uint_as_float(r[k]));
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_W2T + hh * 64 + j0 + 16 * hf, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int kk = 16 * hf + k;
+                *reinterpret_cast<float*>(p + ph[kk & 7] + (kk >> 3) * 1024) = tf32r(__uint_as_float(r[k]));
+            }
+        }
     };
     refresh_w2();
 
+#ifdef TTT_DEBUG_STAGES
+    long long stamp_acc[20] = {};
+    long long stamp_last = clock64();
+#endif
     // One bulk-synchronous MMA stage.  Returns false (uniformly) once a wait has expired.
     auto mma_stage = [&](auto issue) -> bool {
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        if (__syncthreads_or(*abort_flag)) return false;
-        if (tid == 0) {
-            tc::tc_fence_after();
-            issue();
-            tc::mma_commit(bar_mma);
-        }
-        if (!tc::mbar_wait(bar_mma, ph_mma, abort_flag)) {
-            *abort_flag = 1;
-            atomicOr(a.status, kStatusTimeout);
-        }
-        ph_mma ^= 1;
-        tc::tc_fence_after();
-        return true;
-    };
-
-#ifdef TTT_DEBUG_DUMP
-    long long stamp_acc[16] = {};
-    long long stamp_last = clock64();
+#ifdef TTT_DEBUG_STAGES
+        long long t_a = clock64();
 #endif
-    for (int c = 0; c < nchunks; ++c) {
-        int y0, bc;
-        chunk_rows(c, y0, bc);
-        {
-            const bool ok = tc::mbar_wait(bar_k, ph_k, abort_flag) && tc::mbar_wait(bar_q, ph_q, abort_flag) &&
-                            tc::mbar_wait(bar_v, ph_v, abort_flag);
-            ph_k ^= 1;
-            ph_q ^= 1;
-            ph_v ^= 1;
-            if (!ok) {
+        if (__syncthreads_or(*abort_flag)) return false;
+#ifdef TTT_DEBUG_STAGES
+        long long t_b = clock64();
+#endif
+        // Only warp 0 issues and waits; the other warps park in the hardware
+        // barrier below instead of spinning on the mbarrier (spinning warps
+        // starve the issue slots and the load/store pipe of the working ones).
+        if (warp == 0) {
+            if (lane == 0) {
+                tc::tc_fence_after();
+                issue();
+                tc::mma_commit(bar_mma);
+            }
+            __syncwarp();
+#ifdef TTT_DEBUG_STAGES
+            long long t_c = clock64();
+#endif
+            const bool waited = tc::mbar_wait(bar_mma, ph_mma, nullptr);
+#ifdef TTT_DEBUG_STAGES
+            if (tid == 0 && blockIdx.x == 0) {
+                const long long t_d = clock64();
+                stamp_acc[16] += t_b - t_a;
+                stamp_acc[17] += t_c - t_b;
+                stamp_acc[18] += t_d - t_c;
+            }
+#endif
+            if (!waited && lane == 0) {
                 *abort_flag = 1;
                 atomicOr(a.status, kStatusTimeout);
             }
         }
+        ph_mma ^= 1;
+        const int stop = __syncthreads_or(*abort_flag);
+        tc::tc_fence_after();
+        return !stop;
+    };
+
+    for (int c = 0; c < nchunks; ++c) {
+        int y0, bc;
+        chunk_rows(c, y0, bc);
+        STAMP(14);
+        if (warp == 0) {   // the tiles' arrival is published to the other warps by the next barrier
+            const bool ok = tc::mbar_wait(bar_k, ph_k, nullptr) && tc::mbar_wait(bar_q, ph_q, nullptr) &&
+                            tc::mbar_wait(bar_v, ph_v, nullptr);
+            if (!ok && lane == 0) {
+                *abort_flag = 1;
+                atomicOr(a.status, kStatusTimeout);
+            }
+        }
+        ph_k ^= 1;
+        ph_q ^= 1;
+        ph_v ^= 1;
+        STAMP(15);
         if (bc < BT) {   // rows beyond the chunk hold other tokens (or zero fill): clear them
+            __syncthreads();
             for (int idx = tid; idx < (BT - bc) * DH; idx += THREADS) {
                 const int r = bc + idx / DH, j = idx % DH;
                 fK[sw_off(r, j, ST64) / 4] = 0.f;
@@ -300,55 +362,74 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         if (!mma_stage([&] {
                 for (int x = 0; x < 2; ++x)
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_W1 + x * 64 + kk * 8, kdesc(sK, kk, ST64), ID64,
+                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_W1 + x * 64 + kk * 8, kstep(dK, kk, ST64), ID64,
                                         kk > 0);
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ss(tm + TM_S, kdesc(sQ, kk, ST64), kdesc(sK, kk, ST64), ID64, kk > 0);
+                    tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
             }))
             break;
 
         STAMP(1);
         // ---- stage B (threads): G = GELU(A) to shared [t][i] and to tensor memory (G^T), keep G';
         //      K^T copy; M[t][s] = -S[t][s] for s after t
-        float gp[32];
+        __half2 gp[16];   // GELU'(A): |values| < 1.2, kept at fp16 (the same 11-bit significand as tf32)
         {
             const int t0 = 32 * (g & 1);
-            const uint32_t addr = tm + lane_base + TM_X + hh * 64 + t0;
-            uint32_t r[32];
-            tc::tmem_ld_32x32b_x32(addr, r);
-            tc::tmem_wait_ld();
-            uint32_t o[16];
+            uint32_t ph[8];
+            col_phases(i_row, 16384, ph);
+            uint8_t* p = sm + OFF_W2G + ((64 + t0) >> 3) * 1024;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                DBG(DBG_AT, i_row, t0 + k, 64, __uint_as_float(r[k]));
-                float gg;
-                gelu_as(__uint_as_float(r[k]), gg, gp[k], true);
-                gg = tf32r(gg);
-                fW2G[sw_off(64 + t0 + k, i_row, 16384) / 4] = gg;
-                r[k] = __float_as_uint(gg);
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t addr = tm + lane_base + TM_X + hh * 64 + t0 + 16 * hf;
+                uint32_t r[16];
+                tc::tmem_ld_32x32b_x16(addr, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    const int k = 16 * hf + 2 * k2;
+                    DBG(DBG_AT, i_row, t0 + k, 64, __uint_as_float(r[2 * k2]));
+                    DBG(DBG_AT, i_row, t0 + k + 1, 64, __uint_as_float(r[2 * k2 + 1]));
+                    float g0, g1, d0, d1;
+                    gelu_as(__uint_as_float(r[2 * k2]), g0, d0, true);
+                    gelu_as(__uint_as_float(r[2 * k2 + 1]), g1, d1, true);
+                    gp[8 * hf + k2] = __floats2half2_rn(d0, d1);
+                    g0 = tf32r(g0);
+                    g1 = tf32r(g1);
+                    *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) = g0;
+                    *reinterpret_cast<float*>(p + ph[(k + 1) & 7] + ((k + 1) >> 3) * 1024) = g1;
+                    r[2 * k2] = __float_as_uint(g0);
+                    r[2 * k2 + 1] = __float_as_uint(g1);
+                }
+                tc::tmem_st_32x32b_x16(addr, r);   // G^T in place: A operand of the W2^T update
             }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = r[k];
-            tc::tmem_st_32x32b_x16(addr, o);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) o[k] = r[16 + k];
-            tc::tmem_st_32x32b_x16(addr + 16, o);
         }
-        for (int idx = tid; idx < BT * DH; idx += THREADS) {
-            const int j = idx / BT, t = idx % BT;
-            fX1[sw_off(j, t, ST64) / 4] = fK[sw_off(t, j, ST64) / 4];
+        {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
+            const int j = tid & 63, tb = tid >> 6;
+            uint32_t ph[8];
+            col_phases(j, ST64, ph);
+            const uint8_t* src = sm + OFF_K + tb * 1024;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
+            st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
+            st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
         }
         if (q < 2) {
             const int t = 32 * q + lane, s0 = 16 * g;
             uint32_t r[16];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
             tc::tmem_wait_ld();
+            float m[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int s = s0 + k;
                 DBG(DBG_S, t, s, 64, __uint_as_float(r[k]));
-                fX2[sw_off(t, s, ST64) / 4] = after(s, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
+                m[k] = after(s, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
             }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                st4(sm + OFF_X2 + row4_off(t, s0 + 4 * c4, ST64), m[4 * c4], m[4 * c4 + 1], m[4 * c4 + 2],
+                    m[4 * c4 + 3]);
         }
         tc::tmem_wait_st();
 
@@ -356,7 +437,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         // ---- stage C: Y^T = W2 G^T  (A = rows 0..127 of W2G; rows 64.. give unused output rows)
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 32; ++kk)
-                    tc::mma_tf32_ss(tm + TM_Y, kdesc(sW2G, kk, 16384), kdesc(sW2G + 8192, kk, 16384), ID64, kk > 0);
+                    tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
             }))
             break;
 
@@ -364,18 +445,25 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         // ---- stage D (threads): D2' = -2 eta (Y - V) as [t][j] (over K) and [j][t]
         if (q < 2) {
             const int j = 32 * q + lane, t0 = 16 * g;
-            uint32_t r[16];
+            uint32_t r[16], ph[8];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_Y + t0, r);
+            col_phases(j, ST64, ph);
+            const uint32_t rg = (t0 >> 3) * 1024;
             tc::tmem_wait_ld();
+            float d2[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = t0 + k;
                 DBG(DBG_YT, j, t, 64, __uint_as_float(r[k]));
-                const float v = fV[sw_off(t, j, ST64) / 4];
-                const float d2 = (t < bc) ? tf32r(-2.0f * eta * (__uint_as_float(r[k]) - v)) : 0.f;
-                fK[sw_off(t, j, ST64) / 4] = d2;
-                fX3[sw_off(j, t, ST64) / 4] = d2;
+                const uint32_t off = rg + ph[k & 7] + (k >> 3) * 1024;
+                const float v = *reinterpret_cast<const float*>(sm + OFF_V + off);
+                d2[k] = (t < bc) ? tf32r(-2.0f * eta * (__uint_as_float(r[k]) - v)) : 0.f;
+                *reinterpret_cast<float*>(sm + OFF_K + off) = d2[k];
             }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                st4(sm + OFF_X3 + row4_off(j, t0 + 4 * c4, ST64), d2[4 * c4], d2[4 * c4 + 1], d2[4 * c4 + 2],
+                    d2[4 * c4 + 3]);
         }
 
         STAMP(4);
@@ -383,7 +471,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         if (!mma_stage([&] {
                 for (int x = 0; x < 2; ++x)
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_P + x * 64, tm + TM_W2T + x * 64 + kk * 8, kdesc(sK, kk, ST64), ID64,
+                        tc::mma_tf32_ts(tm + TM_P + x * 64, tm + TM_W2T + x * 64 + kk * 8, kstep(dK, kk, ST64), ID64,
                                         kk > 0);
             }))
             break;
@@ -397,32 +485,33 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         // ---- stage F (threads): Dl = P * G', written back in place (A operand of stage G)
         {
             const int t0 = 32 * (g & 1);
-            const uint32_t addr = tm + lane_base + TM_P + hh * 64 + t0;
-            uint32_t r[32];
-            tc::tmem_ld_32x32b_x32(addr, r);
-            tc::tmem_wait_ld();
-            uint32_t o0[16], o1[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                DBG(DBG_PT, i_row, t0 + k, 64, __uint_as_float(r[k]));
-                DBG(DBG_PT, i_row, t0 + 16 + k, 64, __uint_as_float(r[16 + k]));
-                o0[k] = __float_as_uint(tf32r(__uint_as_float(r[k]) * gp[k]));
-                o1[k] = __float_as_uint(tf32r(__uint_as_float(r[16 + k]) * gp[16 + k]));
+            for (int hf = 0; hf < 2; ++hf) {
+                const uint32_t addr = tm + lane_base + TM_P + hh * 64 + t0 + 16 * hf;
+                uint32_t r[16];
+                tc::tmem_ld_32x32b_x16(addr, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    DBG(DBG_PT, i_row, t0 + 16 * hf + 2 * k2, 64, __uint_as_float(r[2 * k2]));
+                    DBG(DBG_PT, i_row, t0 + 16 * hf + 2 * k2 + 1, 64, __uint_as_float(r[2 * k2 + 1]));
+                    const float2 d = __half22float2(gp[8 * hf + k2]);
+                    r[2 * k2] = __float_as_uint(tf32r(__uint_as_float(r[2 * k2]) * d.x));
+                    r[2 * k2 + 1] = __float_as_uint(tf32r(__uint_as_float(r[2 * k2 + 1]) * d.y));
+                }
+                tc::tmem_st_32x32b_x16(addr, r);
             }
-            tc::tmem_st_32x32b_x16(addr, o0);
-            tc::tmem_st_32x32b_x16(addr + 16, o1);
             tc::tmem_wait_st();
         }
 
-        STAMP(6);
         // ---- stage G: W1 += Dl^T K;  W2^T += G^T D2'
         if (!mma_stage([&] {
                 for (int x = 0; x < 2; ++x) {
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_W1 + x * 64, tm + TM_P + x * 64 + kk * 8, kdesc(sX1, kk, ST64), ID64,
+                        tc::mma_tf32_ts(tm + TM_W1 + x * 64, tm + TM_P + x * 64 + kk * 8, kstep(dX1, kk, ST64), ID64,
                                         1);
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_W2T + x * 64, tm + TM_X + x * 64 + kk * 8, kdesc(sX3, kk, ST64),
+                        tc::mma_tf32_ts(tm + TM_W2T + x * 64, tm + TM_X + x * 64 + kk * 8, kstep(dX3, kk, ST64),
                                         ID64, 1);
                 }
             }))
@@ -433,10 +522,10 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         if (!mma_stage([&] {
                 for (int x = 0; x < 2; ++x) {
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_W1 + x * 64 + kk * 8, kdesc(sQ, kk, ST64), ID64,
+                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_W1 + x * 64 + kk * 8, kstep(dQ, kk, ST64), ID64,
                                         kk > 0);
                     for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_P + x * 64 + kk * 8, kdesc(sX2, kk, ST64), ID64,
+                        tc::mma_tf32_ts(tm + TM_X + x * 64, tm + TM_P + x * 64 + kk * 8, kstep(dX2, kk, ST64), ID64,
                                         1);
                 }
             }))
@@ -469,20 +558,22 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         for (int u = 0; u < 2 && !stopped; ++u) {
             {
                 const int t0 = 32 * u + 16 * (g & 1);
-                uint32_t r[16];
+                uint32_t r[16], ph[8];
                 tc::tmem_ld_32x32b_x16(tm + lane_base + TM_X + hh * 64 + t0, r);
+                col_phases(i_row, 4096, ph);
+                uint8_t* p = sm + OFF_GQ + 2 * (g & 1) * 1024;
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     DBG(DBG_AQT, i_row, t0 + k, 64, __uint_as_float(r[k]));
                     float gg, unused;
                     gelu_as(__uint_as_float(r[k]), gg, unused, false);
-                    fGQ[sw_off(t0 - 32 * u + k, i_row, 4096) / 4] = tf32r(gg);
+                    *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) = tf32r(gg);
                 }
             }
             if (!mma_stage([&] {
                     for (int kk = 0; kk < 32; ++kk)
-                        tc::mma_tf32_ss(tm + TM_ZN + 32 * u, kdesc(sW2G, kk, 16384), kdesc(sGQ, kk, 4096), ID32,
+                        tc::mma_tf32_ss(tm + TM_ZN + 32 * u, kstep(dW2, kk, 16384), kstep(dGQ, kk, 4096), ID32,
                                         kk > 0);
                 }))
                 stopped = true;
@@ -498,14 +589,17 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         // ---- stage K (threads): Nm[t][s] = -N[s][t] for s after t  (into X1: K^T is dead)
         if (q >= 2) {
             const int s = 32 * (q - 2) + lane, t0 = 16 * g;
-            uint32_t r[16];
+            uint32_t r[16], ph[8];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
+            col_phases(s, ST64, ph);
+            uint8_t* p = sm + OFF_X1 + (t0 >> 3) * 1024;
             tc::tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = t0 + k;
                 DBG(DBG_N, s, t, 64, __uint_as_float(r[k]));
-                fX1[sw_off(t, s, ST64) / 4] = after(s, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
+                *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
+                    after(s, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
             }
         }
 
@@ -513,7 +607,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         // ---- stage L: Z^T += D2'^T Nm^T
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ss(tm + TM_ZN, kdesc(sX3, kk, ST64), kdesc(sX1, kk, ST64), ID64, 1);
+                    tc::mma_tf32_ss(tm + TM_ZN, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID64, 1);
             }))
             break;
 
@@ -524,14 +618,32 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
             uint32_t r[16];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
             tc::tmem_wait_ld();
+            STAMP(13);
+            // All 16 loads are issued before any is used: one dtype branch around
+            // the whole batch (a per-element branch would wait on each load).
             float xv[16];
+            const long long xrow = (long long)h * a.x_hs + (long long)y0 * a.x_ts + j;
+            if (a.xin_bf16) {
+                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.Xin) + xrow;
+                __nv_bfloat16 raw[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {   // all loads before any store (the output may alias nothing,
-                const int t = t0 + k;        // but the compiler cannot know that)
-                xv[k] = (t < bc) ? load_elem(a.Xin, (long long)h * a.x_hs + (long long)(y0 + t) * a.x_ts + j,
-                                             a.xin_bf16)
-                                 : 0.f;
+                for (int k = 0; k < 16; ++k)
+                    raw[k] = (t0 + k < bc) ? xb[(long long)(t0 + k) * a.x_ts] : __float2bfloat16_rn(0.f);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = __bfloat162float(raw[k]);
+            } else {
+                const float* xf = reinterpret_cast<const float*>(a.Xin) + xrow;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = (t0 + k < bc) ? xf[(long long)(t0 + k) * a.x_ts] : 0.f;
             }
+#ifdef TTT_DEBUG_STAGES
+            {
+                float sum = 0.f;
+                for (int k = 0; k < 16; ++k) sum += xv[k];
+                asm volatile("" ::"f"(sum));
+            }
+            STAMP(19);
+#endif
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = t0 + k;
@@ -549,11 +661,11 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc_kernel(const __grid_consta
         }
     }
 
-#ifdef TTT_DEBUG_DUMP
+#ifdef TTT_DEBUG_STAGES
     if (tid == 0 && blockIdx.x == 0 && g_dbg) {
         STAMP(13);
-        for (int k = 0; k < 16; ++k) g_dbg[11 * 16384 + 16000 + k] = (float)stamp_acc[k];
-        g_dbg[11 * 16384 + 16020] = (float)nchunks;
+        for (int k = 0; k < 20; ++k) g_dbg[11 * 16384 + 16000 + k] = (float)stamp_acc[k];
+        g_dbg[11 * 16384 + 16030] = (float)nchunks;
     }
 #endif
     if (*abort_flag) {
@@ -616,7 +728,7 @@ bool make_stream_map(CUtensorMap* m, const float* base, const ScanArgs& a, bool 
 
 }  // namespace
 
-#ifdef TTT_DEBUG_DUMP
+#if defined(TTT_DEBUG_DUMP) || defined(TTT_DEBUG_STAGES)
 extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump(float* p) {
     return (int)cudaMemcpyToSymbol(g_dbg, &p, sizeof(p));
 }

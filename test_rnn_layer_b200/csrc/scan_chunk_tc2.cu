@@ -1,0 +1,642 @@
+// Chunked TTT-MLP scan on the tcgen05 tensor cores with each head split over
+// a cluster of two CTAs (d = 64, m = 256, b <= 64).
+//
+// CTA r of the pair owns hidden units i in [128 r, 128 r + 128): its halves of
+// W1 [i][j] and W2^T [i][j] live in its tensor memory as fp32 accumulators for
+// the whole sequence (A operands of the MMAs that multiply by them, updated by
+// accumulate-MMAs), with a K-major copy of its W2 columns [j][i] in shared
+// memory.  Every product whose contraction runs over j or over the chunk's
+// tokens stays inside the CTA; the two that run over i are split and their
+// partial sums exchanged through distributed shared memory:
+//   Y^T  = W2 G^T           both CTAs receive the peer's [64 x 64] partial,
+//                           so both form the same D2' (fp32 a + b == b + a);
+//   [Z1^T; N] = [W2; G] Gq^T  each CTA owns 32 of the 64 tokens and receives
+//                           the peer's partial for those columns only.
+// The algebra per chunk (tokens t, s of the chunk in walking order; see the
+// one-CTA kernel for the derivation; paper notes page, "关键设计 / TTT-MLP 层"):
+//   A^T = W1 K^T, G = GELU(A), Y^T = W2 G^T, D2' = -2 eta (Y - V),
+//   P^T = W2^T D2'^T, Dl = P * GELU'(A), W1 += Dl^T K, W2^T += G^T D2',
+//   Aq^T = W1 Q^T + Dl^T M^T (M[t,s] = -q_t.k_s, s after t), Gq = GELU(Aq),
+//   [Z1^T; N] = [W2; G] Gq^T, Z^T = Z1^T + D2'^T Nm^T (Nm[t,s] = -N[s,t], s after t),
+//   out = x + tanh(alpha) z.
+// All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
+// shared-memory operands with the 128-byte swizzle.  Waits are bounded.
+//
+// Ordering of the exchange buffers (no handshake needed): the peer writes my
+// RY for chunk c+1 only after it received my [Z1;N] partial of chunk c, which
+// I send after I have read RY of chunk c; it writes my RZ for chunk c+1 only
+// after it received my Y partial of chunk c+1, which I send after I have read
+// RZ of chunk c.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_prims.cuh"
+
+namespace ttt {
+namespace {
+
+constexpr int BT = 64, DH = 64, MH = 256, MLOC = 128, THREADS = 512;
+
+// Shared memory (bytes from a 1024-aligned base), 128-byte-swizzled atoms of
+// 8 rows x 32 fp32 columns (atoms down the rows 1024 B apart).  A 64-row tile
+// read as a 128-row MMA operand spills into the next 16 KB, hence the order.
+constexpr int OFF_W2G = 0;        // 128 x 128: rows 0-63 my W2 columns [j][i], rows 64-127 G [t][i]; stride 16384
+constexpr int OFF_GQ = 65536;     // 64 x 128: Gq [t][i]; stride 8192
+constexpr int OFF_Q = 98304;      // 64 x 64: Q [t][j] (TMA)
+constexpr int OFF_K = 114688;     // 64 x 64: K [t][j] (TMA); then D2' [t][j]
+constexpr int OFF_X3 = 131072;    // 64 x 64: D2'^T [j][t]
+constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Nm [t_own][s] (32 rows)
+constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s]
+constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
+constexpr int OFF_RY = 196608;    // 64 x 64 fp32 plain [t][j]: the peer's Y^T partial
+constexpr int OFF_RZ = 212992;    // 32 x 128 fp32 plain [t_own][lane]: the peer's [Z1; N] partial for my tokens
+constexpr int OFF_BAR = 229376;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr int ST64 = 8192;
+
+// Tensor memory (128 lanes x 32-bit columns).
+constexpr uint32_t TM_W1 = 0;     // my W1 rows: [i][j]
+constexpr uint32_t TM_W2T = 64;   // my W2^T rows: [i][j]
+constexpr uint32_t TM_X = 128;    // A^T -> G^T -> Aq^T: [i][t]
+constexpr uint32_t TM_S = 192;    // S[t][s] (lanes t < 64)
+constexpr uint32_t TM_Y = 256;    // my Y^T partial [j][t] (lanes j < 64)
+constexpr uint32_t TM_P = 320;    // P^T -> Dl^T: [i][t]
+constexpr uint32_t TM_ZN = 384;   // [Z1^T; N] partial: [j | s][t]
+
+struct ScanTc2Args {
+    CUtensorMap mapQ, mapK, mapV;
+    ScanArgs a;
+    int full;
+};
+
+__device__ __forceinline__ float tf32r(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// erf-GELU (and GELU') with erf from Abramowitz & Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26: |error| <= 1.5e-7, far below the
+// tf32 rounding the results get; GELU and GELU' share one exponential.
+__device__ __forceinline__ void gelu_as(float a, float& g, float& gp, bool want_prime) {
+    const float x = fabsf(a) * 0.70710678118654752f;
+    const float u = __frcp_rn(fmaf(0.3275911f, x, 1.0f));
+    const float e = __expf(-0.5f * a * a);
+    float poly = fmaf(1.061405429f, u, -1.453152027f);
+    poly = fmaf(poly, u, 1.421413741f);
+    poly = fmaf(poly, u, -0.284496736f);
+    poly = fmaf(poly, u, 0.254829592f);
+    poly *= u;
+    const float erf_abs = 1.0f - poly * e;
+    const float Phi = 0.5f + 0.5f * copysignf(erf_abs, a);
+    g = a * Phi;
+    if (want_prime) gp = fmaf(a * 0.39894228040143268f, e, Phi);
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(tc::smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(tc::smem_u32(bar))
+        : "memory");
+}
+
+// A K-major operand descriptor advanced to K-step kk (8 tf32 = 32 bytes per step).
+__device__ __forceinline__ uint64_t kstep(uint64_t d0, int kk, uint32_t stride) {
+    return d0 + (uint64_t)(((kk >> 2) * stride + (kk & 3) * 32) >> 4);
+}
+
+// Column-fixed swizzled addressing: element (R, c) at ph[R & 7] + (R >> 3) * 1024.
+__device__ __forceinline__ void col_phases(int c, int stride, uint32_t (&ph)[8]) {
+    const uint32_t base = (uint32_t)((c >> 5) * stride + (c & 3) * 4);
+    const uint32_t cq = (uint32_t)((c & 31) >> 2);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) ph[r] = base + r * 128 + ((cq ^ r) << 4);
+}
+
+// Byte offset of the 16-byte chunk holding columns c .. c+3 (c a multiple of 4) of row R.
+__device__ __forceinline__ uint32_t row4_off(int R, int c, int stride) {
+    return (uint32_t)((c >> 5) * stride + (R >> 3) * 1024 + (R & 7) * 128 + ((((c & 31) >> 2) ^ (R & 7)) << 4));
+}
+
+__device__ __forceinline__ void st4(uint8_t* p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_constant__ ScanTc2Args P) {
+    const ScanArgs& a = P.a;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_k = bar_mma + 1;
+    uint64_t* bar_q = bar_mma + 2;
+    uint64_t* bar_v = bar_mma + 3;
+    uint64_t* bar_ry = bar_mma + 4;   // the peer's Y^T partial has landed in RY
+    uint64_t* bar_rz = bar_mma + 5;   // the peer's [Z1; N] partial has landed in RZ
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 6);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, g = warp >> 2;       // TMEM lane quarter; token group (16 tokens)
+    const uint32_t r_cta = tc::cluster_ctarank();
+    const uint32_t r_peer = r_cta ^ 1u;
+    const int i_loc = 32 * q + lane;             // my hidden row in the i-lane tiles
+    const int h = blockIdx.x >> 1;
+    const int T = a.T, b = a.b;
+    const int nchunks = (T + b - 1) / b;
+    const float eta = a.eta;
+    const bool my_tokens = (g >> 1) == (int)r_cta;   // tokens 16g .. 16g+15 belong to this CTA
+
+    const uint32_t sW2G = tc::smem_u32(sm + OFF_W2G), sGQ = tc::smem_u32(sm + OFF_GQ);
+    const uint32_t sQ = tc::smem_u32(sm + OFF_Q), sK = tc::smem_u32(sm + OFF_K);
+    const uint32_t sX1 = tc::smem_u32(sm + OFF_X1), sX2 = tc::smem_u32(sm + OFF_X2);
+    const uint32_t sX3 = tc::smem_u32(sm + OFF_X3);
+    // the peer's receive buffers and barriers
+    const uint32_t peer_ry = tc::mapa_shared(tc::smem_u32(sm + OFF_RY), r_peer);
+    const uint32_t peer_rz = tc::mapa_shared(tc::smem_u32(sm + OFF_RZ), r_peer);
+    const uint32_t peer_bar_ry = tc::mapa_shared(tc::smem_u32(bar_ry), r_peer);
+    const uint32_t peer_bar_rz = tc::mapa_shared(tc::smem_u32(bar_rz), r_peer);
+
+    if (tid == 0) {
+        tc::mbar_init(bar_mma, 1);
+        tc::mbar_init(bar_k, 1);
+        tc::mbar_init(bar_q, 1);
+        tc::mbar_init(bar_v, 1);
+        tc::mbar_init(bar_ry, 256);   // one arrival per peer thread holding Y^T rows
+        tc::mbar_init(bar_rz, 256);   // one arrival per peer thread holding my tokens' columns
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tmem_slot, 512);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    tc::cluster_sync();   // both CTAs' barriers exist before either arrives remotely
+    tc::tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+
+    auto chunk_rows = [&](int c, int& y0, int& bc) {
+        bc = min(b, T - c * b);
+        y0 = a.reverse ? (T - c * b - bc) : c * b;
+    };
+    auto load_tile = [&](const CUtensorMap* map, uint32_t dst_off, uint64_t* bar, int y0) {
+        tc::mbar_arrive_expect_tx(bar, BT * DH * 4);
+        for (int half = 0; half < 2; ++half) {
+            if (P.full) tma_load_3d(sm + dst_off + half * ST64, map, half * 32, h, y0, bar);
+            else tma_load_3d(sm + dst_off + half * ST64, map, half * 32, y0, h, bar);
+        }
+    };
+    auto after = [&](int s, int t) -> bool { return a.reverse ? (s < t) : (s > t); };
+
+    // ---- initial state: my rows of W1 and W2^T -> tensor memory
+    {
+        const int j0 = 16 * g;
+        const int ig = (int)r_cta * MLOC + i_loc;
+        const float* w1 = a.W1_0 + ((long long)h * MH + ig) * DH + j0;
+        const float* w2 = a.W2_0 + (long long)h * DH * MH + ig;   // W2[j][i] at j * MH + i
+        uint32_t r1[16], r2[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            r1[k] = __float_as_uint(w1[k]);
+            r2[k] = __float_as_uint(w2[(long long)(j0 + k) * MH]);
+        }
+        tc::tmem_st_32x32b_x16(tm + lane_base + TM_W1 + j0, r1);
+        tc::tmem_st_32x32b_x16(tm + lane_base + TM_W2T + j0, r2);
+        tc::tmem_wait_st();
+    }
+    if (tid == 0) {
+        int y0, bc;
+        chunk_rows(0, y0, bc);
+        load_tile(&P.mapK, OFF_K, bar_k, y0);
+        load_tile(&P.mapQ, OFF_Q, bar_q, y0);
+        load_tile(&P.mapV, OFF_V, bar_v, y0);
+    }
+
+    float tanh_a = 0.f;
+    if (q < 2) tanh_a = tanhf(a.alpha[h * DH + 32 * q + lane]);
+    int nonfinite = 0;
+    uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0;
+
+    constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
+    constexpr uint32_t ID32 = tc::instr_desc(2, 128, 32, 0, 0);
+    const uint64_t dK = tc::smem_desc(sK, 16, 1024), dQ = tc::smem_desc(sQ, 16, 1024);
+    const uint64_t dW2 = tc::smem_desc(sW2G, 16, 1024), dG = tc::smem_desc(sW2G + 8192, 16, 1024);
+    const uint64_t dX1 = tc::smem_desc(sX1, 16, 1024), dX2 = tc::smem_desc(sX2, 16, 1024);
+    const uint64_t dX3 = tc::smem_desc(sX3, 16, 1024), dGQ = tc::smem_desc(sGQ, 16, 1024);
+
+    // W2 [j][i] (tf32 copy, K-major) from my W2^T rows in tensor memory.
+    auto refresh_w2 = [&]() {
+        const int j0 = 16 * g;
+        uint32_t ph[8], r[16];
+        tc::tmem_ld_32x32b_x16(tm + lane_base + TM_W2T + j0, r);
+        col_phases(i_loc, 16384, ph);
+        uint8_t* p = sm + OFF_W2G + (j0 >> 3) * 1024;
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) = tf32r(__uint_as_float(r[k]));
+    };
+    refresh_w2();
+
+    // One MMA stage: all threads' operand writes become visible, warp 0 issues
+    // and waits for completion, the others park in the hardware barrier.
+    auto mma_stage = [&](auto issue) -> bool {
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        if (__syncthreads_or(*abort_flag)) return false;
+        if (warp == 0) {
+            if (lane == 0) {
+                tc::tc_fence_after();
+                issue();
+                tc::mma_commit(bar_mma);
+            }
+            __syncwarp();
+            if (!tc::mbar_wait(bar_mma, ph_mma, nullptr) && lane == 0) {
+                *abort_flag = 1;
+                atomicOr(a.status, kStatusTimeout);
+            }
+        }
+        ph_mma ^= 1;
+        const int stop = __syncthreads_or(*abort_flag);
+        tc::tc_fence_after();
+        return !stop;
+    };
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusTimeout);
+    };
+
+    for (int c = 0; c < nchunks; ++c) {
+        int y0, bc;
+        chunk_rows(c, y0, bc);
+        if (warp == 0) {
+            const bool ok = tc::mbar_wait(bar_k, ph_k, nullptr) && tc::mbar_wait(bar_q, ph_q, nullptr) &&
+                            tc::mbar_wait(bar_v, ph_v, nullptr);
+            if (!ok && lane == 0) give_up();
+        }
+        ph_k ^= 1;
+        ph_q ^= 1;
+        ph_v ^= 1;
+        if (bc < BT) {   // rows beyond the chunk hold other tokens (or zero fill): clear them
+            __syncthreads();
+            float* fK = reinterpret_cast<float*>(sm + OFF_K);
+            float* fQ = reinterpret_cast<float*>(sm + OFF_Q);
+            for (int idx = tid; idx < (BT - bc) * DH; idx += THREADS) {
+                const int rr = bc + idx / DH, j = idx % DH;
+                const uint32_t o = row4_off(rr, j & ~3, ST64) + (j & 3) * 4;
+                fK[o / 4] = 0.f;
+                fQ[o / 4] = 0.f;
+            }
+        }
+
+        // ---- A: A^T = W1 K^T (my rows);  S = Q K^T
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
+            }))
+            break;
+
+        // ---- B: G = GELU(A) to shared [t][i] and in place (G^T); G' kept; K^T; M mask
+        __half2 gp[8];
+        {
+            const int t0 = 16 * g;
+            uint32_t ph[8], r[16];
+            const uint32_t addr = tm + lane_base + TM_X + t0;
+            tc::tmem_ld_32x32b_x16(addr, r);
+            col_phases(i_loc, 16384, ph);
+            uint8_t* p = sm + OFF_W2G + ((64 + t0) >> 3) * 1024;
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+                const int k = 2 * k2;
+                float g0, g1, d0, d1;
+                gelu_as(__uint_as_float(r[k]), g0, d0, true);
+                gelu_as(__uint_as_float(r[k + 1]), g1, d1, true);
+                gp[k2] = __floats2half2_rn(d0, d1);
+                g0 = tf32r(g0);
+                g1 = tf32r(g1);
+                *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) = g0;
+                *reinterpret_cast<float*>(p + ph[(k + 1) & 7] + ((k + 1) >> 3) * 1024) = g1;
+                r[k] = __float_as_uint(g0);
+                r[k + 1] = __float_as_uint(g1);
+            }
+            tc::tmem_st_32x32b_x16(addr, r);
+        }
+        {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
+            const int j = tid & 63, tb = tid >> 6;
+            uint32_t ph[8];
+            col_phases(j, ST64, ph);
+            const uint8_t* src = sm + OFF_K + tb * 1024;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
+            st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
+            st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
+        }
+        if (q < 2) {   // M[t][s] = -S[t][s] for s after t
+            const int t = 32 * q + lane, s0 = 16 * g;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
+            tc::tmem_wait_ld();
+            float m[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) m[k] = after(s0 + k, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                st4(sm + OFF_X2 + row4_off(t, s0 + 4 * c4, ST64), m[4 * c4], m[4 * c4 + 1], m[4 * c4 + 2],
+                    m[4 * c4 + 3]);
+        }
+        tc::tmem_wait_st();
+
+        // ---- C: my Y^T partial = W2[:, mine] G[:, mine]^T  (rows 64.. of the A operand are unused)
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 16; ++kk)
+                    tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
+            }))
+            break;
+
+        // ---- D: exchange the Y^T partials; D2' = -2 eta (Y - V) as [t][j] (over K) and [j][t]
+        if (q < 2) {
+            const int j = 32 * q + lane, t0 = 16 * g;
+            uint32_t r[16], ph[8];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_Y + t0, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) tc::st_cluster_f32(peer_ry + ((t0 + k) * 64 + j) * 4, __uint_as_float(r[k]));
+            tc::mbar_arrive_remote(peer_bar_ry);
+            col_phases(j, ST64, ph);
+            const uint32_t rg = (t0 >> 3) * 1024;
+            if (!tc::mbar_wait_cluster(bar_ry, ph_ry)) give_up();
+            const float* ry = reinterpret_cast<const float*>(sm + OFF_RY);
+            float d2[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = t0 + k;
+                const uint32_t off = rg + ph[k & 7] + (k >> 3) * 1024;
+                const float y = __uint_as_float(r[k]) + ry[t * 64 + j];
+                const float v = *reinterpret_cast<const float*>(sm + OFF_V + off);
+                d2[k] = (t < bc) ? tf32r(-2.0f * eta * (y - v)) : 0.f;
+                *reinterpret_cast<float*>(sm + OFF_K + off) = d2[k];
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                st4(sm + OFF_X3 + row4_off(j, t0 + 4 * c4, ST64), d2[4 * c4], d2[4 * c4 + 1], d2[4 * c4 + 2],
+                    d2[4 * c4 + 3]);
+        }
+        ph_ry ^= 1;
+
+        // ---- E: P^T = W2^T D2'^T (my rows)
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+            }))
+            break;
+        if (tid == 0 && c + 1 < nchunks) {   // K and V buffers are free: fetch the next chunk's
+            int ny0, nbc;
+            chunk_rows(c + 1, ny0, nbc);
+            load_tile(&P.mapK, OFF_K, bar_k, ny0);
+            load_tile(&P.mapV, OFF_V, bar_v, ny0);
+        }
+
+        // ---- F: Dl = P * G' in place
+        {
+            const uint32_t addr = tm + lane_base + TM_P + 16 * g;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(addr, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+                const float2 d = __half22float2(gp[k2]);
+                r[2 * k2] = __float_as_uint(tf32r(__uint_as_float(r[2 * k2]) * d.x));
+                r[2 * k2 + 1] = __float_as_uint(tf32r(__uint_as_float(r[2 * k2 + 1]) * d.y));
+            }
+            tc::tmem_st_32x32b_x16(addr, r);
+            tc::tmem_wait_st();
+        }
+
+        // ---- G: W1 += Dl^T K;  W2^T += G^T D2'
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_W1, tm + TM_P + kk * 8, kstep(dX1, kk, ST64), ID64, 1);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_W2T, tm + TM_X + kk * 8, kstep(dX3, kk, ST64), ID64, 1);
+            }))
+            break;
+
+        // ---- H: Aq^T = W1_new Q^T + Dl^T M^T
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_X, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
+            }))
+            break;
+        if (tid == 0 && c + 1 < nchunks) {   // Q is free: fetch the next chunk's queries
+            int ny0, nbc;
+            chunk_rows(c + 1, ny0, nbc);
+            load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
+        }
+
+        // ---- I: W2 copy from the updated master; Gq = GELU(Aq) to shared [t][i]
+        refresh_w2();
+        {
+            const int t0 = 16 * g;
+            uint32_t ph[8], r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_X + t0, r);
+            col_phases(i_loc, ST64, ph);
+            uint8_t* p = sm + OFF_GQ + (t0 >> 3) * 1024;
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float gg, unused;
+                gelu_as(__uint_as_float(r[k]), gg, unused, false);
+                *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) = tf32r(gg);
+            }
+        }
+
+        // ---- J: my [Z1^T; N] partial = [W2; G][:, mine] Gq[:, mine]^T
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 16; ++kk)
+                    tc::mma_tf32_ss(tm + TM_ZN, kstep(dW2, kk, 16384), kstep(dGQ, kk, ST64), ID64, kk > 0);
+            }))
+            break;
+
+        // ---- K: exchange token halves of the partials; rows 0-63 -> full Z1^T back to tensor
+        //      memory, rows 64-127 -> Nm[t_own][s] = -N[s][t] for s after t
+        {
+            const int t0 = 16 * g;
+            const uint32_t addr = tm + lane_base + TM_ZN + t0;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(addr, r);
+            tc::tmem_wait_ld();
+            if (!my_tokens) {
+                const int tl0 = t0 - 32 * (int)r_peer;   // the peer's local token index
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    tc::st_cluster_f32(peer_rz + ((tl0 + k) * 128 + i_loc) * 4, __uint_as_float(r[k]));
+                tc::mbar_arrive_remote(peer_bar_rz);
+            } else {
+                const int tl0 = t0 - 32 * (int)r_cta;
+                if (!tc::mbar_wait_cluster(bar_rz, ph_rz)) give_up();
+                const float* rz = reinterpret_cast<const float*>(sm + OFF_RZ);
+                float v[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]) + rz[(tl0 + k) * 128 + i_loc];
+                if (q < 2) {   // Z1^T rows: the full sums become the accumulator of stage L
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(v[k]);
+                    tc::tmem_st_32x32b_x16(addr, r);
+                    tc::tmem_wait_st();
+                } else {       // N rows
+                    const int s = i_loc - 64;
+                    uint32_t ph[8];
+                    col_phases(s, ST64, ph);
+                    uint8_t* p = sm + OFF_X1 + (tl0 >> 3) * 1024;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
+                            after(s, t0 + k) ? tf32r(-v[k]) : 0.f;
+                }
+            }
+        }
+        ph_rz ^= 1;
+
+        // ---- L: Z^T (my tokens) += D2'^T Nm^T
+        if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID32, 1);
+            }))
+            break;
+
+        // ---- M: gate and stores (my tokens)
+        if (q < 2 && my_tokens) {
+            const int j = 32 * q + lane, t0 = 16 * g;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
+            float xv[16];
+            const long long xrow = (long long)h * a.x_hs + (long long)y0 * a.x_ts + j;
+            if (a.xin_bf16) {
+                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.Xin) + xrow;
+                __nv_bfloat16 raw[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    raw[k] = (t0 + k < bc) ? xb[(long long)(t0 + k) * a.x_ts] : __float2bfloat16_rn(0.f);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = __bfloat162float(raw[k]);
+            } else {
+                const float* xf = reinterpret_cast<const float*>(a.Xin) + xrow;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = (t0 + k < bc) ? xf[(long long)(t0 + k) * a.x_ts] : 0.f;
+            }
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = t0 + k;
+                if (t < bc) {
+                    const float z = __uint_as_float(r[k]);
+                    const long long xo = xrow + (long long)t * a.x_ts;
+                    const float dz = tanh_a * z;
+                    store_elem(a.Out, xo, a.out_bf16, xv[k] + dz);
+                    if (a.Delta) a.Delta[xo] = __float2bfloat16_rn(dz);
+                    if (a.Zdbg) a.Zdbg[xo] = z;
+                    nonfinite |= !isfinite(z);
+                }
+            }
+        }
+    }
+
+    if (*abort_flag) {
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (tc::globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
+    } else {
+        tc::tc_fence_before();
+        __syncthreads();
+        tc::tc_fence_after();
+        const int j0 = 16 * g;
+        const int ig = (int)r_cta * MLOC + i_loc;
+        uint32_t w[16], v[16];
+        tc::tmem_ld_32x32b_x16(tm + lane_base + TM_W1 + j0, w);
+        tc::tmem_ld_32x32b_x16(tm + lane_base + TM_W2T + j0, v);
+        tc::tmem_wait_ld();
+        if (a.W1_T) {
+            float* dst = a.W1_T + ((long long)h * MH + ig) * DH + j0;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) dst[k] = __uint_as_float(w[k]);
+        }
+        if (a.W2_T) {
+            float* dst = a.W2_T + (long long)h * DH * MH + ig;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) dst[(long long)(j0 + k) * MH] = __uint_as_float(v[k]);
+        }
+    }
+    if (nonfinite) atomicOr(a.status, kStatusNonFinite);
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tm, 512);
+    }
+    tc::cluster_sync();   // neither CTA leaves while the peer may still write into its shared memory
+}
+
+bool make_stream_map(CUtensorMap* m, const float* base, const ScanArgs& a, bool full) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+        return false;
+    auto fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cuuint64_t dims[3];
+    cuuint64_t strides[2];
+    cuuint32_t box[3];
+    if (full) {   // element (j, h, t) at t * D + h * d + j
+        dims[0] = DH; dims[1] = a.H; dims[2] = a.T;
+        strides[0] = DH * 4; strides[1] = (cuuint64_t)a.qkv_ts * 4;
+        box[0] = 32; box[1] = 1; box[2] = BT;
+    } else {      // element (j, t, h) at (h * T + t) * d + j
+        dims[0] = DH; dims[1] = a.T; dims[2] = a.H;
+        strides[0] = DH * 4; strides[1] = (cuuint64_t)a.qkv_hs * 4;
+        box[0] = 32; box[1] = BT; box[2] = 1;
+    }
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s) {
+    ScanTc2Args P{};
+    P.a = a;
+    P.full = (a.qkv_ts != DH) ? 1 : 0;
+    if (!make_stream_map(&P.mapQ, a.Q, a, P.full) || !make_stream_map(&P.mapK, a.K, a, P.full) ||
+        !make_stream_map(&P.mapV, a.V, a, P.full))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(scan_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * a.H);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope scope("scan_chunk_tc2", s);
+    e = cudaLaunchKernelEx(&cfg, scan_tc2_kernel, P);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace ttt

@@ -174,3 +174,15 @@ def test_full_layer_eta_zero_isolates_projection(impl, T):
     o = run_oracle(w, inp, eta=0.0)
     assert maxrel(to_np(g["Z"][0]), o["Z_f"]) < 1e-5
     assert maxrel(to_np(g["Z"][1]), o["Z_r"]) < 2e-4
+
+
+@pytest.mark.parametrize("w", [S.MINIBATCH.with_T(1000), S.SCALE18S.with_T(1000), S.FULL63S.with_T(777)],
+                         ids=["b16-per-head", "b64-per-head", "full-layer"])
+def test_one_cta_tensor_core_scan(w):
+    """The tensor-core scan with one CTA per head (the default runs each head on
+    a two-CTA cluster) against the oracle."""
+    L.check(L.ttt_mlp_select_kernels(3, 0), "select")
+    try:
+        _check(w)
+    finally:
+        L.ttt_mlp_select_kernels(0, 0)
