@@ -16,7 +16,7 @@
 // one-CTA kernel for the derivation; paper notes page, "关键设计 / TTT-MLP 层"):
 //   A^T = W1 K^T, G = GELU(A), Y^T = W2 G^T, D2' = -2 eta (Y - V),
 //   P^T = W2^T D2'^T, Dl = P * GELU'(A), W1 += Dl^T K, W2^T += G^T D2',
-//   Aq^T = W1 Q^T + Dl^T M^T (M[t,s] = -q_t.k_s, s after t), Gq = GELU(Aq),
+//   Aq^T = W1_old Q^T + Dl^T M^T (M[t,s] = q_t.k_s, s not after t), Gq = GELU(Aq),
 //   [Z1^T; N] = [W2; G] Gq^T, Z^T = Z1^T + D2'^T Nm^T (Nm[t,s] = -N[s,t], s after t),
 //   out = x + tanh(alpha) z.
 // All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
@@ -48,7 +48,7 @@ constexpr int OFF_Q = 98304;      // 64 x 64: Q [t][j] (TMA)
 constexpr int OFF_K = 114688;     // 64 x 64: K [t][j] (TMA); then D2' [t][j]
 constexpr int OFF_X3 = 131072;    // 64 x 64: D2'^T [j][t]
 constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Nm [t_own][s] (32 rows)
-constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s]
+constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s] (prefix mask)
 constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
 constexpr int OFF_RY = 196608;    // 64 x 64 fp32 plain [t][j]: the peer's Y^T partial
 constexpr int OFF_RZ = 212992;    // 32 x 128 fp32 plain [t_own][lane]: the peer's [Z1; N] partial for my tokens
@@ -59,11 +59,29 @@ constexpr int ST64 = 8192;
 // Tensor memory (128 lanes x 32-bit columns).
 constexpr uint32_t TM_W1 = 0;     // my W1 rows: [i][j]
 constexpr uint32_t TM_W2T = 64;   // my W2^T rows: [i][j]
-constexpr uint32_t TM_X = 128;    // A^T -> G^T -> Aq^T: [i][t]
+constexpr uint32_t TM_X = 128;    // A^T -> G^T: [i][t]
 constexpr uint32_t TM_S = 192;    // S[t][s] (lanes t < 64)
 constexpr uint32_t TM_Y = 256;    // my Y^T partial [j][t] (lanes j < 64)
 constexpr uint32_t TM_P = 320;    // P^T -> Dl^T: [i][t]
 constexpr uint32_t TM_ZN = 384;   // [Z1^T; N] partial: [j | s][t]
+constexpr uint32_t TM_AQ = 448;   // Aq^T: [i][t]
+
+#ifdef TTT_DEBUG_STAGES
+// Debug builds only: cycles thread 0 of CTA 0 spends between stage boundaries.
+__device__ float* g_dbg2 = nullptr;
+#define STAMP(k)                                                      \
+    do {                                                              \
+        if (tid == 0 && blockIdx.x == 0) {                            \
+            const long long now_ = clock64();                         \
+            stamp_acc[k] += now_ - stamp_last;                        \
+            stamp_last = now_;                                        \
+        }                                                             \
+    } while (0)
+#else
+#define STAMP(k) \
+    do {         \
+    } while (0)
+#endif
 
 struct ScanTc2Args {
     CUtensorMap mapQ, mapK, mapV;
@@ -242,6 +260,10 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     };
     refresh_w2();
 
+#ifdef TTT_DEBUG_STAGES
+    long long stamp_acc[20] = {};
+    long long stamp_last = clock64();
+#endif
     // One MMA stage: all threads' operand writes become visible, warp 0 issues
     // and waits for completion, the others park in the hardware barrier.
     auto mma_stage = [&](auto issue) -> bool {
@@ -265,14 +287,79 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::tc_fence_after();
         return !stop;
     };
+    // The same, with `work` (touching nothing the MMAs read or write) run by all
+    // threads while the tensor core computes.
+    auto mma_stage_with = [&](auto issue, auto work) -> bool {
+        tc::fence_proxy_async_smem();
+        tc::tc_fence_before();
+        if (__syncthreads_or(*abort_flag)) return false;
+        if (tid == 0) {
+            tc::tc_fence_after();
+            issue();
+            tc::mma_commit(bar_mma);
+        }
+        work();
+        if (warp == 0) {
+            __syncwarp();
+            if (!tc::mbar_wait(bar_mma, ph_mma, nullptr) && lane == 0) {
+                *abort_flag = 1;
+                atomicOr(a.status, kStatusTimeout);
+            }
+        }
+        ph_mma ^= 1;
+        const int stop = __syncthreads_or(*abort_flag);
+        tc::tc_fence_after();
+        return !stop;
+    };
     auto give_up = [&]() {
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeout);
     };
 
+    // Gate and stores of a finished chunk (rows y0c .. y0c + bcc - 1), my tokens;
+    // reads only the Z columns of tensor memory and global memory.
+    auto gate_chunk = [&](int y0c, int bcc) {
+        if (q < 2 && my_tokens) {
+            const int j = 32 * q + lane, t0 = 16 * g;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
+            float xv[16];
+            const long long xrow = (long long)h * a.x_hs + (long long)y0c * a.x_ts + j;
+            if (a.xin_bf16) {
+                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.Xin) + xrow;
+                __nv_bfloat16 raw[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    raw[k] = (t0 + k < bcc) ? xb[(long long)(t0 + k) * a.x_ts] : __float2bfloat16_rn(0.f);
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = __bfloat162float(raw[k]);
+            } else {
+                const float* xf = reinterpret_cast<const float*>(a.Xin) + xrow;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) xv[k] = (t0 + k < bcc) ? xf[(long long)(t0 + k) * a.x_ts] : 0.f;
+            }
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int t = t0 + k;
+                if (t < bcc) {
+                    const float z = __uint_as_float(r[k]);
+                    const long long xo = xrow + (long long)t * a.x_ts;
+                    const float dz = tanh_a * z;
+                    store_elem(a.Out, xo, a.out_bf16, xv[k] + dz);
+                    if (a.Delta) a.Delta[xo] = __float2bfloat16_rn(dz);
+                    if (a.Zdbg) a.Zdbg[xo] = z;
+                    nonfinite |= !isfinite(z);
+                }
+            }
+        }
+    };
+    int prev_y0 = 0, prev_bc = 0;   // the chunk whose gate is still pending (prev_bc == 0: none)
+
     for (int c = 0; c < nchunks; ++c) {
         int y0, bc;
         chunk_rows(c, y0, bc);
+        STAMP(13);
         if (warp == 0) {
             const bool ok = tc::mbar_wait(bar_k, ph_k, nullptr) && tc::mbar_wait(bar_q, ph_q, nullptr) &&
                             tc::mbar_wait(bar_v, ph_v, nullptr);
@@ -293,15 +380,29 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             }
         }
 
+        STAMP(0);
         // ---- A: A^T = W1 K^T (my rows);  S = Q K^T
-        if (!mma_stage([&] {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
-            }))
+        if (!mma_stage_with(
+                [&] {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_AQ, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
+                },
+                [&] {
+                    if (prev_bc) gate_chunk(prev_y0, prev_bc);
+                }))
             break;
+        prev_bc = 0;
+        if (tid == 0 && c + 1 < nchunks) {   // Q is free: fetch the next chunk's queries
+            int ny0, nbc;
+            chunk_rows(c + 1, ny0, nbc);
+            load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
+        }
 
+        STAMP(1);
         // ---- B: G = GELU(A) to shared [t][i] and in place (G^T); G' kept; K^T; M mask
         __half2 gp[8];
         {
@@ -328,39 +429,44 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             }
             tc::tmem_st_32x32b_x16(addr, r);
         }
-        {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
-            const int j = tid & 63, tb = tid >> 6;
-            uint32_t ph[8];
-            col_phases(j, ST64, ph);
-            const uint8_t* src = sm + OFF_K + tb * 1024;
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
-            st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
-            st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
-        }
-        if (q < 2) {   // M[t][s] = -S[t][s] for s after t
-            const int t = 32 * q + lane, s0 = 16 * g;
-            uint32_t r[16];
-            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
-            tc::tmem_wait_ld();
-            float m[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) m[k] = after(s0 + k, t) ? tf32r(-__uint_as_float(r[k])) : 0.f;
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                st4(sm + OFF_X2 + row4_off(t, s0 + 4 * c4, ST64), m[4 * c4], m[4 * c4 + 1], m[4 * c4 + 2],
-                    m[4 * c4 + 3]);
-        }
         tc::tmem_wait_st();
 
+        STAMP(2);
         // ---- C: my Y^T partial = W2[:, mine] G[:, mine]^T  (rows 64.. of the A operand are unused)
-        if (!mma_stage([&] {
-                for (int kk = 0; kk < 16; ++kk)
-                    tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
-            }))
+        if (!mma_stage_with(
+                [&] {
+                    for (int kk = 0; kk < 16; ++kk)
+                        tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
+                },
+                [&] {
+        {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
+                        const int j = tid & 63, tb = tid >> 6;
+                        uint32_t ph[8];
+                        col_phases(j, ST64, ph);
+                        const uint8_t* src = sm + OFF_K + tb * 1024;
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
+                        st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
+                        st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
+                    }
+                    if (q < 2) {   // M[t][s] = S[t][s] for s not after t (prefix)
+                        const int t = 32 * q + lane, s0 = 16 * g;
+                        uint32_t r[16];
+                        tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
+                        tc::tmem_wait_ld();
+                        float m[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) m[k] = after(s0 + k, t) ? 0.f : tf32r(__uint_as_float(r[k]));
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4)
+                            st4(sm + OFF_X2 + row4_off(t, s0 + 4 * c4, ST64), m[4 * c4], m[4 * c4 + 1], m[4 * c4 + 2],
+                                m[4 * c4 + 3]);
+                    }
+                }))
             break;
 
+        STAMP(3);
         // ---- D: exchange the Y^T partials; D2' = -2 eta (Y - V) as [t][j] (over K) and [j][t]
         if (q < 2) {
             const int j = 32 * q + lane, t0 = 16 * g;
@@ -391,19 +497,21 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         }
         ph_ry ^= 1;
 
+        STAMP(4);
         // ---- E: P^T = W2^T D2'^T (my rows)
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
             }))
             break;
-        if (tid == 0 && c + 1 < nchunks) {   // K and V buffers are free: fetch the next chunk's
+        if (tid == 0 && c + 1 < nchunks) {   // K and V buffers are free: fetch the next chunk's tiles
             int ny0, nbc;
             chunk_rows(c + 1, ny0, nbc);
             load_tile(&P.mapK, OFF_K, bar_k, ny0);
             load_tile(&P.mapV, OFF_V, bar_v, ny0);
         }
 
+        STAMP(5);
         // ---- F: Dl = P * G' in place
         {
             const uint32_t addr = tm + lane_base + TM_P + 16 * g;
@@ -420,35 +528,25 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             tc::tmem_wait_st();
         }
 
-        // ---- G: W1 += Dl^T K;  W2^T += G^T D2'
+        STAMP(6);
+        // ---- G: W1 += Dl^T K;  W2^T += G^T D2';  Aq^T += Dl^T M^T
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_W1, tm + TM_P + kk * 8, kstep(dX1, kk, ST64), ID64, 1);
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_W2T, tm + TM_X + kk * 8, kstep(dX3, kk, ST64), ID64, 1);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_AQ, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
             }))
             break;
 
-        // ---- H: Aq^T = W1_new Q^T + Dl^T M^T
-        if (!mma_stage([&] {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_X, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
-            }))
-            break;
-        if (tid == 0 && c + 1 < nchunks) {   // Q is free: fetch the next chunk's queries
-            int ny0, nbc;
-            chunk_rows(c + 1, ny0, nbc);
-            load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
-        }
-
+        STAMP(8);
         // ---- I: W2 copy from the updated master; Gq = GELU(Aq) to shared [t][i]
         refresh_w2();
         {
             const int t0 = 16 * g;
             uint32_t ph[8], r[16];
-            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_X + t0, r);
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_AQ + t0, r);
             col_phases(i_loc, ST64, ph);
             uint8_t* p = sm + OFF_GQ + (t0 >> 3) * 1024;
             tc::tmem_wait_ld();
@@ -460,6 +558,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             }
         }
 
+        STAMP(9);
         // ---- J: my [Z1^T; N] partial = [W2; G][:, mine] Gq[:, mine]^T
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 16; ++kk)
@@ -467,6 +566,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             }))
             break;
 
+        STAMP(10);
         // ---- K: exchange token halves of the partials; rows 0-63 -> full Z1^T back to tensor
         //      memory, rows 64-127 -> Nm[t_own][s] = -N[s][t] for s after t
         {
@@ -507,50 +607,27 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         }
         ph_rz ^= 1;
 
+        STAMP(11);
         // ---- L: Z^T (my tokens) += D2'^T Nm^T
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID32, 1);
             }))
             break;
+        prev_y0 = y0;
+        prev_bc = bc;
 
-        // ---- M: gate and stores (my tokens)
-        if (q < 2 && my_tokens) {
-            const int j = 32 * q + lane, t0 = 16 * g;
-            uint32_t r[16];
-            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
-            float xv[16];
-            const long long xrow = (long long)h * a.x_hs + (long long)y0 * a.x_ts + j;
-            if (a.xin_bf16) {
-                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.Xin) + xrow;
-                __nv_bfloat16 raw[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    raw[k] = (t0 + k < bc) ? xb[(long long)(t0 + k) * a.x_ts] : __float2bfloat16_rn(0.f);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) xv[k] = __bfloat162float(raw[k]);
-            } else {
-                const float* xf = reinterpret_cast<const float*>(a.Xin) + xrow;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) xv[k] = (t0 + k < bc) ? xf[(long long)(t0 + k) * a.x_ts] : 0.f;
-            }
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = t0 + k;
-                if (t < bc) {
-                    const float z = __uint_as_float(r[k]);
-                    const long long xo = xrow + (long long)t * a.x_ts;
-                    const float dz = tanh_a * z;
-                    store_elem(a.Out, xo, a.out_bf16, xv[k] + dz);
-                    if (a.Delta) a.Delta[xo] = __float2bfloat16_rn(dz);
-                    if (a.Zdbg) a.Zdbg[xo] = z;
-                    nonfinite |= !isfinite(z);
-                }
-            }
-        }
+        STAMP(12);
     }
 
+    if (prev_bc && !*abort_flag) gate_chunk(prev_y0, prev_bc);   // the last chunk's gate
+
+#ifdef TTT_DEBUG_STAGES
+    if (tid == 0 && blockIdx.x == 0 && g_dbg2) {
+        for (int k = 0; k < 20; ++k) g_dbg2[k] = (float)stamp_acc[k];
+        g_dbg2[30] = (float)nchunks;
+    }
+#endif
     if (*abort_flag) {
         const uint64_t t0 = tc::globaltimer_ns();
         while (tc::globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
@@ -611,6 +688,12 @@ bool make_stream_map(CUtensorMap* m, const float* base, const ScanArgs& a, bool 
 }
 
 }  // namespace
+
+#ifdef TTT_DEBUG_STAGES
+extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump2(float* p) {
+    return (int)cudaMemcpyToSymbol(g_dbg2, &p, sizeof(p));
+}
+#endif
 
 cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s) {
     ScanTc2Args P{};
