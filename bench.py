@@ -61,10 +61,12 @@ def _src_hash(*files) -> str:
 KERNEL_SRC = {
     "scan_chunk_simt": ("scan_chunk_simt.cu",),
     "scan_chunk_tc": ("scan_chunk_tc.cu",),
+    "scan_chunk_tc2": ("scan_chunk_tc2.cu",),
     "scan_token": ("scan_token.cu",),
     "proj_full_simt": ("proj_simt.cu",),
     "proj_full_tc": ("proj_tc.cu",),
     "proj_per_head": ("proj_simt.cu",),
+    "gate": ("gate.cu",),
 }
 
 
@@ -151,11 +153,15 @@ def _algorithmic(w):
     proj_flops = 2.0 * T * D * 3 * D
     return {
         "scan_chunk_tc": ("tensor_tf32", scan_flops),
+        "scan_chunk_tc2": ("tensor_tf32", scan_flops),
         "scan_chunk_simt": ("alu", scan_flops),
         "scan_token": ("alu", H * T * 7 * 2 * d * m),
         "proj_full_tc": ("tensor_bf16", proj_flops),
         "proj_full_simt": ("alu", proj_flops),
         "proj_per_head": ("hbm", T * D * (2 + 12)),
+        # x (bf16) + z (fp32) read, out (bf16) written; the forward launch also
+        # writes the bf16 increment: 10 B and 8 B per element, 9 on average
+        "gate": ("hbm", T * D * 9),
     }
 
 
@@ -182,6 +188,28 @@ def _roofline(name, ms_per_launch, w, peaks, clocks):
     return {"kernel": name, "bound": kind, "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": _traffic(name, units), "peak_note": note,
             "ms_per_launch": round(ms_per_launch, 4), "work_per_launch": work}
+
+
+# ------------------------------------------------------------------ multi-rank bookkeeping
+def rank_seed(rank: int) -> int:
+    """Each replica draws its own sequence."""
+    return rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's value (all ranks call this in the same order)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens of all replicas per second, timed by the slowest rank."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
 # ------------------------------------------------------------------ CPU side (oracle)
@@ -248,7 +276,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = _workload(args)
-    inp = S.make_inputs(w, seed=rank, device=dev)
+    inp = S.make_inputs(w, seed=rank_seed(rank), device=dev)
     desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
     direction = L.DIRS[w.dirs]
     ws = L.alloc_workspace(desc, w.b, direction, dev, host_io=True)
@@ -266,13 +294,6 @@ def run_ours(args, rank, world, local_rank):
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local_rank])
-
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step()
@@ -295,10 +316,10 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     launches = L.ttt_launch_count() - n_launch0
     clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1))
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
     ms_per_step = ms / args.steps
-    value = world * w.T / (ms_per_step * 1e-3)
+    value = whole_job_tokens_per_s(world, w.T, ms_per_step)
 
     # per-kernel device times over a second timed pass (events on the launch stream)
     L.ttt_kernel_timing(True)
@@ -335,9 +356,9 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(ns):
             e2e_step()
         barrier()
-        e2e_s = max_over_ranks(time.perf_counter() - t0) / ns
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
         nbytes = Xh.numel() * Xh.element_size()
-        e2e = {"value": world * w.T / e2e_s, "unit": UNIT, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
                "ms_per_step": e2e_s * 1e3, "steps": ns}
 
     cpu = None

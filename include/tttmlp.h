@@ -186,6 +186,17 @@ TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void*
  */
 TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);
 
+/*
+ * Fault injection for tests (process-wide).  While enabled, the two-CTA
+ * tensor-core scan kernel (the default for bf16 inputs) first waits on an
+ * mbarrier that nothing arrives on, with a 1 ms limit; the wait expires, the
+ * kernel records TTT_ERR_TIMEOUT in the status word, lets its copies in
+ * flight land, frees its tensor memory and returns (that call's outputs are
+ * invalid).  It exercises the bounded-wait failure path without stalling the
+ * GPU; the CUDA context stays usable.
+ */
+TTT_API ttt_status ttt_debug_inject_wait_timeout(int enable);
+
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 TTT_API const char* ttt_last_error(void);
 

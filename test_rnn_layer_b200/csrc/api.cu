@@ -50,6 +50,7 @@ LaunchScope::~LaunchScope() {
 }
 
 static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
+static std::atomic<int> g_inject_timeout{0};
 
 }  // namespace ttt
 
@@ -117,7 +118,7 @@ ttt_status check_desc(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
 }
 
 struct Layout {
-    size_t status, qkv[3], xp, delta, scratch, total;
+    size_t status, qkv[3], xp, delta, scratch, zbuf, total;
     long long scratch_per_head;
     bool split_reverse;   // reverse projection as theta X + theta bf16(X' - X)
 };
@@ -137,6 +138,9 @@ Layout plan(const ttt_mlp_desc& q, int b, ttt_direction dir) {
     // the SIMT chunk kernel may run for any b (it is selectable for b = 1 too)
     L.scratch_per_head = scan_chunk_simt_scratch_floats(q.d, q.m, b);
     off = align_up(off + (size_t)q.H * L.scratch_per_head * sizeof(float));
+    // z of one direction for the cluster tensor-core scan, whose gate runs separately
+    L.zbuf = off;
+    if (scan_chunk_tc_supported(q.d, b)) off = align_up(off + n * sizeof(float));
     L.total = off;
     return L;
 }
@@ -193,6 +197,7 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
     a.status = reinterpret_cast<int*>(ws + L.status);
     a.scratch = reinterpret_cast<float*>(ws + L.scratch);
     a.scratch_per_head = L.scratch_per_head;
+    a.inject_timeout = g_inject_timeout.load();
     // Kernel choice: the tf32 tensor-core scan serves bf16-input layers (whose
     // tolerance is 2e-2); fp32-input layers keep the fp32 kernels unless the
     // tensor-core kernel is requested explicitly.
@@ -203,7 +208,10 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
         if (!tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
         CUDA_TRY(launch_scan_chunk_tc(a, s));
     } else if (impl == 2 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+        a.Zscan = dd.zdbg ? dd.zdbg : reinterpret_cast<float*>(ws + L.zbuf);
         CUDA_TRY(launch_scan_chunk_tc2(a, s));
+        CUDA_TRY(launch_gate(dd.xin, dd.xin_bf16, a.Zscan, dd.alpha, dd.out, dd.out_bf16, dd.delta, a.status, q.T,
+                             q.H, q.d, q.per_head_input, s));
     } else if (b == 1 && impl != 1) {
         CUDA_TRY(launch_scan_token(a, s));
     } else {
@@ -402,6 +410,11 @@ int ttt_kernel_times(int max_kernels, char* names, size_t names_cap, double* tot
         names[names_cap - 1] = '\0';
     }
     return (int)keys.size();
+}
+
+ttt_status ttt_debug_inject_wait_timeout(int enable) {
+    g_inject_timeout.store(enable ? 1 : 0);
+    return TTT_OK;
 }
 
 const char* ttt_last_error(void) { return t_err.c_str(); }

@@ -37,6 +37,8 @@ struct ScanArgs {
     float eta;
     int* status;            // OR-ed status bits
     float* scratch;         // per-head scratch (chunk SIMT kernel)
+    int inject_timeout;     // tests: make the first bounded wait expire (cluster scan)
+    float* Zscan;           // cluster scan: where it stores z (the gate runs as its own kernel)
     long long scratch_per_head;  // floats
 };
 
@@ -63,6 +65,10 @@ cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const t
 bool proj_full_tc_supported(int N, int K);
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
                                 int accumulate, int* status, cudaStream_t s);
+
+// out = x + tanh(alpha) z (+ bf16 increment, + non-finite check) over one direction.
+cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* alpha, void* Out, int out_bf16,
+                        __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, cudaStream_t s);
 
 // Records a message for ttt_last_error() on this thread and returns `code`.
 ttt_status set_error(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));

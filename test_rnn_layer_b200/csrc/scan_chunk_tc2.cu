@@ -17,8 +17,9 @@
 //   A^T = W1 K^T, G = GELU(A), Y^T = W2 G^T, D2' = -2 eta (Y - V),
 //   P^T = W2^T D2'^T, Dl = P * GELU'(A), W1 += Dl^T K, W2^T += G^T D2',
 //   Aq^T = W1_old Q^T + Dl^T M^T (M[t,s] = q_t.k_s, s not after t), Gq = GELU(Aq),
-//   [Z1^T; N] = [W2; G] Gq^T, Z^T = Z1^T + D2'^T Nm^T (Nm[t,s] = -N[s,t], s after t),
-//   out = x + tanh(alpha) z.
+//   [Z1^T; N] = [W2; G] Gq^T, Z^T = Z1^T + D2'^T Nm^T (Nm[t,s] = -N[s,t], s after t).
+// The kernel stores z; the gate out = x + tanh(alpha) z is a separate
+// bandwidth-bound kernel, keeping global loads off the scan's dependent chain.
 // All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
 // shared-memory operands with the 128-byte swizzle.  Waits are bounded.
 //
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint64_t* bar_v = bar_mma + 3;
     uint64_t* bar_ry = bar_mma + 4;   // the peer's Y^T partial has landed in RY
     uint64_t* bar_rz = bar_mma + 5;   // the peer's [Z1; N] partial has landed in RZ
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 6);
+    uint64_t* bar_never = bar_mma + 6;   // fault injection: nothing ever arrives here
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -184,6 +186,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::mbar_init(bar_v, 1);
         tc::mbar_init(bar_ry, 256);   // one arrival per peer thread holding Y^T rows
         tc::mbar_init(bar_rz, 256);   // one arrival per peer thread holding my tokens' columns
+        tc::mbar_init(bar_never, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -234,9 +237,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         load_tile(&P.mapV, OFF_V, bar_v, y0);
     }
 
-    float tanh_a = 0.f;
-    if (q < 2) tanh_a = tanhf(a.alpha[h * DH + 32 * q + lane]);
-    int nonfinite = 0;
     uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0;
 
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
@@ -316,45 +316,26 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         atomicOr(a.status, kStatusTimeout);
     };
 
-    // Gate and stores of a finished chunk (rows y0c .. y0c + bcc - 1), my tokens;
-    // reads only the Z columns of tensor memory and global memory.
-    auto gate_chunk = [&](int y0c, int bcc) {
+    // Stores of a finished chunk's z (rows y0c .. y0c + bcc - 1), my tokens: reads
+    // only the Z columns of tensor memory; no global loads on this path (the gate
+    // x + tanh(alpha) z runs afterwards as a separate elementwise kernel).
+    auto store_z_chunk = [&](int y0c, int bcc) {
         if (q < 2 && my_tokens) {
             const int j = 32 * q + lane, t0 = 16 * g;
             uint32_t r[16];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
-            float xv[16];
-            const long long xrow = (long long)h * a.x_hs + (long long)y0c * a.x_ts + j;
-            if (a.xin_bf16) {
-                const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(a.Xin) + xrow;
-                __nv_bfloat16 raw[16];
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    raw[k] = (t0 + k < bcc) ? xb[(long long)(t0 + k) * a.x_ts] : __float2bfloat16_rn(0.f);
-#pragma unroll
-                for (int k = 0; k < 16; ++k) xv[k] = __bfloat162float(raw[k]);
-            } else {
-                const float* xf = reinterpret_cast<const float*>(a.Xin) + xrow;
-#pragma unroll
-                for (int k = 0; k < 16; ++k) xv[k] = (t0 + k < bcc) ? xf[(long long)(t0 + k) * a.x_ts] : 0.f;
-            }
             tc::tmem_wait_ld();
+            float* zrow = a.Zscan + (long long)h * a.x_hs + (long long)y0c * a.x_ts + j;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = t0 + k;
-                if (t < bcc) {
-                    const float z = __uint_as_float(r[k]);
-                    const long long xo = xrow + (long long)t * a.x_ts;
-                    const float dz = tanh_a * z;
-                    store_elem(a.Out, xo, a.out_bf16, xv[k] + dz);
-                    if (a.Delta) a.Delta[xo] = __float2bfloat16_rn(dz);
-                    if (a.Zdbg) a.Zdbg[xo] = z;
-                    nonfinite |= !isfinite(z);
-                }
-            }
+            for (int k = 0; k < 16; ++k)
+                if (t0 + k < bcc) zrow[(long long)(t0 + k) * a.x_ts] = __uint_as_float(r[k]);
         }
     };
-    int prev_y0 = 0, prev_bc = 0;   // the chunk whose gate is still pending (prev_bc == 0: none)
+    int prev_y0 = 0, prev_bc = 0;   // the chunk whose z is still to be stored (prev_bc == 0: none)
+
+    if (a.inject_timeout && warp == 0) {   // tests: a bounded wait that expires (1 ms)
+        if (!tc::mbar_wait(bar_never, 0, nullptr, 1000000ull) && lane == 0) give_up();
+    }
 
     for (int c = 0; c < nchunks; ++c) {
         int y0, bc;
@@ -392,7 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                         tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
                 },
                 [&] {
-                    if (prev_bc) gate_chunk(prev_y0, prev_bc);
+                    if (prev_bc) store_z_chunk(prev_y0, prev_bc);
                 }))
             break;
         prev_bc = 0;
@@ -620,7 +601,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         STAMP(12);
     }
 
-    if (prev_bc && !*abort_flag) gate_chunk(prev_y0, prev_bc);   // the last chunk's gate
+    if (prev_bc && !*abort_flag) store_z_chunk(prev_y0, prev_bc);   // the last chunk's z
 
 #ifdef TTT_DEBUG_STAGES
     if (tid == 0 && blockIdx.x == 0 && g_dbg2) {
@@ -652,7 +633,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             for (int k = 0; k < 16; ++k) dst[(long long)(j0 + k) * MH] = __uint_as_float(v[k]);
         }
     }
-    if (nonfinite) atomicOr(a.status, kStatusNonFinite);
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 0) {

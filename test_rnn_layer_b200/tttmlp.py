@@ -24,7 +24,7 @@ DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
-            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc"]
+            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_debug_inject_wait_timeout"]
 
 
 class TTTError(RuntimeError):
@@ -73,6 +73,8 @@ def lib():
         L.ttt_last_error.argtypes = []
         L.ttt_launch_count.restype = ctypes.c_uint64
         L.ttt_launch_count.argtypes = []
+        L.ttt_debug_inject_wait_timeout.restype = i
+        L.ttt_debug_inject_wait_timeout.argtypes = [i]
         L.ttt_kernel_timing.restype = i
         L.ttt_kernel_timing.argtypes = [i]
         L.ttt_kernel_times.restype = i
@@ -105,6 +107,10 @@ def ttt_last_error() -> str:
 
 def ttt_launch_count() -> int:
     return int(lib().ttt_launch_count())
+
+
+def ttt_debug_inject_wait_timeout(enable: bool) -> int:
+    return int(lib().ttt_debug_inject_wait_timeout(1 if enable else 0))
 
 
 def ttt_kernel_timing(enable: bool) -> int:
