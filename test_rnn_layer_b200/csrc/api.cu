@@ -6,6 +6,7 @@
 // the forward scan runs on X and its gate writes X' = X + tanh(alpha_f) z_f;
 // the reverse scan runs on X' (same theta, same W_0) and its gate writes
 // Y = X' + tanh(alpha_r) z_r.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cmath>
@@ -118,7 +119,7 @@ ttt_status check_desc(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
 }
 
 struct Layout {
-    size_t status, qkv[3], xp, delta, scratch, zbuf, total;
+    size_t status, qkv[3], xp, delta, scratch, zbuf, state, total;
     long long scratch_per_head;
     bool split_reverse;   // reverse projection as theta X + theta bf16(X' - X)
 };
@@ -141,6 +142,9 @@ Layout plan(const ttt_mlp_desc& q, int b, ttt_direction dir) {
     // z of one direction for the cluster tensor-core scan, whose gate runs separately
     L.zbuf = off;
     if (scan_chunk_tc_supported(q.d, b)) off = align_up(off + n * sizeof(float));
+    // W1 and W2 of every head between two segments of a pipelined direction
+    L.state = off;
+    if (scan_chunk_tc_supported(q.d, b)) off = align_up(off + 2 * (size_t)q.H * q.m * q.d * sizeof(float));
     L.total = off;
     return L;
 }
@@ -171,15 +175,15 @@ ttt_status project(const ttt_mlp_desc& q, const void* src, int src_bf16, const v
     if (impl == 2 && !tc_ok)
         return fail(TTT_ERR_UNSUPPORTED, "tensor-core projection needs bf16 inputs, D %% 256 == 0");
     if (tc_ok && impl != 1) {
-        CUDA_TRY(launch_proj_full_tc(src, th, out, q.T, q.D, q.D, accumulate, status, s));
+        CUDA_TRY(launch_proj_full_tc(src, th, out, q.T, q.D, q.D, accumulate, status, 0, s));
     } else {
         CUDA_TRY(launch_proj_full_simt(src, src_bf16, th, th_bf16, out, q.T, q.D, q.D, accumulate, s));
     }
     return TTT_OK;
 }
 
-ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W1_0, const float* W2_0,
-                float eta, int b, const Dir& dd, cudaStream_t s) {
+ScanArgs scan_args(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W1_0, const float* W2_0,
+                   float eta, int b, const Dir& dd) {
     ScanArgs a{};
     a.Q = reinterpret_cast<const float*>(ws + L.qkv[0]);
     a.K = reinterpret_cast<const float*>(ws + L.qkv[1]);
@@ -198,6 +202,12 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
     a.scratch = reinterpret_cast<float*>(ws + L.scratch);
     a.scratch_per_head = L.scratch_per_head;
     a.inject_timeout = g_inject_timeout.load();
+    return a;
+}
+
+ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W1_0, const float* W2_0,
+                float eta, int b, const Dir& dd, cudaStream_t s) {
+    ScanArgs a = scan_args(q, L, ws, W1_0, W2_0, eta, b, dd);
     // Kernel choice: the tf32 tensor-core scan serves bf16-input layers (whose
     // tolerance is 2e-2); fp32-input layers keep the fp32 kernels unless the
     // tensor-core kernel is requested explicitly.
@@ -211,12 +221,192 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
         a.Zscan = dd.zdbg ? dd.zdbg : reinterpret_cast<float*>(ws + L.zbuf);
         CUDA_TRY(launch_scan_chunk_tc2(a, s));
         CUDA_TRY(launch_gate(dd.xin, dd.xin_bf16, a.Zscan, dd.alpha, dd.out, dd.out_bf16, dd.delta, a.status, q.T,
-                             q.H, q.d, q.per_head_input, s));
+                             q.H, q.d, q.per_head_input, 0, s));
     } else if (b == 1 && impl != 1) {
         CUDA_TRY(launch_scan_token(a, s));
     } else {
         CUDA_TRY(launch_scan_chunk_simt(a, s));
     }
+    return TTT_OK;
+}
+
+// ---------------------------------------------------------------- pipelined full layer
+// With the full-width projection on the tensor cores and the cluster scan, a
+// direction runs as a sequence of chunk segments so that the projection and
+// the gate use the SMs the scan leaves free (the scan holds two SMs per head):
+//   side stream : proj(seg 0), proj(seg 1), ...  then, after scan(seg k), gate(seg k)
+//   scan stream : after proj(seg k), scan(seg k) -- the state W1, W2 is carried
+//                 from one segment to the next in the workspace
+// Only stream order and events connect the two streams (no kernel waits on
+// another).  Projection and gate launches next to a running scan are capped
+// to the free SMs less a margin, so that every CTA pair of the next scan
+// segment finds room; the scan stream has the higher priority.
+struct Pipe {
+    cudaStream_t scan = nullptr, side = nullptr;
+    std::vector<cudaEvent_t> ev;
+    int sms = 0;
+};
+std::mutex g_pipe_mu;
+Pipe g_pipes[64];
+
+constexpr int kPipeMinSegChunks = 16;
+constexpr int kPipeSmMargin = 8;
+
+// Chunk ranges [begin, end) of a walk over `nchunks` chunks: segments grow
+// by 3/2 from 16 chunks at both ends (short exposed head and tail), with
+// pieces of about nchunks / 12 in between.
+std::vector<std::pair<int, int>> pipe_segments(int nchunks) {
+    const int cap = std::max(kPipeMinSegChunks, (nchunks + 11) / 12);
+    std::vector<int> front, back;
+    int rem = nchunks;
+    for (int sz = kPipeMinSegChunks; sz < cap && rem > 0; sz = sz * 3 / 2) {
+        int t = std::min(sz, rem);
+        front.push_back(t);
+        rem -= t;
+        if (rem <= 0) break;
+        t = std::min(sz, rem);
+        back.push_back(t);
+        rem -= t;
+    }
+    while (rem > 0) {
+        const int t = std::min(cap, rem);
+        front.push_back(t);
+        rem -= t;
+    }
+    front.insert(front.end(), back.rbegin(), back.rend());
+    std::vector<std::pair<int, int>> out;
+    int c = 0;
+    for (int sz : front) {
+        out.emplace_back(c, c + sz);
+        c += sz;
+    }
+    return out;
+}
+
+// SMs the projection and gate may use next to a running scan (0: no pipelining).
+int pipe_side_sms(const ttt_mlp_desc& q) {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    const int side = sms - 2 * q.H - kPipeSmMargin;
+    return side >= 16 ? side : 0;
+}
+
+bool pipe_eligible(const ttt_mlp_desc& q, const Layout& L, int b, ttt_direction dir) {
+    const int si = g_scan_impl.load(), pi = g_proj_impl.load();
+    if (q.per_head_input || q.x_dtype != TTT_BF16) return false;
+    if (!(si == 0 || si == 2) || !scan_chunk_tc_supported(q.d, b)) return false;
+    if (pi == 1 || !proj_full_tc_supported(q.D, q.D)) return false;
+    if (dir == TTT_BIDIR && !L.split_reverse) return false;
+    return pipe_side_sms(q) > 0;
+}
+
+ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, const void* X, const void* const th[3],
+                             float* const qkv[3], const float* W1_0, const float* W2_0, float eta, int b,
+                             ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
+                             float* W1_T, float* W2_T, cudaStream_t s) {
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(TTT_ERR_UNSUPPORTED, "device index %d", dev);
+    Pipe& P = g_pipes[dev];
+    if (!P.scan) {
+        int lo = 0, hi = 0;
+        CUDA_TRY(cudaDeviceGetStreamPriorityRange(&lo, &hi));
+        CUDA_TRY(cudaStreamCreateWithPriority(&P.scan, cudaStreamNonBlocking, hi));
+        CUDA_TRY(cudaStreamCreateWithPriority(&P.side, cudaStreamNonBlocking, lo));
+    }
+    const int side_sms = pipe_side_sms(q);
+    const int nch = (q.T + b - 1) / b;
+    const auto seg = pipe_segments(nch);
+    const int ns = (int)seg.size();
+    const int ndir = dir == TTT_BIDIR ? 2 : 1;
+    const size_t need_ev = 3 + (size_t)ndir * 2 * ns;
+    while (P.ev.size() < need_ev) {
+        cudaEvent_t e;
+        CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        P.ev.push_back(e);
+    }
+    size_t next_ev = 0;
+    auto new_ev = [&]() { return P.ev[next_ev++]; };
+
+    cudaEvent_t fork = new_ev();
+    CUDA_TRY(cudaEventRecord(fork, s));
+    CUDA_TRY(cudaStreamWaitEvent(P.scan, fork, 0));
+    CUDA_TRY(cudaStreamWaitEvent(P.side, fork, 0));
+
+    const size_t n = (size_t)q.T * q.D;
+    const size_t nW = (size_t)q.H * q.m * q.d;
+    const int D = q.D;
+    float* xp = reinterpret_cast<float*>(ws + L.xp);
+    __nv_bfloat16* delta = reinterpret_cast<__nv_bfloat16*>(ws + L.delta);
+    float* st1 = reinterpret_cast<float*>(ws + L.state);
+    float* st2 = st1 + nW;
+    int* status = reinterpret_cast<int*>(ws + L.status);
+
+    for (int di = 0; di < ndir; ++di) {
+        Dir dd{};
+        dd.reverse = (dir == TTT_REV || di == 1) ? 1 : 0;
+        const bool second = di == 1;
+        dd.xin = second ? static_cast<const void*>(xp) : X;
+        dd.xin_bf16 = second ? 0 : 1;
+        dd.alpha = dd.reverse ? alpha_r : alpha_f;
+        if (dir == TTT_BIDIR && !second) { dd.out = xp; dd.out_bf16 = 0; dd.delta = delta; }
+        else { dd.out = Y; dd.out_bf16 = 1; dd.delta = nullptr; }
+        dd.zdbg = Z_out ? Z_out + di * n : nullptr;
+        const void* psrc = second ? static_cast<const void*>(delta) : X;   // both bf16
+        const int pacc = second ? 1 : 0;
+        float* zscan = Z_out ? Z_out + di * n : reinterpret_cast<float*>(ws + L.zbuf);
+
+        std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns);
+        for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); }
+        auto rows = [&](int k, int& r0, int& r1) {
+            const int lo = seg[k].first * b, hi = std::min(seg[k].second * b, q.T);
+            if (dd.reverse) { r0 = q.T - hi; r1 = q.T - lo; }
+            else { r0 = lo; r1 = hi; }
+        };
+        // projections (the first runs alone on the whole GPU)
+        for (int k = 0; k < ns; ++k) {
+            int r0, r1;
+            rows(k, r0, r1);
+            const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
+            float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
+            CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
+            CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
+        }
+        // scan segments, state carried in the workspace
+        for (int k = 0; k < ns; ++k) {
+            CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k], 0));
+            ScanArgs a = scan_args(q, L, ws, k == 0 ? W1_0 : st1, k == 0 ? W2_0 : st2, eta, b, dd);
+            a.Zscan = zscan;
+            a.c_begin = seg[k].first;
+            a.c_end = seg[k].second;
+            const bool last = k == ns - 1;
+            a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
+            a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
+            CUDA_TRY(launch_scan_chunk_tc2(a, P.scan));
+            CUDA_TRY(cudaEventRecord(ev_scan[k], P.scan));
+        }
+        // gates, each after its segment's scan
+        for (int k = 0; k < ns; ++k) {
+            int r0, r1;
+            rows(k, r0, r1);
+            CUDA_TRY(cudaStreamWaitEvent(P.side, ev_scan[k], 0));
+            const size_t o = (size_t)r0 * D;
+            const void* xin = static_cast<const char*>(dd.xin) + o * (dd.xin_bf16 ? 2 : 4);
+            void* out = static_cast<char*>(dd.out) + o * (dd.out_bf16 ? 2 : 4);
+            const bool last = k == ns - 1;
+            CUDA_TRY(launch_gate(xin, dd.xin_bf16, zscan + o, dd.alpha, out, dd.out_bf16,
+                                 dd.delta ? dd.delta + o : nullptr, status, r1 - r0, q.H, q.d, 0,
+                                 last ? 0 : side_sms * 4, P.side));
+        }
+    }
+    cudaEvent_t j1 = new_ev(), j2 = new_ev();
+    CUDA_TRY(cudaEventRecord(j1, P.scan));
+    CUDA_TRY(cudaEventRecord(j2, P.side));
+    CUDA_TRY(cudaStreamWaitEvent(s, j1, 0));
+    CUDA_TRY(cudaStreamWaitEvent(s, j2, 0));
     return TTT_OK;
 }
 
@@ -289,6 +479,10 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     const size_t nW = (size_t)q.H * q.m * q.d;
     float* xp = reinterpret_cast<float*>(ws + L.xp);
     int* status = reinterpret_cast<int*>(ws + L.status);
+
+    if (pipe_eligible(q, L, b, dir))
+        return forward_pipelined(q, L, ws, X, th, qkv, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
+                                 W2_T, s);
 
     // first (or only) direction
     Dir d0{};

@@ -67,7 +67,8 @@ __global__ void __launch_bounds__(256) gate_kernel(GateArgs g) {
 }  // namespace
 
 cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* alpha, void* Out, int out_bf16,
-                        __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, cudaStream_t s) {
+                        __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, int max_blocks,
+                        cudaStream_t s) {
     GateArgs g{};
     g.X = X; g.x_bf16 = x_bf16; g.Z = Z; g.alpha = alpha; g.Out = Out; g.out_bf16 = out_bf16;
     g.Delta = Delta; g.status = status;
@@ -78,7 +79,8 @@ cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     long long blocks = (g.n / 4 + 255) / 256;
-    if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+    if (blocks > (long long)sms * 6) blocks = (long long)sms * 6;
+    if (max_blocks > 0 && blocks > max_blocks) blocks = max_blocks;
     LaunchScope scope("gate", s);
     gate_kernel<<<(unsigned)blocks, 256, 0, s>>>(g);
     return cudaGetLastError();

@@ -39,6 +39,8 @@ struct ScanArgs {
     float* scratch;         // per-head scratch (chunk SIMT kernel)
     int inject_timeout;     // tests: make the first bounded wait expire (cluster scan)
     float* Zscan;           // cluster scan: where it stores z (the gate runs as its own kernel)
+    int c_begin, c_end;     // cluster scan: chunks [c_begin, c_end) of the walk (c_end 0: to the end);
+                            // state from W1_0/W2_0, final state to W1_T/W2_T
     long long scratch_per_head;  // floats
 };
 
@@ -64,11 +66,12 @@ cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const t
 // tcgen05 projections (bf16 A and Theta, N % 256 == 0, K % 64 == 0), same contract.
 bool proj_full_tc_supported(int N, int K);
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
-                                int accumulate, int* status, cudaStream_t s);
+                                int accumulate, int* status, int max_ctas, cudaStream_t s);
 
 // out = x + tanh(alpha) z (+ bf16 increment, + non-finite check) over one direction.
 cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* alpha, void* Out, int out_bf16,
-                        __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, cudaStream_t s);
+                        __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, int max_blocks,
+                        cudaStream_t s);
 
 // Records a message for ttt_last_error() on this thread and returns `code`.
 ttt_status set_error(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));

@@ -216,7 +216,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 bool proj_full_tc_supported(int N, int K) { return N % BN == 0 && K % BK == 0 && N > 0 && K > 0; }
 
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
-                                int accumulate, int* status, cudaStream_t s) {
+                                int accumulate, int* status, int max_ctas, cudaStream_t s) {
     ProjTcArgs p{};
     bool ok = make_map(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, T, (uint64_t)K * 2, BK, BM);
     for (int w = 0; w < 3 && ok; ++w) {
@@ -236,7 +236,8 @@ cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float
     cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     LaunchScope scope("proj_full_tc", s);
-    const int grid = p.tiles < sms ? p.tiles : sms;
+    int grid = p.tiles < sms ? p.tiles : sms;
+    if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
     proj_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
 }

@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     const int h = blockIdx.x >> 1;
     const int T = a.T, b = a.b;
     const int nchunks = (T + b - 1) / b;
+    const int c_first = a.c_begin, c_last = a.c_end > 0 ? min(a.c_end, nchunks) : nchunks;
     const float eta = a.eta;
     const bool my_tokens = (g >> 1) == (int)r_cta;   // tokens 16g .. 16g+15 belong to this CTA
 
@@ -231,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     }
     if (tid == 0) {
         int y0, bc;
-        chunk_rows(0, y0, bc);
+        chunk_rows(c_first, y0, bc);
         load_tile(&P.mapK, OFF_K, bar_k, y0);
         load_tile(&P.mapQ, OFF_Q, bar_q, y0);
         load_tile(&P.mapV, OFF_V, bar_v, y0);
@@ -337,7 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         if (!tc::mbar_wait(bar_never, 0, nullptr, 1000000ull) && lane == 0) give_up();
     }
 
-    for (int c = 0; c < nchunks; ++c) {
+    for (int c = c_first; c < c_last; ++c) {
         int y0, bc;
         chunk_rows(c, y0, bc);
         STAMP(13);
@@ -377,7 +378,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                 }))
             break;
         prev_bc = 0;
-        if (tid == 0 && c + 1 < nchunks) {   // Q is free: fetch the next chunk's queries
+        if (tid == 0 && c + 1 < c_last) {   // Q is free: fetch the next chunk's queries
             int ny0, nbc;
             chunk_rows(c + 1, ny0, nbc);
             load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                     tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
             }))
             break;
-        if (tid == 0 && c + 1 < nchunks) {   // K and V buffers are free: fetch the next chunk's tiles
+        if (tid == 0 && c + 1 < c_last) {   // K and V buffers are free: fetch the next chunk's tiles
             int ny0, nbc;
             chunk_rows(c + 1, ny0, nbc);
             load_tile(&P.mapK, OFF_K, bar_k, ny0);
@@ -606,7 +607,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
 #ifdef TTT_DEBUG_STAGES
     if (tid == 0 && blockIdx.x == 0 && g_dbg2) {
         for (int k = 0; k < 20; ++k) g_dbg2[k] = (float)stamp_acc[k];
-        g_dbg2[30] = (float)nchunks;
+        g_dbg2[30] = (float)(c_last - c_first);
     }
 #endif
     if (*abort_flag) {
@@ -676,6 +677,9 @@ extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump2(float*
 #endif
 
 cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s) {
+    const int nchunks = (a.T + a.b - 1) / a.b;
+    const int c_end = a.c_end > 0 ? a.c_end : nchunks;
+    if (a.c_begin < 0 || c_end > nchunks || a.c_begin >= c_end) return cudaErrorInvalidValue;
     ScanTc2Args P{};
     P.a = a;
     P.full = (a.qkv_ts != DH) ? 1 : 0;

@@ -75,6 +75,16 @@ def test_full_layer_short(impl):
     _check(S.FULL63S.with_T(777))
 
 
+@pytest.mark.parametrize("T", [3000, 64 * 50])
+@pytest.mark.parametrize("dirs", ["bidir", "rev"])
+def test_full_layer_segmented_pipeline(T, dirs):
+    """On the tensor-core path the full layer runs each direction as several
+    chunk segments (state carried between launches, projection and gate on a
+    second stream): lengths that give three segments, with and without a
+    ragged last chunk, checked with the final state."""
+    _check(S.FULL63S.with_(T=T, H=4, D=256, dirs=dirs))
+
+
 @pytest.mark.parametrize("dirs", ["fwd", "rev", "bidir"])
 @pytest.mark.parametrize("b", [1, 5, 64])
 def test_directions_and_chunks_f32(impl, dirs, b):
