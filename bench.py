@@ -147,7 +147,8 @@ def _config(w, extra=None):
 
 
 def _algorithmic(w):
-    """Algorithmic work per launch of each kernel kind (one direction)."""
+    """Algorithmic work of each kernel kind over one direction of the layer
+    (all of that direction's launches together)."""
     T, D, H, d, m, b = w.T, w.model_dim, w.H, w.d, w.m, w.b
     scan_flops = H * T * (7 * 2 * d * m + 2 * b * (d + m))
     proj_flops = 2.0 * T * D * 3 * D
@@ -165,8 +166,13 @@ def _algorithmic(w):
     }
 
 
-def _roofline(name, ms_per_launch, w, peaks, clocks):
-    bound, work = _algorithmic(w)[name]
+def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):
+    """Roofline of one launch of `name`: the step's algorithmic work for that
+    kernel (both directions for a bidirectional layer) divided evenly over its
+    launches, against the average launch duration."""
+    bound, work_dir = _algorithmic(w)[name]
+    ndir = 2 if w.dirs == "bidir" else 1
+    work = work_dir * ndir / launches_per_step
     sus = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     src = "of " + peaks["_source"]
     if bound == "tensor_bf16":
@@ -184,7 +190,7 @@ def _roofline(name, ms_per_launch, w, peaks, clocks):
     else:
         peak, unit, kind, note = peaks["hbm_gbs"], "GB/s", "hbm", f"HBM copy {src}"
         achieved = work / (ms_per_launch * 1e-3) / 1e9
-    units = w.T / 1024.0   # traffic records are stored per 1024 tokens
+    units = w.T * ndir / launches_per_step / 1024.0   # traffic records are stored per 1024 tokens
     return {"kernel": name, "bound": kind, "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
             "frac": round(achieved / peak, 4), "traffic": _traffic(name, units), "peak_note": note,
             "ms_per_launch": round(ms_per_launch, 4), "work_per_launch": work}
@@ -332,8 +338,9 @@ def run_ours(args, rank, world, local_rank):
     total = sum(v[0] for v in ktimes.values()) or 1.0
     top = max(ktimes, key=lambda k: ktimes[k][0])
     peaks = _peaks()
-    roof = _roofline(top, ktimes[top][0] / ktimes[top][1], w, peaks, clocks)
-    roof["share"] = round(ktimes[top][0] / total, 4)
+    roof = _roofline(top, ktimes[top][0] / ktimes[top][1], ktimes[top][1] / kpass, w, peaks, clocks)
+    roof["share"] = round(ktimes[top][0] / total, 4)   # of the summed kernel time (streams overlap)
+    roof["ms_per_step"] = round(ktimes[top][0] / kpass, 3)
     kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
                    "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
 
