@@ -137,6 +137,10 @@ TTT_API size_t ttt_mlp_host_io_workspace_size(const ttt_mlp_desc* desc, int b, t
  * copy speed); everything else as in ttt_mlp_forward (device pointers).
  * Copies X_host to the device, runs the layer, copies Y back to Y_host,
  * synchronises `stream` and returns the status as ttt_mlp_status would.
+ * Where the layer runs in chunk segments (full-width bf16 input on the
+ * tensor-core path) the copies overlap the computation: X goes over segment
+ * by segment ahead of its projection, Y comes back segment by segment after
+ * its last gate.
  */
 TTT_API ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host,
                                 const void* theta_q, const void* theta_k, const void* theta_v,

@@ -242,7 +242,7 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
 // to the free SMs less a margin, so that every CTA pair of the next scan
 // segment finds room; the scan stream has the higher priority.
 struct Pipe {
-    cudaStream_t scan = nullptr, side = nullptr;
+    cudaStream_t scan = nullptr, side = nullptr, copy = nullptr;
     std::vector<cudaEvent_t> ev;
     int sms = 0;
 };
@@ -305,7 +305,7 @@ bool pipe_eligible(const ttt_mlp_desc& q, const Layout& L, int b, ttt_direction 
 ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, const void* X, const void* const th[3],
                              float* const qkv[3], const float* W1_0, const float* W2_0, float eta, int b,
                              ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
-                             float* W1_T, float* W2_T, cudaStream_t s) {
+                             float* W1_T, float* W2_T, cudaStream_t s, const void* X_host, void* Y_host) {
     std::lock_guard<std::mutex> lk(g_pipe_mu);
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
@@ -316,13 +316,14 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
         CUDA_TRY(cudaDeviceGetStreamPriorityRange(&lo, &hi));
         CUDA_TRY(cudaStreamCreateWithPriority(&P.scan, cudaStreamNonBlocking, hi));
         CUDA_TRY(cudaStreamCreateWithPriority(&P.side, cudaStreamNonBlocking, lo));
+        CUDA_TRY(cudaStreamCreateWithPriority(&P.copy, cudaStreamNonBlocking, lo));
     }
     const int side_sms = pipe_side_sms(q);
     const int nch = (q.T + b - 1) / b;
     const auto seg = pipe_segments(nch);
     const int ns = (int)seg.size();
     const int ndir = dir == TTT_BIDIR ? 2 : 1;
-    const size_t need_ev = 3 + (size_t)ndir * 2 * ns;
+    const size_t need_ev = 4 + (size_t)ndir * 4 * ns;
     while (P.ev.size() < need_ev) {
         cudaEvent_t e;
         CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
@@ -335,6 +336,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
     CUDA_TRY(cudaEventRecord(fork, s));
     CUDA_TRY(cudaStreamWaitEvent(P.scan, fork, 0));
     CUDA_TRY(cudaStreamWaitEvent(P.side, fork, 0));
+    CUDA_TRY(cudaStreamWaitEvent(P.copy, fork, 0));
 
     const size_t n = (size_t)q.T * q.D;
     const size_t nW = (size_t)q.H * q.m * q.d;
@@ -359,17 +361,30 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
         const int pacc = second ? 1 : 0;
         float* zscan = Z_out ? Z_out + di * n : reinterpret_cast<float*>(ws + L.zbuf);
 
-        std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns);
-        for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); }
+        std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns), ev_h2d(ns), ev_gate(ns);
+        for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); ev_h2d[k] = new_ev(); ev_gate[k] = new_ev(); }
+        const bool copy_in = X_host && di == 0;           // X arrives segment by segment
+        const bool copy_out = Y_host && di == ndir - 1;   // Y leaves segment by segment
         auto rows = [&](int k, int& r0, int& r1) {
             const int lo = seg[k].first * b, hi = std::min(seg[k].second * b, q.T);
             if (dd.reverse) { r0 = q.T - hi; r1 = q.T - lo; }
             else { r0 = lo; r1 = hi; }
         };
+        if (copy_in) {
+            for (int k = 0; k < ns; ++k) {
+                int r0, r1;
+                rows(k, r0, r1);
+                const size_t o = (size_t)r0 * D * 2, nb = (size_t)(r1 - r0) * D * 2;
+                CUDA_TRY(cudaMemcpyAsync(const_cast<char*>(static_cast<const char*>(X)) + o,
+                                         static_cast<const char*>(X_host) + o, nb, cudaMemcpyHostToDevice, P.copy));
+                CUDA_TRY(cudaEventRecord(ev_h2d[k], P.copy));
+            }
+        }
         // projections (the first runs alone on the whole GPU)
         for (int k = 0; k < ns; ++k) {
             int r0, r1;
             rows(k, r0, r1);
+            if (copy_in) CUDA_TRY(cudaStreamWaitEvent(P.side, ev_h2d[k], 0));
             const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
             float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
             CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
@@ -400,13 +415,21 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
             CUDA_TRY(launch_gate(xin, dd.xin_bf16, zscan + o, dd.alpha, out, dd.out_bf16,
                                  dd.delta ? dd.delta + o : nullptr, status, r1 - r0, q.H, q.d, 0,
                                  last ? 0 : side_sms * 4, P.side));
+            if (copy_out) {
+                CUDA_TRY(cudaEventRecord(ev_gate[k], P.side));
+                CUDA_TRY(cudaStreamWaitEvent(P.copy, ev_gate[k], 0));
+                CUDA_TRY(cudaMemcpyAsync(static_cast<char*>(Y_host) + o * 2, static_cast<const char*>(Y) + o * 2,
+                                         (size_t)(r1 - r0) * D * 2, cudaMemcpyDeviceToHost, P.copy));
+            }
         }
     }
-    cudaEvent_t j1 = new_ev(), j2 = new_ev();
+    cudaEvent_t j1 = new_ev(), j2 = new_ev(), j3 = new_ev();
     CUDA_TRY(cudaEventRecord(j1, P.scan));
     CUDA_TRY(cudaEventRecord(j2, P.side));
+    CUDA_TRY(cudaEventRecord(j3, P.copy));
     CUDA_TRY(cudaStreamWaitEvent(s, j1, 0));
     CUDA_TRY(cudaStreamWaitEvent(s, j2, 0));
+    CUDA_TRY(cudaStreamWaitEvent(s, j3, 0));
     return TTT_OK;
 }
 
@@ -429,24 +452,16 @@ ttt_status check_ptrs(const ttt_mlp_desc& q, const void* X, const void* tq, cons
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-size_t ttt_mlp_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
-    if (check_desc(desc, b, dir) != TTT_OK) return 0;
-    return plan(*desc, b, dir).total;
-}
-
-size_t ttt_mlp_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
-    if (check_desc(desc, b, dir) != TTT_OK) return 0;
-    const size_t io = align_up((size_t)desc->T * desc->D * elem_size(desc->x_dtype));
-    return plan(*desc, b, dir).total + 2 * io;
-}
-
-ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
-                           const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
-                           ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
-                           float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes,
-                           ttt_stream_t stream_) {
+// The layer on device buffers; with X_host / Y_host (host buffers) X is first
+// copied into the device buffer X and Y copied back out, overlapped with the
+// computation on the pipelined path.
+ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                        const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                        ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
+                        float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes, ttt_stream_t stream_,
+                        const void* X_host, void* Y_host) {
     ttt_status st = check_desc(desc, b, dir);
     if (st != TTT_OK) return st;
     const ttt_mlp_desc& q = *desc;
@@ -482,7 +497,12 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
 
     if (pipe_eligible(q, L, b, dir))
         return forward_pipelined(q, L, ws, X, th, qkv, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
-                                 W2_T, s);
+                                 W2_T, s, X_host, Y_host);
+    if (X_host) CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(X), X_host, xbytes, cudaMemcpyHostToDevice, s));
+    auto finish = [&]() -> ttt_status {
+        if (Y_host) CUDA_TRY(cudaMemcpyAsync(Y_host, Y, xbytes, cudaMemcpyDeviceToHost, s));
+        return TTT_OK;
+    };
 
     // first (or only) direction
     Dir d0{};
@@ -497,7 +517,7 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     if (st != TTT_OK) return st;
     st = scan(q, L, ws, W1_0, W2_0, eta, b, d0, s);
     if (st != TTT_OK) return st;
-    if (dir != TTT_BIDIR) return TTT_OK;
+    if (dir != TTT_BIDIR) return finish();
 
     // reverse direction on X' = X + tanh(alpha_f) z_f
     if (L.split_reverse) {
@@ -516,7 +536,33 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
     d1.zdbg = Z_out ? Z_out + n : nullptr;
     d1.w1t = W1_T ? W1_T + nW : nullptr;
     d1.w2t = W2_T ? W2_T + nW : nullptr;
-    return scan(q, L, ws, W1_0, W2_0, eta, b, d1, s);
+    st = scan(q, L, ws, W1_0, W2_0, eta, b, d1, s);
+    if (st != TTT_OK) return st;
+    return finish();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ttt_mlp_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc(desc, b, dir) != TTT_OK) return 0;
+    return plan(*desc, b, dir).total;
+}
+
+size_t ttt_mlp_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc(desc, b, dir) != TTT_OK) return 0;
+    const size_t io = align_up((size_t)desc->T * desc->D * elem_size(desc->x_dtype));
+    return plan(*desc, b, dir).total + 2 * io;
+}
+
+ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                           const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                           ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
+                           float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes,
+                           ttt_stream_t stream_) {
+    return forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
+                        W2_T, workspace, workspace_bytes, stream_, nullptr, nullptr);
 }
 
 ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {
@@ -547,12 +593,9 @@ ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, co
     char* ws = static_cast<char*>(workspace);
     void* Xd = ws + L.total;
     void* Yd = ws + L.total + align_up(xbytes);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
-    CUDA_TRY(cudaMemcpyAsync(Xd, X_host, xbytes, cudaMemcpyHostToDevice, s));
-    st = ttt_mlp_forward(desc, Xd, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Yd,
-                         nullptr, nullptr, nullptr, workspace, L.total, stream_);
+    st = forward_impl(desc, Xd, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Yd, nullptr,
+                      nullptr, nullptr, workspace, L.total, stream_, X_host, Y_host);
     if (st != TTT_OK) return st;
-    CUDA_TRY(cudaMemcpyAsync(Y_host, Yd, xbytes, cudaMemcpyDeviceToHost, s));
     return ttt_mlp_status(workspace, stream_);
 }
 

@@ -147,18 +147,24 @@ def test_reverse_equals_flipped_forward_on_gpu():
     assert maxrel(to_np(g_rev["Z"][0]), to_np(g_fwd["Z"][0].flip(1))) < 1e-3
 
 
-def test_host_io_entry_point_matches_device_entry_point():
-    w = S.MINIBATCH.with_(T=500, H=4)
+@pytest.mark.parametrize("w", [S.MINIBATCH.with_(T=500, H=4), S.FULL63S.with_(T=3000, H=4, D=256),
+                               S.FULL63S.with_(T=3000, H=4, D=256, dirs="rev")],
+                         ids=["per-head", "full-layer-segmented", "full-layer-segmented-rev"])
+def test_host_io_entry_point_matches_device_entry_point(w):
+    """Host buffers in and out (copied segment by segment, overlapped with the
+    computation, on the segmented full-layer path) give the device entry
+    point's result bit for bit."""
     inp = S.make_inputs(w)
     dev = torch.device("cuda")
     gd = {k: v.to(dev) for k, v in inp.items()}
     ref = run_gpu(w, inp)["Y"].cpu()
-    desc = L.make_desc(w.T, w.H, w.d, True, True)
-    ws = L.alloc_workspace(desc, w.b, L.TTT_BIDIR, dev, host_io=True)
+    desc = L.make_desc(w.T, w.H, w.d, w.per_head, True)
+    direction = L.DIRS[w.dirs]
+    ws = L.alloc_workspace(desc, w.b, direction, dev, host_io=True)
     Xh = inp["X"].pin_memory()
     Yh = torch.empty_like(Xh).pin_memory()
     st = L.ttt_mlp_forward_host(desc, Xh, gd["theta_q"], gd["theta_k"], gd["theta_v"], gd["W1_0"], gd["W2_0"],
-                                w.eta_eff, w.b, L.TTT_BIDIR, gd["alpha_f"], gd["alpha_r"], Yh, ws, ws.numel())
+                                w.eta_eff, w.b, direction, gd["alpha_f"], gd["alpha_r"], Yh, ws, ws.numel())
     L.check(st, "ttt_mlp_forward_host")
     assert torch.equal(Yh, ref)
 
