@@ -17,7 +17,11 @@
 //   A^T = W1 K^T, G = GELU(A), Y^T = W2 G^T, D2' = -2 eta (Y - V),
 //   P^T = W2^T D2'^T, Dl = P * GELU'(A), W1 += Dl^T K, W2^T += G^T D2',
 //   Aq^T = W1_old Q^T + Dl^T M^T (M[t,s] = q_t.k_s, s not after t), Gq = GELU(Aq),
-//   [Z1^T; N] = [W2; G] Gq^T, Z^T = Z1^T + D2'^T Nm^T (Nm[t,s] = -N[s,t], s after t).
+//   [Z1^T; N] = [W2_old; G] Gq^T, Z^T = Z1^T + D2'^T Np^T (Np[t,s] = N[s,t], s not after t):
+//   token t sees W2_old plus the updates of the tokens up to and including t.
+// The MMAs a later stage does not need at once are committed separately (the
+// first stage's Aq0 and S, the update stage's W1 and W2^T), and the shared
+// copy of the updated W2 is refreshed while the last MMA of the chunk runs.
 // The kernel stores z; the gate out = x + tanh(alpha) z is a separate
 // bandwidth-bound kernel, keeping global loads off the scan's dependent chain.
 // All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
@@ -48,7 +52,7 @@ constexpr int OFF_GQ = 65536;     // 64 x 128: Gq [t][i]; stride 8192
 constexpr int OFF_Q = 98304;      // 64 x 64: Q [t][j] (TMA)
 constexpr int OFF_K = 114688;     // 64 x 64: K [t][j] (TMA); then D2' [t][j]
 constexpr int OFF_X3 = 131072;    // 64 x 64: D2'^T [j][t]
-constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Nm [t_own][s] (32 rows)
+constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Np [t_own][s] (32 rows)
 constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s] (prefix mask)
 constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
 constexpr int OFF_RY = 196608;    // 64 x 64 fp32 plain [t][j]: the peer's Y^T partial
@@ -156,6 +160,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint64_t* bar_rz = bar_mma + 5;   // the peer's [Z1; N] partial has landed in RZ
     uint64_t* bar_never = bar_mma + 6;   // fault injection: nothing ever arrives here
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 7);
+    uint64_t* bar_a2 = bar_mma + 8;      // the first stage's second group (Aq0, S)
+    uint64_t* bar_g2 = bar_mma + 9;      // the update stage's second group (W1, W2^T)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -188,6 +194,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::mbar_init(bar_ry, 256);   // one arrival per peer thread holding Y^T rows
         tc::mbar_init(bar_rz, 256);   // one arrival per peer thread holding my tokens' columns
         tc::mbar_init(bar_never, 1);
+        tc::mbar_init(bar_a2, 1);
+        tc::mbar_init(bar_g2, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         load_tile(&P.mapV, OFF_V, bar_v, y0);
     }
 
-    uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0;
+    uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0, ph_a2 = 0, ph_g2 = 0;
 
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
     constexpr uint32_t ID32 = tc::instr_desc(2, 128, 32, 0, 0);
@@ -265,31 +273,21 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     long long stamp_acc[20] = {};
     long long stamp_last = clock64();
 #endif
-    // One MMA stage: all threads' operand writes become visible, warp 0 issues
-    // and waits for completion, the others park in the hardware barrier.
-    auto mma_stage = [&](auto issue) -> bool {
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        if (__syncthreads_or(*abort_flag)) return false;
-        if (warp == 0) {
-            if (lane == 0) {
-                tc::tc_fence_after();
-                issue();
-                tc::mma_commit(bar_mma);
-            }
-            __syncwarp();
-            if (!tc::mbar_wait(bar_mma, ph_mma, nullptr) && lane == 0) {
-                *abort_flag = 1;
-                atomicOr(a.status, kStatusTimeout);
-            }
-        }
-        ph_mma ^= 1;
-        const int stop = __syncthreads_or(*abort_flag);
-        tc::tc_fence_after();
-        return !stop;
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        atomicOr(a.status, kStatusTimeout);
     };
-    // The same, with `work` (touching nothing the MMAs read or write) run by all
-    // threads while the tensor core computes.
+    // Every thread waits for an MMA group itself (no block barrier after the
+    // MMAs); a thread whose wait expires raises the abort flag, which the next
+    // stage's leading barrier turns into a uniform exit.
+    auto wait_mma = [&](uint64_t* bar, uint32_t& ph) {
+        if (!tc::mbar_wait(bar, ph, abort_flag)) give_up();
+        ph ^= 1;
+        tc::tc_fence_after();
+    };
+    // One MMA stage: all threads' operand writes become visible, thread 0
+    // issues (and commits: the group the stage waits for goes to bar_mma),
+    // `work` (touching nothing the MMAs read or write) runs meanwhile.
     auto mma_stage_with = [&](auto issue, auto work) -> bool {
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
@@ -297,26 +295,12 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         if (tid == 0) {
             tc::tc_fence_after();
             issue();
-            tc::mma_commit(bar_mma);
         }
         work();
-        if (warp == 0) {
-            __syncwarp();
-            if (!tc::mbar_wait(bar_mma, ph_mma, nullptr) && lane == 0) {
-                *abort_flag = 1;
-                atomicOr(a.status, kStatusTimeout);
-            }
-        }
-        ph_mma ^= 1;
-        const int stop = __syncthreads_or(*abort_flag);
-        tc::tc_fence_after();
-        return !stop;
+        wait_mma(bar_mma, ph_mma);
+        return true;
     };
-    auto give_up = [&]() {
-        *abort_flag = 1;
-        atomicOr(a.status, kStatusTimeout);
-    };
-
+    auto mma_stage = [&](auto issue) -> bool { return mma_stage_with(issue, [] {}); };
     // Stores of a finished chunk's z (rows y0c .. y0c + bcc - 1), my tokens: reads
     // only the Z columns of tensor memory; no global loads on this path (the gate
     // x + tanh(alpha) z runs afterwards as a separate elementwise kernel).
@@ -363,29 +347,39 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         }
 
         STAMP(0);
-        // ---- A: A^T = W1 K^T (my rows);  S = Q K^T
+        // ---- A: A^T = W1 K^T (my rows); then Aq0^T = W1 Q^T, S = Q K^T (bar_a2).  Meanwhile:
+        //      the previous chunk's z out, K^T into X1 (nothing later in the chunk writes K or X1
+        //      before a block barrier)
         if (!mma_stage_with(
                 [&] {
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                    tc::mma_commit(bar_mma);
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_tf32_ts(tm + TM_AQ, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
+                    tc::mma_commit(bar_a2);
                 },
                 [&] {
                     if (prev_bc) store_z_chunk(prev_y0, prev_bc);
+                    {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
+                        const int j = tid & 63, tb = tid >> 6;
+                        uint32_t ph[8];
+                        col_phases(j, ST64, ph);
+                        const uint8_t* src = sm + OFF_K + tb * 1024;
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
+                        st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
+                        st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
+                    }
                 }))
             break;
         prev_bc = 0;
-        if (tid == 0 && c + 1 < c_last) {   // Q is free: fetch the next chunk's queries
-            int ny0, nbc;
-            chunk_rows(c + 1, ny0, nbc);
-            load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
-        }
 
         STAMP(1);
-        // ---- B: G = GELU(A) to shared [t][i] and in place (G^T); G' kept; K^T; M mask
+        // ---- B: G = GELU(A) to shared [t][i] and in place (G^T); G' kept
         __half2 gp[8];
         {
             const int t0 = 16 * g;
@@ -414,23 +408,20 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::tmem_wait_st();
 
         STAMP(2);
-        // ---- C: my Y^T partial = W2[:, mine] G[:, mine]^T  (rows 64.. of the A operand are unused)
+        // ---- C: my Y^T partial = W2[:, mine] G[:, mine]^T  (rows 64.. of the A operand are unused);
+        //      meanwhile the prefix mask M from S (the next stage writes neither S nor X2)
         if (!mma_stage_with(
                 [&] {
                     for (int kk = 0; kk < 16; ++kk)
                         tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
+                    tc::mma_commit(bar_mma);
                 },
                 [&] {
-        {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
-                        const int j = tid & 63, tb = tid >> 6;
-                        uint32_t ph[8];
-                        col_phases(j, ST64, ph);
-                        const uint8_t* src = sm + OFF_K + tb * 1024;
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
-                        st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
-                        st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
+                    wait_mma(bar_a2, ph_a2);   // S is ready; Q and K are no longer read
+                    if (tid == 0 && c + 1 < c_last) {   // Q is free: fetch the next chunk's queries
+                        int ny0, nbc;
+                        chunk_rows(c + 1, ny0, nbc);
+                        load_tile(&P.mapQ, OFF_Q, bar_q, ny0);
                     }
                     if (q < 2) {   // M[t][s] = S[t][s] for s not after t (prefix)
                         const int t = 32 * q + lane, s0 = 16 * g;
@@ -484,6 +475,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                tc::mma_commit(bar_mma);
             }))
             break;
         if (tid == 0 && c + 1 < c_last) {   // K and V buffers are free: fetch the next chunk's tiles
@@ -511,20 +503,21 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         }
 
         STAMP(6);
-        // ---- G: W1 += Dl^T K;  W2^T += G^T D2';  Aq^T += Dl^T M^T
+        // ---- G: Aq^T += Dl^T M^T (waited for); then W1 += Dl^T K, W2^T += G^T D2' (bar_g2)
         if (!mma_stage([&] {
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + TM_AQ, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
+                tc::mma_commit(bar_mma);
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_W1, tm + TM_P + kk * 8, kstep(dX1, kk, ST64), ID64, 1);
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_W2T, tm + TM_X + kk * 8, kstep(dX3, kk, ST64), ID64, 1);
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_AQ, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
+                tc::mma_commit(bar_g2);
             }))
             break;
 
         STAMP(8);
-        // ---- I: W2 copy from the updated master; Gq = GELU(Aq) to shared [t][i]
-        refresh_w2();
+        // ---- I: Gq = GELU(Aq) to shared [t][i]
         {
             const int t0 = 16 * g;
             uint32_t ph[8], r[16];
@@ -545,12 +538,13 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         if (!mma_stage([&] {
                 for (int kk = 0; kk < 16; ++kk)
                     tc::mma_tf32_ss(tm + TM_ZN, kstep(dW2, kk, 16384), kstep(dGQ, kk, ST64), ID64, kk > 0);
+                tc::mma_commit(bar_mma);
             }))
             break;
 
         STAMP(10);
         // ---- K: exchange token halves of the partials; rows 0-63 -> full Z1^T back to tensor
-        //      memory, rows 64-127 -> Nm[t_own][s] = -N[s][t] for s after t
+        //      memory, rows 64-127 -> Np[t_own][s] = N[s][t] for s not after t
         {
             const int t0 = 16 * g;
             const uint32_t addr = tm + lane_base + TM_ZN + t0;
@@ -583,18 +577,25 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
 #pragma unroll
                     for (int k = 0; k < 16; ++k)
                         *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
-                            after(s, t0 + k) ? tf32r(-v[k]) : 0.f;
+                            after(s, t0 + k) ? 0.f : tf32r(v[k]);
                 }
             }
         }
         ph_rz ^= 1;
 
         STAMP(11);
-        // ---- L: Z^T (my tokens) += D2'^T Nm^T
-        if (!mma_stage([&] {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID32, 1);
-            }))
+        // ---- L: Z^T (my tokens) += D2'^T Np^T; meanwhile the shared W2 copy takes the update
+        if (!mma_stage_with(
+                [&] {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID32,
+                                        1);
+                    tc::mma_commit(bar_mma);
+                },
+                [&] {
+                    wait_mma(bar_g2, ph_g2);
+                    refresh_w2();
+                }))
             break;
         prev_y0 = y0;
         prev_bc = bc;
