@@ -27,6 +27,9 @@
 // All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
 // shared-memory operands with the 128-byte swizzle.  Waits are bounded.
 //
+// The partials travel as asynchronous 16-byte stores into the peer's shared
+// memory that complete bytes on the peer's receive barrier (armed by one local
+// thread with the expected 16 KB right after the previous phase completed).
 // Ordering of the exchange buffers (no handshake needed): the peer writes my
 // RY for chunk c+1 only after it received my [Z1;N] partial of chunk c, which
 // I send after I have read RY of chunk c; it writes my RZ for chunk c+1 only
@@ -55,8 +58,9 @@ constexpr int OFF_X3 = 131072;    // 64 x 64: D2'^T [j][t]
 constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Np [t_own][s] (32 rows)
 constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s] (prefix mask)
 constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
-constexpr int OFF_RY = 196608;    // 64 x 64 fp32 plain [t][j]: the peer's Y^T partial
-constexpr int OFF_RZ = 212992;    // 32 x 128 fp32 plain [t_own][lane]: the peer's [Z1; N] partial for my tokens
+constexpr int OFF_RY = 196608;    // 64 x 64 fp32 [j][t]: the peer's Y^T partial (ry_off)
+constexpr int OFF_RZ = 212992;    // 128 x 32 fp32 [lane][t_own]: the peer's [Z1; N] partial for my tokens (rz_off)
+constexpr uint32_t XCHG_BYTES = 16384;   // each exchange moves 16 KB each way
 constexpr int OFF_BAR = 229376;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr int ST64 = 8192;
@@ -100,12 +104,18 @@ __device__ __forceinline__ float tf32r(float x) {
     return __uint_as_float(r);
 }
 
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // erf-GELU (and GELU') with erf from Abramowitz & Stegun, Handbook of
 // Mathematical Functions, formula 7.1.26: |error| <= 1.5e-7, far below the
 // tf32 rounding the results get; GELU and GELU' share one exponential.
 __device__ __forceinline__ void gelu_as(float a, float& g, float& gp, bool want_prime) {
     const float x = fabsf(a) * 0.70710678118654752f;
-    const float u = __frcp_rn(fmaf(0.3275911f, x, 1.0f));
+    const float u = rcp_approx(fmaf(0.3275911f, x, 1.0f));   // argument >= 1
     const float e = __expf(-0.5f * a * a);
     float poly = fmaf(1.061405429f, u, -1.453152027f);
     poly = fmaf(poly, u, 1.421413741f);
@@ -143,6 +153,11 @@ __device__ __forceinline__ void col_phases(int c, int stride, uint32_t (&ph)[8])
 __device__ __forceinline__ uint32_t row4_off(int R, int c, int stride) {
     return (uint32_t)((c >> 5) * stride + (R >> 3) * 1024 + (R & 7) * 128 + ((((c & 31) >> 2) ^ (R & 7)) << 4));
 }
+
+// Receive buffers: rows of 16-byte chunks, chunk index XOR-ed with the row so
+// that 32 threads on consecutive rows hit distinct banks.  t a multiple of 4.
+__device__ __forceinline__ uint32_t ry_off(int j, int t) { return (uint32_t)(j * 256 + (((t >> 2) ^ (j & 15)) << 4)); }
+__device__ __forceinline__ uint32_t rz_off(int i, int t) { return (uint32_t)(i * 128 + (((t >> 2) ^ (i & 7)) << 4)); }
 
 __device__ __forceinline__ void st4(uint8_t* p, float a, float b, float c, float d) {
     *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
@@ -191,12 +206,14 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::mbar_init(bar_k, 1);
         tc::mbar_init(bar_q, 1);
         tc::mbar_init(bar_v, 1);
-        tc::mbar_init(bar_ry, 256);   // one arrival per peer thread holding Y^T rows
-        tc::mbar_init(bar_rz, 256);   // one arrival per peer thread holding my tokens' columns
+        tc::mbar_init(bar_ry, 1);   // one local arrival with expect_tx; the peer's stores complete the bytes
+        tc::mbar_init(bar_rz, 1);
         tc::mbar_init(bar_never, 1);
         tc::mbar_init(bar_a2, 1);
         tc::mbar_init(bar_g2, 1);
         *abort_flag = 0;
+        tc::mbar_arrive_expect_tx(bar_ry, XCHG_BYTES);   // arm phase 0 of both receive barriers
+        tc::mbar_arrive_expect_tx(bar_rz, XCHG_BYTES);
         tc::fence_mbar_init();
     }
     if (warp == 0) {
@@ -447,18 +464,28 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_Y + t0, r);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int k = 0; k < 16; ++k) tc::st_cluster_f32(peer_ry + ((t0 + k) * 64 + j) * 4, __uint_as_float(r[k]));
-            tc::mbar_arrive_remote(peer_bar_ry);
+            for (int c4 = 0; c4 < 4; ++c4)
+                tc::st_async_v4(peer_ry + ry_off(j, t0 + 4 * c4), r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2], r[4 * c4 + 3],
+                                peer_bar_ry);
             col_phases(j, ST64, ph);
             const uint32_t rg = (t0 >> 3) * 1024;
             if (!tc::mbar_wait_cluster(bar_ry, ph_ry)) give_up();
-            const float* ry = reinterpret_cast<const float*>(sm + OFF_RY);
+            if (tid == 0) tc::mbar_arrive_expect_tx(bar_ry, XCHG_BYTES);   // arm the next phase
+            float ry[16];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(sm + OFF_RY + ry_off(j, t0 + 4 * c4));
+                ry[4 * c4] = v4.x;
+                ry[4 * c4 + 1] = v4.y;
+                ry[4 * c4 + 2] = v4.z;
+                ry[4 * c4 + 3] = v4.w;
+            }
             float d2[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int t = t0 + k;
                 const uint32_t off = rg + ph[k & 7] + (k >> 3) * 1024;
-                const float y = __uint_as_float(r[k]) + ry[t * 64 + j];
+                const float y = __uint_as_float(r[k]) + ry[k];
                 const float v = *reinterpret_cast<const float*>(sm + OFF_V + off);
                 d2[k] = (t < bc) ? tf32r(-2.0f * eta * (y - v)) : 0.f;
                 *reinterpret_cast<float*>(sm + OFF_K + off) = d2[k];
@@ -554,16 +581,22 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             if (!my_tokens) {
                 const int tl0 = t0 - 32 * (int)r_peer;   // the peer's local token index
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    tc::st_cluster_f32(peer_rz + ((tl0 + k) * 128 + i_loc) * 4, __uint_as_float(r[k]));
-                tc::mbar_arrive_remote(peer_bar_rz);
+                for (int c4 = 0; c4 < 4; ++c4)
+                    tc::st_async_v4(peer_rz + rz_off(i_loc, tl0 + 4 * c4), r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2],
+                                    r[4 * c4 + 3], peer_bar_rz);
             } else {
                 const int tl0 = t0 - 32 * (int)r_cta;
                 if (!tc::mbar_wait_cluster(bar_rz, ph_rz)) give_up();
-                const float* rz = reinterpret_cast<const float*>(sm + OFF_RZ);
+                if (tid == 256 * (int)r_cta) tc::mbar_arrive_expect_tx(bar_rz, XCHG_BYTES);   // arm the next phase
                 float v[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]) + rz[(tl0 + k) * 128 + i_loc];
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(sm + OFF_RZ + rz_off(i_loc, tl0 + 4 * c4));
+                    v[4 * c4] = __uint_as_float(r[4 * c4]) + v4.x;
+                    v[4 * c4 + 1] = __uint_as_float(r[4 * c4 + 1]) + v4.y;
+                    v[4 * c4 + 2] = __uint_as_float(r[4 * c4 + 2]) + v4.z;
+                    v[4 * c4 + 3] = __uint_as_float(r[4 * c4 + 3]) + v4.w;
+                }
                 if (q < 2) {   // Z1^T rows: the full sums become the accumulator of stage L
 #pragma unroll
                     for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(v[k]);
