@@ -28,8 +28,10 @@
 // shared-memory operands with the 128-byte swizzle.  Waits are bounded.
 //
 // The partials travel as asynchronous 16-byte stores into the peer's shared
-// memory that complete bytes on the peer's receive barrier (armed by one local
-// thread with the expected 16 KB right after the previous phase completed).
+// memory that complete bytes on a receive barrier of the peer.  Each receiving
+// warp reads exactly what one sending warp of the peer wrote, so every warp
+// pair has a barrier of its own (2 KB per phase, armed by the receiving warp's
+// lane 0 right after the previous phase completed).
 // Ordering of the exchange buffers (no handshake needed): the peer writes my
 // RY for chunk c+1 only after it received my [Z1;N] partial of chunk c, which
 // I send after I have read RY of chunk c; it writes my RZ for chunk c+1 only
@@ -60,7 +62,7 @@ constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s] (prefix mask)
 constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
 constexpr int OFF_RY = 196608;    // 64 x 64 fp32 [j][t]: the peer's Y^T partial (ry_off)
 constexpr int OFF_RZ = 212992;    // 128 x 32 fp32 [lane][t_own]: the peer's [Z1; N] partial for my tokens (rz_off)
-constexpr uint32_t XCHG_BYTES = 16384;   // each exchange moves 16 KB each way
+constexpr uint32_t XCHG_WARP_BYTES = 2048;   // each exchange: 8 warps x 2 KB each way
 constexpr int OFF_BAR = 229376;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr int ST64 = 8192;
@@ -76,11 +78,14 @@ constexpr uint32_t TM_ZN = 384;   // [Z1^T; N] partial: [j | s][t]
 constexpr uint32_t TM_AQ = 448;   // Aq^T: [i][t]
 
 #ifdef TTT_DEBUG_STAGES
-// Debug builds only: cycles thread 0 of CTA 0 spends between stage boundaries.
+// Debug builds only: cycles thread 0 of CTA TTT_STAMP_CTA spends between stage boundaries.
+#ifndef TTT_STAMP_CTA
+#define TTT_STAMP_CTA 0
+#endif
 __device__ float* g_dbg2 = nullptr;
 #define STAMP(k)                                                      \
     do {                                                              \
-        if (tid == 0 && blockIdx.x == 0) {                            \
+        if (tid == 0 && blockIdx.x == TTT_STAMP_CTA) {                \
             const long long now_ = clock64();                         \
             stamp_acc[k] += now_ - stamp_last;                        \
             stamp_last = now_;                                        \
@@ -171,8 +176,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint64_t* bar_k = bar_mma + 1;
     uint64_t* bar_q = bar_mma + 2;
     uint64_t* bar_v = bar_mma + 3;
-    uint64_t* bar_ry = bar_mma + 4;   // the peer's Y^T partial has landed in RY
-    uint64_t* bar_rz = bar_mma + 5;   // the peer's [Z1; N] partial has landed in RZ
+    uint64_t* bar_ryw = bar_mma + 10;   // [8] a peer warp's part of the Y^T partial has landed in RY
+    uint64_t* bar_rzw = bar_mma + 18;   // [8] a peer warp's part of the [Z1; N] partial has landed in RZ
     uint64_t* bar_never = bar_mma + 6;   // fault injection: nothing ever arrives here
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 7);
     uint64_t* bar_a2 = bar_mma + 8;      // the first stage's second group (Aq0, S)
@@ -198,22 +203,28 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     // the peer's receive buffers and barriers
     const uint32_t peer_ry = tc::mapa_shared(tc::smem_u32(sm + OFF_RY), r_peer);
     const uint32_t peer_rz = tc::mapa_shared(tc::smem_u32(sm + OFF_RZ), r_peer);
-    const uint32_t peer_bar_ry = tc::mapa_shared(tc::smem_u32(bar_ry), r_peer);
-    const uint32_t peer_bar_rz = tc::mapa_shared(tc::smem_u32(bar_rz), r_peer);
+    // exchange warp pairs: D pairs the q < 2 warps, K pairs the warps of one token half
+    const int wx_y = 2 * g + (q & 1), wx_z = 4 * (g & 1) + q;
+    const uint32_t peer_bar_ry = tc::mapa_shared(tc::smem_u32(bar_ryw + wx_y), r_peer);
+    const uint32_t peer_bar_rz = tc::mapa_shared(tc::smem_u32(bar_rzw + wx_z), r_peer);
 
     if (tid == 0) {
         tc::mbar_init(bar_mma, 1);
         tc::mbar_init(bar_k, 1);
         tc::mbar_init(bar_q, 1);
         tc::mbar_init(bar_v, 1);
-        tc::mbar_init(bar_ry, 1);   // one local arrival with expect_tx; the peer's stores complete the bytes
-        tc::mbar_init(bar_rz, 1);
+        for (int w = 0; w < 8; ++w) {   // one local arrival with expect_tx; the peer's stores complete the bytes
+            tc::mbar_init(bar_ryw + w, 1);
+            tc::mbar_init(bar_rzw + w, 1);
+        }
         tc::mbar_init(bar_never, 1);
-        tc::mbar_init(bar_a2, 1);
-        tc::mbar_init(bar_g2, 1);
+        tc::mbar_init(bar_a2, 2);   // two issuing threads commit to each
+        tc::mbar_init(bar_g2, 2);
         *abort_flag = 0;
-        tc::mbar_arrive_expect_tx(bar_ry, XCHG_BYTES);   // arm phase 0 of both receive barriers
-        tc::mbar_arrive_expect_tx(bar_rz, XCHG_BYTES);
+        for (int w = 0; w < 8; ++w) {   // arm phase 0 of the receive barriers
+            tc::mbar_arrive_expect_tx(bar_ryw + w, XCHG_WARP_BYTES);
+            tc::mbar_arrive_expect_tx(bar_rzw + w, XCHG_WARP_BYTES);
+        }
         tc::fence_mbar_init();
     }
     if (warp == 0) {
@@ -287,7 +298,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     refresh_w2();
 
 #ifdef TTT_DEBUG_STAGES
-    long long stamp_acc[20] = {};
+    long long stamp_acc[28] = {};
     long long stamp_last = clock64();
 #endif
     auto give_up = [&]() {
@@ -302,17 +313,17 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         ph ^= 1;
         tc::tc_fence_after();
     };
-    // One MMA stage: all threads' operand writes become visible, thread 0
-    // issues (and commits: the group the stage waits for goes to bar_mma),
-    // `work` (touching nothing the MMAs read or write) runs meanwhile.
+    // One MMA stage: all threads' operand writes become visible, the issuing
+    // threads issue (and commit: the group the stage waits for goes to
+    // bar_mma), `work` (touching nothing the MMAs read or write) runs meanwhile.
+    // Accumulators that do not depend on one another are issued by different
+    // threads (lane 0 of warps 0, 1, 2) so that their issue overlaps.
     auto mma_stage_with = [&](auto issue, auto work) -> bool {
         tc::fence_proxy_async_smem();
         tc::tc_fence_before();
         if (__syncthreads_or(*abort_flag)) return false;
-        if (tid == 0) {
-            tc::tc_fence_after();
-            issue();
-        }
+        tc::tc_fence_after();
+        issue();
         work();
         wait_mma(bar_mma, ph_mma);
         return true;
@@ -369,14 +380,20 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         //      before a block barrier)
         if (!mma_stage_with(
                 [&] {
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
-                    tc::mma_commit(bar_mma);
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_AQ, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
-                    tc::mma_commit(bar_a2);
+                    if (tid == 0) {
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_tf32_ts(tm + TM_X, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                        tc::mma_commit(bar_mma);
+                        STAMP(14);
+                    } else if (tid == 32) {
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_tf32_ts(tm + TM_AQ, tm + TM_W1 + kk * 8, kstep(dQ, kk, ST64), ID64, kk > 0);
+                        tc::mma_commit(bar_a2);
+                    } else if (tid == 64) {
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID64, kk > 0);
+                        tc::mma_commit(bar_a2);
+                    }
                 },
                 [&] {
                     if (prev_bc) store_z_chunk(prev_y0, prev_bc);
@@ -429,9 +446,12 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         //      meanwhile the prefix mask M from S (the next stage writes neither S nor X2)
         if (!mma_stage_with(
                 [&] {
-                    for (int kk = 0; kk < 16; ++kk)
-                        tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
-                    tc::mma_commit(bar_mma);
+                    if (tid == 0) {
+                        for (int kk = 0; kk < 16; ++kk)
+                            tc::mma_tf32_ss(tm + TM_Y, kstep(dW2, kk, 16384), kstep(dG, kk, 16384), ID64, kk > 0);
+                        tc::mma_commit(bar_mma);
+                        STAMP(15);
+                    }
                 },
                 [&] {
                     wait_mma(bar_a2, ph_a2);   // S is ready; Q and K are no longer read
@@ -469,8 +489,15 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                                 peer_bar_ry);
             col_phases(j, ST64, ph);
             const uint32_t rg = (t0 >> 3) * 1024;
-            if (!tc::mbar_wait_cluster(bar_ry, ph_ry)) give_up();
-            if (tid == 0) tc::mbar_arrive_expect_tx(bar_ry, XCHG_BYTES);   // arm the next phase
+            STAMP(20);
+            float vv[16];   // V first: no load waits behind a store below
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                vv[k] = *reinterpret_cast<const float*>(sm + OFF_V + rg + ph[k & 7] + (k >> 3) * 1024);
+            if (!tc::mbar_wait_cluster(bar_ryw + wx_y, ph_ry)) give_up();
+            STAMP(21);
+            if (lane == 0) tc::mbar_arrive_expect_tx(bar_ryw + wx_y, XCHG_WARP_BYTES);   // arm the next phase
+            STAMP(24);
             float ry[16];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) {
@@ -480,16 +507,17 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                 ry[4 * c4 + 2] = v4.z;
                 ry[4 * c4 + 3] = v4.w;
             }
+            STAMP(25);
             float d2[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const int t = t0 + k;
-                const uint32_t off = rg + ph[k & 7] + (k >> 3) * 1024;
                 const float y = __uint_as_float(r[k]) + ry[k];
-                const float v = *reinterpret_cast<const float*>(sm + OFF_V + off);
-                d2[k] = (t < bc) ? tf32r(-2.0f * eta * (y - v)) : 0.f;
-                *reinterpret_cast<float*>(sm + OFF_K + off) = d2[k];
+                d2[k] = (t0 + k < bc) ? tf32r(-2.0f * eta * (y - vv[k])) : 0.f;
             }
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                *reinterpret_cast<float*>(sm + OFF_K + rg + ph[k & 7] + (k >> 3) * 1024) = d2[k];
+            STAMP(26);
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4)
                 st4(sm + OFF_X3 + row4_off(j, t0 + 4 * c4, ST64), d2[4 * c4], d2[4 * c4 + 1], d2[4 * c4 + 2],
@@ -500,9 +528,12 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         STAMP(4);
         // ---- E: P^T = W2^T D2'^T (my rows)
         if (!mma_stage([&] {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
-                tc::mma_commit(bar_mma);
+                if (tid == 0) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_P, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID64, kk > 0);
+                    tc::mma_commit(bar_mma);
+                    STAMP(16);
+                }
             }))
             break;
         if (tid == 0 && c + 1 < c_last) {   // K and V buffers are free: fetch the next chunk's tiles
@@ -532,14 +563,20 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         STAMP(6);
         // ---- G: Aq^T += Dl^T M^T (waited for); then W1 += Dl^T K, W2^T += G^T D2' (bar_g2)
         if (!mma_stage([&] {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_AQ, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
-                tc::mma_commit(bar_mma);
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_W1, tm + TM_P + kk * 8, kstep(dX1, kk, ST64), ID64, 1);
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_W2T, tm + TM_X + kk * 8, kstep(dX3, kk, ST64), ID64, 1);
-                tc::mma_commit(bar_g2);
+                if (tid == 0) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_AQ, tm + TM_P + kk * 8, kstep(dX2, kk, ST64), ID64, 1);
+                    tc::mma_commit(bar_mma);
+                    STAMP(17);
+                } else if (tid == 32) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_W1, tm + TM_P + kk * 8, kstep(dX1, kk, ST64), ID64, 1);
+                    tc::mma_commit(bar_g2);
+                } else if (tid == 64) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        tc::mma_tf32_ts(tm + TM_W2T, tm + TM_X + kk * 8, kstep(dX3, kk, ST64), ID64, 1);
+                    tc::mma_commit(bar_g2);
+                }
             }))
             break;
 
@@ -562,11 +599,17 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
 
         STAMP(9);
         // ---- J: my [Z1^T; N] partial = [W2; G][:, mine] Gq[:, mine]^T
-        if (!mma_stage([&] {
-                for (int kk = 0; kk < 16; ++kk)
-                    tc::mma_tf32_ss(tm + TM_ZN, kstep(dW2, kk, 16384), kstep(dGQ, kk, ST64), ID64, kk > 0);
-                tc::mma_commit(bar_mma);
-            }))
+        //      meanwhile: the W1 and W2^T updates have landed (X1 is rewritten next, W2^T read in L)
+        if (!mma_stage_with(
+                [&] {
+                    if (tid == 0) {
+                        for (int kk = 0; kk < 16; ++kk)
+                            tc::mma_tf32_ss(tm + TM_ZN, kstep(dW2, kk, 16384), kstep(dGQ, kk, ST64), ID64, kk > 0);
+                        tc::mma_commit(bar_mma);
+                        STAMP(18);
+                    }
+                },
+                [&] { wait_mma(bar_g2, ph_g2); }))
             break;
 
         STAMP(10);
@@ -586,8 +629,10 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                                     r[4 * c4 + 3], peer_bar_rz);
             } else {
                 const int tl0 = t0 - 32 * (int)r_cta;
-                if (!tc::mbar_wait_cluster(bar_rz, ph_rz)) give_up();
-                if (tid == 256 * (int)r_cta) tc::mbar_arrive_expect_tx(bar_rz, XCHG_BYTES);   // arm the next phase
+                STAMP(22);
+                if (!tc::mbar_wait_cluster(bar_rzw + wx_z, ph_rz)) give_up();
+                STAMP(23);
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar_rzw + wx_z, XCHG_WARP_BYTES);   // arm the next phase
                 float v[16];
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
@@ -620,15 +665,15 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         // ---- L: Z^T (my tokens) += D2'^T Np^T; meanwhile the shared W2 copy takes the update
         if (!mma_stage_with(
                 [&] {
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID32,
-                                        1);
-                    tc::mma_commit(bar_mma);
+                    if (tid == 0) {
+                        for (int kk = 0; kk < 8; ++kk)
+                            tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64),
+                                            ID32, 1);
+                        tc::mma_commit(bar_mma);
+                        STAMP(19);
+                    }
                 },
-                [&] {
-                    wait_mma(bar_g2, ph_g2);
-                    refresh_w2();
-                }))
+                [&] { refresh_w2(); }))
             break;
         prev_y0 = y0;
         prev_bc = bc;
@@ -639,8 +684,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     if (prev_bc && !*abort_flag) store_z_chunk(prev_y0, prev_bc);   // the last chunk's z
 
 #ifdef TTT_DEBUG_STAGES
-    if (tid == 0 && blockIdx.x == 0 && g_dbg2) {
-        for (int k = 0; k < 20; ++k) g_dbg2[k] = (float)stamp_acc[k];
+    if (tid == 0 && blockIdx.x == TTT_STAMP_CTA && g_dbg2) {
+        for (int k = 0; k < 28; ++k) g_dbg2[k] = (float)stamp_acc[k];
         g_dbg2[30] = (float)(c_last - c_first);
     }
 #endif
