@@ -49,7 +49,8 @@ typedef enum {
     TTT_ERR_INVALID_ARG = 1,   /* a pointer, size or value violates the contract below */
     TTT_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. a head dim other than 16/32/64) */
     TTT_ERR_CUDA = 3,          /* a CUDA runtime call failed; ttt_last_error() has its message */
-    TTT_ERR_NONFINITE = 4,     /* (ttt_mlp_status) an output z was NaN/Inf: the scan diverged */
+    TTT_ERR_NONFINITE = 4,     /* (ttt_mlp_status) a NaN/Inf in the inputs, projections or outputs z:
+                                  bad inputs or a diverged scan; outputs invalid */
     TTT_ERR_TIMEOUT = 5        /* (ttt_mlp_status) a bounded on-chip wait expired; outputs invalid */
 } ttt_status;
 
@@ -120,8 +121,9 @@ TTT_API ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X,
 
 /*
  * Synchronises `stream`, reads and clears the status word a previous
- * ttt_mlp_forward left in `workspace`: TTT_OK, TTT_ERR_NONFINITE (an output
- * was NaN/Inf, e.g. eta too large for the squared-norm loss) or
+ * ttt_mlp_forward left in `workspace`: TTT_OK, TTT_ERR_NONFINITE (a NaN/Inf
+ * in X, theta or W_0, in the projections, or in an output, e.g. eta too large
+ * for the squared-norm loss) or
  * TTT_ERR_TIMEOUT (a bounded wait inside a kernel expired; outputs invalid).
  */
 TTT_API ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream);

@@ -167,7 +167,7 @@ ttt_status project(const ttt_mlp_desc& q, const void* src, int src_bf16, const v
     const int th_bf16 = q.x_dtype == TTT_BF16;
     if (q.per_head_input) {
         if (accumulate) return fail(TTT_ERR_UNSUPPORTED, "internal: accumulate in per-head projection");
-        CUDA_TRY(launch_proj_per_head(src, src_bf16, th, th_bf16, out, q.T, q.H, q.d, s));
+        CUDA_TRY(launch_proj_per_head(src, src_bf16, th, th_bf16, out, q.T, q.H, q.d, status, s));
         return TTT_OK;
     }
     const int impl = g_proj_impl.load();
@@ -177,7 +177,7 @@ ttt_status project(const ttt_mlp_desc& q, const void* src, int src_bf16, const v
     if (tc_ok && impl != 1) {
         CUDA_TRY(launch_proj_full_tc(src, th, out, q.T, q.D, q.D, accumulate, status, 0, s));
     } else {
-        CUDA_TRY(launch_proj_full_simt(src, src_bf16, th, th_bf16, out, q.T, q.D, q.D, accumulate, s));
+        CUDA_TRY(launch_proj_full_simt(src, src_bf16, th, th_bf16, out, q.T, q.D, q.D, accumulate, status, s));
     }
     return TTT_OK;
 }
@@ -573,7 +573,8 @@ ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {
     CUDA_TRY(cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost));
     CUDA_TRY(cudaMemset(workspace, 0, sizeof(int)));
     if (word & kStatusTimeout) return fail(TTT_ERR_TIMEOUT, "a bounded wait inside a scan kernel expired");
-    if (word & kStatusNonFinite) return fail(TTT_ERR_NONFINITE, "the scan produced non-finite outputs");
+    if (word & kStatusNonFinite)
+        return fail(TTT_ERR_NONFINITE, "non-finite values in the inputs, projections or outputs");
     return TTT_OK;
 }
 

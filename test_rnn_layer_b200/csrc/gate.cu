@@ -1,7 +1,7 @@
 // The gate out = x + tanh(alpha) * z over a whole direction's outputs
 // (paper notes page, "关键设计 / 门控 + 双向机制"), with the optional bf16
 // increment tanh(alpha) * z that the full layer's reverse projection uses, and
-// the non-finite check of z.  Bandwidth-bound: four elements per thread and
+// the non-finite check of x and z.  Bandwidth-bound: four elements per thread and
 // iteration, grid-stride over the flat arrays (all in X's layout).
 #include "common.cuh"
 #include "internal.h"
@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(256) gate_kernel(GateArgs g) {
         const float4 dz = make_float4(tanhf(al.x) * z.x, tanhf(al.y) * z.y, tanhf(al.z) * z.z, tanhf(al.w) * z.w);
         store4(g.Out, i, g.out_bf16, make_float4(x.x + dz.x, x.y + dz.y, x.z + dz.z, x.w + dz.w));
         if (g.Delta) store4(g.Delta, i, 1, dz);
-        nonfinite |= !(isfinite(z.x) && isfinite(z.y) && isfinite(z.z) && isfinite(z.w));
+        nonfinite |= !(isfinite(z.x) && isfinite(z.y) && isfinite(z.z) && isfinite(z.w) && isfinite(x.x) &&
+                       isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
     }
     if (__syncthreads_or(nonfinite) && threadIdx.x == 0) atomicOr(g.status, kStatusNonFinite);
 }

@@ -55,12 +55,12 @@ cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s);   // a clu
 
 // Per-head projections: U[which][h, t, e] = sum_j theta_which[h][e][j] x[h, t, j].
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
-                                 float* const out[3], int T, int H, int d, cudaStream_t s);
+                                 float* const out[3], int T, int H, int d, int* status, cudaStream_t s);
 
 // Full-mode projections: C_which[t, n] (+)= sum_c A[t, c] Theta_which[n, c],
 // A [T, Dm] row-major, Theta [N, Dm] row-major, C [T, N] fp32.
 cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
-                                  float* const out[3], int T, int N, int Dm, int accumulate,
+                                  float* const out[3], int T, int N, int Dm, int accumulate, int* status,
                                   cudaStream_t s);
 
 // tcgen05 projections (bf16 A and Theta, N % 256 == 0, K % 64 == 0), same contract.

@@ -16,7 +16,7 @@ constexpr int kPhThreads = 256;
 
 __global__ void __launch_bounds__(kPhThreads)
 proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk, const void* thv,
-                     int th_bf16, float* oq, float* ok, float* ov, int T, int d) {
+                     int th_bf16, float* oq, float* ok, float* ov, int T, int d, int* status) {
     extern __shared__ float sm[];
     float* th = sm;                     // [3][d][d]
     float* xs = sm + 3 * d * d;         // [kPhTok][d]
@@ -32,6 +32,7 @@ proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk
         xs[p] = load_elem(X, ((long long)h * T + t0) * d + p, x_bf16);
     __syncthreads();
     float* outs[3] = {oq, ok, ov};
+    int bad = 0;   // a non-finite input reaches every projection of its token
     for (int p = threadIdx.x; p < 3 * nt * d; p += blockDim.x) {
         const int w = p / (nt * d), q = p % (nt * d);
         const int r = q / d, e = q % d;
@@ -40,7 +41,9 @@ proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk
         float acc = 0.f;
         for (int j = 0; j < d; ++j) acc = fmaf(row[j], x[j], acc);
         outs[w][((long long)h * T + t0 + r) * d + e] = acc;
+        bad |= !isfinite(acc);
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kStatusNonFinite);
 }
 
 // C[t, n] (+)= sum_c A[t, c] B[n, c]; 64 x 64 tile, 16-deep k steps, 4 x 4 per thread.
@@ -48,7 +51,7 @@ constexpr int kGT = 64, kGK = 16;
 
 __global__ void __launch_bounds__(256)
 proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1, const void* B2, int b_bf16,
-                      float* C0, float* C1, float* C2, int T, int N, int Dm, int accumulate) {
+                      float* C0, float* C1, float* C2, int T, int N, int Dm, int accumulate, int* status) {
     __shared__ float As[kGK][kGT + 4];
     __shared__ float Bs[kGK][kGT + 4];
     const void* B = blockIdx.z == 0 ? B0 : (blockIdx.z == 1 ? B1 : B2);
@@ -76,6 +79,7 @@ proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1,
         }
         __syncthreads();
     }
+    int bad = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int t = t0 + ty * 4 + u;
@@ -86,14 +90,16 @@ proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1,
             if (n >= N) continue;
             float* dst = C + (long long)t * N + n;
             *dst = accumulate ? *dst + acc[u][v] : acc[u][v];
+            bad |= !isfinite(acc[u][v]);
         }
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kStatusNonFinite);
 }
 
 }  // namespace
 
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
-                                 float* const out[3], int T, int H, int d, cudaStream_t s) {
+                                 float* const out[3], int T, int H, int d, int* status, cudaStream_t s) {
     const size_t smem = sizeof(float) * (3 * (size_t)d * d + (size_t)kPhTok * d);
     cudaError_t e = cudaFuncSetAttribute(proj_per_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -101,17 +107,17 @@ cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const th
     LaunchScope scope("proj_per_head", s);
     dim3 grid((T + kPhTok - 1) / kPhTok, H);
     proj_per_head_kernel<<<grid, kPhThreads, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16,
-                                                        out[0], out[1], out[2], T, d);
+                                                        out[0], out[1], out[2], T, d, status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,
-                                  float* const out[3], int T, int N, int Dm, int accumulate,
+                                  float* const out[3], int T, int N, int Dm, int accumulate, int* status,
                                   cudaStream_t s) {
     LaunchScope scope("proj_full_simt", s);
     dim3 grid((N + kGT - 1) / kGT, (T + kGT - 1) / kGT, 3);
     proj_full_simt_kernel<<<grid, 256, 0, s>>>(A, a_bf16, theta[0], theta[1], theta[2], th_bf16, out[0], out[1],
-                                                out[2], T, N, Dm, accumulate);
+                                                out[2], T, N, Dm, accumulate, status);
     return cudaGetLastError();
 }
 

@@ -134,19 +134,26 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
         // ---------------- epilogue (warps 2..5 -> TMEM lane quarters 2, 3, 0, 1)
         const int q = warp % 4;
         uint8_t* bufs = epi_base + (warp - 2) * 2 * EPI_BUF;
-        int it = 0, nbuf = 0;
+        int it = 0, nbuf = 0, nonfinite = 0;
         for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             const int mt = tile / n_tiles, nt = tile % n_tiles;
             const int which = nt / p.n_tiles_per;
             const int n0 = (nt % p.n_tiles_per) * BN;
-            if (!tc::mbar_wait(&tmem_full[acc], acc_phase, abort_flag)) { give_up(); break; }
+            // the whole warp leaves together (it meets __syncwarp below and __any_sync after the loop)
+            const bool got = tc::mbar_wait(&tmem_full[acc], acc_phase, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) {
+                if (lane == 0) give_up();
+                break;
+            }
             tc::tc_fence_after();
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + acc * BN + c * 32, r);
                 tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) nonfinite |= (r[j] & 0x7f800000u) == 0x7f800000u;
                 uint8_t* buf = bufs + nbuf * EPI_BUF;
                 if (lane == 0) tc::bulk_wait_group_read<1>();   // the store that last used `buf` has read it
                 __syncwarp();
@@ -170,6 +177,8 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
             if (lane == 0) tc::mbar_arrive(&tmem_empty[acc]);
         }
         if (lane == 0) tc::bulk_wait_group<0>();
+        // a non-finite input (X, theta or the increment) reaches the projections
+        if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(p.status, kStatusNonFinite);
     }
 
     if (*abort_flag) {

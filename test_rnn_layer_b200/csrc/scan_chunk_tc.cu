@@ -108,10 +108,19 @@ enum { DBG_AT = 0, DBG_S, DBG_YT, DBG_PT, DBG_W1, DBG_DW2T, DBG_AQT, DBG_ZN, DBG
     } while (0)
 #endif
 
+// Round to the nearest tf32 value, ties away from zero: add half a unit of the
+// 13 dropped mantissa bits, then clear them (a carry into the exponent is the
+// correct result, infinities stay infinite).  NaN is passed through as it is:
+// the GPU's NaN 0x7fffffff would carry into the sign bit.
 __device__ __forceinline__ float tf32r(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    const float r = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+    return x != x ? x : r;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 // erf-GELU and its derivative with erf from Abramowitz & Stegun, Handbook of
@@ -122,7 +131,7 @@ __device__ __forceinline__ float tf32r(float x) {
 // exponential, so GELU and GELU' share one exponential and one reciprocal.
 __device__ __forceinline__ void gelu_as(float a, float& g, float& gp, bool want_prime) {
     const float x = fabsf(a) * 0.70710678118654752f;
-    const float u = __frcp_rn(fmaf(0.3275911f, x, 1.0f));
+    const float u = rcp_approx(fmaf(0.3275911f, x, 1.0f));   // argument >= 1
     const float e = __expf(-0.5f * a * a);
     float poly = fmaf(1.061405429f, u, -1.453152027f);
     poly = fmaf(poly, u, 1.421413741f);

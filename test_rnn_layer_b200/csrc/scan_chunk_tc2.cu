@@ -103,10 +103,14 @@ struct ScanTc2Args {
     int full;
 };
 
+// Round to the nearest tf32 value, ties away from zero: add half a unit of the
+// 13 dropped mantissa bits, then clear them (a carry into the exponent is the
+// correct result, infinities stay infinite).  Two integer operations.  A NaN
+// may come out as zero (the GPU's NaN 0x7fffffff carries into the sign bit), so
+// non-finite values are detected where they enter instead: the projections
+// check Q, K, V, this kernel checks W1_0 and W2_0, the gate checks x and z.
 __device__ __forceinline__ float tf32r(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -262,6 +266,11 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             r1[k] = __float_as_uint(w1[k]);
             r2[k] = __float_as_uint(w2[(long long)(j0 + k) * MH]);
         }
+        int bad = 0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+            bad |= ((r1[k] & 0x7f800000u) == 0x7f800000u) | ((r2[k] & 0x7f800000u) == 0x7f800000u);
+        if (bad) atomicOr(a.status, kStatusNonFinite);
         tc::tmem_st_32x32b_x16(tm + lane_base + TM_W1 + j0, r1);
         tc::tmem_st_32x32b_x16(tm + lane_base + TM_W2T + j0, r2);
         tc::tmem_wait_st();

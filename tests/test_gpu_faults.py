@@ -28,9 +28,26 @@ def test_expired_wait_reports_timeout_and_context_survives():
     assert maxrel(to_np(g["Y"]), o["Y"]) <= tol(w)
 
 
-@pytest.mark.parametrize("w", [S.MINIBATCH.with_(T=200, H=2), S.TINY], ids=["tensor-core", "per-token"])
-def test_nonfinite_input_reports_nonfinite(w):
+def _poison(inp, key, value):
+    t = inp[key]
+    flat = t.view(-1)
+    flat[flat.numel() // 3] = value
+
+
+@pytest.mark.parametrize("w,key,value", [
+    (S.MINIBATCH.with_(T=200, H=2), "X", float("nan")),
+    (S.TINY, "X", float("nan")),
+    (S.FULL63S.with_(T=700, H=4, D=256), "X", float("nan")),
+    (S.FULL63S.with_(T=700, H=4, D=256), "theta_k", float("inf")),
+    (S.MINIBATCH.with_(T=200, H=2), "theta_v", float("nan")),
+    (S.MINIBATCH.with_(T=200, H=2), "W1_0", float("nan")),
+    (S.FULL63S.with_(T=700, H=4, D=256), "W2_0", float("-inf")),
+], ids=["per-head-X", "per-token-X", "full-layer-X", "full-layer-theta_k", "per-head-theta_v", "per-head-W1_0",
+        "full-layer-W2_0"])
+def test_nonfinite_input_reports_nonfinite(w, key, value):
+    """A NaN or Inf anywhere in the inputs comes back as TTT_ERR_NONFINITE,
+    whichever kernel it meets first (projection, scan state load, gate)."""
     inp = S.make_inputs(w)
-    inp["X"][0, 5, 3] = float("nan")
+    _poison(inp, key, value)
     g = run_gpu(w, inp, check_status=False)
     assert L.ttt_mlp_status(g["workspace"]) == L.TTT_ERR_NONFINITE
