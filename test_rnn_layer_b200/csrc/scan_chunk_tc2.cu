@@ -10,8 +10,14 @@
 // partial sums exchanged through distributed shared memory:
 //   Y^T  = W2 G^T           both CTAs receive the peer's [64 x 64] partial,
 //                           so both form the same D2' (fp32 a + b == b + a);
-//   [Z1^T; N] = [W2; G] Gq^T  each CTA owns 32 of the 64 tokens and receives
-//                           the peer's partial for those columns only.
+//   [Z1^T; N] = [W2; G] Gq^T  kept as partials (see below); each CTA owns 32 of
+//                           the 64 tokens of z and receives the peer's partial
+//                           z for those columns only.
+// The final z is also a sum over the pair: the masked correction is linear in N,
+// so each CTA adds D2'^T Np_r^T built from its own partial N_r to its own Z1
+// partial, and only the z partials for the peer's tokens cross (8 KB).  No
+// later stage depends on z, so the peer's half is received and stored while
+// the next chunk's first MMAs run.
 // The algebra per chunk (tokens t, s of the chunk in walking order; see the
 // one-CTA kernel for the derivation; paper notes page, "关键设计 / TTT-MLP 层"):
 //   A^T = W1 K^T, G = GELU(A), Y^T = W2 G^T, D2' = -2 eta (Y - V),
@@ -61,7 +67,7 @@ constexpr int OFF_X1 = 147456;    // 64 x 64: K^T [j][t]; then Np [t_own][s] (32
 constexpr int OFF_X2 = 163840;    // 64 x 64: M [t][s] (prefix mask)
 constexpr int OFF_V = 180224;     // 64 x 64: V [t][j] (TMA)
 constexpr int OFF_RY = 196608;    // 64 x 64 fp32 [j][t]: the peer's Y^T partial (ry_off)
-constexpr int OFF_RZ = 212992;    // 128 x 32 fp32 [lane][t_own]: the peer's [Z1; N] partial for my tokens (rz_off)
+constexpr int OFF_RZ = 212992;    // 64 x 32 fp32 [j][t_own]: the peer's z partial for my tokens (rz_off)
 constexpr uint32_t XCHG_WARP_BYTES = 2048;   // each exchange: 8 warps x 2 KB each way
 constexpr int OFF_BAR = 229376;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -166,7 +172,7 @@ __device__ __forceinline__ uint32_t row4_off(int R, int c, int stride) {
 // Receive buffers: rows of 16-byte chunks, chunk index XOR-ed with the row so
 // that 32 threads on consecutive rows hit distinct banks.  t a multiple of 4.
 __device__ __forceinline__ uint32_t ry_off(int j, int t) { return (uint32_t)(j * 256 + (((t >> 2) ^ (j & 15)) << 4)); }
-__device__ __forceinline__ uint32_t rz_off(int i, int t) { return (uint32_t)(i * 128 + (((t >> 2) ^ (i & 7)) << 4)); }
+__device__ __forceinline__ uint32_t rz_off(int j, int t) { return (uint32_t)(j * 128 + (((t >> 2) ^ (j & 7)) << 4)); }
 
 __device__ __forceinline__ void st4(uint8_t* p, float a, float b, float c, float d) {
     *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
@@ -181,7 +187,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint64_t* bar_q = bar_mma + 2;
     uint64_t* bar_v = bar_mma + 3;
     uint64_t* bar_ryw = bar_mma + 10;   // [8] a peer warp's part of the Y^T partial has landed in RY
-    uint64_t* bar_rzw = bar_mma + 18;   // [8] a peer warp's part of the [Z1; N] partial has landed in RZ
+    uint64_t* bar_rzw = bar_mma + 18;   // [4] a peer warp's part of the z partial has landed in RZ
     uint64_t* bar_never = bar_mma + 6;   // fault injection: nothing ever arrives here
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 7);
     uint64_t* bar_a2 = bar_mma + 8;      // the first stage's second group (Aq0, S)
@@ -207,8 +213,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     // the peer's receive buffers and barriers
     const uint32_t peer_ry = tc::mapa_shared(tc::smem_u32(sm + OFF_RY), r_peer);
     const uint32_t peer_rz = tc::mapa_shared(tc::smem_u32(sm + OFF_RZ), r_peer);
-    // exchange warp pairs: D pairs the q < 2 warps, K pairs the warps of one token half
-    const int wx_y = 2 * g + (q & 1), wx_z = 4 * (g & 1) + q;
+    // exchange warp pairs: both exchanges pair q < 2 warps (Y: all token groups, z: one token half)
+    const int wx_y = 2 * g + (q & 1), wx_z = 2 * (g & 1) + (q & 1);
     const uint32_t peer_bar_ry = tc::mapa_shared(tc::smem_u32(bar_ryw + wx_y), r_peer);
     const uint32_t peer_bar_rz = tc::mapa_shared(tc::smem_u32(bar_rzw + wx_z), r_peer);
 
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::mbar_init(bar_v, 1);
         for (int w = 0; w < 8; ++w) {   // one local arrival with expect_tx; the peer's stores complete the bytes
             tc::mbar_init(bar_ryw + w, 1);
-            tc::mbar_init(bar_rzw + w, 1);
+            if (w < 4) tc::mbar_init(bar_rzw + w, 1);
         }
         tc::mbar_init(bar_never, 1);
         tc::mbar_init(bar_a2, 2);   // two issuing threads commit to each
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         *abort_flag = 0;
         for (int w = 0; w < 8; ++w) {   // arm phase 0 of the receive barriers
             tc::mbar_arrive_expect_tx(bar_ryw + w, XCHG_WARP_BYTES);
-            tc::mbar_arrive_expect_tx(bar_rzw + w, XCHG_WARP_BYTES);
+            if (w < 4) tc::mbar_arrive_expect_tx(bar_rzw + w, XCHG_WARP_BYTES);
         }
         tc::fence_mbar_init();
     }
@@ -286,7 +292,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0, ph_a2 = 0, ph_g2 = 0;
 
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
-    constexpr uint32_t ID32 = tc::instr_desc(2, 128, 32, 0, 0);
     const uint64_t dK = tc::smem_desc(sK, 16, 1024), dQ = tc::smem_desc(sQ, 16, 1024);
     const uint64_t dW2 = tc::smem_desc(sW2G, 16, 1024), dG = tc::smem_desc(sW2G + 8192, 16, 1024);
     const uint64_t dX1 = tc::smem_desc(sX1, 16, 1024), dX2 = tc::smem_desc(sX2, 16, 1024);
@@ -338,19 +343,48 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         return true;
     };
     auto mma_stage = [&](auto issue) -> bool { return mma_stage_with(issue, [] {}); };
-    // Stores of a finished chunk's z (rows y0c .. y0c + bcc - 1), my tokens: reads
-    // only the Z columns of tensor memory; no global loads on this path (the gate
-    // x + tanh(alpha) z runs afterwards as a separate elementwise kernel).
+    // A finished chunk's z for my tokens (rows y0c .. y0c + bcc - 1): my partial
+    // from tensor memory plus the peer's from RZ, stored to global memory; no
+    // global loads on this path (the gate x + tanh(alpha) z runs afterwards as a
+    // separate elementwise kernel).  Called by all threads.
     auto store_z_chunk = [&](int y0c, int bcc) {
         if (q < 2 && my_tokens) {
-            const int j = 32 * q + lane, t0 = 16 * g;
+            const int j = 32 * q + lane, t0 = 16 * g, tl0 = t0 - 32 * (int)r_cta;
             uint32_t r[16];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
             tc::tmem_wait_ld();
-            float* zrow = a.Zscan + (long long)h * a.x_hs + (long long)y0c * a.x_ts + j;
+            if (tc::mbar_wait_cluster(bar_rzw + wx_z, ph_rz)) {
+                if (lane == 0) tc::mbar_arrive_expect_tx(bar_rzw + wx_z, XCHG_WARP_BYTES);   // arm the next phase
+                float v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (t0 + k < bcc) zrow[(long long)(t0 + k) * a.x_ts] = __uint_as_float(r[k]);
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(sm + OFF_RZ + rz_off(j, tl0 + 4 * c4));
+                    v[4 * c4] = __uint_as_float(r[4 * c4]) + v4.x;
+                    v[4 * c4 + 1] = __uint_as_float(r[4 * c4 + 1]) + v4.y;
+                    v[4 * c4 + 2] = __uint_as_float(r[4 * c4 + 2]) + v4.z;
+                    v[4 * c4 + 3] = __uint_as_float(r[4 * c4 + 3]) + v4.w;
+                }
+                float* zrow = a.Zscan + (long long)h * a.x_hs + (long long)y0c * a.x_ts + j;
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    if (t0 + k < bcc) zrow[(long long)(t0 + k) * a.x_ts] = v[k];
+            } else {
+                give_up();
+            }
+        }
+        ph_rz ^= 1;
+    };
+    // My partial z for the peer's tokens -> the peer's RZ (right after the chunk's last MMA).
+    auto send_z_chunk = [&]() {
+        if (q < 2 && !my_tokens) {
+            const int j = 32 * q + lane, t0 = 16 * g, tl0 = t0 - 32 * (int)r_peer;
+            uint32_t r[16];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4)
+                tc::st_async_v4(peer_rz + rz_off(j, tl0 + 4 * c4), r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2],
+                                r[4 * c4 + 3], peer_bar_rz);
         }
     };
     int prev_y0 = 0, prev_bc = 0;   // the chunk whose z is still to be stored (prev_bc == 0: none)
@@ -622,68 +656,35 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             break;
 
         STAMP(10);
-        // ---- K: exchange token halves of the partials; rows 0-63 -> full Z1^T back to tensor
-        //      memory, rows 64-127 -> Np[t_own][s] = N[s][t] for s not after t
-        {
-            const int t0 = 16 * g;
-            const uint32_t addr = tm + lane_base + TM_ZN + t0;
-            uint32_t r[16];
-            tc::tmem_ld_32x32b_x16(addr, r);
+        // ---- K: Np_r[t][s] = N_r[s][t] for s not after t, from my partial N_r (rows 64-127), all tokens
+        if (q >= 2) {
+            const int t0 = 16 * g, s = i_loc - 64;
+            uint32_t r[16], ph[8];
+            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
+            col_phases(s, ST64, ph);
+            uint8_t* p = sm + OFF_X1 + (t0 >> 3) * 1024;
             tc::tmem_wait_ld();
-            if (!my_tokens) {
-                const int tl0 = t0 - 32 * (int)r_peer;   // the peer's local token index
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4)
-                    tc::st_async_v4(peer_rz + rz_off(i_loc, tl0 + 4 * c4), r[4 * c4], r[4 * c4 + 1], r[4 * c4 + 2],
-                                    r[4 * c4 + 3], peer_bar_rz);
-            } else {
-                const int tl0 = t0 - 32 * (int)r_cta;
-                STAMP(22);
-                if (!tc::mbar_wait_cluster(bar_rzw + wx_z, ph_rz)) give_up();
-                STAMP(23);
-                if (lane == 0) tc::mbar_arrive_expect_tx(bar_rzw + wx_z, XCHG_WARP_BYTES);   // arm the next phase
-                float v[16];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(sm + OFF_RZ + rz_off(i_loc, tl0 + 4 * c4));
-                    v[4 * c4] = __uint_as_float(r[4 * c4]) + v4.x;
-                    v[4 * c4 + 1] = __uint_as_float(r[4 * c4 + 1]) + v4.y;
-                    v[4 * c4 + 2] = __uint_as_float(r[4 * c4 + 2]) + v4.z;
-                    v[4 * c4 + 3] = __uint_as_float(r[4 * c4 + 3]) + v4.w;
-                }
-                if (q < 2) {   // Z1^T rows: the full sums become the accumulator of stage L
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(v[k]);
-                    tc::tmem_st_32x32b_x16(addr, r);
-                    tc::tmem_wait_st();
-                } else {       // N rows
-                    const int s = i_loc - 64;
-                    uint32_t ph[8];
-                    col_phases(s, ST64, ph);
-                    uint8_t* p = sm + OFF_X1 + (tl0 >> 3) * 1024;
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
-                            after(s, t0 + k) ? 0.f : tf32r(v[k]);
-                }
-            }
+            for (int k = 0; k < 16; ++k)
+                *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
+                    after(s, t0 + k) ? 0.f : tf32r(__uint_as_float(r[k]));
         }
-        ph_rz ^= 1;
 
         STAMP(11);
-        // ---- L: Z^T (my tokens) += D2'^T Np^T; meanwhile the shared W2 copy takes the update
+        // ---- L: my partial Z^T (all tokens) += D2'^T Np_r^T (rows 64.. of the A operand are unused and
+        //      land on the consumed N rows); meanwhile the shared W2 copy takes the update
         if (!mma_stage_with(
                 [&] {
                     if (tid == 0) {
                         for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_tf32_ss(tm + TM_ZN + 32 * r_cta, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64),
-                                            ID32, 1);
+                            tc::mma_tf32_ss(tm + TM_ZN, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID64, 1);
                         tc::mma_commit(bar_mma);
                         STAMP(19);
                     }
                 },
                 [&] { refresh_w2(); }))
             break;
+        send_z_chunk();
         prev_y0 = y0;
         prev_bc = bc;
 
