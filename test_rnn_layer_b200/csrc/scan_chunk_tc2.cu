@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
     uint64_t* bar_v = bar_mma + 3;
     uint64_t* bar_ryw = bar_mma + 10;   // [8] a peer warp's part of the Y^T partial has landed in RY
     uint64_t* bar_rzw = bar_mma + 18;   // [4] a peer warp's part of the z partial has landed in RZ
+    uint64_t* bar_l = bar_mma + 26;     // the z correction MMA of the previous chunk
     uint64_t* bar_never = bar_mma + 6;   // fault injection: nothing ever arrives here
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 7);
     uint64_t* bar_a2 = bar_mma + 8;      // the first stage's second group (Aq0, S)
@@ -230,6 +231,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         tc::mbar_init(bar_never, 1);
         tc::mbar_init(bar_a2, 2);   // two issuing threads commit to each
         tc::mbar_init(bar_g2, 2);
+        tc::mbar_init(bar_l, 1);
         *abort_flag = 0;
         for (int w = 0; w < 8; ++w) {   // arm phase 0 of the receive barriers
             tc::mbar_arrive_expect_tx(bar_ryw + w, XCHG_WARP_BYTES);
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         load_tile(&P.mapV, OFF_V, bar_v, y0);
     }
 
-    uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0, ph_a2 = 0, ph_g2 = 0;
+    uint32_t ph_mma = 0, ph_k = 0, ph_q = 0, ph_v = 0, ph_ry = 0, ph_rz = 0, ph_a2 = 0, ph_g2 = 0, ph_l = 0;
 
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
     const uint64_t dK = tc::smem_desc(sK, 16, 1024), dQ = tc::smem_desc(sQ, 16, 1024);
@@ -439,7 +441,10 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                     }
                 },
                 [&] {
-                    if (prev_bc) store_z_chunk(prev_y0, prev_bc);
+                    if (prev_bc) {   // the previous chunk's z correction has run: send the peer its half
+                        wait_mma(bar_l, ph_l);
+                        send_z_chunk();
+                    }
                     {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
                         const int j = tid & 63, tb = tid >> 6;
                         uint32_t ph[8];
@@ -451,6 +456,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                         st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
                         st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
                     }
+                    refresh_w2();   // the previous chunk's W2 update (landed, see J) into the copy stage C reads
+                    if (prev_bc) store_z_chunk(prev_y0, prev_bc);   // + the peer's half, for my tokens
                 }))
             break;
         prev_bc = 0;
@@ -656,42 +663,44 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
             break;
 
         STAMP(10);
-        // ---- K: Np_r[t][s] = N_r[s][t] for s not after t, from my partial N_r (rows 64-127), all tokens
+        // ---- K: Np_r[t][s] = N_r[s][t] for s not after t, from my partial N_r (rows 64-127), all
+        //      tokens, into X2 (M is consumed).  Then the z correction, my partial Z^T += D2'^T Np_r^T
+        //      (rows 64.. of the A operand are unused and land on the consumed N rows), is issued by
+        //      one of these warps after a barrier of the eight alone: no later stage of the chain
+        //      needs z, so the block moves on to the next chunk while it runs (bar_l).
         if (q >= 2) {
             const int t0 = 16 * g, s = i_loc - 64;
             uint32_t r[16], ph[8];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
             col_phases(s, ST64, ph);
-            uint8_t* p = sm + OFF_X1 + (t0 >> 3) * 1024;
+            uint8_t* p = sm + OFF_X2 + (t0 >> 3) * 1024;
             tc::tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 16; ++k)
                 *reinterpret_cast<float*>(p + ph[k & 7] + (k >> 3) * 1024) =
                     after(s, t0 + k) ? 0.f : tf32r(__uint_as_float(r[k]));
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            asm volatile("bar.sync 1, 256;" ::: "memory");   // the eight q >= 2 warps
+            if (tid == 64) {
+                tc::tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ss(tm + TM_ZN, kstep(dX3, kk, ST64), kstep(dX2, kk, ST64), ID64, 1);
+                tc::mma_commit(bar_l);
+            }
         }
-
         STAMP(11);
-        // ---- L: my partial Z^T (all tokens) += D2'^T Np_r^T (rows 64.. of the A operand are unused and
-        //      land on the consumed N rows); meanwhile the shared W2 copy takes the update
-        if (!mma_stage_with(
-                [&] {
-                    if (tid == 0) {
-                        for (int kk = 0; kk < 8; ++kk)
-                            tc::mma_tf32_ss(tm + TM_ZN, kstep(dX3, kk, ST64), kstep(dX1, kk, ST64), ID64, 1);
-                        tc::mma_commit(bar_mma);
-                        STAMP(19);
-                    }
-                },
-                [&] { refresh_w2(); }))
-            break;
-        send_z_chunk();
         prev_y0 = y0;
         prev_bc = bc;
 
         STAMP(12);
     }
 
-    if (prev_bc && !*abort_flag) store_z_chunk(prev_y0, prev_bc);   // the last chunk's z
+    if (prev_bc && !*abort_flag) {   // the last chunk's z
+        wait_mma(bar_l, ph_l);
+        send_z_chunk();
+        store_z_chunk(prev_y0, prev_bc);
+    }
 
 #ifdef TTT_DEBUG_STAGES
     if (tid == 0 && blockIdx.x == TTT_STAMP_CTA && g_dbg2) {
