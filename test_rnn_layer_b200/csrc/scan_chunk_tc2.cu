@@ -128,10 +128,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // erf-GELU (and GELU') with erf from Abramowitz & Stegun, Handbook of
 // Mathematical Functions, formula 7.1.26: |error| <= 1.5e-7, far below the
 // tf32 rounding the results get; GELU and GELU' share one exponential.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 __device__ __forceinline__ void gelu_as(float a, float& g, float& gp, bool want_prime) {
-    const float x = fabsf(a) * 0.70710678118654752f;
-    const float u = rcp_approx(fmaf(0.3275911f, x, 1.0f));   // argument >= 1
-    const float e = __expf(-0.5f * a * a);
+    // u = 1 / (1 + p |a| / sqrt 2), the two constants folded into one
+    const float u = rcp_approx(fmaf(0.3275911f * 0.70710678118654752f, fabsf(a), 1.0f));   // argument >= 1
+    const float e = ex2_approx(a * (a * -0.72134752044448170f));   // exp(-a^2 / 2) = 2^(-a^2 log2(e) / 2)
     float poly = fmaf(1.061405429f, u, -1.453152027f);
     poly = fmaf(poly, u, 1.421413741f);
     poly = fmaf(poly, u, -0.284496736f);
@@ -456,7 +462,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
                         st4(sm + OFF_X1 + row4_off(j, 8 * tb, ST64), v[0], v[1], v[2], v[3]);
                         st4(sm + OFF_X1 + row4_off(j, 8 * tb + 4, ST64), v[4], v[5], v[6], v[7]);
                     }
-                    refresh_w2();   // the previous chunk's W2 update (landed, see J) into the copy stage C reads
+                    if (q >= 2) refresh_w2();   // the other half of the W2 copy (lanes 0-63 refreshed in K)
                     if (prev_bc) store_z_chunk(prev_y0, prev_bc);   // + the peer's half, for my tokens
                 }))
             break;
@@ -668,7 +674,9 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc2_kernel(const __grid_const
         //      (rows 64.. of the A operand are unused and land on the consumed N rows), is issued by
         //      one of these warps after a barrier of the eight alone: no later stage of the chain
         //      needs z, so the block moves on to the next chunk while it runs (bar_l).
-        if (q >= 2) {
+        if (q < 2) {
+            refresh_w2();   // my lanes' part of the W2 update (landed, see J) into the copy stage C reads
+        } else {
             const int t0 = 16 * g, s = i_loc - 64;
             uint32_t r[16], ph[8];
             tc::tmem_ld_32x32b_x16(tm + lane_base + TM_ZN + t0, r);
