@@ -338,98 +338,104 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
     CUDA_TRY(cudaStreamWaitEvent(P.side, fork, 0));
     CUDA_TRY(cudaStreamWaitEvent(P.copy, fork, 0));
 
-    const size_t n = (size_t)q.T * q.D;
-    const size_t nW = (size_t)q.H * q.m * q.d;
-    const int D = q.D;
-    float* xp = reinterpret_cast<float*>(ws + L.xp);
-    __nv_bfloat16* delta = reinterpret_cast<__nv_bfloat16*>(ws + L.delta);
-    float* st1 = reinterpret_cast<float*>(ws + L.state);
-    float* st2 = st1 + nW;
-    int* status = reinterpret_cast<int*>(ws + L.status);
+    auto enqueue = [&]() -> ttt_status {
+        const size_t n = (size_t)q.T * q.D;
+        const size_t nW = (size_t)q.H * q.m * q.d;
+        const int D = q.D;
+        float* xp = reinterpret_cast<float*>(ws + L.xp);
+        __nv_bfloat16* delta = reinterpret_cast<__nv_bfloat16*>(ws + L.delta);
+        float* st1 = reinterpret_cast<float*>(ws + L.state);
+        float* st2 = st1 + nW;
+        int* status = reinterpret_cast<int*>(ws + L.status);
 
-    for (int di = 0; di < ndir; ++di) {
-        Dir dd{};
-        dd.reverse = (dir == TTT_REV || di == 1) ? 1 : 0;
-        const bool second = di == 1;
-        dd.xin = second ? static_cast<const void*>(xp) : X;
-        dd.xin_bf16 = second ? 0 : 1;
-        dd.alpha = dd.reverse ? alpha_r : alpha_f;
-        if (dir == TTT_BIDIR && !second) { dd.out = xp; dd.out_bf16 = 0; dd.delta = delta; }
-        else { dd.out = Y; dd.out_bf16 = 1; dd.delta = nullptr; }
-        dd.zdbg = Z_out ? Z_out + di * n : nullptr;
-        const void* psrc = second ? static_cast<const void*>(delta) : X;   // both bf16
-        const int pacc = second ? 1 : 0;
-        float* zscan = Z_out ? Z_out + di * n : reinterpret_cast<float*>(ws + L.zbuf);
+        for (int di = 0; di < ndir; ++di) {
+            Dir dd{};
+            dd.reverse = (dir == TTT_REV || di == 1) ? 1 : 0;
+            const bool second = di == 1;
+            dd.xin = second ? static_cast<const void*>(xp) : X;
+            dd.xin_bf16 = second ? 0 : 1;
+            dd.alpha = dd.reverse ? alpha_r : alpha_f;
+            if (dir == TTT_BIDIR && !second) { dd.out = xp; dd.out_bf16 = 0; dd.delta = delta; }
+            else { dd.out = Y; dd.out_bf16 = 1; dd.delta = nullptr; }
+            dd.zdbg = Z_out ? Z_out + di * n : nullptr;
+            const void* psrc = second ? static_cast<const void*>(delta) : X;   // both bf16
+            const int pacc = second ? 1 : 0;
+            float* zscan = Z_out ? Z_out + di * n : reinterpret_cast<float*>(ws + L.zbuf);
 
-        std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns), ev_h2d(ns), ev_gate(ns);
-        for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); ev_h2d[k] = new_ev(); ev_gate[k] = new_ev(); }
-        const bool copy_in = X_host && di == 0;           // X arrives segment by segment
-        const bool copy_out = Y_host && di == ndir - 1;   // Y leaves segment by segment
-        auto rows = [&](int k, int& r0, int& r1) {
-            const int lo = seg[k].first * b, hi = std::min(seg[k].second * b, q.T);
-            if (dd.reverse) { r0 = q.T - hi; r1 = q.T - lo; }
-            else { r0 = lo; r1 = hi; }
-        };
-        if (copy_in) {
+            std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns), ev_h2d(ns), ev_gate(ns);
+            for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); ev_h2d[k] = new_ev(); ev_gate[k] = new_ev(); }
+            const bool copy_in = X_host && di == 0;           // X arrives segment by segment
+            const bool copy_out = Y_host && di == ndir - 1;   // Y leaves segment by segment
+            auto rows = [&](int k, int& r0, int& r1) {
+                const int lo = seg[k].first * b, hi = std::min(seg[k].second * b, q.T);
+                if (dd.reverse) { r0 = q.T - hi; r1 = q.T - lo; }
+                else { r0 = lo; r1 = hi; }
+            };
+            if (copy_in) {
+                for (int k = 0; k < ns; ++k) {
+                    int r0, r1;
+                    rows(k, r0, r1);
+                    const size_t o = (size_t)r0 * D * 2, nb = (size_t)(r1 - r0) * D * 2;
+                    CUDA_TRY(cudaMemcpyAsync(const_cast<char*>(static_cast<const char*>(X)) + o,
+                                             static_cast<const char*>(X_host) + o, nb, cudaMemcpyHostToDevice, P.copy));
+                    CUDA_TRY(cudaEventRecord(ev_h2d[k], P.copy));
+                }
+            }
+            // projections (the first runs alone on the whole GPU)
             for (int k = 0; k < ns; ++k) {
                 int r0, r1;
                 rows(k, r0, r1);
-                const size_t o = (size_t)r0 * D * 2, nb = (size_t)(r1 - r0) * D * 2;
-                CUDA_TRY(cudaMemcpyAsync(const_cast<char*>(static_cast<const char*>(X)) + o,
-                                         static_cast<const char*>(X_host) + o, nb, cudaMemcpyHostToDevice, P.copy));
-                CUDA_TRY(cudaEventRecord(ev_h2d[k], P.copy));
+                if (copy_in) CUDA_TRY(cudaStreamWaitEvent(P.side, ev_h2d[k], 0));
+                const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
+                float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
+                CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
+                CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
+            }
+            // scan segments, state carried in the workspace
+            for (int k = 0; k < ns; ++k) {
+                CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k], 0));
+                ScanArgs a = scan_args(q, L, ws, k == 0 ? W1_0 : st1, k == 0 ? W2_0 : st2, eta, b, dd);
+                a.Zscan = zscan;
+                a.c_begin = seg[k].first;
+                a.c_end = seg[k].second;
+                const bool last = k == ns - 1;
+                a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
+                a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
+                CUDA_TRY(launch_scan_chunk_tc2(a, P.scan));
+                CUDA_TRY(cudaEventRecord(ev_scan[k], P.scan));
+            }
+            // gates, each after its segment's scan
+            for (int k = 0; k < ns; ++k) {
+                int r0, r1;
+                rows(k, r0, r1);
+                CUDA_TRY(cudaStreamWaitEvent(P.side, ev_scan[k], 0));
+                const size_t o = (size_t)r0 * D;
+                const void* xin = static_cast<const char*>(dd.xin) + o * (dd.xin_bf16 ? 2 : 4);
+                void* out = static_cast<char*>(dd.out) + o * (dd.out_bf16 ? 2 : 4);
+                const bool last = k == ns - 1;
+                CUDA_TRY(launch_gate(xin, dd.xin_bf16, zscan + o, dd.alpha, out, dd.out_bf16,
+                                     dd.delta ? dd.delta + o : nullptr, status, r1 - r0, q.H, q.d, 0,
+                                     last ? 0 : side_sms * 4, P.side));
+                if (copy_out) {
+                    CUDA_TRY(cudaEventRecord(ev_gate[k], P.side));
+                    CUDA_TRY(cudaStreamWaitEvent(P.copy, ev_gate[k], 0));
+                    CUDA_TRY(cudaMemcpyAsync(static_cast<char*>(Y_host) + o * 2, static_cast<const char*>(Y) + o * 2,
+                                             (size_t)(r1 - r0) * D * 2, cudaMemcpyDeviceToHost, P.copy));
+                }
             }
         }
-        // projections (the first runs alone on the whole GPU)
-        for (int k = 0; k < ns; ++k) {
-            int r0, r1;
-            rows(k, r0, r1);
-            if (copy_in) CUDA_TRY(cudaStreamWaitEvent(P.side, ev_h2d[k], 0));
-            const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
-            float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
-            CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
-            CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
-        }
-        // scan segments, state carried in the workspace
-        for (int k = 0; k < ns; ++k) {
-            CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k], 0));
-            ScanArgs a = scan_args(q, L, ws, k == 0 ? W1_0 : st1, k == 0 ? W2_0 : st2, eta, b, dd);
-            a.Zscan = zscan;
-            a.c_begin = seg[k].first;
-            a.c_end = seg[k].second;
-            const bool last = k == ns - 1;
-            a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
-            a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
-            CUDA_TRY(launch_scan_chunk_tc2(a, P.scan));
-            CUDA_TRY(cudaEventRecord(ev_scan[k], P.scan));
-        }
-        // gates, each after its segment's scan
-        for (int k = 0; k < ns; ++k) {
-            int r0, r1;
-            rows(k, r0, r1);
-            CUDA_TRY(cudaStreamWaitEvent(P.side, ev_scan[k], 0));
-            const size_t o = (size_t)r0 * D;
-            const void* xin = static_cast<const char*>(dd.xin) + o * (dd.xin_bf16 ? 2 : 4);
-            void* out = static_cast<char*>(dd.out) + o * (dd.out_bf16 ? 2 : 4);
-            const bool last = k == ns - 1;
-            CUDA_TRY(launch_gate(xin, dd.xin_bf16, zscan + o, dd.alpha, out, dd.out_bf16,
-                                 dd.delta ? dd.delta + o : nullptr, status, r1 - r0, q.H, q.d, 0,
-                                 last ? 0 : side_sms * 4, P.side));
-            if (copy_out) {
-                CUDA_TRY(cudaEventRecord(ev_gate[k], P.side));
-                CUDA_TRY(cudaStreamWaitEvent(P.copy, ev_gate[k], 0));
-                CUDA_TRY(cudaMemcpyAsync(static_cast<char*>(Y_host) + o * 2, static_cast<const char*>(Y) + o * 2,
-                                         (size_t)(r1 - r0) * D * 2, cudaMemcpyDeviceToHost, P.copy));
-            }
-        }
-    }
+        return TTT_OK;
+    };
+    const ttt_status st = enqueue();
+    // Join the library's streams back into the caller's stream, after a failed
+    // enqueue too: nothing launched on them may outlive the caller's view of the call.
     cudaEvent_t j1 = new_ev(), j2 = new_ev(), j3 = new_ev();
-    CUDA_TRY(cudaEventRecord(j1, P.scan));
-    CUDA_TRY(cudaEventRecord(j2, P.side));
-    CUDA_TRY(cudaEventRecord(j3, P.copy));
-    CUDA_TRY(cudaStreamWaitEvent(s, j1, 0));
-    CUDA_TRY(cudaStreamWaitEvent(s, j2, 0));
-    CUDA_TRY(cudaStreamWaitEvent(s, j3, 0));
+    const cudaError_t je[6] = {cudaEventRecord(j1, P.scan), cudaEventRecord(j2, P.side), cudaEventRecord(j3, P.copy),
+                               cudaStreamWaitEvent(s, j1, 0), cudaStreamWaitEvent(s, j2, 0),
+                               cudaStreamWaitEvent(s, j3, 0)};
+    if (st != TTT_OK) return st;
+    for (cudaError_t e : je)
+        if (e != cudaSuccess) return fail(TTT_ERR_CUDA, "joining the library's streams: %s", cudaGetErrorString(e));
     return TTT_OK;
 }
 
