@@ -160,9 +160,9 @@ def _algorithmic(w):
         "proj_full_tc": ("tensor_bf16", proj_flops),
         "proj_full_simt": ("alu", proj_flops),
         "proj_per_head": ("hbm", T * D * (2 + 12)),
-        # x (bf16) + z (fp32) read, out (bf16) written; the forward launch also
-        # writes the bf16 increment: 10 B and 8 B per element, 9 on average
-        "gate": ("hbm", T * D * 9),
+        # forward: x bf16 + z fp32 read, X' fp32 + bf16 increment written (12 B);
+        # reverse: X' fp32 + z fp32 read, Y bf16 written (10 B); 11 B on average
+        "gate": ("hbm", T * D * 11),
     }
 
 

@@ -415,7 +415,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
                 const bool last = k == ns - 1;
                 CUDA_TRY(launch_gate(xin, dd.xin_bf16, zscan + o, dd.alpha, out, dd.out_bf16,
                                      dd.delta ? dd.delta + o : nullptr, status, r1 - r0, q.H, q.d, 0,
-                                     last ? 0 : side_sms * 4, P.side));
+                                     last ? 0 : side_sms * 6, P.side));
                 if (copy_out) {
                     CUDA_TRY(cudaEventRecord(ev_gate[k], P.side));
                     CUDA_TRY(cudaStreamWaitEvent(P.copy, ev_gate[k], 0));

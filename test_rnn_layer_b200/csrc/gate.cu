@@ -1,8 +1,10 @@
 // The gate out = x + tanh(alpha) * z over a whole direction's outputs
 // (paper notes page, "关键设计 / 门控 + 双向机制"), with the optional bf16
 // increment tanh(alpha) * z that the full layer's reverse projection uses, and
-// the non-finite check of x and z.  Bandwidth-bound: four elements per thread and
-// iteration, grid-stride over the flat arrays (all in X's layout).
+// the non-finite check of x and z.  Bandwidth-bound: four elements per thread,
+// two grid-stride steps per iteration with all their loads issued before any
+// store (bytes in flight are what limit a launch capped to a few SMs), over the
+// flat arrays (all in X's layout).
 #include "common.cuh"
 #include "internal.h"
 
@@ -48,19 +50,34 @@ __device__ __forceinline__ void store4(void* p, long long i, int bf16, float4 v)
 }
 
 __global__ void __launch_bounds__(256) gate_kernel(GateArgs g) {
+    constexpr int U = 2;
     int nonfinite = 0;
     const long long stride = (long long)gridDim.x * blockDim.x * 4;
-    for (long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < g.n; i += stride) {
-        // channel of element i (4 consecutive elements share the row; d is a multiple of 4)
-        const long long ch = g.per_head ? (i / g.Td) * g.d + (i % g.d) : (i % g.D);
-        const float4 x = load4(g.X, i, g.x_bf16);
-        const float4 z = *reinterpret_cast<const float4*>(g.Z + i);
-        const float4 al = *reinterpret_cast<const float4*>(g.alpha + ch);
-        const float4 dz = make_float4(tanhf(al.x) * z.x, tanhf(al.y) * z.y, tanhf(al.z) * z.z, tanhf(al.w) * z.w);
-        store4(g.Out, i, g.out_bf16, make_float4(x.x + dz.x, x.y + dz.y, x.z + dz.z, x.w + dz.w));
-        if (g.Delta) store4(g.Delta, i, 1, dz);
-        nonfinite |= !(isfinite(z.x) && isfinite(z.y) && isfinite(z.z) && isfinite(z.w) && isfinite(x.x) &&
-                       isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+    for (long long i0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) * 4; i0 < g.n; i0 += U * stride) {
+        float4 x[U], z[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = i0 + u * stride;
+            if (i < g.n) {
+                x[u] = load4(g.X, i, g.x_bf16);
+                z[u] = *reinterpret_cast<const float4*>(g.Z + i);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long i = i0 + u * stride;
+            if (i >= g.n) break;
+            // channel of element i (4 consecutive elements share the row; d is a multiple of 4)
+            const long long ch = g.per_head ? (i / g.Td) * g.d + (i % g.d) : (i % g.D);
+            const float4 al = *reinterpret_cast<const float4*>(g.alpha + ch);
+            const float4 zz = z[u], xx = x[u];
+            const float4 dz =
+                make_float4(tanhf(al.x) * zz.x, tanhf(al.y) * zz.y, tanhf(al.z) * zz.z, tanhf(al.w) * zz.w);
+            store4(g.Out, i, g.out_bf16, make_float4(xx.x + dz.x, xx.y + dz.y, xx.z + dz.z, xx.w + dz.w));
+            if (g.Delta) store4(g.Delta, i, 1, dz);
+            nonfinite |= !(isfinite(zz.x) && isfinite(zz.y) && isfinite(zz.z) && isfinite(zz.w) && isfinite(xx.x) &&
+                           isfinite(xx.y) && isfinite(xx.z) && isfinite(xx.w));
+        }
     }
     if (__syncthreads_or(nonfinite) && threadIdx.x == 0) atomicOr(g.status, kStatusNonFinite);
 }
