@@ -203,3 +203,81 @@ int ttt_ref_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ---------------------------------------------------------------- TTT-Linear
+ * The linear variant of the layer (paper notes page, "实验关键数据 / 消融实验":
+ * TTT-Linear, the same layer with a linear hidden state):
+ *     f(u; W) = W u,  W: [d x d],
+ * with the loss, the gradient step, the prefix reading inside a chunk, the
+ * gate and the two directions exactly as for the MLP state above.  For the
+ * loss l(W) = || W k - v ||^2 the gradient is grad_W = 2 (W k - v) k^T.
+ */
+
+/* l(W; k, v) and its gradient G [d x d] (row-major). */
+double ttt_ref_linear_grad(int d, const double* W, const double* k, const double* v, double* G) {
+    double loss = 0.0;
+    for (int i = 0; i < d; ++i) {
+        double e = -v[i];
+        for (int j = 0; j < d; ++j) e += W[(size_t)i * d + j] * k[j];
+        loss += e * e;
+        for (int j = 0; j < d; ++j) G[(size_t)i * d + j] = 2.0 * e * k[j];
+    }
+    return loss;
+}
+
+/* z = W u. */
+void ttt_ref_linear_apply(int d, const double* W, const double* u, double* z) {
+    for (int i = 0; i < d; ++i) {
+        double s = 0.0;
+        for (int j = 0; j < d; ++j) s += W[(size_t)i * d + j] * u[j];
+        z[i] = s;
+    }
+}
+
+/* The per-token rule: W_t = W_{t-1} - eta grad l(W_{t-1}; x_t), z_t = W_t q_t. */
+void ttt_ref_linear_scan_per_token(int T, int d, int reverse, double eta, const double* Q, const double* K,
+                                   const double* V, double* W, double* Z) {
+    const size_t n = (size_t)d * d;
+    double* G = (double*)malloc(sizeof(double) * n);
+    for (int s = 0; s < T; ++s) {
+        const int t = reverse ? (T - 1 - s) : s;
+        ttt_ref_linear_grad(d, W, K + (size_t)t * d, V + (size_t)t * d, G);
+        for (size_t p = 0; p < n; ++p) W[p] -= eta * G[p];
+        ttt_ref_linear_apply(d, W, Q + (size_t)t * d, Z + (size_t)t * d);
+    }
+    free(G);
+}
+
+/* Mini-batch form: gradients at the chunk-start state, prefix reading. */
+void ttt_ref_linear_scan_chunked(int T, int d, int b, int reverse, double eta, const double* Q, const double* K,
+                                 const double* V, double* W, double* Z) {
+    const size_t n = (size_t)d * d;
+    double* Wc = (double*)malloc(sizeof(double) * n);
+    double* G = (double*)malloc(sizeof(double) * n);
+    for (int s0 = 0; s0 < T; s0 += b) {
+        const int s1 = (s0 + b < T) ? (s0 + b) : T;
+        memcpy(Wc, W, sizeof(double) * n);
+        for (int s = s0; s < s1; ++s) {
+            const int t = reverse ? (T - 1 - s) : s;
+            ttt_ref_linear_grad(d, Wc, K + (size_t)t * d, V + (size_t)t * d, G);
+            for (size_t p = 0; p < n; ++p) W[p] -= eta * G[p];
+            ttt_ref_linear_apply(d, W, Q + (size_t)t * d, Z + (size_t)t * d);
+        }
+    }
+    free(Wc); free(G);
+}
+
+/* H independent heads ([H x T x d] streams, W [H x d x d]), one OpenMP task each. */
+void ttt_ref_linear_scan_heads(int H, int T, int d, int b, int reverse, double eta, const double* Q,
+                               const double* K, const double* V, double* W, double* Z) {
+    const size_t sT = (size_t)T * d, sW = (size_t)d * d;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < H; ++h) {
+        if (b == 1)
+            ttt_ref_linear_scan_per_token(T, d, reverse, eta, Q + h * sT, K + h * sT, V + h * sT, W + h * sW,
+                                          Z + h * sT);
+        else
+            ttt_ref_linear_scan_chunked(T, d, b, reverse, eta, Q + h * sT, K + h * sT, V + h * sT, W + h * sW,
+                                        Z + h * sT);
+    }
+}

@@ -70,6 +70,16 @@ def _load():
         lib.ttt_ref_scan_heads.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 6
         lib.ttt_ref_num_threads.restype = ctypes.c_int
         lib.ttt_ref_num_threads.argtypes = []
+        lib.ttt_ref_linear_grad.restype = ctypes.c_double
+        lib.ttt_ref_linear_grad.argtypes = [ctypes.c_int, _dp, _dp, _dp, _dp]
+        lib.ttt_ref_linear_apply.restype = None
+        lib.ttt_ref_linear_apply.argtypes = [ctypes.c_int, _dp, _dp, _dp]
+        lib.ttt_ref_linear_scan_per_token.restype = None
+        lib.ttt_ref_linear_scan_per_token.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double] + [_dp] * 5
+        lib.ttt_ref_linear_scan_chunked.restype = None
+        lib.ttt_ref_linear_scan_chunked.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [_dp] * 5
+        lib.ttt_ref_linear_scan_heads.restype = None
+        lib.ttt_ref_linear_scan_heads.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_dp] * 5
         _lib = lib
     return _lib
 
@@ -255,3 +265,84 @@ def full_mode_heads(X, theta_q, theta_k, theta_v, W1_0, W2_0, eta: float, b: int
     W1 = _f64(W1_0)[list(heads)]; W2 = _f64(W2_0)[list(heads)]
     Zh, W1T, W2T = scan_heads(Q, K, V, W1, W2, eta, b, reverse)
     return _full_from_heads(Zh), W1T, W2T
+
+
+# ---------------------------------------------------------------- TTT-Linear
+# The linear variant (paper notes page, "实验关键数据 / 消融实验": TTT-Linear):
+# f(u; W) = W u with W [d, d]; loss, update rule, prefix reading, gate and
+# directions as for the MLP state.
+def linear_grad(W, k, v):
+    """Loss ||W k - v||^2 and its gradient 2 (W k - v) k^T."""
+    W, k, v = _f64(W), _f64(k), _f64(v)
+    d = W.shape[0]
+    G = np.empty((d, d))
+    loss = _load().ttt_ref_linear_grad(d, _ptr(W), _ptr(k), _ptr(v), _ptr(G))
+    return float(loss), G
+
+
+def linear_apply(W, u) -> np.ndarray:
+    """f(u; W) = W u."""
+    W, u = _f64(W), _f64(u)
+    z = np.empty(W.shape[0])
+    _load().ttt_ref_linear_apply(W.shape[0], _ptr(W), _ptr(u), _ptr(z))
+    return z
+
+
+def linear_scan(Q, K, V, W_0, eta: float, b: int, reverse: bool = False, per_token: bool = False):
+    """One head, one direction.  Q, K, V: [T, d].  Returns (Z [T, d], W_T)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    W = _f64(W_0).copy()
+    T, d = Q.shape
+    Z = np.zeros((T, d))
+    lib = _load()
+    if per_token:
+        lib.ttt_ref_linear_scan_per_token(T, d, int(reverse), float(eta), _ptr(Q), _ptr(K), _ptr(V), _ptr(W),
+                                          _ptr(Z))
+    else:
+        lib.ttt_ref_linear_scan_chunked(T, d, int(b), int(reverse), float(eta), _ptr(Q), _ptr(K), _ptr(V),
+                                        _ptr(W), _ptr(Z))
+    return Z, W
+
+
+def linear_scan_heads(Q, K, V, W_0, eta: float, b: int, reverse: bool = False):
+    """H heads (OpenMP).  Q, K, V: [H, T, d]; W_0 [H, d, d]."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    W = _f64(W_0).copy()
+    H, T, d = Q.shape
+    Z = np.zeros((H, T, d))
+    _load().ttt_ref_linear_scan_heads(H, T, d, int(b), int(reverse), float(eta), _ptr(Q), _ptr(K), _ptr(V),
+                                      _ptr(W), _ptr(Z))
+    return Z, W
+
+
+def linear_direction(X, theta_q, theta_k, theta_v, W_0, eta: float, b: int, reverse: bool, per_head: bool):
+    """One TTT-Linear direction on input X; returns (Z in X's layout, W_T)."""
+    if per_head:
+        Q = project_per_head(X, theta_q); K = project_per_head(X, theta_k); V = project_per_head(X, theta_v)
+        return linear_scan_heads(Q, K, V, W_0, eta, b, reverse)
+    H, d = W_0.shape[0], W_0.shape[2]
+    Q = _heads_from_full(project_full(X, theta_q), H, d)
+    K = _heads_from_full(project_full(X, theta_k), H, d)
+    V = _heads_from_full(project_full(X, theta_v), H, d)
+    Zh, W = linear_scan_heads(Q, K, V, W_0, eta, b, reverse)
+    return _full_from_heads(Zh), W
+
+
+def linear_layer_forward(X, theta_q, theta_k, theta_v, W_0, eta: float, b: int, dirs: str, alpha_f=None,
+                         alpha_r=None, per_head: bool = True) -> dict:
+    """The gated TTT-Linear layer, composed as layer_forward composes the MLP one."""
+    out = {}
+    if dirs in ("fwd", "bidir"):
+        Zf, Wf = linear_direction(X, theta_q, theta_k, theta_v, W_0, eta, b, False, per_head)
+        Xp = gate(X, Zf, _alpha_layout(alpha_f, X, per_head))
+        out.update(Z_f=Zf, W_f=Wf)
+        if dirs == "fwd":
+            out["Y"] = Xp
+            return out
+        out["Xp"] = Xp
+        src = Xp
+    else:
+        src = _f64(X)
+    Zr, Wr = linear_direction(src, theta_q, theta_k, theta_v, W_0, eta, b, True, per_head)
+    out.update(Z_r=Zr, W_r=Wr, Y=gate(src, Zr, _alpha_layout(alpha_r, X, per_head)))
+    return out
