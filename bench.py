@@ -7,9 +7,10 @@ sequence of width 3072 (48 heads, d = 64, hidden 256, b = 64), inputs already
 resident in HBM.  Multi-GPU (torchrun): each rank runs its own sequence
 (independent replicas, weak scaling, no collective on the data path).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--model mlp|linear]
 
-Prints one JSON line on rank 0.
+Prints one JSON line on rank 0.  --model linear measures the TTT-Linear layer
+(f(u; W) = W u) on the same sequence instead.
 """
 from __future__ import annotations
 
@@ -28,6 +29,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "TTT-MLP tokens/s (48 heads, bidirectional) at T≈313k; % of roofline"
+METRIC_LINEAR = "TTT-Linear tokens/s (48 heads, bidirectional) at T≈313k; % of roofline"
 UNIT = "tokens/s"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "traffic.json")
@@ -67,6 +69,7 @@ KERNEL_SRC = {
     "proj_full_tc": ("proj_tc.cu",),
     "proj_per_head": ("proj_simt.cu",),
     "gate": ("gate.cu",),
+    "scan_linear": ("scan_linear.cu",),
 }
 
 
@@ -163,6 +166,8 @@ def _algorithmic(w):
         # forward: x bf16 + z fp32 read, X' fp32 + bf16 increment written (12 B);
         # reverse: X' fp32 + z fp32 read, Y bf16 written (10 B); 11 B on average
         "gate": ("hbm", T * D * 11),
+        # TTT-Linear per head-token: e = W_c k (2 d^2), update (2 d^2), z = W q (2 d^2)
+        "scan_linear": ("alu", H * T * 6 * d * d),
     }
 
 
@@ -248,19 +253,47 @@ def _cpu_sample(w, tokens: int, seed: int = 0):
     return run, scale, threads, sample
 
 
+def _cpu_sample_linear(w, tokens: int, seed: int = 0):
+    """As _cpu_sample, for the TTT-Linear layer."""
+    import numpy as np
+
+    from oracle import ttt_oracle as O
+    from test_rnn_layer_b200 import synth as S
+
+    threads = O.num_threads()
+    heads = list(range(min(w.H, threads)))
+    inp = S.make_linear_inputs(w.with_T(tokens), seed=seed, device="cpu")
+    X = inp["X"].float().numpy()
+    rows = np.concatenate([np.arange(h * w.d, (h + 1) * w.d) for h in heads])
+    th = [inp[k].float().numpy()[rows] for k in ("theta_q", "theta_k", "theta_v")]
+    W0 = inp["W_0"].double().numpy()[heads]
+
+    def run():
+        t0 = time.perf_counter()
+        Q, K, V = [O.project_full(X, t).reshape(tokens, len(heads), w.d).transpose(1, 0, 2) for t in th]
+        O.linear_scan_heads(Q, K, V, W0, w.eta_eff, w.b)
+        return time.perf_counter() - t0
+
+    scale = len(heads) / (w.H * 2.0)
+    sample = (f"first {tokens} tokens, {len(heads)} of {w.H} heads, forward direction only (fp64 TTT-Linear "
+              f"oracle incl. those heads' Q/K/V projections); tokens/s scaled by {len(heads)}/({w.H}*2)")
+    return run, scale, threads, sample
+
+
 # ------------------------------------------------------------------ arms
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
     w = _workload(args)
     tokens = args.ref_tokens
-    run, scale, threads, sample = _cpu_sample(w, tokens)
+    run, scale, threads, sample = (_cpu_sample_linear if args.model == "linear" else _cpu_sample)(w, tokens)
     for _ in range(args.warmup):
         run()
     times = [run() for _ in range(args.steps)]
     step_s = sum(times) / len(times)
     value = tokens * scale / step_s
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": METRIC_LINEAR if args.model == "linear" else METRIC, "value": value,
+            "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config(w, {"sample": sample}),
@@ -389,12 +422,116 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_ours_linear(args, rank, world, local_rank):
+    """The TTT-Linear layer on the same sequence (fp32 scan), same JSON line."""
+    import torch
+
+    from test_rnn_layer_b200 import synth as S
+    from test_rnn_layer_b200 import tttmlp as L
+
+    L.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = _workload(args)
+    inp = S.make_linear_inputs(w, seed=rank_seed(rank), device=dev)
+    desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
+    direction = L.DIRS[w.dirs]
+    n_ws = L.ttt_linear_workspace_size(desc, w.b, direction)
+    ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
+    Y = torch.empty_like(inp["X"])
+    stream = torch.cuda.current_stream()
+
+    def step(X=None, Yo=None):
+        st = L.ttt_linear_forward(desc, inp["X"] if X is None else X, inp["theta_q"], inp["theta_k"],
+                                  inp["theta_v"], inp["W_0"], w.eta_eff, w.b, direction, inp["alpha_f"],
+                                  inp["alpha_r"], Y if Yo is None else Yo, None, None, ws, n_ws, stream)
+        L.check(st, "ttt_linear_forward")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    L.check(L.ttt_mlp_status(ws, stream), "warm-up status")
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    n_launch0 = L.ttt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = L.ttt_launch_count() - n_launch0
+    clocks = sampler.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
+    ms_per_step = ms / args.steps
+    value = whole_job_tokens_per_s(world, w.T, ms_per_step)
+
+    L.ttt_kernel_timing(True)
+    kpass = max(1, min(args.steps, 3))
+    for _ in range(kpass):
+        step()
+    torch.cuda.synchronize()
+    ktimes = L.ttt_kernel_times()
+    L.ttt_kernel_timing(False)
+    total = sum(v[0] for v in ktimes.values()) or 1.0
+    peaks = _peaks()
+    roof = _roofline("scan_linear", ktimes["scan_linear"][0] / ktimes["scan_linear"][1],
+                     ktimes["scan_linear"][1] / kpass, w, peaks, clocks)
+    roof["share"] = round(ktimes["scan_linear"][0] / total, 4)
+    kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
+                   "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
+
+    e2e = None
+    if not args.no_e2e:   # pinned host X in, host Y out, through the device entry point
+        Xh = inp["X"].cpu().pin_memory()
+        Yh = torch.empty_like(Xh).pin_memory()
+        Xd = torch.empty_like(inp["X"])
+        ns = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            step(Xd, Y)
+            Yh.copy_(Y, non_blocking=True)
+            L.check(L.ttt_mlp_status(ws, stream), "status")
+
+        e2e_step()
+        t0 = time.perf_counter()
+        for _ in range(ns):
+            e2e_step()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
+        nbytes = Xh.numel() * Xh.element_size()
+        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_s * 1e3,
+               "steps": ns}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        run, scale, threads, sample = _cpu_sample_linear(w, args.cpu_tokens)
+        t = run()
+        cpu = {"value": args.cpu_tokens * scale / t, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": sample, "seconds": round(t, 2)}
+    if rank == 0:
+        line = {"metric": METRIC_LINEAR, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16-in/fp32-scan", "data": "synthetic",
+                "config": _config(w, {"model": "ttt-linear", "state": "W [64 x 64] fp32 per head"}),
+                "gpu_launches": launches, "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e,
+                "cpu_baseline": cpu, "impl": "ours"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--model", choices=["mlp", "linear"], default="mlp")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length (quick checks only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -419,6 +556,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.model == "linear":
+            return run_ours_linear(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

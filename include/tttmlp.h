@@ -201,6 +201,28 @@ TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void*
 TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);
 
 /*
+ * TTT-Linear: the same gated layer with a linear hidden state f(u; W) = W u,
+ * W [d x d] per head (paper notes page, "实验关键数据 / 消融实验").  For each
+ * token W_t = W_{t-1} - eta * 2 (W k - v) k^T and z_t = W_t q; the mini-batch
+ * form (gradients at the chunk-start state, prefix reading), the gate and the
+ * directions are those of ttt_mlp_forward.  desc as for ttt_mlp_forward
+ * (desc->m is not used by this layer and is not checked).
+ *
+ *   W_0   [H, d, d] fp32 initial state (both directions).
+ *   W_T   optional (may be NULL) fp32 [n_dir, H, d, d]: the state after each
+ *         direction's last token.
+ *   Every other argument, the status (ttt_mlp_status) and the errors as in
+ *   ttt_mlp_forward; workspace of ttt_linear_workspace_size bytes.  The scan
+ *   runs in fp32 (one CTA per 16 rows of a head's state).
+ */
+TTT_API size_t ttt_linear_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
+TTT_API ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q,
+                              const void* theta_k, const void* theta_v, const float* W_0, float eta, int b,
+                              ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y,
+                              float* Z_out, float* W_T, void* workspace, size_t workspace_bytes,
+                              ttt_stream_t stream);
+
+/*
  * Fault injection for tests (process-wide).  While enabled, the two-CTA
  * tensor-core scan kernel (the default for bf16 inputs) first waits on an
  * mbarrier that nothing arrives on, with a 1 ms limit; the wait expires, the

@@ -549,6 +549,64 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
 
 }  // namespace
 
+namespace {
+
+// ---------------------------------------------------------------- TTT-Linear
+ttt_status check_desc_linear(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (!desc) return fail(TTT_ERR_INVALID_ARG, "desc is NULL");
+    ttt_mlp_desc q = *desc;
+    q.m = 4 * q.d;   // not used by the linear layer
+    return check_desc(&q, b, dir);
+}
+
+struct LinearLayout {
+    size_t status, qkv[3], xp, delta, zbuf, total;
+    bool split_reverse;
+};
+
+LinearLayout plan_linear(const ttt_mlp_desc& q, ttt_direction dir) {
+    LinearLayout L{};
+    const size_t n = (size_t)q.T * q.D;
+    size_t off = 0;
+    L.status = off; off += kAlign;
+    for (int w = 0; w < 3; ++w) { L.qkv[w] = off; off = align_up(off + n * sizeof(float)); }
+    L.split_reverse = (dir == TTT_BIDIR) && !q.per_head_input && q.x_dtype == TTT_BF16;
+    L.xp = off;
+    if (dir == TTT_BIDIR) off = align_up(off + n * sizeof(float));
+    L.delta = off;
+    if (L.split_reverse) off = align_up(off + n * 2);
+    L.zbuf = off;
+    off = align_up(off + n * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+ttt_status linear_direction(const ttt_mlp_desc& q, const LinearLayout& L, char* ws, const void* xin, int xin_bf16,
+                            const void* src, int src_bf16, int accumulate, const void* const th[3],
+                            const float* W_0, float eta, int b, int reverse, const float* alpha, void* out,
+                            int out_bf16, __nv_bfloat16* delta, float* z_out, float* w_t, cudaStream_t s) {
+    int* status = reinterpret_cast<int*>(ws + L.status);
+    float* qkv[3] = {reinterpret_cast<float*>(ws + L.qkv[0]), reinterpret_cast<float*>(ws + L.qkv[1]),
+                     reinterpret_cast<float*>(ws + L.qkv[2])};
+    ttt_status st = project(q, src, src_bf16, th, qkv, accumulate, status, s);
+    if (st != TTT_OK) return st;
+    LinearScanArgs a{};
+    a.Q = qkv[0]; a.K = qkv[1]; a.V = qkv[2];
+    if (q.per_head_input) { a.qkv_hs = (long long)q.T * q.d; a.qkv_ts = q.d; }
+    else { a.qkv_hs = q.d; a.qkv_ts = q.D; }
+    a.x_hs = a.qkv_hs; a.x_ts = a.qkv_ts;
+    a.Z = z_out ? z_out : reinterpret_cast<float*>(ws + L.zbuf);
+    a.W_0 = W_0; a.W_T = w_t;
+    a.T = q.T; a.H = q.H; a.d = q.d; a.b = b; a.reverse = reverse; a.eta = eta;
+    a.status = status;
+    CUDA_TRY(launch_scan_linear(a, s));
+    CUDA_TRY(launch_gate(xin, xin_bf16, a.Z, alpha, out, out_bf16, delta, status, q.T, q.H, q.d,
+                         q.per_head_input, 0, s));
+    return TTT_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t ttt_mlp_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
@@ -569,6 +627,56 @@ ttt_status ttt_mlp_forward(const ttt_mlp_desc* desc, const void* X, const void* 
                            ttt_stream_t stream_) {
     return forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
                         W2_T, workspace, workspace_bytes, stream_, nullptr, nullptr);
+}
+
+size_t ttt_linear_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc_linear(desc, b, dir) != TTT_OK) return 0;
+    return plan_linear(*desc, dir).total;
+}
+
+ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                              const void* theta_v, const float* W_0, float eta, int b, ttt_direction dir,
+                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, float* W_T,
+                              void* workspace, size_t workspace_bytes, ttt_stream_t stream_) {
+    ttt_status st = check_desc_linear(desc, b, dir);
+    if (st != TTT_OK) return st;
+    const ttt_mlp_desc& q = *desc;
+    if (!scan_linear_supported(q.d)) return fail(TTT_ERR_UNSUPPORTED, "head dim d=%d not supported (16, 32, 64)", q.d);
+    st = check_ptrs(q, X, theta_q, theta_k, theta_v, W_0, W_0, eta, dir, alpha_f, alpha_r);
+    if (st != TTT_OK) return st;
+    if (!Y || !workspace) return fail(TTT_ERR_INVALID_ARG, "Y and workspace must be non-NULL");
+    const void* outs[] = {Y, Z_out, W_T};
+    for (const void* p : outs)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "output pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t xbytes = (size_t)q.T * q.D * elem_size(q.x_dtype);
+    {
+        const char* xs = static_cast<const char*>(X);
+        const char* ys = static_cast<const char*>(Y);
+        if (xs < ys + xbytes && ys < xs + xbytes) return fail(TTT_ERR_INVALID_ARG, "Y must not alias X");
+    }
+    const LinearLayout L = plan_linear(q, dir);
+    if (workspace_bytes < L.total)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, L.total);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    char* ws = static_cast<char*>(workspace);
+    CUDA_TRY(cudaMemsetAsync(ws + L.status, 0, 16, s));
+    const int x_bf16 = q.x_dtype == TTT_BF16;
+    const void* th[3] = {theta_q, theta_k, theta_v};
+    const size_t n = (size_t)q.T * q.D, nW = (size_t)q.H * q.d * q.d;
+    float* xp = reinterpret_cast<float*>(ws + L.xp);
+    __nv_bfloat16* delta = L.split_reverse ? reinterpret_cast<__nv_bfloat16*>(ws + L.delta) : nullptr;
+    if (dir != TTT_BIDIR)
+        return linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, dir == TTT_REV,
+                                dir == TTT_REV ? alpha_r : alpha_f, Y, x_bf16, nullptr, Z_out, W_T, s);
+    st = linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, 0, alpha_f, xp, 0, delta, Z_out, W_T,
+                          s);
+    if (st != TTT_OK) return st;
+    // reverse on X' = X + tanh(alpha_f) z_f; theta X' = theta X + theta bf16(X' - X) where X is bf16 and full width
+    return linear_direction(q, L, ws, xp, 0, L.split_reverse ? static_cast<const void*>(delta) : xp,
+                            L.split_reverse ? 1 : 0, L.split_reverse ? 1 : 0, th, W_0, eta, b, 1, alpha_r, Y,
+                            x_bf16, nullptr, Z_out ? Z_out + n : nullptr, W_T ? W_T + nW : nullptr, s);
 }
 
 ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {

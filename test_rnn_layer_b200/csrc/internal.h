@@ -53,6 +53,24 @@ bool scan_chunk_tc_supported(int d, int b);
 cudaError_t launch_scan_chunk_tc(const ScanArgs& a, cudaStream_t s);    // one CTA per head
 cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s);   // a cluster of two CTAs per head
 
+// TTT-Linear scan (f(u; W) = W u, W [d x d] per head): z of one direction into Z
+// (X's layout); state from W_0 [H, d, d], final state to W_T (optional).
+struct LinearScanArgs {
+    const float* Q;
+    const float* K;
+    const float* V;
+    long long qkv_hs, qkv_ts;
+    float* Z;
+    long long x_hs, x_ts;
+    const float* W_0;
+    float* W_T;
+    int T, H, d, b, reverse;
+    float eta;
+    int* status;
+};
+bool scan_linear_supported(int d);
+cudaError_t launch_scan_linear(const LinearScanArgs& a, cudaStream_t s);
+
 // Per-head projections: U[which][h, t, e] = sum_j theta_which[h][e][j] x[h, t, j].
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
                                  float* const out[3], int T, int H, int d, int* status, cudaStream_t s);

@@ -107,3 +107,15 @@ def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu") 
     alpha_r = torch.full((D,), w.alpha, dtype=torch.float32, device=dev)
     return dict(X=X, theta_q=thetas[0], theta_k=thetas[1], theta_v=thetas[2], W1_0=W1_0, W2_0=W2_0,
                 alpha_f=alpha_f, alpha_r=alpha_r)
+
+
+def make_linear_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu") -> dict:
+    """The inputs of make_inputs plus the TTT-Linear initial state W_0 [H, d, d]
+    ~ N(0, 1/d) (fan-in), drawn afterwards from the same generator sequence."""
+    inp = make_inputs(w, seed, device)
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 1_000_003)
+    inp["W_0"] = torch.randn((w.H, w.d, w.d), generator=g, device=dev, dtype=torch.float32).mul_(
+        math.sqrt(1.0 / w.d))
+    return inp

@@ -24,7 +24,8 @@ DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
-            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_debug_inject_wait_timeout"]
+            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_debug_inject_wait_timeout",
+            "ttt_linear_workspace_size", "ttt_linear_forward"]
 
 
 class TTTError(RuntimeError):
@@ -65,6 +66,10 @@ def lib():
         L.ttt_mlp_forward_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_forward_noalloc.restype = i
         L.ttt_mlp_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp]
+        L.ttt_linear_workspace_size.restype = sz
+        L.ttt_linear_workspace_size.argtypes = [dp, i, i]
+        L.ttt_linear_forward.restype = i
+        L.ttt_linear_forward.argtypes = [dp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_status.restype = i
         L.ttt_mlp_status.argtypes = [vp, vp]
         L.ttt_mlp_select_kernels.restype = i
@@ -166,6 +171,17 @@ def ttt_mlp_forward_noalloc(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta,
                                              _p(alpha_r), _p(Y), _p(Z_out), _p(W1_T), _p(W2_T), _stream(stream)))
 
 
+def ttt_linear_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
+    return int(lib().ttt_linear_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_linear_forward(desc, X, theta_q, theta_k, theta_v, W_0, eta, b, direction, alpha_f, alpha_r, Y, Z_out,
+                       W_T, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_linear_forward(ctypes.byref(desc), _p(X), _p(theta_q), _p(theta_k), _p(theta_v), _p(W_0),
+                                        float(eta), int(b), int(direction), _p(alpha_f), _p(alpha_r), _p(Y),
+                                        _p(Z_out), _p(W_T), _p(workspace), int(workspace_bytes), _stream(stream)))
+
+
 def ttt_mlp_status(workspace, stream=None) -> int:
     return int(lib().ttt_mlp_status(_p(workspace), _stream(stream)))
 
@@ -208,6 +224,38 @@ def layer_forward(X, theta_q, theta_k, theta_v, W1_0, W2_0, eta: float, b: int, 
     out = {"Y": Y, "Z": Z, "W1_T": W1T, "W2_T": W2T, "workspace": ws}
     if check_status:
         st = ttt_mlp_status(ws, stream)
+        out["status"] = st
+        check(st, "ttt_mlp_status")
+    return out
+
+
+def linear_layer_forward(X, theta_q, theta_k, theta_v, W_0, eta: float, b: int, dirs: str, alpha_f=None,
+                         alpha_r=None, per_head: bool = True, want_z: bool = False, want_state: bool = False,
+                         workspace: torch.Tensor | None = None, check_status: bool = True, stream=None) -> dict:
+    """Allocate outputs (torch, on X's device) and call ttt_linear_forward once."""
+    dev = X.device
+    if per_head:
+        H, T, d = X.shape
+    else:
+        T, _ = X.shape
+        H, d = W_0.shape[0], W_0.shape[2]
+    desc = make_desc(T, H, d, per_head, X.dtype == torch.bfloat16)
+    direction = DIRS[dirs]
+    nd = 2 if dirs == "bidir" else 1
+    if workspace is None:
+        n = ttt_linear_workspace_size(desc, b, direction)
+        if n == 0:
+            raise TTTError(TTT_ERR_INVALID_ARG, "workspace size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    Y = torch.empty_like(X)
+    Z = torch.empty((nd,) + tuple(X.shape), dtype=torch.float32, device=dev) if want_z else None
+    WT = torch.empty((nd,) + tuple(W_0.shape), dtype=torch.float32, device=dev) if want_state else None
+    st = ttt_linear_forward(desc, X, theta_q, theta_k, theta_v, W_0, eta, b, direction, alpha_f, alpha_r, Y, Z, WT,
+                            workspace, workspace.numel(), stream)
+    check(st, "ttt_linear_forward")
+    out = {"Y": Y, "Z": Z, "W_T": WT, "workspace": workspace}
+    if check_status:
+        st = ttt_mlp_status(workspace, stream)
         out["status"] = st
         check(st, "ttt_mlp_status")
     return out

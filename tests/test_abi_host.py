@@ -118,3 +118,35 @@ def test_kernel_selector_validation():
 
 def test_status_null_workspace():
     assert L.lib().ttt_mlp_status(None, None) == L.TTT_ERR_INVALID_ARG
+
+
+def test_linear_workspace_sizes_and_desc_checks():
+    d = _desc()
+    d.m = 12345   # not used by the linear layer
+    n1 = L.ttt_linear_workspace_size(d, 16, L.TTT_FWD)
+    nb = L.ttt_linear_workspace_size(d, 16, L.TTT_BIDIR)
+    # Q, K, V and z in fp32 (+ X' for both directions)
+    assert n1 >= 4 * 1024 * 256 * 4 and nb >= n1 + 1024 * 256 * 4 and n1 % 256 == 0
+    assert L.ttt_linear_workspace_size(_desc(d=48), 16, L.TTT_FWD) == 0
+    assert L.ttt_linear_workspace_size(_desc(), 0, L.TTT_FWD) == 0
+
+
+def test_linear_forward_argument_errors_before_any_cuda_call():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses are only used where no GPU exists")
+    d = _desc()
+
+    def fwd(**over):
+        a = dict(X=0x1000, tq=0x2000, tk=0x3000, tv=0x4000, W=0x5000, eta=0.01, b=16, dir=L.TTT_BIDIR,
+                 af=0x7000, ar=0x8000, Y=0x90000000, Z=None, WT=None, ws=0x100000000, wsb=1 << 40)
+        a.update(over)
+        return L.ttt_linear_forward(d, a["X"], a["tq"], a["tk"], a["tv"], a["W"], a["eta"], a["b"], a["dir"],
+                                    a["af"], a["ar"], a["Y"], a["Z"], a["WT"], a["ws"], a["wsb"], 0)
+
+    assert fwd(W=None) == L.TTT_ERR_INVALID_ARG
+    assert fwd(af=None) == L.TTT_ERR_INVALID_ARG and "alpha_f" in L.ttt_last_error()
+    assert fwd(eta=float("inf")) == L.TTT_ERR_INVALID_ARG
+    assert fwd(Y=0x1000) == L.TTT_ERR_INVALID_ARG and "alias" in L.ttt_last_error()
+    assert fwd(wsb=4096) == L.TTT_ERR_INVALID_ARG and "too small" in L.ttt_last_error()
+    assert fwd(WT=0x1008) == L.TTT_ERR_INVALID_ARG and "aligned" in L.ttt_last_error()
