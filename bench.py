@@ -70,6 +70,7 @@ KERNEL_SRC = {
     "proj_per_head": ("proj_simt.cu",),
     "gate": ("gate.cu",),
     "scan_linear": ("scan_linear.cu",),
+    "scan_linear_tc": ("scan_linear_tc.cu",),
 }
 
 
@@ -168,6 +169,9 @@ def _algorithmic(w):
         "gate": ("hbm", T * D * 11),
         # TTT-Linear per head-token: e = W_c k (2 d^2), update (2 d^2), z = W q (2 d^2)
         "scan_linear": ("alu", H * T * 6 * d * d),
+        # chunk form on the tensor cores: W K^T, W Q^T, update (3 x 2 d^2) + Q K^T and the masked
+        # correction (2 x 2 b d over the causal half)
+        "scan_linear_tc": ("tensor_tf32", H * T * (6 * d * d + 2 * b * d)),
     }
 
 
@@ -479,9 +483,9 @@ def run_ours_linear(args, rank, world, local_rank):
     L.ttt_kernel_timing(False)
     total = sum(v[0] for v in ktimes.values()) or 1.0
     peaks = _peaks()
-    roof = _roofline("scan_linear", ktimes["scan_linear"][0] / ktimes["scan_linear"][1],
-                     ktimes["scan_linear"][1] / kpass, w, peaks, clocks)
-    roof["share"] = round(ktimes["scan_linear"][0] / total, 4)
+    scan = "scan_linear_tc" if "scan_linear_tc" in ktimes else "scan_linear"
+    roof = _roofline(scan, ktimes[scan][0] / ktimes[scan][1], ktimes[scan][1] / kpass, w, peaks, clocks)
+    roof["share"] = round(ktimes[scan][0] / total, 4)
     kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
                    "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
 
@@ -517,7 +521,9 @@ def run_ours_linear(args, rank, world, local_rank):
     if rank == 0:
         line = {"metric": METRIC_LINEAR, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16-in/fp32-scan", "data": "synthetic",
+                "vs_baseline": None,
+                "dtype": "bf16-in/tf32-mma/fp32-state" if scan == "scan_linear_tc" else "bf16-in/fp32-scan",
+                "data": "synthetic",
                 "config": _config(w, {"model": "ttt-linear", "state": "W [64 x 64] fp32 per head"}),
                 "gpu_launches": launches, "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e,
                 "cpu_baseline": cpu, "impl": "ours"}

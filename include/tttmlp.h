@@ -213,7 +213,10 @@ TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);
  *         direction's last token.
  *   Every other argument, the status (ttt_mlp_status) and the errors as in
  *   ttt_mlp_forward; workspace of ttt_linear_workspace_size bytes.  The scan
- *   runs in fp32 (one CTA per 16 rows of a head's state).
+ *   takes the chunk form on the tensor cores (tf32 operands, fp32 state) for
+ *   bf16 inputs with d = 64 and 2 <= b <= 64, else runs in fp32 (one CTA per
+ *   16 rows of a head's state); ttt_mlp_select_kernels(1, .) forces the fp32
+ *   scan.
  */
 TTT_API size_t ttt_linear_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
 TTT_API ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q,

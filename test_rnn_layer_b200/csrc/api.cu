@@ -599,7 +599,12 @@ ttt_status linear_direction(const ttt_mlp_desc& q, const LinearLayout& L, char* 
     a.W_0 = W_0; a.W_T = w_t;
     a.T = q.T; a.H = q.H; a.d = q.d; a.b = b; a.reverse = reverse; a.eta = eta;
     a.status = status;
-    CUDA_TRY(launch_scan_linear(a, s));
+    // bf16-input layers (tolerance 2e-2) take the tensor-core chunk form; fp32 inputs, b = 1 and
+    // ttt_mlp_select_kernels(1, .) keep the fp32 SIMT scan
+    if (g_scan_impl.load() != 1 && q.x_dtype == TTT_BF16 && scan_linear_tc_supported(q.d, b))
+        CUDA_TRY(launch_scan_linear_tc(a, s));
+    else
+        CUDA_TRY(launch_scan_linear(a, s));
     CUDA_TRY(launch_gate(xin, xin_bf16, a.Z, alpha, out, out_bf16, delta, status, q.T, q.H, q.d,
                          q.per_head_input, 0, s));
     return TTT_OK;

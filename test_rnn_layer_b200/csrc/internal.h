@@ -69,7 +69,10 @@ struct LinearScanArgs {
     int* status;
 };
 bool scan_linear_supported(int d);
-cudaError_t launch_scan_linear(const LinearScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan_linear(const LinearScanArgs& a, cudaStream_t s);   // fp32 SIMT, any b
+// tcgen05 chunk form (tf32 contractions, fp32 state): d = 64, 2 <= b <= 64.
+bool scan_linear_tc_supported(int d, int b);
+cudaError_t launch_scan_linear_tc(const LinearScanArgs& a, cudaStream_t s);
 
 // Per-head projections: U[which][h, t, e] = sum_j theta_which[h][e][j] x[h, t, j].
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
