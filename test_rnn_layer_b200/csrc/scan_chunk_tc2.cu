@@ -26,8 +26,11 @@
 //   [Z1^T; N] = [W2_old; G] Gq^T, Z^T = Z1^T + D2'^T Np^T (Np[t,s] = N[s,t], s not after t):
 //   token t sees W2_old plus the updates of the tokens up to and including t.
 // The MMAs a later stage does not need at once are committed separately (the
-// first stage's Aq0 and S, the update stage's W1 and W2^T), and the shared
-// copy of the updated W2 is refreshed while the last MMA of the chunk runs.
+// first stage's Aq0 and S, the update stage's W1 and W2^T), independent
+// accumulators are issued by different threads, the z correction MMA is issued
+// behind a barrier of only the warps that build its operand, and the shared
+// copy of the updated W2 is refreshed off the chain (lanes 0-63 in the stage
+// after [Z1; N], lanes 64-127 during the next chunk's first MMAs).
 // The kernel stores z; the gate out = x + tanh(alpha) z is a separate
 // bandwidth-bound kernel, keeping global loads off the scan's dependent chain.
 // All contractions are kind::tf32 MMAs (fp32 accumulate) on K-major
@@ -39,10 +42,10 @@
 // pair has a barrier of its own (2 KB per phase, armed by the receiving warp's
 // lane 0 right after the previous phase completed).
 // Ordering of the exchange buffers (no handshake needed): the peer writes my
-// RY for chunk c+1 only after it received my [Z1;N] partial of chunk c, which
-// I send after I have read RY of chunk c; it writes my RZ for chunk c+1 only
-// after it received my Y partial of chunk c+1, which I send after I have read
-// RZ of chunk c.
+// RY for chunk c+1 only after it received my z partial of chunk c (before a
+// block barrier that precedes its Y send), which I send after I have read RY
+// of chunk c; it writes my RZ for chunk c+1 only after it received my Y
+// partial of chunk c+1, which I send after I have read RZ of chunk c.
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
