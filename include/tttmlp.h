@@ -236,6 +236,14 @@ TTT_API ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, c
  */
 TTT_API ttt_status ttt_debug_inject_wait_timeout(int enable);
 
+/*
+ * Tests only: the chunk segments [begin, end) the pipelined full-width layer
+ * uses for a walk of `nchunks` chunks, written as begin/end pairs into `out`
+ * (room for `max_segments` pairs).  Returns the number of segments (which may
+ * exceed max_segments: only that many are written), or -1 if nchunks < 1.
+ */
+TTT_API int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments);
+
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 TTT_API const char* ttt_last_error(void);
 

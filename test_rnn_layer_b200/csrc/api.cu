@@ -253,8 +253,9 @@ constexpr int kPipeMinSegChunks = 16;
 constexpr int kPipeSmMargin = 8;
 
 // Chunk ranges [begin, end) of a walk over `nchunks` chunks: segments grow
-// by 3/2 from 16 chunks at both ends (short exposed head and tail), with
-// pieces of about nchunks / 12 in between.
+// by 3/2 from 16 chunks at both ends (short exposed head and tail: 16, 24,
+// 36, ... and ..., 36, 24, 16), with equal pieces of at most
+// max(16, ceil(nchunks / 12)) chunks in between.
 std::vector<std::pair<int, int>> pipe_segments(int nchunks) {
     const int cap = std::max(kPipeMinSegChunks, (nchunks + 11) / 12);
     std::vector<int> front, back;
@@ -268,10 +269,9 @@ std::vector<std::pair<int, int>> pipe_segments(int nchunks) {
         back.push_back(t);
         rem -= t;
     }
-    while (rem > 0) {
-        const int t = std::min(cap, rem);
-        front.push_back(t);
-        rem -= t;
+    if (rem > 0) {   // the middle in equal pieces (no short leftover segment)
+        const int n = (rem + cap - 1) / cap;
+        for (int k = 0; k < n; ++k) front.push_back(rem / n + (k < rem % n ? 1 : 0));
     }
     front.insert(front.end(), back.rbegin(), back.rend());
     std::vector<std::pair<int, int>> out;
@@ -767,6 +767,16 @@ int ttt_kernel_times(int max_kernels, char* names, size_t names_cap, double* tot
         names[names_cap - 1] = '\0';
     }
     return (int)keys.size();
+}
+
+int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments) {
+    if (nchunks < 1) return -1;
+    const auto seg = pipe_segments(nchunks);
+    for (int k = 0; k < (int)seg.size() && k < max_segments && out; ++k) {
+        out[2 * k] = seg[k].first;
+        out[2 * k + 1] = seg[k].second;
+    }
+    return (int)seg.size();
 }
 
 ttt_status ttt_debug_inject_wait_timeout(int enable) {

@@ -25,7 +25,7 @@ DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
             "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_debug_inject_wait_timeout",
-            "ttt_linear_workspace_size", "ttt_linear_forward"]
+            "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments"]
 
 
 class TTTError(RuntimeError):
@@ -78,6 +78,8 @@ def lib():
         L.ttt_last_error.argtypes = []
         L.ttt_launch_count.restype = ctypes.c_uint64
         L.ttt_launch_count.argtypes = []
+        L.ttt_debug_pipe_segments.restype = i
+        L.ttt_debug_pipe_segments.argtypes = [i, ctypes.POINTER(ctypes.c_int), i]
         L.ttt_debug_inject_wait_timeout.restype = i
         L.ttt_debug_inject_wait_timeout.argtypes = [i]
         L.ttt_kernel_timing.restype = i
@@ -116,6 +118,15 @@ def ttt_launch_count() -> int:
 
 def ttt_debug_inject_wait_timeout(enable: bool) -> int:
     return int(lib().ttt_debug_inject_wait_timeout(1 if enable else 0))
+
+
+def ttt_debug_pipe_segments(nchunks: int, max_segments: int = 256) -> list:
+    """Chunk segments [(begin, end), ...] of the pipelined full-width layer (tests)."""
+    buf = (ctypes.c_int * (2 * max_segments))()
+    n = int(lib().ttt_debug_pipe_segments(int(nchunks), buf, max_segments))
+    if n < 0:
+        raise TTTError(TTT_ERR_INVALID_ARG, "ttt_debug_pipe_segments")
+    return [(buf[2 * k], buf[2 * k + 1]) for k in range(min(n, max_segments))]
 
 
 def ttt_kernel_timing(enable: bool) -> int:

@@ -150,3 +150,31 @@ def test_linear_forward_argument_errors_before_any_cuda_call():
     assert fwd(Y=0x1000) == L.TTT_ERR_INVALID_ARG and "alias" in L.ttt_last_error()
     assert fwd(wsb=4096) == L.TTT_ERR_INVALID_ARG and "too small" in L.ttt_last_error()
     assert fwd(WT=0x1008) == L.TTT_ERR_INVALID_ARG and "aligned" in L.ttt_last_error()
+
+
+@pytest.mark.parametrize("nchunks", [1, 15, 16, 17, 47, 128, 1000, 1603, 4896])
+def test_pipeline_segments_tile_the_walk(nchunks):
+    """The pipelined full-width layer splits a direction's walk into chunk
+    segments: contiguous, non-empty, covering [0, nchunks) exactly; the first
+    and last segments are the shortest (their projection or gate is not
+    overlapped), no segment exceeds max(16, ceil(nchunks / 12))."""
+    seg = L.ttt_debug_pipe_segments(nchunks)
+    assert seg[0][0] == 0 and seg[-1][1] == nchunks
+    for (a0, a1), (b0, _) in zip(seg, seg[1:]):
+        assert a1 == b0
+    sizes = [e - b for b, e in seg]
+    assert min(sizes) >= 1
+    cap = max(16, -(-nchunks // 12))
+    assert max(sizes) <= cap
+    if len(seg) > 2:
+        assert sizes[0] <= min(sizes[1:-1]) and sizes[-1] <= min(sizes[1:-1])
+    assert L.lib().ttt_debug_pipe_segments(0, None, 0) == -1
+
+
+def test_pipeline_segments_of_the_benchmark_layer():
+    """313,344 tokens in 64-token chunks: 4,896 chunks; the ramp grows by 3/2
+    from 16 at both ends and the middle is split into equal pieces."""
+    sizes = [e - b for b, e in L.ttt_debug_pipe_segments(4896)]
+    assert sizes[:4] == [16, 24, 36, 54] and sizes[-4:] == [54, 36, 24, 16]
+    middle = sizes[9:-9]   # between the two ramps (9 segments each, capped at 408 = 4896 / 12)
+    assert max(middle) - min(middle) <= 1 and max(middle) <= 408
