@@ -13,9 +13,9 @@ Sources (One-Minute Video Generation with Test-Time Training):
     tanh(alpha) * TTT(X) + X with alpha a learned vector; a forward TTT pass,
     then a reverse one, sharing theta but each with its own gate.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * the reverse pass runs on the gated forward output X' (sequential
-    composition, "first forward, then reverse");
+    composition: the forward pass first, the reverse pass after it);
   * both directions start from the same W_0 and use the same theta;
   * per-head mode: X is [H, T, d] and theta is [H, d, d] (one projection per
     head); full mode: X is [T, D] and theta is [H*d, D] (nn.Linear layout),
