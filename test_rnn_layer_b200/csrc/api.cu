@@ -8,6 +8,7 @@
 // Y = X' + tanh(alpha_r) z_r.
 #include <algorithm>
 #include <atomic>
+#include <functional>
 #include <cstdarg>
 #include <cmath>
 #include <cstdio>
@@ -283,13 +284,14 @@ std::vector<std::pair<int, int>> pipe_segments(int nchunks) {
     return out;
 }
 
-// SMs the projection and gate may use next to a running scan (0: no pipelining).
-int pipe_side_sms(const ttt_mlp_desc& q) {
+// SMs the projection and gate may use next to a running scan that holds
+// `scan_sms_per_head` SMs per head (0: no pipelining).
+int pipe_side_sms(const ttt_mlp_desc& q, int scan_sms_per_head) {
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return 0;
-    const int side = sms - 2 * q.H - kPipeSmMargin;
+    const int side = sms - scan_sms_per_head * q.H - kPipeSmMargin;
     return side >= 16 ? side : 0;
 }
 
@@ -299,13 +301,25 @@ bool pipe_eligible(const ttt_mlp_desc& q, const Layout& L, int b, ttt_direction 
     if (!(si == 0 || si == 2) || !scan_chunk_tc_supported(q.d, b)) return false;
     if (pi == 1 || !proj_full_tc_supported(q.D, q.D)) return false;
     if (dir == TTT_BIDIR && !L.split_reverse) return false;
-    return pipe_side_sms(q) > 0;
+    return pipe_side_sms(q, 2) > 0;
 }
 
-ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, const void* X, const void* const th[3],
-                             float* const qkv[3], const float* W1_0, const float* W2_0, float eta, int b,
-                             ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
-                             float* W1_T, float* W2_T, cudaStream_t s, const void* X_host, void* Y_host) {
+// Workspace buffers the pipeline uses (layer-independent).
+struct PipeBufs {
+    int* status;
+    float* xp;              // X' (fp32) between the directions
+    __nv_bfloat16* delta;   // bf16 gate increment (reverse projection input)
+    float* zbuf;            // z of one direction when the caller wants none
+};
+// Launches the scan over chunks [c_begin, c_end) of direction `di` (first/last:
+// the segment starts from W_0 / leaves the final state for the caller).
+using SegScan = std::function<cudaError_t(int di, const struct Dir& dd, int c_begin, int c_end, bool first,
+                                          bool last, float* zscan, cudaStream_t s)>;
+
+ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_sms_per_head, const SegScan& seg_scan,
+                             const void* X, const void* const th[3], float* const qkv[3], int b, ttt_direction dir,
+                             const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, cudaStream_t s,
+                             const void* X_host, void* Y_host) {
     std::lock_guard<std::mutex> lk(g_pipe_mu);
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
@@ -318,7 +332,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
         CUDA_TRY(cudaStreamCreateWithPriority(&P.side, cudaStreamNonBlocking, lo));
         CUDA_TRY(cudaStreamCreateWithPriority(&P.copy, cudaStreamNonBlocking, lo));
     }
-    const int side_sms = pipe_side_sms(q);
+    const int side_sms = pipe_side_sms(q, scan_sms_per_head);
     const int nch = (q.T + b - 1) / b;
     const auto seg = pipe_segments(nch);
     const int ns = (int)seg.size();
@@ -340,13 +354,10 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
 
     auto enqueue = [&]() -> ttt_status {
         const size_t n = (size_t)q.T * q.D;
-        const size_t nW = (size_t)q.H * q.m * q.d;
         const int D = q.D;
-        float* xp = reinterpret_cast<float*>(ws + L.xp);
-        __nv_bfloat16* delta = reinterpret_cast<__nv_bfloat16*>(ws + L.delta);
-        float* st1 = reinterpret_cast<float*>(ws + L.state);
-        float* st2 = st1 + nW;
-        int* status = reinterpret_cast<int*>(ws + L.status);
+        float* xp = B.xp;
+        __nv_bfloat16* delta = B.delta;
+        int* status = B.status;
 
         for (int di = 0; di < ndir; ++di) {
             Dir dd{};
@@ -360,7 +371,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
             dd.zdbg = Z_out ? Z_out + di * n : nullptr;
             const void* psrc = second ? static_cast<const void*>(delta) : X;   // both bf16
             const int pacc = second ? 1 : 0;
-            float* zscan = Z_out ? Z_out + di * n : reinterpret_cast<float*>(ws + L.zbuf);
+            float* zscan = Z_out ? Z_out + di * n : B.zbuf;
 
             std::vector<cudaEvent_t> ev_proj(ns), ev_scan(ns), ev_h2d(ns), ev_gate(ns);
             for (int k = 0; k < ns; ++k) { ev_proj[k] = new_ev(); ev_scan[k] = new_ev(); ev_h2d[k] = new_ev(); ev_gate[k] = new_ev(); }
@@ -391,17 +402,10 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const Layout& L, char* ws, c
                 CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
                 CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
             }
-            // scan segments, state carried in the workspace
+            // scan segments, the state carried by the launcher
             for (int k = 0; k < ns; ++k) {
                 CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k], 0));
-                ScanArgs a = scan_args(q, L, ws, k == 0 ? W1_0 : st1, k == 0 ? W2_0 : st2, eta, b, dd);
-                a.Zscan = zscan;
-                a.c_begin = seg[k].first;
-                a.c_end = seg[k].second;
-                const bool last = k == ns - 1;
-                a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
-                a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
-                CUDA_TRY(launch_scan_chunk_tc2(a, P.scan));
+                CUDA_TRY(seg_scan(di, dd, seg[k].first, seg[k].second, k == 0, k == ns - 1, zscan, P.scan));
                 CUDA_TRY(cudaEventRecord(ev_scan[k], P.scan));
             }
             // gates, each after its segment's scan
@@ -501,9 +505,26 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
     float* xp = reinterpret_cast<float*>(ws + L.xp);
     int* status = reinterpret_cast<int*>(ws + L.status);
 
-    if (pipe_eligible(q, L, b, dir))
-        return forward_pipelined(q, L, ws, X, th, qkv, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
-                                 W2_T, s, X_host, Y_host);
+    if (pipe_eligible(q, L, b, dir)) {
+        // the cluster scan, the state W1, W2 carried between segments through the workspace
+        const size_t nW = (size_t)q.H * q.m * q.d;
+        float* st1 = reinterpret_cast<float*>(ws + L.state);
+        float* st2 = st1 + nW;
+        const SegScan seg_scan = [&](int di, const Dir& dd, int cb, int ce, bool first, bool last, float* zscan,
+                                     cudaStream_t ss) {
+            ScanArgs a = scan_args(q, L, ws, first ? W1_0 : st1, first ? W2_0 : st2, eta, b, dd);
+            a.Zscan = zscan;
+            a.c_begin = cb;
+            a.c_end = ce;
+            a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
+            a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
+            return launch_scan_chunk_tc2(a, ss);
+        };
+        const PipeBufs bufs{status, xp, reinterpret_cast<__nv_bfloat16*>(ws + L.delta),
+                            reinterpret_cast<float*>(ws + L.zbuf)};
+        return forward_pipelined(q, bufs, 2, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, X_host,
+                                 Y_host);
+    }
     if (X_host) CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(X), X_host, xbytes, cudaMemcpyHostToDevice, s));
     auto finish = [&]() -> ttt_status {
         if (Y_host) CUDA_TRY(cudaMemcpyAsync(Y_host, Y, xbytes, cudaMemcpyDeviceToHost, s));
@@ -560,7 +581,7 @@ ttt_status check_desc_linear(const ttt_mlp_desc* desc, int b, ttt_direction dir)
 }
 
 struct LinearLayout {
-    size_t status, qkv[3], xp, delta, zbuf, total;
+    size_t status, qkv[3], xp, delta, zbuf, state, total;
     bool split_reverse;
 };
 
@@ -577,6 +598,8 @@ LinearLayout plan_linear(const ttt_mlp_desc& q, ttt_direction dir) {
     if (L.split_reverse) off = align_up(off + n * 2);
     L.zbuf = off;
     off = align_up(off + n * sizeof(float));
+    L.state = off;   // W of every head between two segments of a pipelined direction
+    off = align_up(off + (size_t)q.H * q.d * q.d * sizeof(float));
     L.total = off;
     return L;
 }
@@ -672,6 +695,32 @@ ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const voi
     const size_t n = (size_t)q.T * q.D, nW = (size_t)q.H * q.d * q.d;
     float* xp = reinterpret_cast<float*>(ws + L.xp);
     __nv_bfloat16* delta = L.split_reverse ? reinterpret_cast<__nv_bfloat16*>(ws + L.delta) : nullptr;
+    // the full-width bf16 layer on the tensor cores: chunk segments on two streams, as for the MLP layer
+    if (!q.per_head_input && x_bf16 && g_scan_impl.load() != 1 && scan_linear_tc_supported(q.d, b) &&
+        g_proj_impl.load() != 1 && proj_full_tc_supported(q.D, q.D) && (dir != TTT_BIDIR || L.split_reverse) &&
+        pipe_side_sms(q, 1) > 0) {
+        float* stW = reinterpret_cast<float*>(ws + L.state);
+        int* status = reinterpret_cast<int*>(ws + L.status);
+        float* qkv[3] = {reinterpret_cast<float*>(ws + L.qkv[0]), reinterpret_cast<float*>(ws + L.qkv[1]),
+                         reinterpret_cast<float*>(ws + L.qkv[2])};
+        const SegScan seg_scan = [&](int di, const Dir& dd, int cb, int ce, bool first, bool last, float* zscan,
+                                     cudaStream_t ss) {
+            LinearScanArgs a{};
+            a.Q = qkv[0]; a.K = qkv[1]; a.V = qkv[2];
+            a.qkv_hs = q.d; a.qkv_ts = q.D; a.x_hs = q.d; a.x_ts = q.D;
+            a.Z = zscan;
+            a.W_0 = first ? W_0 : stW;
+            a.W_T = last ? (W_T ? W_T + di * nW : nullptr) : stW;
+            a.T = q.T; a.H = q.H; a.d = q.d; a.b = b; a.reverse = dd.reverse; a.eta = eta;
+            a.status = status;
+            a.c_begin = cb;
+            a.c_end = ce;
+            return launch_scan_linear_tc(a, ss);
+        };
+        const PipeBufs bufs{status, xp, delta, reinterpret_cast<float*>(ws + L.zbuf)};
+        return forward_pipelined(q, bufs, 1, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, nullptr,
+                                 nullptr);
+    }
     if (dir != TTT_BIDIR)
         return linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, dir == TTT_REV,
                                 dir == TTT_REV ? alpha_r : alpha_f, Y, x_bf16, nullptr, Z_out, W_T, s);

@@ -67,6 +67,7 @@ struct LinearScanArgs {
     int T, H, d, b, reverse;
     float eta;
     int* status;
+    int c_begin, c_end;   // tensor-core kernel: chunks [c_begin, c_end) of the walk (c_end 0: to the end)
 };
 bool scan_linear_supported(int d);
 cudaError_t launch_scan_linear(const LinearScanArgs& a, cudaStream_t s);   // fp32 SIMT, any b

@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
     const int h = blockIdx.x;
     const int T = a.T, b = a.b;
     const int nchunks = (T + b - 1) / b;
+    const int c_first = a.c_begin, c_last = a.c_end > 0 ? min(a.c_end, nchunks) : nchunks;
     const float m2eta = -2.0f * a.eta;
 
     if (tid == 0) {
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
     }
     if (tid == 0) {
         int y0, bc;
-        chunk_rows(0, y0, bc);
+        chunk_rows(c_first, y0, bc);
         load_tiles(y0);
     }
 
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
     };
     int prev_y0 = 0, prev_bc = 0;
 
-    for (int c = 0; c < nchunks; ++c) {
+    for (int c = c_first; c < c_last; ++c) {
         int y0, bc;
         chunk_rows(c, y0, bc);
         const uint32_t tz = TM_Z + 64 * (c & 1);
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
                     for (int kk = 0; kk < 8; ++kk)
                         tc::mma_tf32_ts(tm + TM_W, tm + TM_E + kk * 8, kstep(dX1, kk), ID64, 1);
                     tc::mma_commit(bar_mma);
-                    if (c + 1 < nchunks) {
+                    if (c + 1 < c_last) {
                         int ny0, nbc;
                         chunk_rows(c + 1, ny0, nbc);
                         load_tiles(ny0);
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
         prev_y0 = y0;
         prev_bc = bc;
     }
-    if (prev_bc && !*abort_flag) store_z(TM_Z + 64 * ((nchunks - 1) & 1), prev_y0, prev_bc);
+    if (prev_bc && !*abort_flag) store_z(TM_Z + 64 * ((c_last - 1) & 1), prev_y0, prev_bc);
 
     if (*abort_flag) {
         const uint64_t t0 = tc::globaltimer_ns();
@@ -351,6 +352,9 @@ bool scan_linear_tc_supported(int d, int b) { return d == DH && b >= 2 && b <= B
 
 cudaError_t launch_scan_linear_tc(const LinearScanArgs& a, cudaStream_t s) {
     if (!scan_linear_tc_supported(a.d, a.b)) return cudaErrorInvalidValue;
+    const int nchunks = (a.T + a.b - 1) / a.b;
+    const int c_end = a.c_end > 0 ? a.c_end : nchunks;
+    if (a.c_begin < 0 || c_end > nchunks || a.c_begin >= c_end) return cudaErrorInvalidValue;
     LinTcArgs P{};
     P.a = a;
     P.full = (a.qkv_ts != DH) ? 1 : 0;

@@ -22,9 +22,11 @@ CASES = [
     S.CAUSAL.with_(T=300, H=3, d=32, b=5, dirs="rev"),             # fp32, d = 32, reverse only
     S.CAUSAL.with_(T=350, H=2, b=100, dirs="bidir"),               # fp32, chunks spanning two tiles
     S.MINIBATCH.with_(T=1, H=2),                                   # a single token
+    S.FULL63S.with_(T=3000, H=4, D=256),                           # full width, three chunk segments
+    S.FULL63S.with_(T=3000, H=4, D=256, dirs="rev"),               # ... reverse only
 ]
 IDS = ["tiny-d16-b1", "causal-d64-b1", "b16-bidir-bf16", "b64-bidir-bf16", "full-width-bf16", "d32-b5-rev",
-       "b100-bidir", "T1"]
+       "b100-bidir", "T1", "full-width-segmented", "full-width-segmented-rev"]
 
 
 def _oracle(w, inp):
