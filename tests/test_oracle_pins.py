@@ -353,3 +353,23 @@ def test_literal_eta_diverges_and_eta_over_d_does_not():
     assert not np.isfinite(bad["Y"]).all()
     good = O.layer_forward(*args, w.eta_eff, 1, "fwd", alpha_f=inp["alpha_f"].numpy(), per_head=True)
     assert np.isfinite(good["Y"]).all() and np.isfinite(good["W1_f"]).all()
+
+
+@pytest.mark.parametrize("b", [1, 8])
+def test_scan_is_causal_token_by_token(b):
+    """Forward: z_t depends on tokens 0..t only, also inside a chunk (the prefix
+    reading); reverse: on tokens t..T-1 only.  Perturbing token t0 must leave the
+    earlier (forward) or later (reverse) outputs exactly unchanged and change z_t0."""
+    rng = np.random.default_rng(29 + b)
+    T, d, m, t0 = 21, 3, 12, 11
+    Q, K, V = rng.normal(size=(T, d)), rng.normal(size=(T, d)), rng.normal(size=(T, d))
+    W1, W2 = rng.normal(size=(m, d)) / np.sqrt(d), rng.normal(size=(d, m)) / np.sqrt(m)
+    Q2, K2, V2 = Q.copy(), K.copy(), V.copy()
+    K2[t0] += 0.5
+    V2[t0] -= 0.5
+    for reverse in (False, True):
+        Z, _, _ = O.scan(Q, K, V, W1, W2, 0.02, b, reverse=reverse)
+        Zp, _, _ = O.scan(Q2, K2, V2, W1, W2, 0.02, b, reverse=reverse)
+        same = slice(t0 + 1, T) if reverse else slice(0, t0)
+        np.testing.assert_array_equal(Z[same], Zp[same])
+        assert np.abs(Z[t0] - Zp[t0]).max() > 1e-6

@@ -191,3 +191,20 @@ def test_linear_full_mode_with_block_diagonal_theta_equals_per_head_mode():
     ph = O.linear_layer_forward(Xh, *th_h, W0, 0.01, 3, "bidir", alpha_f=a, alpha_r=a, per_head=True)
     fm = O.linear_layer_forward(Xf, *th_f, W0, 0.01, 3, "bidir", alpha_f=a, alpha_r=a, per_head=False)
     np.testing.assert_allclose(fm["Y"], ph["Y"].transpose(1, 0, 2).reshape(T, D), rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("b", [1, 8])
+def test_linear_scan_is_causal_token_by_token(b):
+    rng = np.random.default_rng(31 + b)
+    T, d, t0 = 21, 4, 11
+    Q, K, V = _rand((T, d), rng), _rand((T, d), rng), _rand((T, d), rng)
+    W0 = _rand((d, d), rng, 0.5)
+    K2, V2 = K.copy(), V.copy()
+    K2[t0] += 0.5
+    V2[t0] -= 0.5
+    for reverse in (False, True):
+        Z, _ = O.linear_scan(Q, K, V, W0, 0.02, b, reverse=reverse)
+        Zp, _ = O.linear_scan(Q, K2, V2, W0, 0.02, b, reverse=reverse)
+        same = slice(t0 + 1, T) if reverse else slice(0, t0)
+        np.testing.assert_array_equal(Z[same], Zp[same])
+        assert np.abs(Z[t0] - Zp[t0]).max() > 1e-6
