@@ -316,6 +316,8 @@ def run_ours(args, rank, world, local_rank):
     from test_rnn_layer_b200 import tttmlp as L
 
     L.lib()   # loud failure if the CUDA library is missing
+    if args.kernels == "simt":
+        L.check(L.ttt_mlp_select_kernels(1, 1), "ttt_mlp_select_kernels")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = _workload(args)
@@ -538,6 +540,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--model", choices=["mlp", "linear"], default="mlp")
+    ap.add_argument("--kernels", choices=["auto", "simt"], default="auto",
+                    help="simt: the fp32 SIMT scan and projection kernels (reference kernels)")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length (quick checks only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
