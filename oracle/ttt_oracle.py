@@ -50,37 +50,42 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
+def configure(lib):
+    """Declare the argument and result types of the C functions on a loaded
+    ctypes library (the oracle's own, or a copy built from another source)."""
+    lib.ttt_ref_gelu.restype = ctypes.c_double
+    lib.ttt_ref_gelu.argtypes = [ctypes.c_double]
+    lib.ttt_ref_gelu_prime.restype = ctypes.c_double
+    lib.ttt_ref_gelu_prime.argtypes = [ctypes.c_double]
+    lib.ttt_ref_inner_loss_grad.restype = ctypes.c_double
+    lib.ttt_ref_inner_loss_grad.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp]
+    lib.ttt_ref_mlp_apply.restype = None
+    lib.ttt_ref_mlp_apply.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp]
+    lib.ttt_ref_scan_per_token.restype = None
+    lib.ttt_ref_scan_per_token.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [_dp] * 6
+    lib.ttt_ref_scan_chunked.restype = None
+    lib.ttt_ref_scan_chunked.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 6
+    lib.ttt_ref_scan_heads.restype = None
+    lib.ttt_ref_scan_heads.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 6
+    lib.ttt_ref_num_threads.restype = ctypes.c_int
+    lib.ttt_ref_num_threads.argtypes = []
+    lib.ttt_ref_linear_grad.restype = ctypes.c_double
+    lib.ttt_ref_linear_grad.argtypes = [ctypes.c_int, _dp, _dp, _dp, _dp]
+    lib.ttt_ref_linear_apply.restype = None
+    lib.ttt_ref_linear_apply.argtypes = [ctypes.c_int, _dp, _dp, _dp]
+    lib.ttt_ref_linear_scan_per_token.restype = None
+    lib.ttt_ref_linear_scan_per_token.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double] + [_dp] * 5
+    lib.ttt_ref_linear_scan_chunked.restype = None
+    lib.ttt_ref_linear_scan_chunked.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [_dp] * 5
+    lib.ttt_ref_linear_scan_heads.restype = None
+    lib.ttt_ref_linear_scan_heads.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_dp] * 5
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
-        lib.ttt_ref_gelu.restype = ctypes.c_double
-        lib.ttt_ref_gelu.argtypes = [ctypes.c_double]
-        lib.ttt_ref_gelu_prime.restype = ctypes.c_double
-        lib.ttt_ref_gelu_prime.argtypes = [ctypes.c_double]
-        lib.ttt_ref_inner_loss_grad.restype = ctypes.c_double
-        lib.ttt_ref_inner_loss_grad.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp]
-        lib.ttt_ref_mlp_apply.restype = None
-        lib.ttt_ref_mlp_apply.argtypes = [ctypes.c_int, ctypes.c_int, _dp, _dp, _dp, _dp]
-        lib.ttt_ref_scan_per_token.restype = None
-        lib.ttt_ref_scan_per_token.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [_dp] * 6
-        lib.ttt_ref_scan_chunked.restype = None
-        lib.ttt_ref_scan_chunked.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 6
-        lib.ttt_ref_scan_heads.restype = None
-        lib.ttt_ref_scan_heads.argtypes = [ctypes.c_int] * 6 + [ctypes.c_double] + [_dp] * 6
-        lib.ttt_ref_num_threads.restype = ctypes.c_int
-        lib.ttt_ref_num_threads.argtypes = []
-        lib.ttt_ref_linear_grad.restype = ctypes.c_double
-        lib.ttt_ref_linear_grad.argtypes = [ctypes.c_int, _dp, _dp, _dp, _dp]
-        lib.ttt_ref_linear_apply.restype = None
-        lib.ttt_ref_linear_apply.argtypes = [ctypes.c_int, _dp, _dp, _dp]
-        lib.ttt_ref_linear_scan_per_token.restype = None
-        lib.ttt_ref_linear_scan_per_token.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double] + [_dp] * 5
-        lib.ttt_ref_linear_scan_chunked.restype = None
-        lib.ttt_ref_linear_scan_chunked.argtypes = [ctypes.c_int] * 4 + [ctypes.c_double] + [_dp] * 5
-        lib.ttt_ref_linear_scan_heads.restype = None
-        lib.ttt_ref_linear_scan_heads.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double] + [_dp] * 5
-        _lib = lib
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
 
 

@@ -373,3 +373,22 @@ def test_scan_is_causal_token_by_token(b):
         same = slice(t0 + 1, T) if reverse else slice(0, t0)
         np.testing.assert_array_equal(Z[same], Zp[same])
         assert np.abs(Z[t0] - Zp[t0]).max() > 1e-6
+
+
+def test_heads_equal_single_head_runs():
+    """The multi-head driver (OpenMP over heads, [H, T, d] streams) equals H
+    separate single-head scans with eta > 0: fixes its head strides for Q, K, V,
+    W1, W2 and Z, for the per-token rule (b = 1) and the chunk form, both ways."""
+    rng = np.random.default_rng(21)
+    H, T, d = 3, 29, 4
+    m = 4 * d
+    Q, K, V = (rng.normal(size=(H, T, d)) for _ in range(3))
+    W1 = rng.normal(size=(H, m, d)) / math.sqrt(d)
+    W2 = rng.normal(size=(H, d, m)) / math.sqrt(m)
+    for b in (1, 6):
+        for reverse in (False, True):
+            Z, W1T, W2T = O.scan_heads(Q, K, V, W1, W2, 0.05 / d, b, reverse)
+            for h in range(H):
+                z, w1, w2 = O.scan(Q[h], K[h], V[h], W1[h], W2[h], 0.05 / d, b, reverse=reverse, per_token=b == 1)
+                assert np.array_equal(Z[h], z) and np.array_equal(W1T[h], w1) and np.array_equal(W2T[h], w2)
+            assert np.abs(W1T - W1).max() > 1e-6   # the state moved
