@@ -48,6 +48,8 @@ def _check(w, dirs=None, eta=None, impl=None, **inp_kw):
     g = run_gpu(w, inp, dirs=dirs, eta=eta, want_z=True, want_state=True)
     o = run_oracle(w, inp, dirs=dirs, eta=eta)
     errs = _compare(w, g, o, dirs)
+    print(f"PARITY {w.name} T={w.T} b={w.b} {dirs or w.dirs} " + " ".join(f"{k}={v:.3e}" for k, v in errs.items()),
+          flush=True)
     bad = {k: v for k, v in errs.items() if not v <= tol(w)}
     assert not bad, f"{w.name}: {errs}"
     return errs
