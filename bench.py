@@ -8,9 +8,14 @@ resident in HBM.  Multi-GPU (torchrun): each rank runs its own sequence
 (independent replicas, weak scaling, no collective on the data path).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--model mlp|linear]
+                    [--workload full63s|scale18s|minibatch|causal|tiny]
 
-Prints one JSON line on rank 0.  --model linear measures the TTT-Linear layer
-(f(u; W) = W u) on the same sequence instead.
+Prints one JSON line on rank 0.  With --gpus N > 1 and no torchrun
+environment, bench.py starts N ranks itself (torch.distributed.run, one
+process per GPU).  --model linear measures the TTT-Linear layer
+(f(u; W) = W u) on the same sequence instead.  --workload picks one of the
+other workloads of the description (default: the 313,344-token layer); the
+b = 1 per-token workloads also report the time per token.
 """
 from __future__ import annotations
 
@@ -64,6 +69,7 @@ KERNEL_SRC = {
     "scan_chunk_simt": ("scan_chunk_simt.cu",),
     "scan_chunk_tc": ("scan_chunk_tc.cu",),
     "scan_chunk_tc2": ("scan_chunk_tc2.cu",),
+    "scan_chunk_tc3": ("scan_chunk_tc3.cu",),
     "scan_token": ("scan_token.cu",),
     "proj_full_simt": ("proj_simt.cu",),
     "proj_full_tc": ("proj_tc.cu",),
@@ -74,13 +80,20 @@ KERNEL_SRC = {
 }
 
 
-def _traffic(name: str, units_scale: float):
+def _layout_key(w) -> str:
+    return f"{'head' if w.per_head else 'full'}-H{w.H}-d{w.d}"
+
+
+def _traffic(name: str, units_scale: float, w=None):
     """DRAM bytes per launch of `name` from the committed ncu summary, or None
-    if absent or taken on a different version of the kernel's source."""
+    if absent, taken on a different version of the kernel's source, or taken
+    on another layout (head count, per-head vs full width) than `w`'s."""
     try:
         with open(TRAFFIC_PATH) as f:
             rec = json.load(f).get(name)
         if not rec or rec.get("src_hash") != _src_hash(*KERNEL_SRC[name]):
+            return None
+        if w is not None and rec.get("layout", "full-H48-d64") != _layout_key(w):
             return None
         return rec["bytes_per_launch_per_unit"] * units_scale
     except (OSError, KeyError, ValueError):
@@ -130,21 +143,42 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ workload
+WORKLOAD_NAMES = ("full63s", "scale18s", "minibatch", "causal", "tiny")
+
+
 def _workload(args):
     from test_rnn_layer_b200 import synth as S
-    w = S.FULL63S
+    w = {"full63s": S.FULL63S, "scale18s": S.SCALE18S, "minibatch": S.MINIBATCH, "causal": S.CAUSAL,
+         "tiny": S.TINY}[args.workload]
     if args.T:
         w = w.with_T(args.T)
     return w
 
 
+def _metric(w, model: str) -> str:
+    from test_rnn_layer_b200 import synth as S
+    if w.name == S.FULL63S.name:
+        return METRIC_LINEAR if model == "linear" else METRIC
+    kind = "TTT-Linear" if model == "linear" else "TTT-MLP"
+    return f"{kind} tokens/s ({w.H} heads, {w.dirs}, b={w.b}, {w.dtype}) at T={w.T}; % of roofline"
+
+
+def _input_bytes(w) -> int:
+    return w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) if w.per_head else w.T * w.model_dim * 2
+
+
 def _config(w, extra=None):
+    """The workload description; identical in both arms for the same workload."""
+    th = f"theta~N(0,1/{'d' if w.per_head else 'D'})"
+    xb = _input_bytes(w)
+    l2 = ("no flush: every input is larger than the 126 MB L2" if xb > 126e6 else
+          "no flush: the inputs fit in L2 (a small workload; reported for its per-token latency)")
     cfg = {"workload": w.name, "T": w.T, "D": w.model_dim, "H": w.H, "d": w.d, "hidden": w.m, "b": w.b,
            "dirs": w.dirs, "x_dtype": w.dtype, "state": "fp32", "eta": f"{w.eta}/d", "alpha": w.alpha,
-           "inputs": "seeded Gaussian stand-ins for video tokens (X~N(0,1), theta~N(0,1/D), W1_0~N(0,1/d), "
+           "layout": "per-head X [H,T,d]" if w.per_head else "full width X [T,D]",
+           "inputs": f"seeded Gaussian stand-ins for video tokens (X~N(0,1), {th}, W1_0~N(0,1/d), "
                      "W2_0~N(0,1/4d))",
-           "l2": "no flush: every input is larger than the 126 MB L2 (X 1.9 GB, Q/K/V 11.5 GB)",
-           "parallelism": "replicas (one sequence per GPU)"}
+           "l2": l2, "parallelism": "replicas (one sequence per GPU)"}
     if extra:
         cfg.update(extra)
     return cfg
@@ -159,6 +193,8 @@ def _algorithmic(w):
     return {
         "scan_chunk_tc": ("tensor_tf32", scan_flops),
         "scan_chunk_tc2": ("tensor_tf32", scan_flops),
+        # tf32 for the three d-by-m products that read the fp32 state (A, Aq0, P), fp16 for the rest
+        "scan_chunk_tc3": ("tensor_mixed", scan_flops),
         "scan_chunk_simt": ("alu", scan_flops),
         "scan_token": ("alu", H * T * 7 * 2 * d * m),
         "proj_full_tc": ("tensor_bf16", proj_flops),
@@ -175,6 +211,12 @@ def _algorithmic(w):
     }
 
 
+def _tf32_share(w) -> float:
+    """Share of the scan's algorithmic flops that the split-group kernel runs
+    with tf32 operands: A^T = W1 K^T, Aq0 = W1 Q^T and P^T = W2^T D2'^T."""
+    return 3 * 2 * w.d * w.m / (7 * 2 * w.d * w.m + 2 * w.b * (w.d + w.m))
+
+
 def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):
     """Roofline of one launch of `name`: the step's algorithmic work for that
     kernel (both directions for a bidirectional layer) divided evenly over its
@@ -186,6 +228,13 @@ def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):
     src = "of " + peaks["_source"]
     if bound == "tensor_bf16":
         peak, unit, kind, note = sus, "TFLOP/s", "tensor", f"bf16 dense sustained {src}"
+        achieved = work / (ms_per_launch * 1e-3) / 1e12
+    elif bound == "tensor_mixed":
+        f = _tf32_share(w)
+        peak = 1.0 / (f / (sus * TF32_PER_BF16) + (1.0 - f) / sus)
+        unit, kind = "TFLOP/s", "tensor"
+        note = (f"{f:.3f} of the flops at tf32 (bf16 sustained {src} x 1.1/2.25), the rest at fp16 (= bf16 "
+                f"sustained {src}): the time-weighted peak")
         achieved = work / (ms_per_launch * 1e-3) / 1e12
     elif bound == "tensor_tf32":
         peak, unit, kind = sus * TF32_PER_BF16, "TFLOP/s", "tensor"
@@ -201,7 +250,7 @@ def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):
         achieved = work / (ms_per_launch * 1e-3) / 1e9
     units = w.T * ndir / launches_per_step / 1024.0   # traffic records are stored per 1024 tokens
     return {"kernel": name, "bound": kind, "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": _traffic(name, units), "peak_note": note,
+            "frac": round(achieved / peak, 4), "traffic": _traffic(name, units, w), "peak_note": note,
             "ms_per_launch": round(ms_per_launch, 4), "work_per_launch": work}
 
 
@@ -228,37 +277,25 @@ def whole_job_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float)
 
 
 # ------------------------------------------------------------------ CPU side (oracle)
-def _cpu_sample(w, tokens: int, seed: int = 0):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _cpu_sample(w, tokens: int, model: str = "mlp", seed: int = 0):
     """A bounded sample of the workload for the fp64 oracle: the first `tokens`
-    tokens of the sequence, forward direction, `heads` heads (one OpenMP thread
-    each), with their share of the projections."""
-    import numpy as np
-    import torch
-
-    from oracle import ttt_oracle as O
-    from test_rnn_layer_b200 import synth as S
-
-    threads = O.num_threads()
-    heads = list(range(min(w.H, threads)))
-    inp = S.make_inputs(w.with_T(tokens), seed=seed, device="cpu")
-    X = inp["X"].float().numpy()
-    th = [inp[k].float().numpy() for k in ("theta_q", "theta_k", "theta_v")]
-    W1, W2 = inp["W1_0"].double().numpy(), inp["W2_0"].double().numpy()
-
-    def run():
-        t0 = time.perf_counter()
-        O.full_mode_heads(X, *th, W1, W2, w.eta_eff, w.b, heads)
-        return time.perf_counter() - t0
-
-    # metric units: tokens through all H heads in both directions
-    scale = len(heads) / (w.H * 2.0)
-    sample = (f"first {tokens} tokens, {len(heads)} of {w.H} heads, forward direction only (fp64 oracle incl. "
-              f"those heads' Q/K/V projections); tokens/s scaled by {len(heads)}/({w.H}*2)")
-    return run, scale, threads, sample
-
-
-def _cpu_sample_linear(w, tokens: int, seed: int = 0):
-    """As _cpu_sample, for the TTT-Linear layer."""
+    tokens of the sequence, the first direction only, as many heads as the
+    oracle has threads (one OpenMP thread per head), with those heads' share of
+    the projections.  Both the reference arm and the CPU baseline time exactly
+    this sample.  Returns (run, scale, threads, description): run() times one
+    pass in seconds; tokens x scale / seconds is in the metric's units (tokens
+    through all heads and directions)."""
     import numpy as np
 
     from oracle import ttt_oracle as O
@@ -266,22 +303,59 @@ def _cpu_sample_linear(w, tokens: int, seed: int = 0):
 
     threads = O.num_threads()
     heads = list(range(min(w.H, threads)))
-    inp = S.make_linear_inputs(w.with_T(tokens), seed=seed, device="cpu")
-    X = inp["X"].float().numpy()
-    rows = np.concatenate([np.arange(h * w.d, (h + 1) * w.d) for h in heads])
-    th = [inp[k].float().numpy()[rows] for k in ("theta_q", "theta_k", "theta_v")]
-    W0 = inp["W_0"].double().numpy()[heads]
+    tokens = min(tokens, w.T)
+    ws = w.with_T(tokens)
+    inp = (S.make_linear_inputs if model == "linear" else S.make_inputs)(ws, seed=seed, device="cpu")
+    reverse = w.dirs == "rev"
+    ndir = 2 if w.dirs == "bidir" else 1
+    if w.per_head:
+        X = inp["X"].double().numpy()[heads]
+        th = [inp[k].double().numpy()[heads] for k in ("theta_q", "theta_k", "theta_v")]
+    else:
+        X = inp["X"].float().numpy()
+        rows = np.concatenate([np.arange(h * w.d, (h + 1) * w.d) for h in heads])
+        th = [inp[k].float().numpy()[rows] for k in ("theta_q", "theta_k", "theta_v")]
+
+    if model == "linear":
+        W0 = inp["W_0"].double().numpy()[heads]
+
+        def work():
+            if w.per_head:
+                O.linear_direction(X, *th, W0, w.eta_eff, w.b, reverse, per_head=True)
+            else:
+                Q, K, V = [O.project_full(X, t).reshape(tokens, len(heads), w.d).transpose(1, 0, 2) for t in th]
+                O.linear_scan_heads(Q, K, V, W0, w.eta_eff, w.b, reverse)
+    else:
+        W1, W2 = inp["W1_0"].double().numpy()[heads], inp["W2_0"].double().numpy()[heads]
+
+        def work():
+            if w.per_head:
+                O.direction(X, *th, W1, W2, w.eta_eff, w.b, reverse, per_head=True)
+            else:
+                O.full_mode_heads(X, *th, W1, W2, w.eta_eff, w.b, list(range(len(heads))), reverse=reverse)
 
     def run():
         t0 = time.perf_counter()
-        Q, K, V = [O.project_full(X, t).reshape(tokens, len(heads), w.d).transpose(1, 0, 2) for t in th]
-        O.linear_scan_heads(Q, K, V, W0, w.eta_eff, w.b)
+        work()
         return time.perf_counter() - t0
 
-    scale = len(heads) / (w.H * 2.0)
-    sample = (f"first {tokens} tokens, {len(heads)} of {w.H} heads, forward direction only (fp64 TTT-Linear "
-              f"oracle incl. those heads' Q/K/V projections); tokens/s scaled by {len(heads)}/({w.H}*2)")
+    scale = len(heads) / (w.H * float(ndir))
+    kind = "TTT-Linear" if model == "linear" else "TTT-MLP"
+    sample = (f"first {tokens} tokens, {len(heads)} of {w.H} heads, {'reverse' if reverse else 'forward'} direction "
+              f"only (fp64 {kind} oracle incl. those heads' Q/K/V projections); tokens/s scaled by "
+              f"{len(heads)}/({w.H}*{ndir})")
     return run, scale, threads, sample
+
+
+def cpu_baseline(w, args) -> dict:
+    """The oracle on this host's cores, on the reference arm's sample, repeated
+    args.cpu_reps times (about 10-30 s of CPU work at the full layer)."""
+    run, scale, threads, sample = _cpu_sample(w, args.sample_tokens, args.model)
+    times = [run() for _ in range(args.cpu_reps)]
+    t = sum(times) / len(times)
+    tokens = min(args.sample_tokens, w.T)
+    return {"value": tokens * scale / t, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+            "seconds": round(sum(times), 2), "reps": len(times), "cpu_model": cpu_model()}
 
 
 # ------------------------------------------------------------------ arms
@@ -289,23 +363,64 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     w = _workload(args)
-    tokens = args.ref_tokens
-    run, scale, threads, sample = (_cpu_sample_linear if args.model == "linear" else _cpu_sample)(w, tokens)
+    run, scale, threads, sample = _cpu_sample(w, args.sample_tokens, args.model)
+    tokens = min(args.sample_tokens, w.T)
     for _ in range(args.warmup):
         run()
     times = [run() for _ in range(args.steps)]
     step_s = sum(times) / len(times)
     value = tokens * scale / step_s
-    line = {"impl": "reference", "metric": METRIC_LINEAR if args.model == "linear" else METRIC, "value": value,
-            "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": _config(w, {"sample": sample}),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+    line = {"impl": "reference", "metric": _metric(w, args.model), "value": value, "unit": UNIT,
+            "n_gpus": max(world, args.gpus), "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": _config(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _timed_steps(step, args, world, local_rank, stream, flush_l2):
+    """W untimed warm-up steps, then K timed steps between barriers and
+    synchronisations, timed by CUDA events on `stream`; the maximum over
+    ranks.  With flush_l2 a buffer larger than L2 is written before each
+    step and every step is timed alone (the flush outside the timed spans)."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    scrub = torch.empty(64 << 22, dtype=torch.float32, device=stream.device) if flush_l2 else None   # 1 GiB
+    barrier()
+    torch.cuda.synchronize()
+    if flush_l2:
+        ms = 0.0
+        for _ in range(args.steps):
+            scrub.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            e1.synchronize()
+            ms += e0.elapsed_time(e1)
+    else:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1)
+    torch.cuda.synchronize()
+    barrier()
+    return max_over_ranks(ms, world, torch.device("cuda", local_rank))
 
 
 def run_ours(args, rank, world, local_rank):
@@ -316,30 +431,40 @@ def run_ours(args, rank, world, local_rank):
     from test_rnn_layer_b200 import tttmlp as L
 
     L.lib()   # loud failure if the CUDA library is missing
-    if args.kernels == "simt":
-        L.check(L.ttt_mlp_select_kernels(1, 1), "ttt_mlp_select_kernels")
+    sel = {"auto": None, "simt": (1, 1), "cluster": (2, 0), "split": (4, 0)}[args.kernels]
+    if sel:
+        L.check(L.ttt_mlp_select_kernels(*sel), "ttt_mlp_select_kernels")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = _workload(args)
-    inp = S.make_inputs(w, seed=rank_seed(rank), device=dev)
+    linear = args.model == "linear"
+    inp = (S.make_linear_inputs if linear else S.make_inputs)(w, seed=rank_seed(rank), device=dev)
     desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
     direction = L.DIRS[w.dirs]
-    ws = L.alloc_workspace(desc, w.b, direction, dev, host_io=True)
-    ws_dev_bytes = L.ttt_mlp_workspace_size(desc, w.b, direction)
+    if linear:
+        ws_dev_bytes = L.ttt_linear_workspace_size(desc, w.b, direction)
+        ws = torch.empty(ws_dev_bytes, dtype=torch.uint8, device=dev)
+    else:
+        ws = L.alloc_workspace(desc, w.b, direction, dev, host_io=True)
+        ws_dev_bytes = L.ttt_mlp_workspace_size(desc, w.b, direction)
     Y = torch.empty_like(inp["X"])
     stream = torch.cuda.current_stream()
 
-    def step():
-        st = L.ttt_mlp_forward(desc, inp["X"], inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W1_0"],
-                               inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"], Y, None, None,
-                               None, ws, ws_dev_bytes, stream)
+    def step(X=None, Yo=None):
+        X = inp["X"] if X is None else X
+        Yo = Y if Yo is None else Yo
+        if linear:
+            st = L.ttt_linear_forward(desc, X, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W_0"],
+                                      w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"], Yo, None, None, ws,
+                                      ws_dev_bytes, stream)
+        else:
+            st = L.ttt_mlp_forward(desc, X, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W1_0"],
+                                   inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"], Yo, None,
+                                   None, None, ws, ws_dev_bytes, stream)
         if st != L.TTT_OK:
-            raise L.TTTError(st, "ttt_mlp_forward")
+            raise L.TTTError(st, "ttt_linear_forward" if linear else "ttt_mlp_forward")
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
-
+    flush_l2 = _input_bytes(w) <= 126e6
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -349,19 +474,10 @@ def run_ours(args, rank, world, local_rank):
     sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
     sampler.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
     n_launch0 = L.ttt_launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    ms = _timed_steps(step, argparse.Namespace(warmup=0, steps=args.steps), world, local_rank, stream, flush_l2)
     launches = L.ttt_launch_count() - n_launch0
     clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
     ms_per_step = ms / args.steps
     value = whole_job_tokens_per_s(world, w.T, ms_per_step)
@@ -375,7 +491,8 @@ def run_ours(args, rank, world, local_rank):
     ktimes = L.ttt_kernel_times()
     L.ttt_kernel_timing(False)
     total = sum(v[0] for v in ktimes.values()) or 1.0
-    top = max(ktimes, key=lambda k: ktimes[k][0])
+    scans = [k for k in ktimes if k.startswith("scan")]
+    top = max(scans or ktimes, key=lambda k: ktimes[k][0]) if linear else max(ktimes, key=lambda k: ktimes[k][0])
     peaks = _peaks()
     roof = _roofline(top, ktimes[top][0] / ktimes[top][1], ktimes[top][1] / kpass, w, peaks, clocks)
     roof["share"] = round(ktimes[top][0] / total, 4)   # of the summed kernel time (streams overlap)
@@ -383,154 +500,97 @@ def run_ours(args, rank, world, local_rank):
     kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
                    "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
 
-    # end to end through the public host-buffer entry point: H2D of X, layer, D2H of Y
+    # end to end through the public API with pinned host buffers: H2D of X, layer, D2H of Y
     e2e = None
     if not args.no_e2e:
-        Xh = inp["X"].cpu().pin_memory()
-        Yh = torch.empty_like(Xh).pin_memory()
-        ns = max(1, min(args.steps, args.e2e_steps))
-
-        def e2e_step():
-            st = L.ttt_mlp_forward_host(desc, Xh, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W1_0"],
-                                        inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"], Yh, ws,
-                                        ws.numel(), stream)
-            L.check(st, "ttt_mlp_forward_host")
-
-        e2e_step()
-        barrier()
-        t0 = time.perf_counter()
-        for _ in range(ns):
-            e2e_step()
-        barrier()
-        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
-        nbytes = Xh.numel() * Xh.element_size()
-        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
-               "ms_per_step": e2e_s * 1e3, "steps": ns}
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu:
-        run, scale, threads, sample = _cpu_sample(w, args.cpu_tokens)
-        t = run()
-        cpu = {"value": args.cpu_tokens * scale / t, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": sample, "seconds": round(t, 2)}
-
-    if rank == 0:
-        scan_impl = "tensor-core" if any(k.endswith("_tc") for k in ktimes) else "simt"
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None,
-                "dtype": "bf16-in/tf32-mma/fp32-state" if scan_impl == "tensor-core" else "fp32",
-                "data": "synthetic",
-                "config": _config(w, {"kernels": scan_impl}), "gpu_launches": launches,
-                "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e, "cpu_baseline": cpu,
-                "impl": "ours"}
-        print(json.dumps(line), flush=True)
-    return 0
-
-
-def run_ours_linear(args, rank, world, local_rank):
-    """The TTT-Linear layer on the same sequence (fp32 scan), same JSON line."""
-    import torch
-
-    from test_rnn_layer_b200 import synth as S
-    from test_rnn_layer_b200 import tttmlp as L
-
-    L.lib()
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = _workload(args)
-    inp = S.make_linear_inputs(w, seed=rank_seed(rank), device=dev)
-    desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
-    direction = L.DIRS[w.dirs]
-    n_ws = L.ttt_linear_workspace_size(desc, w.b, direction)
-    ws = torch.empty(n_ws, dtype=torch.uint8, device=dev)
-    Y = torch.empty_like(inp["X"])
-    stream = torch.cuda.current_stream()
-
-    def step(X=None, Yo=None):
-        st = L.ttt_linear_forward(desc, inp["X"] if X is None else X, inp["theta_q"], inp["theta_k"],
-                                  inp["theta_v"], inp["W_0"], w.eta_eff, w.b, direction, inp["alpha_f"],
-                                  inp["alpha_r"], Y if Yo is None else Yo, None, None, ws, n_ws, stream)
-        L.check(st, "ttt_linear_forward")
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    L.check(L.ttt_mlp_status(ws, stream), "warm-up status")
-    uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
-    sampler.start()
-    time.sleep(0.3)
-    torch.cuda.synchronize()
-    n_launch0 = L.ttt_launch_count()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    launches = L.ttt_launch_count() - n_launch0
-    clocks = sampler.stop()
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
-    ms_per_step = ms / args.steps
-    value = whole_job_tokens_per_s(world, w.T, ms_per_step)
-
-    L.ttt_kernel_timing(True)
-    kpass = max(1, min(args.steps, 3))
-    for _ in range(kpass):
-        step()
-    torch.cuda.synchronize()
-    ktimes = L.ttt_kernel_times()
-    L.ttt_kernel_timing(False)
-    total = sum(v[0] for v in ktimes.values()) or 1.0
-    peaks = _peaks()
-    scan = "scan_linear_tc" if "scan_linear_tc" in ktimes else "scan_linear"
-    roof = _roofline(scan, ktimes[scan][0] / ktimes[scan][1], ktimes[scan][1] / kpass, w, peaks, clocks)
-    roof["share"] = round(ktimes[scan][0] / total, 4)
-    kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
-                   "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
-
-    e2e = None
-    if not args.no_e2e:   # pinned host X in, host Y out, through the device entry point
         Xh = inp["X"].cpu().pin_memory()
         Yh = torch.empty_like(Xh).pin_memory()
         Xd = torch.empty_like(inp["X"])
         ns = max(1, min(args.steps, args.e2e_steps))
 
         def e2e_step():
-            Xd.copy_(Xh, non_blocking=True)
-            step(Xd, Y)
-            Yh.copy_(Y, non_blocking=True)
-            L.check(L.ttt_mlp_status(ws, stream), "status")
+            if linear:   # the TTT-Linear layer has no host-buffer entry point: copies around the device call
+                Xd.copy_(Xh, non_blocking=True)
+                step(Xd, Y)
+                Yh.copy_(Y, non_blocking=True)
+                L.check(L.ttt_mlp_status(ws, stream), "status")
+            else:
+                st = L.ttt_mlp_forward_host(desc, Xh, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W1_0"],
+                                            inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"],
+                                            Yh, ws, ws.numel(), stream)
+                L.check(st, "ttt_mlp_forward_host")
 
         e2e_step()
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
         t0 = time.perf_counter()
         for _ in range(ns):
             e2e_step()
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
         e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
         nbytes = Xh.numel() * Xh.element_size()
-        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT,
-               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_s * 1e3,
-               "steps": ns}
+        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+               "d2h_bytes_per_step": nbytes, "ms_per_step": e2e_s * 1e3, "steps": ns}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        run, scale, threads, sample = _cpu_sample_linear(w, args.cpu_tokens)
-        t = run()
-        cpu = {"value": args.cpu_tokens * scale / t, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": sample, "seconds": round(t, 2)}
+        cpu = cpu_baseline(w, args)
+
     if rank == 0:
-        line = {"metric": METRIC_LINEAR, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None,
-                "dtype": "bf16-in/tf32-mma/fp32-state" if scan == "scan_linear_tc" else "bf16-in/fp32-scan",
-                "data": "synthetic",
-                "config": _config(w, {"model": "ttt-linear", "state": "W [64 x 64] fp32 per head"}),
-                "gpu_launches": launches, "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e,
-                "cpu_baseline": cpu, "impl": "ours"}
+        tc = any(k.endswith("_tc") or k.endswith("_tc2") for k in ktimes)
+        scan_name = next((k for k in ktimes if k.startswith("scan")), "")
+        if linear:
+            dtype = "bf16-in/tf32-mma/fp32-state" if tc else f"{w.dtype}-in/fp32-scan"
+        else:
+            dtype = "bf16-in/tf32-mma/fp32-state" if tc else "fp32"
+        line = {"metric": _metric(w, args.model), "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic", "config": _config(w),
+                "kernels_impl": "tensor-core" if tc else "simt", "gpu_launches": launches, "clocks": clocks,
+                "roofline": roof, "kernels": kernels, "e2e": e2e, "cpu_baseline": cpu, "impl": "ours"}
+        if w.b == 1:   # the per-token rule: the sequential chain per token
+            line["ns_per_token"] = ms_per_step * 1e6 / w.T
+            line["scan_ns_per_token"] = ktimes[scan_name][0] / kpass * 1e6 / (w.T * (2 if w.dirs == "bidir" else 1))
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_dry_host(args, rank, world):
+    """Host plumbing only (no GPU, no library): the rank layout, the process
+    group (gloo), the barrier-bracketed timing of `steps` steps that sleep
+    (10 ms x (rank + 1)), the maximum over ranks and rank 0's JSON line.
+    Used by the CPU tests of the launcher."""
+    import torch
+    import torch.distributed as dist
+    w = _workload(args)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.010 * (rank + 1))
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks((time.perf_counter() - t0) * 1e3, world, torch.device("cpu"))
+    if rank == 0:
+        ms_per_step = ms / args.steps
+        print(json.dumps({"metric": _metric(w, args.model), "value": whole_job_tokens_per_s(world, w.T, ms_per_step),
+                          "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": ms_per_step, "dry_run": True, "config": _config(w)}), flush=True)
+    return 0
+
+
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_command(argv, n: int, port: int) -> list:
+    """torch.distributed.run command that runs this script as n ranks on one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
 
 
 def main():
@@ -540,38 +600,50 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--model", choices=["mlp", "linear"], default="mlp")
-    ap.add_argument("--kernels", choices=["auto", "simt"], default="auto",
-                    help="simt: the fp32 SIMT scan and projection kernels (reference kernels)")
+    ap.add_argument("--workload", choices=WORKLOAD_NAMES, default="full63s")
+    ap.add_argument("--kernels", choices=["auto", "simt", "cluster", "split"], default="auto",
+                    help="simt: the fp32 SIMT scan and projection kernels (reference kernels); cluster / split: "
+                         "the two-CTA tensor-core scan with all warps on every stage / with state and output warp "
+                         "groups a chunk apart")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length (quick checks only)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-tokens", type=int, default=65536)
-    ap.add_argument("--ref-tokens", type=int, default=8192)
+    ap.add_argument("--sample-tokens", type=int, default=16384,
+                    help="tokens of the oracle's sample (reference arm and CPU baseline alike)")
+    ap.add_argument("--cpu-reps", type=int, default=4, help="passes of the oracle's sample for the CPU baseline")
+    ap.add_argument("--dry-run-host", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1 and args.impl == "ours":
+        # one process per GPU: start the ranks and wait for them (rank 0 prints the line)
+        return subprocess.call(spawn_command(sys.argv[1:], args.gpus, _free_port()))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
-    if world > 1:
-        import datetime
+    import datetime
 
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local_rank))
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        if args.dry_run_host:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        else:
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
     try:
-        if args.model == "linear":
-            return run_ours_linear(args, rank, world, local_rank)
+        if args.dry_run_host:
+            return run_dry_host(args, rank, world)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
-            import torch.distributed as dist
             dist.destroy_process_group()
 
 

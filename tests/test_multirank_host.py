@@ -56,3 +56,23 @@ def test_single_rank_bookkeeping_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
     assert bench.whole_job_tokens_per_s(1, 313344, 200.0) == pytest.approx(313344 / 0.2)
+
+
+def test_bench_starts_its_own_ranks_and_reports_the_slowest():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself; rank 0
+    alone prints the line, with n_gpus 2 and the slower rank's time (the host
+    plumbing only: each step sleeps 10 ms x (rank + 1), gloo, no GPU)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--steps", "3", "--warmup", "3", "--dry-run-host",
+                        "--workload", "tiny"], capture_output=True, text=True, timeout=240, cwd=root, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["n_gpus"] == 2 and line["dry_run"] is True
+    assert line["ms_per_step"] >= 20.0                       # the second rank sleeps 20 ms per step
+    assert line["value"] == pytest.approx(2 * 256 / (line["ms_per_step"] * 1e-3))
