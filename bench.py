@@ -208,6 +208,13 @@ def _algorithmic(w):
         # chunk form on the tensor cores: W K^T, W Q^T, update (3 x 2 d^2) + Q K^T and the masked
         # correction (2 x 2 b d over the causal half)
         "scan_linear_tc": ("tensor_tf32", H * T * (6 * d * d + 2 * b * d)),
+        # backward of the scan: the forward chunk recomputed plus its reverse-mode derivative, counted
+        # as three forward passes (the kernel does more: the state walk for the checkpoints and the
+        # rebuild of each segment's chunk-start states)
+        "scan_backward": ("alu", 3 * H * T * (7 * 2 * d * m + 2 * b * (d + m))),
+        # projections' gradients: dX += dU theta and dtheta += dU^T X for the three projections
+        "grad_gemm": ("alu", 2 * 3 * 2.0 * T * D * (d if w.per_head else D)),
+        "gate_backward": ("hbm", T * D * 16),
     }
 
 
@@ -538,10 +545,12 @@ def run_ours(args, rank, world, local_rank):
         cpu = cpu_baseline(w, args)
 
     if rank == 0:
-        tc = any(k.endswith("_tc") or k.endswith("_tc2") for k in ktimes)
+        tc = any("_tc" in k for k in ktimes)
         scan_name = next((k for k in ktimes if k.startswith("scan")), "")
         if linear:
             dtype = "bf16-in/tf32-mma/fp32-state" if tc else f"{w.dtype}-in/fp32-scan"
+        elif "scan_chunk_tc3" in ktimes:
+            dtype = "bf16-in/tf32+fp16-mma/fp32-state"
         else:
             dtype = "bf16-in/tf32-mma/fp32-state" if tc else "fp32"
         line = {"metric": _metric(w, args.model), "value": value, "unit": UNIT, "n_gpus": world,
@@ -554,6 +563,135 @@ def run_ours(args, rank, world, local_rank):
             line["scan_ns_per_token"] = ktimes[scan_name][0] / kpass * 1e6 / (w.T * (2 if w.dirs == "bidir" else 1))
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_backward(args, rank, world, local_rank):
+    """One training step of the layer: ttt_mlp_backward (the forward pass
+    recomputed inside, then the gradients of every input) for a seeded
+    upstream gradient dY; tokens/s of that step."""
+    import torch
+
+    from test_rnn_layer_b200 import synth as S
+    from test_rnn_layer_b200 import tttmlp as L
+
+    L.lib()
+    sel = {"auto": None, "simt": (1, 1), "cluster": (2, 0), "split": (4, 0)}[args.kernels]
+    if sel:
+        L.check(L.ttt_mlp_select_kernels(*sel), "ttt_mlp_select_kernels")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = _workload(args)
+    inp = S.make_inputs(w, seed=rank_seed(rank), device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    dY = torch.randn(inp["X"].shape, generator=gen, device=dev, dtype=torch.float32)
+    desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
+    direction = L.DIRS[w.dirs]
+    nbytes = L.ttt_mlp_backward_workspace_size(desc, w.b, direction)
+    if nbytes == 0:
+        raise L.TTTError(L.TTT_ERR_INVALID_ARG, "ttt_mlp_backward_workspace_size: " + L.ttt_last_error())
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    outs = [torch.empty(inp["X"].shape, **f32)] + [torch.empty(inp[k].shape, **f32) for k in
+                                                   ("theta_q", "theta_k", "theta_v", "W1_0", "W2_0")]
+    da_f, da_r = torch.empty(w.model_dim, **f32), torch.empty(w.model_dim, **f32)
+    stream = torch.cuda.current_stream()
+
+    def step(X=None, dy=None, dX=None):
+        st = L.ttt_mlp_backward(desc, inp["X"] if X is None else X, inp["theta_q"], inp["theta_k"], inp["theta_v"],
+                                inp["W1_0"], inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"],
+                                dY if dy is None else dy, outs[0] if dX is None else dX, *outs[1:], da_f, da_r, ws,
+                                nbytes, stream)
+        if st != L.TTT_OK:
+            raise L.TTTError(st, "ttt_mlp_backward")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    L.check(L.ttt_mlp_status(ws, stream), "warm-up status")
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    time.sleep(0.3)
+    n_launch0 = L.ttt_launch_count()
+    ms = _timed_steps(step, argparse.Namespace(warmup=0, steps=args.steps), world, local_rank, stream,
+                      _input_bytes(w) <= 126e6)
+    launches = L.ttt_launch_count() - n_launch0
+    clocks = sampler.stop()
+    L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
+    ms_per_step = ms / args.steps
+    L.ttt_kernel_timing(True)
+    step()
+    torch.cuda.synchronize()
+    ktimes = L.ttt_kernel_times()
+    L.ttt_kernel_timing(False)
+    total = sum(v[0] for v in ktimes.values()) or 1.0
+    top = max(ktimes, key=lambda k: ktimes[k][0])
+    roof = None
+    if top in _algorithmic(w):
+        roof = _roofline(top, ktimes[top][0] / ktimes[top][1], ktimes[top][1], w, _peaks(), clocks)
+        roof["share"] = round(ktimes[top][0] / total, 4)
+    kernels = {k: {"ms_per_step": round(v[0], 3), "launches_per_step": v[1], "share": round(v[0] / total, 4)}
+               for k, v in ktimes.items()}
+    e2e = None
+    if not args.no_e2e:   # X and dY from pinned host memory, dX back to it
+        Xh, dYh = inp["X"].cpu().pin_memory(), dY.cpu().pin_memory()
+        dXh = torch.empty(dYh.shape, dtype=torch.float32).pin_memory()
+        Xd, dYd = torch.empty_like(inp["X"]), torch.empty_like(dY)
+        ns = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            dYd.copy_(dYh, non_blocking=True)
+            step(Xd, dYd)
+            dXh.copy_(outs[0], non_blocking=True)
+            L.check(L.ttt_mlp_status(ws, stream), "status")
+
+        e2e_step()
+        t0 = time.perf_counter()
+        for _ in range(ns):
+            e2e_step()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
+        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": Xh.numel() * Xh.element_size() + dYh.numel() * 4,
+               "d2h_bytes_per_step": dXh.numel() * 4, "ms_per_step": e2e_s * 1e3, "steps": ns}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_backward(w, args)
+    if rank == 0:
+        line = {"metric": "TTT-MLP training step (forward + backward) " + _metric(w, "mlp"),
+                "value": whole_job_tokens_per_s(world, w.T, ms_per_step), "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "fp32-backward", "data": "synthetic",
+                "config": _config(w, {"step": "forward recomputed + backward of every input"}),
+                "gpu_launches": launches, "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e,
+                "cpu_baseline": cpu, "impl": "ours"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline_backward(w, args) -> dict:
+    """The backward oracle (fp64 autograd) on a bounded sample: the first
+    sample_tokens // 32 tokens (at most 512) of two heads."""
+    import numpy as np
+    import torch
+
+    from oracle import ttt_backward as B
+    from test_rnn_layer_b200 import synth as S
+
+    tokens = min(w.T, max(16, min(512, args.sample_tokens // 32)))
+    heads = min(w.H, 2)
+    ws = w.with_(T=tokens, H=heads, D=heads * w.d if not w.per_head else 0)
+    inp = S.make_inputs(ws, seed=0)
+    dY = np.random.default_rng(0).normal(size=tuple(inp["X"].shape))
+    t0 = time.perf_counter()
+    B.layer_backward({k: inp[k].double().numpy() for k in B.NAMES}, dY, w.eta_eff, w.b, w.dirs, w.per_head)
+    t = time.perf_counter() - t0
+    scale = heads / w.H
+    return {"value": tokens * scale / t, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+            "sample": f"first {tokens} tokens, {heads} of {w.H} heads (fp64 autograd of the oracle's forward, "
+                      f"{'the full width reduced to those heads' if not w.per_head else 'per-head inputs'}); "
+                      f"tokens/s scaled by {heads}/{w.H}", "seconds": round(t, 2), "cpu_model": cpu_model()}
 
 
 def run_dry_host(args, rank, world):
@@ -612,6 +750,8 @@ def main():
     ap.add_argument("--sample-tokens", type=int, default=16384,
                     help="tokens of the oracle's sample (reference arm and CPU baseline alike)")
     ap.add_argument("--cpu-reps", type=int, default=4, help="passes of the oracle's sample for the CPU baseline")
+    ap.add_argument("--backward", action="store_true",
+                    help="time one training step (forward recomputed + backward) instead of the forward layer")
     ap.add_argument("--dry-run-host", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -641,6 +781,8 @@ def main():
     try:
         if args.dry_run_host:
             return run_dry_host(args, rank, world)
+        if args.backward:
+            return run_backward(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -160,27 +160,62 @@ TTT_API ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_
                                 ttt_stream_t stream);
 
 /*
+ * Backward pass of the layer (training: the paper notes page, "损失函数 /
+ * 训练策略", fine-tunes the TTT layers and their gates): for a scalar loss with
+ * upstream gradient dY = dLoss/dY, the gradients with respect to X, theta_Q/K/V,
+ * W1_0, W2_0, alpha_f and alpha_r.  The layer's arguments are those of
+ * ttt_mlp_forward (1 <= b <= 64); the forward pass is recomputed inside.
+ *
+ *   dY        fp32, X's layout.
+ *   dX        fp32, X's layout.
+ *   dtheta_q/k/v  fp32, theta's layout ([H, d, d] or [H*d, D]).
+ *   dW1_0 [H, m, d], dW2_0 [H, d, m]  fp32.
+ *   dalpha_f, dalpha_r  fp32 [D]; required for the directions that use them
+ *             (may be NULL otherwise).
+ *   workspace ttt_mlp_backward_workspace_size(desc, b, dir) bytes, 256-byte
+ *             aligned; ttt_mlp_status(workspace, stream) reports non-finite
+ *             values and expired waits as for ttt_mlp_forward.
+ * Every gradient output is overwritten.  The scan's backward runs in fp32 on
+ * the SIMT cores (one CTA per head, the chunk-start states rebuilt from
+ * checkpoints every 32 chunks), the projections' gradients as fp32 GEMMs.
+ * Returns TTT_ERR_UNSUPPORTED for b > 64.
+ */
+TTT_API size_t ttt_mlp_backward_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
+TTT_API ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, const void* theta_q,
+                                    const void* theta_k, const void* theta_v, const float* W1_0, const float* W2_0,
+                                    float eta, int b, ttt_direction dir, const float* alpha_f,
+                                    const float* alpha_r, const float* dY, float* dX, float* dtheta_q,
+                                    float* dtheta_k, float* dtheta_v, float* dW1_0, float* dW2_0, float* dalpha_f,
+                                    float* dalpha_r, void* workspace, size_t workspace_bytes,
+                                    ttt_stream_t stream);
+
+/*
  * ttt_mlp_forward for callers that cannot allocate device memory.
  *
  * The paper has no counterpart: this is a deployment aid.  Code embedded in a
  * host framework that owns the allocator, plug-ins forbidden to call
  * cudaMalloc, or services that must not allocate after start-up cannot obtain
  * a workspace.  This entry point takes the same arguments as ttt_mlp_forward
- * except the workspace and runs the same kernels; its scratch is a fixed
- * 32 MiB array in the library's own device memory, held by every GPU that
- * loads the library until the process exits.
+ * except the workspace and runs the same kernels with the same arithmetic;
+ * its scratch is a fixed 32 MiB array in the library's own device memory,
+ * held by every GPU that loads the library until the process exits.
  *   - Shapes whose ttt_mlp_workspace_size exceeds 32 MiB are rejected with
  *     TTT_ERR_UNSUPPORTED and a message saying so.
- *   - It calls no cudaMalloc, cudaFree or other allocating routine.  (If the
- *     caller switched ttt_kernel_timing on, that hook still creates events.)
- *   - The first call on a device looks up the array's device address (once
- *     per device, with that device current); make that first call before any
- *     stream capture.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine, and it
+ *     creates no streams or events: every kernel runs on `stream` itself
+ *     (also for the full-width bf16 layer, which ttt_mlp_forward runs in
+ *     chunk segments on streams of its own).  If the caller switched
+ *     ttt_kernel_timing on, that hook still creates its timing events.
+ *   - The first call on a device (of this function or of
+ *     ttt_mlp_noalloc_status) looks up the array's device address, once per
+ *     device, with that device current; make that first call before any
+ *     stream capture.  The address is kept for the life of the process, so
+ *     these two functions must not be used after cudaDeviceReset.
  *   - Every call shares the one array and it keeps the last call's contents;
  *     the status word is cleared at the start of each call.  Calls whose GPU
  *     work overlaps (other streams, other host threads) race on it: order them.
- *   - Divergence and expired waits are recorded in that array but not
- *     reported: check the outputs for NaN/Inf where that matters.
+ *   - Divergence and expired waits are recorded in that array: read them with
+ *     ttt_mlp_noalloc_status.
  */
 TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void* X,
                                            const void* theta_q, const void* theta_k, const void* theta_v,
@@ -190,12 +225,22 @@ TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void*
                                            ttt_stream_t stream);
 
 /*
+ * ttt_mlp_status for ttt_mlp_forward_noalloc: synchronises `stream`, then
+ * reads and clears the status word in the library's fixed scratch array of
+ * the current device (TTT_OK, TTT_ERR_NONFINITE or TTT_ERR_TIMEOUT, as
+ * ttt_mlp_status).  The word belongs to the last no-alloc call on this device.
+ */
+TTT_API ttt_status ttt_mlp_noalloc_status(ttt_stream_t stream);
+
+/*
  * Kernel selection, process-wide (for tests and comparisons): 0 = automatic
  * (the fastest kernel that takes the shape), 1 = the FP32 SIMT kernels,
  * 2 = the tensor-core kernels (a later ttt_mlp_forward returns
  * TTT_ERR_UNSUPPORTED if the shape is outside them), and for the scan only
  * 3 = the tensor-core scan with one CTA per head instead of a two-CTA
- * cluster.  scan_impl selects the scan kernel, proj_impl the full-mode
+ * cluster, 4 = the two-CTA tensor-core scan whose CTAs each run the state
+ * chain and the output of the chunk before on separate warp groups.
+ * scan_impl selects the scan kernel, proj_impl the full-mode
  * projection kernel.
  */
 TTT_API ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl);

@@ -52,6 +52,13 @@ LaunchScope::~LaunchScope() {
 }
 
 static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
+
+// The split-group cluster scan applies the gate in its output group (1) or
+// leaves it to the separate gate kernel (0).
+#ifndef TTT_SPLIT_SCAN_GATES
+#define TTT_SPLIT_SCAN_GATES 0
+#endif
+constexpr bool kSplitScanGates = TTT_SPLIT_SCAN_GATES != 0;
 static std::atomic<int> g_inject_timeout{0};
 
 }  // namespace ttt
@@ -209,20 +216,28 @@ ScanArgs scan_args(const ttt_mlp_desc& q, const Layout& L, char* ws, const float
 ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W1_0, const float* W2_0,
                 float eta, int b, const Dir& dd, cudaStream_t s) {
     ScanArgs a = scan_args(q, L, ws, W1_0, W2_0, eta, b, dd);
-    // Kernel choice: the tf32 tensor-core scan serves bf16-input layers (whose
-    // tolerance is 2e-2); fp32-input layers keep the fp32 kernels unless the
-    // tensor-core kernel is requested explicitly.
+    // Kernel choice: the tensor-core scan (the split-group cluster kernel)
+    // serves bf16-input layers (whose tolerance is 2e-2); fp32-input layers
+    // keep the fp32 kernels unless a tensor-core kernel is requested explicitly.
     const int impl = g_scan_impl.load();
     const bool tc_ok = scan_chunk_tc_supported(q.d, b);
     if (impl == 2 && !tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
     if (impl == 3) {
         if (!tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
         CUDA_TRY(launch_scan_chunk_tc(a, s));
-    } else if (impl == 2 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+    } else if (impl == 2 || impl == 4 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
+        if (impl == 4 && !tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
+        const bool split = impl != 2;   // automatic: the split-group cluster scan
         a.Zscan = dd.zdbg ? dd.zdbg : reinterpret_cast<float*>(ws + L.zbuf);
-        CUDA_TRY(launch_scan_chunk_tc2(a, s));
-        CUDA_TRY(launch_gate(dd.xin, dd.xin_bf16, a.Zscan, dd.alpha, dd.out, dd.out_bf16, dd.delta, a.status, q.T,
-                             q.H, q.d, q.per_head_input, 0, s));
+        if (split && kSplitScanGates) {   // the split-group scan applies the gate itself
+            a.fuse_gate = 1;
+            CUDA_TRY(launch_scan_chunk_tc3(a, s));
+        } else {
+            if (split) CUDA_TRY(launch_scan_chunk_tc3(a, s));
+            else CUDA_TRY(launch_scan_chunk_tc2(a, s));
+            CUDA_TRY(launch_gate(dd.xin, dd.xin_bf16, a.Zscan, dd.alpha, dd.out, dd.out_bf16, dd.delta, a.status,
+                                 q.T, q.H, q.d, q.per_head_input, 0, s));
+        }
     } else if (b == 1 && impl != 1) {
         CUDA_TRY(launch_scan_token(a, s));
     } else {
@@ -252,6 +267,14 @@ Pipe g_pipes[64];
 
 constexpr int kPipeMinSegChunks = 16;
 constexpr int kPipeSmMargin = 8;
+// When the scan applies the gate itself, the projections of the segments that
+// cover the first kPipeFrontPercent of a direction's chunks run on the whole
+// GPU before that direction's scan starts (a head start: the scan then walks
+// faster than the projection can follow on the SMs the scan leaves free).
+#ifndef TTT_PIPE_FRONT_PERCENT
+#define TTT_PIPE_FRONT_PERCENT 30
+#endif
+constexpr int kPipeFrontPercent = TTT_PIPE_FRONT_PERCENT;
 
 // Chunk ranges [begin, end) of a walk over `nchunks` chunks: segments grow
 // by 3/2 from 16 chunks at both ends (short exposed head and tail: 16, 24,
@@ -298,7 +321,7 @@ int pipe_side_sms(const ttt_mlp_desc& q, int scan_sms_per_head) {
 bool pipe_eligible(const ttt_mlp_desc& q, const Layout& L, int b, ttt_direction dir) {
     const int si = g_scan_impl.load(), pi = g_proj_impl.load();
     if (q.per_head_input || q.x_dtype != TTT_BF16) return false;
-    if (!(si == 0 || si == 2) || !scan_chunk_tc_supported(q.d, b)) return false;
+    if (!(si == 0 || si == 2 || si == 4) || !scan_chunk_tc_supported(q.d, b)) return false;
     if (pi == 1 || !proj_full_tc_supported(q.D, q.D)) return false;
     if (dir == TTT_BIDIR && !L.split_reverse) return false;
     return pipe_side_sms(q, 2) > 0;
@@ -319,7 +342,7 @@ using SegScan = std::function<cudaError_t(int di, const struct Dir& dd, int c_be
 ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_sms_per_head, const SegScan& seg_scan,
                              const void* X, const void* const th[3], float* const qkv[3], int b, ttt_direction dir,
                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, cudaStream_t s,
-                             const void* X_host, void* Y_host) {
+                             const void* X_host, void* Y_host, bool scan_gates = false) {
     std::lock_guard<std::mutex> lk(g_pipe_mu);
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
@@ -355,6 +378,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_
     auto enqueue = [&]() -> ttt_status {
         const size_t n = (size_t)q.T * q.D;
         const int D = q.D;
+        cudaEvent_t prev_dir_done = nullptr;   // the previous direction's last scan segment
         float* xp = B.xp;
         __nv_bfloat16* delta = B.delta;
         int* status = B.status;
@@ -392,28 +416,45 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_
                     CUDA_TRY(cudaEventRecord(ev_h2d[k], P.copy));
                 }
             }
-            // projections (the first runs alone on the whole GPU)
+            // projections: the first runs alone on the whole GPU (with a gating scan, the segments of the
+            // first kPipeFrontPercent of the chunks); the reverse ones after the forward scan wrote X'
+            if (prev_dir_done) CUDA_TRY(cudaStreamWaitEvent(P.side, prev_dir_done, 0));
+            const int front_chunks = scan_gates ? nch * kPipeFrontPercent / 100 : 0;
+            int last_front = 0;   // the first scan segment waits for the projections of the head start
+            for (int k = 0; k < ns; ++k)
+                if (seg[k].second <= front_chunks) last_front = k;
             for (int k = 0; k < ns; ++k) {
                 int r0, r1;
                 rows(k, r0, r1);
                 if (copy_in) CUDA_TRY(cudaStreamWaitEvent(P.side, ev_h2d[k], 0));
                 const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
                 float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
-                CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, k == 0 ? 0 : side_sms, P.side));
+                const bool whole_gpu = k == 0 || seg[k].second <= front_chunks;
+                CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, whole_gpu ? 0 : side_sms, P.side));
                 CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
             }
             // scan segments, the state carried by the launcher
             for (int k = 0; k < ns; ++k) {
-                CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k], 0));
+                CUDA_TRY(cudaStreamWaitEvent(P.scan, ev_proj[k == 0 ? last_front : k], 0));
                 CUDA_TRY(seg_scan(di, dd, seg[k].first, seg[k].second, k == 0, k == ns - 1, zscan, P.scan));
                 CUDA_TRY(cudaEventRecord(ev_scan[k], P.scan));
             }
-            // gates, each after its segment's scan
+            prev_dir_done = ev_scan[ns - 1];
+            // gates, each after its segment's scan (or in the scan itself)
             for (int k = 0; k < ns; ++k) {
                 int r0, r1;
                 rows(k, r0, r1);
-                CUDA_TRY(cudaStreamWaitEvent(P.side, ev_scan[k], 0));
                 const size_t o = (size_t)r0 * D;
+                if (scan_gates) {
+                    if (copy_out) {
+                        CUDA_TRY(cudaStreamWaitEvent(P.copy, ev_scan[k], 0));
+                        CUDA_TRY(cudaMemcpyAsync(static_cast<char*>(Y_host) + o * 2,
+                                                 static_cast<const char*>(Y) + o * 2, (size_t)(r1 - r0) * D * 2,
+                                                 cudaMemcpyDeviceToHost, P.copy));
+                    }
+                    continue;
+                }
+                CUDA_TRY(cudaStreamWaitEvent(P.side, ev_scan[k], 0));
                 const void* xin = static_cast<const char*>(dd.xin) + o * (dd.xin_bf16 ? 2 : 4);
                 void* out = static_cast<char*>(dd.out) + o * (dd.out_bf16 ? 2 : 4);
                 const bool last = k == ns - 1;
@@ -471,7 +512,7 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
                         const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
                         ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
                         float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes, ttt_stream_t stream_,
-                        const void* X_host, void* Y_host) {
+                        const void* X_host, void* Y_host, bool allow_pipeline = true) {
     ttt_status st = check_desc(desc, b, dir);
     if (st != TTT_OK) return st;
     const ttt_mlp_desc& q = *desc;
@@ -505,11 +546,12 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
     float* xp = reinterpret_cast<float*>(ws + L.xp);
     int* status = reinterpret_cast<int*>(ws + L.status);
 
-    if (pipe_eligible(q, L, b, dir)) {
+    if (allow_pipeline && pipe_eligible(q, L, b, dir)) {
         // the cluster scan, the state W1, W2 carried between segments through the workspace
         const size_t nW = (size_t)q.H * q.m * q.d;
         float* st1 = reinterpret_cast<float*>(ws + L.state);
         float* st2 = st1 + nW;
+        const bool split_groups = g_scan_impl.load() != 2;   // automatic: the split-group cluster scan
         const SegScan seg_scan = [&](int di, const Dir& dd, int cb, int ce, bool first, bool last, float* zscan,
                                      cudaStream_t ss) {
             ScanArgs a = scan_args(q, L, ws, first ? W1_0 : st1, first ? W2_0 : st2, eta, b, dd);
@@ -518,12 +560,16 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
             a.c_end = ce;
             a.W1_T = last ? (W1_T ? W1_T + di * nW : nullptr) : st1;
             a.W2_T = last ? (W2_T ? W2_T + di * nW : nullptr) : st2;
+            if (split_groups) {
+                a.fuse_gate = kSplitScanGates ? 1 : 0;
+                return launch_scan_chunk_tc3(a, ss);
+            }
             return launch_scan_chunk_tc2(a, ss);
         };
         const PipeBufs bufs{status, xp, reinterpret_cast<__nv_bfloat16*>(ws + L.delta),
                             reinterpret_cast<float*>(ws + L.zbuf)};
         return forward_pipelined(q, bufs, 2, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, X_host,
-                                 Y_host);
+                                 Y_host, split_groups && kSplitScanGates);
     }
     if (X_host) CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(X), X_host, xbytes, cudaMemcpyHostToDevice, s));
     auto finish = [&]() -> ttt_status {
@@ -566,6 +612,58 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
     st = scan(q, L, ws, W1_0, W2_0, eta, b, d1, s);
     if (st != TTT_OK) return st;
     return finish();
+}
+
+}  // namespace
+
+ttt_status ttt::forward_single_stream(const ttt_mlp_desc* desc, const void* X, const void* theta_q,
+                                      const void* theta_k, const void* theta_v, const float* W1_0, const float* W2_0,
+                                      float eta, int b, ttt_direction dir, const float* alpha_f,
+                                      const float* alpha_r, void* Y, float* Z_out, float* W1_T, float* W2_T,
+                                      void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+    return forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W1_T,
+                        W2_T, workspace, workspace_bytes, stream, nullptr, nullptr, false);
+}
+
+namespace {
+
+// ---------------------------------------------------------------- backward pass
+struct BwdLayout {
+    size_t fwd, y, zs, xp, u[3], du[3], g, dz, scratch, total;
+};
+
+BwdLayout plan_backward(const ttt_mlp_desc& q, int b, ttt_direction dir) {
+    BwdLayout L{};
+    const size_t n = (size_t)q.T * q.D;
+    const int nd = dir == TTT_BIDIR ? 2 : 1;
+    size_t off = 0;
+    L.fwd = off; off = align_up(off + plan(q, b, dir).total);
+    L.y = off; off = align_up(off + n * elem_size(q.x_dtype));
+    L.zs = off; off = align_up(off + nd * n * sizeof(float));
+    L.xp = off; if (dir == TTT_BIDIR) off = align_up(off + n * sizeof(float));
+    for (int w = 0; w < 3; ++w) { L.u[w] = off; off = align_up(off + n * sizeof(float)); }
+    for (int w = 0; w < 3; ++w) { L.du[w] = off; off = align_up(off + n * sizeof(float)); }
+    L.g = off; off = align_up(off + n * sizeof(float));
+    L.dz = off; off = align_up(off + n * sizeof(float));
+    L.scratch = off; off = align_up(off + (size_t)q.H * scan_backward_scratch_floats(q.d, b, q.T) * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// dX += dU theta (X layout) and dtheta += dU^T src, for one projection.
+ttt_status projection_grads(const ttt_mlp_desc& q, const float* dU, const void* theta, int th_bf16, const void* src,
+                            int src_bf16, float* G, float* dtheta, cudaStream_t s) {
+    const long long T = q.T, D = q.D, d = q.d;
+    if (q.per_head_input) {   // per head: U[h] [T x d] = X[h] theta[h]^T
+        CUDA_TRY(launch_grad_gemm(G, d, T * d, dU, 0, d, 1, T * d, theta, th_bf16, d, 1, d * d, q.H, (int)T, (int)d, d,
+                                  1, s));
+        CUDA_TRY(launch_grad_gemm(dtheta, d, d * d, dU, 0, 1, d, T * d, src, src_bf16, d, 1, T * d, q.H, (int)d,
+                                  (int)d, T, 1, s));
+    } else {                  // full width: U [T x D] = X theta^T, theta [D x D]
+        CUDA_TRY(launch_grad_gemm(G, D, 0, dU, 0, D, 1, 0, theta, th_bf16, D, 1, 0, 1, (int)T, (int)D, D, 1, s));
+        CUDA_TRY(launch_grad_gemm(dtheta, D, 0, dU, 0, 1, D, 0, src, src_bf16, D, 1, 0, 1, (int)D, (int)D, T, 1, s));
+    }
+    return TTT_OK;
 }
 
 }  // namespace
@@ -733,6 +831,94 @@ ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const voi
                             x_bf16, nullptr, Z_out ? Z_out + n : nullptr, W_T ? W_T + nW : nullptr, s);
 }
 
+size_t ttt_mlp_backward_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc(desc, b, dir) != TTT_OK) return 0;
+    if (b > 64) {
+        fail(TTT_ERR_UNSUPPORTED, "backward pass: chunk size b=%d above 64", b);
+        return 0;
+    }
+    return plan_backward(*desc, b, dir).total;
+}
+
+ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                            const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                            ttt_direction dir, const float* alpha_f, const float* alpha_r, const float* dY, float* dX,
+                            float* dtheta_q, float* dtheta_k, float* dtheta_v, float* dW1_0, float* dW2_0,
+                            float* dalpha_f, float* dalpha_r, void* workspace, size_t workspace_bytes,
+                            ttt_stream_t stream_) {
+    ttt_status st = check_desc(desc, b, dir);
+    if (st != TTT_OK) return st;
+    const ttt_mlp_desc& q = *desc;
+    if (b > 64) return fail(TTT_ERR_UNSUPPORTED, "backward pass: chunk size b=%d above 64", b);
+    st = check_ptrs(q, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, dir, alpha_f, alpha_r);
+    if (st != TTT_OK) return st;
+    const bool uses_f = dir != TTT_REV, uses_r = dir != TTT_FWD;
+    if (!dY || !dX || !dtheta_q || !dtheta_k || !dtheta_v || !dW1_0 || !dW2_0 || (uses_f && !dalpha_f) ||
+        (uses_r && !dalpha_r) || !workspace)
+        return fail(TTT_ERR_INVALID_ARG, "dY, every gradient output of this direction and workspace must be non-NULL");
+    const void* ps[] = {dY, dX, dtheta_q, dtheta_k, dtheta_v, dW1_0, dW2_0, dalpha_f, dalpha_r};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const BwdLayout B = plan_backward(q, b, dir);
+    if (workspace_bytes < B.total)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, B.total);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    char* ws = static_cast<char*>(workspace);
+    const size_t n = (size_t)q.T * q.D;
+    const int x_bf16 = q.x_dtype == TTT_BF16;
+    float* zs = reinterpret_cast<float*>(ws + B.zs);
+
+    // the forward pass, keeping each direction's z (its status word lands at the workspace start)
+    st = forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, ws + B.y, zs,
+                      nullptr, nullptr, ws + B.fwd, plan(q, b, dir).total, stream_, nullptr, nullptr);
+    if (st != TTT_OK) return st;
+    int* status = reinterpret_cast<int*>(ws + B.fwd);
+    const size_t th_elems = q.per_head_input ? (size_t)q.H * q.d * q.d : (size_t)q.D * q.D;
+    const size_t w_elems = (size_t)q.H * q.m * q.d;
+    float* dth[3] = {dtheta_q, dtheta_k, dtheta_v};
+    for (float* p : dth) CUDA_TRY(cudaMemsetAsync(p, 0, th_elems * sizeof(float), s));
+    CUDA_TRY(cudaMemsetAsync(dW1_0, 0, w_elems * sizeof(float), s));
+    CUDA_TRY(cudaMemsetAsync(dW2_0, 0, w_elems * sizeof(float), s));
+    if (dalpha_f && uses_f) CUDA_TRY(cudaMemsetAsync(dalpha_f, 0, q.D * sizeof(float), s));
+    if (dalpha_r && uses_r) CUDA_TRY(cudaMemsetAsync(dalpha_r, 0, q.D * sizeof(float), s));
+    float* G = reinterpret_cast<float*>(ws + B.g);   // gradient with respect to the current gate's output
+    CUDA_TRY(cudaMemcpyAsync(G, dY, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    float* xp = reinterpret_cast<float*>(ws + B.xp);
+    if (dir == TTT_BIDIR)   // X' = X + tanh(alpha_f) z_f, the reverse direction's input
+        CUDA_TRY(launch_gate(X, x_bf16, zs, alpha_f, xp, 0, nullptr, status, q.T, q.H, q.d, q.per_head_input, 0, s));
+    const void* th[3] = {theta_q, theta_k, theta_v};
+    float* U[3] = {reinterpret_cast<float*>(ws + B.u[0]), reinterpret_cast<float*>(ws + B.u[1]),
+                   reinterpret_cast<float*>(ws + B.u[2])};
+    float* dU[3] = {reinterpret_cast<float*>(ws + B.du[0]), reinterpret_cast<float*>(ws + B.du[1]),
+                    reinterpret_cast<float*>(ws + B.du[2])};
+    float* dz = reinterpret_cast<float*>(ws + B.dz);
+    const long long qkv_hs = q.per_head_input ? (long long)q.T * q.d : q.d;
+    const long long qkv_ts = q.per_head_input ? q.d : q.D;
+    // directions from the last to the first
+    const int ndir = dir == TTT_BIDIR ? 2 : 1;
+    for (int k = ndir - 1; k >= 0; --k) {
+        const bool reverse = dir == TTT_REV || k == 1;
+        const bool on_xp = dir == TTT_BIDIR && k == 1;
+        const void* src = on_xp ? static_cast<const void*>(xp) : X;
+        const int src_bf16 = on_xp ? 0 : x_bf16;
+        CUDA_TRY(launch_gate_backward(G, zs + k * n, reverse ? alpha_r : alpha_f, dz, reverse ? dalpha_r : dalpha_f,
+                                      q.T, q.H, q.d, q.per_head_input, s));
+        st = project(q, src, src_bf16, th, U, 0, status, s);
+        if (st != TTT_OK) return st;
+        CUDA_TRY(launch_scan_backward(U[0], U[1], U[2], qkv_hs, qkv_ts, dz, qkv_hs, qkv_ts, W1_0, W2_0, dU[0], dU[1],
+                                      dU[2], dW1_0, dW2_0, reinterpret_cast<float*>(ws + B.scratch), q.T, q.H, q.d, b,
+                                      reverse ? 1 : 0, eta, s));
+        for (int w = 0; w < 3; ++w) {   // the gate's x path keeps G; the projections add theta's share
+            st = projection_grads(q, dU[w], th[w], x_bf16, src, src_bf16, G, dth[w], s);
+            if (st != TTT_OK) return st;
+        }
+    }
+    CUDA_TRY(cudaMemcpyAsync(dX, G, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+    return TTT_OK;
+}
+
 ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {
     if (!workspace) return fail(TTT_ERR_INVALID_ARG, "workspace is NULL");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
@@ -769,10 +955,10 @@ ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, co
 }
 
 ttt_status ttt_mlp_select_kernels(int scan_impl, int proj_impl) {
-    if (scan_impl < 0 || scan_impl > 3 || proj_impl < 0 || proj_impl > 2)
+    if (scan_impl < 0 || scan_impl > 4 || proj_impl < 0 || proj_impl > 2)
         return fail(TTT_ERR_INVALID_ARG,
                     "kernel selector must be 0 (auto), 1 (SIMT), 2 (tensor core) or, for the scan, 3 (tensor core, "
-                    "one CTA per head)");
+                    "one CTA per head) or 4 (tensor core, two warp groups per CTA)");
     g_scan_impl.store(scan_impl);
     g_proj_impl.store(proj_impl);
     return TTT_OK;

@@ -42,6 +42,7 @@ struct ScanArgs {
     int c_begin, c_end;     // cluster scan: chunks [c_begin, c_end) of the walk (c_end 0: to the end);
                             // state from W1_0/W2_0, final state to W1_T/W2_T
     long long scratch_per_head;  // floats
+    int fuse_gate;          // split-group cluster scan: apply the gate itself (Out, Delta, Zdbg; no Zscan)
 };
 
 // Scan kernels.  Each returns a cudaError_t from the launch.
@@ -52,6 +53,10 @@ long long scan_chunk_simt_scratch_floats(int d, int m, int b);
 bool scan_chunk_tc_supported(int d, int b);
 cudaError_t launch_scan_chunk_tc(const ScanArgs& a, cudaStream_t s);    // one CTA per head
 cudaError_t launch_scan_chunk_tc2(const ScanArgs& a, cudaStream_t s);   // a cluster of two CTAs per head
+// A cluster of two CTAs per head, each split into a state warp group and an
+// output warp group that run one chunk apart (fp16 operands for the products
+// of thread-produced values, tf32 for those that read the fp32 state).
+cudaError_t launch_scan_chunk_tc3(const ScanArgs& a, cudaStream_t s);
 
 // TTT-Linear scan (f(u; W) = W u, W [d x d] per head): z of one direction into Z
 // (X's layout); state from W_0 [H, d, d], final state to W_T (optional).
@@ -94,6 +99,31 @@ cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float
 cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* alpha, void* Out, int out_bf16,
                         __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, int max_blocks,
                         cudaStream_t s);
+
+// ttt_mlp_forward with every kernel on `stream` itself: the same kernels and
+// arithmetic, but never the chunk-segment schedule on the library's own
+// streams, so that the call creates no streams or events.
+ttt_status forward_single_stream(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                                 const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                                 ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
+                                 float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes,
+                                 ttt_stream_t stream);
+
+// Backward pass of one direction of the scan (fp32, b <= 64, d = 16/32/64):
+// dQ, dK, dV (qkv layout) from dZ (X layout); dW1, dW2 [H, m, d] / [H, d, m]
+// accumulated; scratch of H * scan_backward_scratch_floats(d, b, T) floats.
+long long scan_backward_scratch_floats(int d, int b, int T);
+cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V, long long qkv_hs, long long qkv_ts,
+                                 const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
+                                 const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
+                                 float* scratch, int T, int H, int d, int b, int reverse, float eta, cudaStream_t s);
+// Gate backward: dz = tanh(alpha) g, dalpha += (1 - tanh^2 alpha) sum_t g z (per channel).
+cudaError_t launch_gate_backward(const float* g, const float* z, const float* alpha, float* dz, float* dalpha, int T,
+                                 int H, int d, int per_head, cudaStream_t s);
+// Batched GEMM C[b] (+)= A[b] [M x K] B[b] [K x N] (fp32 C row-major; A, B bf16 or fp32 via strides).
+cudaError_t launch_grad_gemm(float* C, long long ldc, long long cbs, const void* A, int a_bf16, long long a_rs,
+                             long long a_cs, long long a_bs, const void* B, int b_bf16, long long b_rs, long long b_cs,
+                             long long b_bs, int batch, int M, int N, long long K, int accumulate, cudaStream_t s);
 
 // Records a message for ttt_last_error() on this thread and returns `code`.
 ttt_status set_error(ttt_status code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));

@@ -4,11 +4,13 @@
 // Some callers have no way to obtain a device workspace: code running inside a
 // host framework whose allocator it does not own, plug-ins that may not call
 // cudaMalloc, or environments that forbid allocation after start-up.  This
-// entry point runs exactly the same kernels as ttt_mlp_forward, but its
-// scratch (the Q/K/V streams, X', the chunk intermediates and the status word)
-// lives in one fixed-size array in the library's own device memory instead of
-// a caller-provided workspace.  Every GPU that loads the library holds that
-// array (kNoAllocBytes) until the process exits.
+// entry point runs the same kernels as ttt_mlp_forward, but its scratch (the
+// Q/K/V streams, X', the chunk intermediates and the status word) lives in one
+// fixed-size array in the library's own device memory instead of a
+// caller-provided workspace.  Every GPU that loads the library holds that
+// array (kNoAllocBytes) until the process exits.  Every kernel runs on the
+// caller's stream (never the chunk-segment schedule on the library's own
+// streams), so a call creates no streams or events either.
 #include <mutex>
 
 #include "../../include/tttmlp.h"
@@ -27,6 +29,24 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 std::mutex g_mu;
 void* g_ptr[kMaxDevices] = {};
 
+// Device address of the scratch on the current device, looked up once per
+// device (with that device current) and kept for the life of the process.
+ttt_status scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return ttt::set_error(TTT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return ttt::set_error(TTT_ERR_UNSUPPORTED, "device index %d too large", dev);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return ttt::set_error(TTT_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        g_ptr[dev] = p;
+    }
+    *out = g_ptr[dev];
+    return TTT_OK;
+}
+
 }  // namespace
 
 extern "C" TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, const void* X, const void* theta_q,
@@ -42,24 +62,16 @@ extern "C" TTT_API ttt_status ttt_mlp_forward_noalloc(const ttt_mlp_desc* desc, 
                               "library's fixed %zu bytes; use ttt_mlp_forward with a caller workspace",
                               need, kNoAllocBytes);
     }
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return ttt::set_error(TTT_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kMaxDevices) return ttt::set_error(TTT_ERR_UNSUPPORTED, "device index %d too large", dev);
     void* ws = nullptr;
-    {
-        // One-time set-up per device, with that device current: the device
-        // address of the static scratch.
-        std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_ptr[dev]) {
-            void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-            if (e != cudaSuccess)
-                return ttt::set_error(TTT_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-            g_ptr[dev] = p;
-        }
-        ws = g_ptr[dev];
-    }
-    return ttt_mlp_forward(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out,
-                           W1_T, W2_T, ws, kNoAllocBytes, stream);
+    const ttt_status st = scratch_address(&ws);
+    if (st != TTT_OK) return st;
+    return ttt::forward_single_stream(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, dir, alpha_f, alpha_r,
+                                      Y, Z_out, W1_T, W2_T, ws, kNoAllocBytes, stream);
+}
+
+extern "C" TTT_API ttt_status ttt_mlp_noalloc_status(ttt_stream_t stream) {
+    void* ws = nullptr;
+    const ttt_status st = scratch_address(&ws);
+    if (st != TTT_OK) return st;
+    return ttt_mlp_status(ws, stream);
 }

@@ -1,0 +1,363 @@
+// Backward pass of one direction of the TTT-MLP scan (fp32 SIMT, any b <= 64,
+// d = 16, 32 or 64): given dZ = dLoss/dz for every token, the gradients with
+// respect to the token streams Q, K, V and the initial state W1_0, W2_0.
+//
+// The forward chunk (paper notes page, "关键设计 / TTT-MLP 层"; n tokens in
+// walking order, state W1 [m x d], W2 [d x m] at the chunk start, rows of the
+// matrices below are tokens, tril keeps s <= t in walking order):
+//   A = K W1^T, G = GELU(A), Y = G W2^T, D2 = -2 eta (Y - V), P = D2 W2,
+//   Dl = P * GELU'(A),  W1' = W1 + Dl^T K,  W2' = W2 + D2^T G,
+//   Mk = tril(Q K^T), Aq = Q W1^T + Mk Dl, Gq = GELU(Aq),
+//   Ng = tril(Gq G^T), Z = Gq W2^T + Ng D2
+// is differentiated by hand (reverse-mode chain rule; GELU'' = phi (2 - a^2)),
+// given dZ of the chunk and the gradient with respect to the chunk-end state
+// (carried backward from the next chunk):
+//   dW2 += dZ^T Gq,  dGq = dZ W2 + tril(dZ D2^T) G,  dD2 = Ng^T dZ,  dG = tril(dZ D2^T)^T Gq,
+//   dAq = dGq * GELU'(Aq),  dQ = dAq W1 + tril(dAq Dl^T) K,  dK = tril(dAq Dl^T)^T Q,
+//   dDl = Mk^T dAq + K dW1'^T,  dK += Dl dW1',  dD2 += G dW2'^T,  dG += D2 dW2',
+//   dP = dDl * GELU'(A),  dA = dDl * P * GELU''(A),  dD2 += dP W2^T,
+//   dE = -2 eta dD2,  dV = -dE,  dG += dE W2,  dA += dG * GELU'(A),  dK += dA W1,
+//   dW1 = dW1' + dAq^T Q + dA^T K,  dW2 = dW2' + dZ^T Gq + D2^T dP + dE^T G.
+// The chunk-start states come from checkpoints: the kernel first walks the
+// sequence forward (state updates only) keeping the state every kCkpt chunks,
+// then, segment by segment from the end, rebuilds the segment's chunk-start
+// states from its checkpoint and runs the chunks' backward steps in reverse.
+//
+// One CTA of 512 threads per head; the matrices of a chunk live in a per-head
+// scratch area in global memory (it stays in L2); every product is a block
+// GEMM tiled through shared memory.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ttt {
+namespace {
+
+constexpr int NT = 512;          // threads per CTA
+constexpr int BMAX = 64;         // largest chunk
+constexpr int kCkpt = 32;        // chunks between two checkpoints
+constexpr int TM = 64, TN = 64, TK = 16;   // GEMM tile
+
+struct BwdArgs {
+    const float* Q;
+    const float* K;
+    const float* V;
+    long long qkv_hs, qkv_ts;
+    const float* dZ;             // [tokens] in the X layout
+    long long x_hs, x_ts;
+    const float* W1_0;           // [H, m, d]
+    const float* W2_0;           // [H, d, m]
+    float* dQ;                   // qkv layout (written)
+    float* dK;
+    float* dV;
+    float* dW1;                  // [H, m, d] (accumulated)
+    float* dW2;                  // [H, d, m] (accumulated)
+    float* scratch;              // per head: scratch_per_head floats
+    long long scratch_per_head;
+    int T, H, d, b, reverse;
+    float eta;
+};
+
+// Per-head scratch layout (floats).
+struct Scratch {
+    float *W1, *W2;              // running state
+    float *dW1, *dW2;            // carried state gradient
+    float *ck;                   // checkpoints: [nck][2 m d]
+    float *seg;                  // chunk-start states of one segment: [kCkpt][2 m d]
+    // chunk matrices
+    float *Qc, *Kc, *Vc, *dZc;                 // [n x d]
+    float *A, *G, *P, *Dl, *Aq, *Gq;           // [n x m]
+    float *dA, *dG, *dGq, *dDl;                // [n x m]
+    float *D2, *dD2, *dQc, *dKc;               // [n x d]
+    float *Mk, *Ng, *dNg, *dMk;                // [n x n]
+};
+
+__host__ __device__ inline long long scratch_floats_for(int d, int b, int T) {
+    const long long m = 4LL * d, md = m * d;
+    const long long nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
+    return 4 * md + nck * 2 * md + kCkpt * 2 * md + 4LL * BMAX * d + 10LL * BMAX * m + 4LL * BMAX * d +
+           4LL * BMAX * BMAX + 64;
+}
+
+__device__ Scratch carve(float* base, int d, int nck) {
+    const long long m = 4LL * d, md = m * d;
+    Scratch s;
+    float* p = base;
+    s.W1 = p; p += md;
+    s.W2 = p; p += md;
+    s.dW1 = p; p += md;
+    s.dW2 = p; p += md;
+    s.ck = p; p += (long long)nck * 2 * md;
+    s.seg = p; p += (long long)kCkpt * 2 * md;
+    s.Qc = p; p += BMAX * d;
+    s.Kc = p; p += BMAX * d;
+    s.Vc = p; p += BMAX * d;
+    s.dZc = p; p += BMAX * d;
+    s.A = p; p += BMAX * m;
+    s.G = p; p += BMAX * m;
+    s.P = p; p += BMAX * m;
+    s.Dl = p; p += BMAX * m;
+    s.Aq = p; p += BMAX * m;
+    s.Gq = p; p += BMAX * m;
+    s.dA = p; p += BMAX * m;
+    s.dG = p; p += BMAX * m;
+    s.dGq = p; p += BMAX * m;
+    s.dDl = p; p += BMAX * m;
+    s.D2 = p; p += BMAX * d;
+    s.dD2 = p; p += BMAX * d;
+    s.dQc = p; p += BMAX * d;
+    s.dKc = p; p += BMAX * d;
+    s.Mk = p; p += BMAX * BMAX;
+    s.Ng = p; p += BMAX * BMAX;
+    s.dNg = p; p += BMAX * BMAX;
+    s.dMk = p; p += BMAX * BMAX;
+    return s;
+}
+
+// A matrix operand: element (r, c) of op(X) at X[r * rs + c * cs].
+struct Mat {
+    const float* p;
+    int rs, cs;
+    __device__ float at(int r, int c) const { return p[(long long)r * rs + (long long)c * cs]; }
+};
+__device__ __forceinline__ Mat N_(const float* p, int ld) { return Mat{p, ld, 1}; }   // row-major as is
+__device__ __forceinline__ Mat T_(const float* p, int ld) { return Mat{p, 1, ld}; }   // transposed view
+
+// C[M x N] (+)= alpha * A[M x Kd] B[Kd x N], C row-major with leading dimension ldc.
+// mask: 0 none, 1 keep C[r][c] only for c <= r (lower triangle incl. diagonal).
+// All threads of the CTA call it; it ends with a barrier.
+__device__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha, bool accumulate,
+                     int mask = 0) {
+    __shared__ float sA[TK][TM + 1], sB[TK][TN + 1];
+    const int tid = threadIdx.x;
+    const int tr = tid / 16, tc = tid % 16;          // 32 x 16 threads, 2 x 4 outputs each
+    for (int m0 = 0; m0 < M; m0 += TM) {
+        for (int n0 = 0; n0 < N; n0 += TN) {
+            float acc[2][4] = {};
+            for (int k0 = 0; k0 < Kd; k0 += TK) {
+                __syncthreads();
+                for (int idx = tid; idx < TK * TM; idx += NT) {
+                    const int kk = idx / TM, mm = idx % TM;
+                    sA[kk][mm] = (m0 + mm < M && k0 + kk < Kd) ? A.at(m0 + mm, k0 + kk) : 0.f;
+                }
+                for (int idx = tid; idx < TK * TN; idx += NT) {
+                    const int kk = idx / TN, nn = idx % TN;
+                    sB[kk][nn] = (n0 + nn < N && k0 + kk < Kd) ? B.at(k0 + kk, n0 + nn) : 0.f;
+                }
+                __syncthreads();
+#pragma unroll
+                for (int kk = 0; kk < TK; ++kk) {
+                    const float a0 = sA[kk][2 * tr], a1 = sA[kk][2 * tr + 1];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float bv = sB[kk][tc + 16 * j];
+                        acc[0][j] = fmaf(a0, bv, acc[0][j]);
+                        acc[1][j] = fmaf(a1, bv, acc[1][j]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = m0 + 2 * tr + i, c = n0 + tc + 16 * j;
+                    if (r < M && c < N) {
+                        float v = alpha * acc[i][j];
+                        if (mask == 1 && c > r) v = 0.f;
+                        float* dst = C + (long long)r * ldc + c;
+                        *dst = accumulate ? *dst + v : v;
+                    }
+                }
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
+    return 0.39894228040143268f * expf(-0.5f * a * a) * (2.0f - a * a);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
+    constexpr int M = 4 * D;
+    constexpr long long MD = (long long)M * D;
+    const int h = blockIdx.x, tid = threadIdx.x;
+    const int T = a.T, b = a.b;
+    const int nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
+    Scratch s = carve(a.scratch + (long long)h * a.scratch_per_head, D, nck);
+    const float eta = a.eta;
+
+    auto token = [&](int c, int r) { return a.reverse ? T - 1 - (c * b + r) : c * b + r; };
+    auto load_chunk = [&](int c, int n, bool with_q, bool with_dz) {
+        for (int idx = tid; idx < n * D; idx += NT) {
+            const int r = idx / D, j = idx % D;
+            const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
+            s.Kc[idx] = a.K[off];
+            s.Vc[idx] = a.V[off];
+            if (with_q) s.Qc[idx] = a.Q[off];
+            if (with_dz) s.dZc[idx] = a.dZ[(long long)h * a.x_hs + (long long)token(c, r) * a.x_ts + j];
+        }
+        __syncthreads();
+    };
+    // A = K W1^T, G = GELU(A), D2 = -2 eta (G W2^T - V), P = D2 W2, Dl = P GELU'(A)
+    auto chunk_core = [&](int n) {
+        gemm(s.A, M, N_(s.Kc, D), T_(s.W1, D), n, M, D, 1.f, false);
+        for (int idx = tid; idx < n * M; idx += NT) s.G[idx] = gelu(s.A[idx]);
+        __syncthreads();
+        gemm(s.D2, D, N_(s.G, M), T_(s.W2, M), n, D, M, 1.f, false);
+        for (int idx = tid; idx < n * D; idx += NT) s.D2[idx] = -2.0f * eta * (s.D2[idx] - s.Vc[idx]);
+        __syncthreads();
+        gemm(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
+        for (int idx = tid; idx < n * M; idx += NT) {
+            float g, gp;
+            gelu_and_prime(s.A[idx], g, gp);
+            s.Dl[idx] = s.P[idx] * gp;
+        }
+        __syncthreads();
+    };
+    // W1 += Dl^T K, W2 += D2^T G
+    auto chunk_update = [&](int n) {
+        gemm(s.W1, D, T_(s.Dl, M), N_(s.Kc, D), M, D, n, 1.f, true);
+        gemm(s.W2, M, T_(s.D2, D), N_(s.G, M), D, M, n, 1.f, true);
+    };
+    auto copy = [&](float* dst, const float* src, long long cnt) {
+        for (long long i = tid; i < cnt; i += NT) dst[i] = src[i];
+        __syncthreads();
+    };
+
+    // ---- forward walk: checkpoints of the state every kCkpt chunks
+    copy(s.W1, a.W1_0 + (long long)h * MD, MD);
+    copy(s.W2, a.W2_0 + (long long)h * MD, MD);
+    for (int c = 0; c < nch; ++c) {
+        const int n = min(b, T - c * b);
+        if (c % kCkpt == 0) {
+            copy(s.ck + (long long)(c / kCkpt) * 2 * MD, s.W1, MD);
+            copy(s.ck + (long long)(c / kCkpt) * 2 * MD + MD, s.W2, MD);
+        }
+        load_chunk(c, n, false, false);
+        chunk_core(n);
+        chunk_update(n);
+    }
+
+    // ---- backward, segment by segment from the end
+    for (long long i = tid; i < MD; i += NT) { s.dW1[i] = 0.f; s.dW2[i] = 0.f; }
+    __syncthreads();
+    for (int sg = nck - 1; sg >= 0; --sg) {
+        const int c0 = sg * kCkpt, c1 = min(nch, c0 + kCkpt);
+        copy(s.W1, s.ck + (long long)sg * 2 * MD, MD);
+        copy(s.W2, s.ck + (long long)sg * 2 * MD + MD, MD);
+        for (int c = c0; c < c1; ++c) {   // chunk-start states of the segment
+            copy(s.seg + (long long)(c - c0) * 2 * MD, s.W1, MD);
+            copy(s.seg + (long long)(c - c0) * 2 * MD + MD, s.W2, MD);
+            if (c + 1 < c1) {
+                const int n = min(b, T - c * b);
+                load_chunk(c, n, false, false);
+                chunk_core(n);
+                chunk_update(n);
+            }
+        }
+        for (int c = c1 - 1; c >= c0; --c) {
+            const int n = min(b, T - c * b);
+            copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
+            copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
+            load_chunk(c, n, true, true);
+            // forward intermediates
+            chunk_core(n);
+            gemm(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
+            gemm(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
+            gemm(s.Aq, M, N_(s.Mk, BMAX), N_(s.Dl, M), n, M, n, 1.f, true);
+            for (int idx = tid; idx < n * M; idx += NT) s.Gq[idx] = gelu(s.Aq[idx]);
+            __syncthreads();
+            gemm(s.Ng, BMAX, N_(s.Gq, M), T_(s.G, M), n, n, M, 1.f, false, 1);
+            // output branch
+            gemm(s.dGq, M, N_(s.dZc, D), N_(s.W2, M), n, M, D, 1.f, false);                 // dZ W2
+            gemm(s.dNg, BMAX, N_(s.dZc, D), T_(s.D2, D), n, n, D, 1.f, false, 1);            // tril(dZ D2^T)
+            gemm(s.dD2, D, T_(s.Ng, BMAX), N_(s.dZc, D), n, D, n, 1.f, false);               // Ng^T dZ
+            gemm(s.dGq, M, N_(s.dNg, BMAX), N_(s.G, M), n, M, n, 1.f, true);                 // + dNg G
+            gemm(s.dG, M, T_(s.dNg, BMAX), N_(s.Gq, M), n, M, n, 1.f, false);                // dNg^T Gq
+            for (int idx = tid; idx < n * M; idx += NT) {                                    // dAq (in dGq)
+                float g, gp;
+                gelu_and_prime(s.Aq[idx], g, gp);
+                s.dGq[idx] *= gp;
+            }
+            __syncthreads();
+            gemm(s.dQc, D, N_(s.dGq, M), N_(s.W1, D), n, D, M, 1.f, false);                 // dAq W1
+            gemm(s.dMk, BMAX, N_(s.dGq, M), T_(s.Dl, M), n, n, M, 1.f, false, 1);            // tril(dAq Dl^T)
+            gemm(s.dDl, M, T_(s.Mk, BMAX), N_(s.dGq, M), n, M, n, 1.f, false);               // Mk^T dAq
+            gemm(s.dQc, D, N_(s.dMk, BMAX), N_(s.Kc, D), n, D, n, 1.f, true);                // + dMk K
+            gemm(s.dKc, D, T_(s.dMk, BMAX), N_(s.Qc, D), n, D, n, 1.f, false);               // dMk^T Q
+            // the chunk-end state gradient
+            gemm(s.dDl, M, N_(s.Kc, D), T_(s.dW1, D), n, M, D, 1.f, true);                  // + K dW1'^T
+            gemm(s.dKc, D, N_(s.Dl, M), N_(s.dW1, D), n, D, M, 1.f, true);                  // + Dl dW1'
+            gemm(s.dD2, D, N_(s.G, M), T_(s.dW2, M), n, D, M, 1.f, true);                   // + G dW2'^T
+            gemm(s.dG, M, N_(s.D2, D), N_(s.dW2, M), n, M, D, 1.f, true);                   // + D2 dW2'
+            // dP (in dDl), dA
+            for (int idx = tid; idx < n * M; idx += NT) {
+                float g, gp;
+                gelu_and_prime(s.A[idx], g, gp);
+                const float ddl = s.dDl[idx];
+                s.dA[idx] = ddl * s.P[idx] * gelu_pp(s.A[idx]);
+                s.dDl[idx] = ddl * gp;
+            }
+            __syncthreads();
+            gemm(s.dD2, D, N_(s.dDl, M), T_(s.W2, M), n, D, M, 1.f, true);                  // + dP W2^T
+            for (int idx = tid; idx < n * D; idx += NT) s.dD2[idx] *= -2.0f * eta;            // dE (in dD2)
+            __syncthreads();
+            gemm(s.dG, M, N_(s.dD2, D), N_(s.W2, M), n, M, D, 1.f, true);                   // + dE W2
+            for (int idx = tid; idx < n * M; idx += NT) {                                    // dA += dG GELU'(A)
+                float g, gp;
+                gelu_and_prime(s.A[idx], g, gp);
+                s.dA[idx] += s.dG[idx] * gp;
+            }
+            __syncthreads();
+            gemm(s.dKc, D, N_(s.dA, M), N_(s.W1, D), n, D, M, 1.f, true);                   // + dA W1
+            // the chunk-start state gradient (accumulated onto the chunk-end one)
+            gemm(s.dW2, M, T_(s.dZc, D), N_(s.Gq, M), D, M, n, 1.f, true);                  // dZ^T Gq
+            gemm(s.dW2, M, T_(s.D2, D), N_(s.dDl, M), D, M, n, 1.f, true);                  // D2^T dP
+            gemm(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, 1.f, true);                   // dE^T G
+            gemm(s.dW1, D, T_(s.dGq, M), N_(s.Qc, D), M, D, n, 1.f, true);                  // dAq^T Q
+            gemm(s.dW1, D, T_(s.dA, M), N_(s.Kc, D), M, D, n, 1.f, true);                   // dA^T K
+            // dQ, dK, dV of the chunk's tokens
+            for (int idx = tid; idx < n * D; idx += NT) {
+                const int r = idx / D, j = idx % D;
+                const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
+                a.dQ[off] = s.dQc[idx];
+                a.dK[off] = s.dKc[idx];
+                a.dV[off] = -s.dD2[idx];   // dV = -dE
+            }
+            __syncthreads();
+        }
+    }
+    for (long long i = tid; i < MD; i += NT) {
+        a.dW1[(long long)h * MD + i] += s.dW1[i];
+        a.dW2[(long long)h * MD + i] += s.dW2[i];
+    }
+}
+
+}  // namespace
+
+long long scan_backward_scratch_floats(int d, int b, int T) { return scratch_floats_for(d, b, T); }
+
+cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V, long long qkv_hs, long long qkv_ts,
+                                 const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
+                                 const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
+                                 float* scratch, int T, int H, int d, int b, int reverse, float eta,
+                                 cudaStream_t s) {
+    if (b < 1 || b > BMAX) return cudaErrorInvalidValue;
+    BwdArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.qkv_hs = qkv_hs; a.qkv_ts = qkv_ts;
+    a.dZ = dZ; a.x_hs = x_hs; a.x_ts = x_ts;
+    a.W1_0 = W1_0; a.W2_0 = W2_0;
+    a.dQ = dQ; a.dK = dK; a.dV = dV; a.dW1 = dW1; a.dW2 = dW2;
+    a.scratch = scratch; a.scratch_per_head = scratch_floats_for(d, b, T);
+    a.T = T; a.H = H; a.d = d; a.b = b; a.reverse = reverse; a.eta = eta;
+    LaunchScope scope("scan_backward", s);
+    switch (d) {
+        case 16: scan_bwd_kernel<16><<<H, NT, 0, s>>>(a); break;
+        case 32: scan_bwd_kernel<32><<<H, NT, 0, s>>>(a); break;
+        case 64: scan_bwd_kernel<64><<<H, NT, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ttt

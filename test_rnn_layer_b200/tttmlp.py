@@ -24,8 +24,9 @@ DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
-            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_debug_inject_wait_timeout",
-            "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments"]
+            "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_mlp_noalloc_status", "ttt_debug_inject_wait_timeout",
+            "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments",
+            "ttt_mlp_backward_workspace_size", "ttt_mlp_backward"]
 
 
 class TTTError(RuntimeError):
@@ -66,6 +67,13 @@ def lib():
         L.ttt_mlp_forward_host.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_forward_noalloc.restype = i
         L.ttt_mlp_forward_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp]
+        L.ttt_mlp_backward_workspace_size.restype = sz
+        L.ttt_mlp_backward_workspace_size.argtypes = [dp, i, i]
+        L.ttt_mlp_backward.restype = i
+        L.ttt_mlp_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                       vp, sz, vp]
+        L.ttt_mlp_noalloc_status.restype = i
+        L.ttt_mlp_noalloc_status.argtypes = [vp]
         L.ttt_linear_workspace_size.restype = sz
         L.ttt_linear_workspace_size.argtypes = [dp, i, i]
         L.ttt_linear_forward.restype = i
@@ -180,6 +188,59 @@ def ttt_mlp_forward_noalloc(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta,
     return int(lib().ttt_mlp_forward_noalloc(ctypes.byref(desc), _p(X), _p(theta_q), _p(theta_k), _p(theta_v),
                                              _p(W1_0), _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f),
                                              _p(alpha_r), _p(Y), _p(Z_out), _p(W1_T), _p(W2_T), _stream(stream)))
+
+
+def ttt_mlp_backward_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
+    return int(lib().ttt_mlp_backward_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_mlp_backward(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r, dY, dX,
+                     dtheta_q, dtheta_k, dtheta_v, dW1_0, dW2_0, dalpha_f, dalpha_r, workspace, workspace_bytes,
+                     stream=None) -> int:
+    return int(lib().ttt_mlp_backward(ctypes.byref(desc), _p(X), _p(theta_q), _p(theta_k), _p(theta_v), _p(W1_0),
+                                      _p(W2_0), float(eta), int(b), int(direction), _p(alpha_f), _p(alpha_r), _p(dY),
+                                      _p(dX), _p(dtheta_q), _p(dtheta_k), _p(dtheta_v), _p(dW1_0), _p(dW2_0),
+                                      _p(dalpha_f), _p(dalpha_r), _p(workspace), int(workspace_bytes),
+                                      _stream(stream)))
+
+
+def layer_backward(X, theta_q, theta_k, theta_v, W1_0, W2_0, eta: float, b: int, dirs: str, alpha_f, alpha_r, dY,
+                   per_head: bool = True, workspace: torch.Tensor | None = None, check_status: bool = True,
+                   stream=None) -> dict:
+    """Allocate gradient outputs (fp32, on X's device) and call ttt_mlp_backward once."""
+    dev = X.device
+    if per_head:
+        H, T, d = X.shape
+    else:
+        T, _ = X.shape
+        H, d = W1_0.shape[0], W1_0.shape[2]
+    desc = make_desc(T, H, d, per_head, X.dtype == torch.bfloat16)
+    direction = DIRS[dirs]
+    if workspace is None:
+        n = ttt_mlp_backward_workspace_size(desc, b, direction)
+        if n == 0:
+            raise TTTError(TTT_ERR_INVALID_ARG, "backward workspace size")
+        workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dX": torch.empty(X.shape, **f32), "dtheta_q": torch.empty(theta_q.shape, **f32),
+           "dtheta_k": torch.empty(theta_k.shape, **f32), "dtheta_v": torch.empty(theta_v.shape, **f32),
+           "dW1_0": torch.empty(W1_0.shape, **f32), "dW2_0": torch.empty(W2_0.shape, **f32),
+           "dalpha_f": torch.zeros(alpha_f.shape, **f32), "dalpha_r": torch.zeros(alpha_r.shape, **f32)}
+    st = ttt_mlp_backward(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, direction, alpha_f, alpha_r,
+                          dY.float().contiguous(), out["dX"], out["dtheta_q"], out["dtheta_k"], out["dtheta_v"],
+                          out["dW1_0"], out["dW2_0"], out["dalpha_f"], out["dalpha_r"], workspace, workspace.numel(),
+                          stream)
+    check(st, "ttt_mlp_backward")
+    if check_status:
+        check(ttt_mlp_status(workspace, stream), "ttt_mlp_status")
+    out["workspace"] = workspace
+    return out
+
+
+def ttt_mlp_noalloc_status(stream=None) -> int:
+    """ttt_mlp_status for the no-alloc entry point (its status word lives in
+    the library's fixed scratch array on the current device)."""
+    return int(lib().ttt_mlp_noalloc_status(_stream(stream)))
 
 
 def ttt_linear_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:

@@ -111,7 +111,8 @@ def test_forward_argument_errors_before_any_cuda_call():
 
 
 def test_kernel_selector_validation():
-    assert L.ttt_mlp_select_kernels(4, 0) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_mlp_select_kernels(5, 0) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_mlp_select_kernels(-1, 0) == L.TTT_ERR_INVALID_ARG
     assert L.ttt_mlp_select_kernels(0, 3) == L.TTT_ERR_INVALID_ARG
     assert L.ttt_mlp_select_kernels(0, 0) == L.TTT_OK
 
