@@ -193,7 +193,7 @@ def _algorithmic(w):
     return {
         "scan_chunk_tc": ("tensor_tf32", scan_flops),
         "scan_chunk_tc2": ("tensor_tf32", scan_flops),
-        # tf32 for the three d-by-m products that read the fp32 state (A, Aq0, P), fp16 for the rest
+        # tf32 for the two d-by-m products that read the fp32 state (A, Aq0), fp16 for the rest
         "scan_chunk_tc3": ("tensor_mixed", scan_flops),
         "scan_chunk_simt": ("alu", scan_flops),
         "scan_token": ("alu", H * T * 7 * 2 * d * m),
@@ -220,8 +220,9 @@ def _algorithmic(w):
 
 def _tf32_share(w) -> float:
     """Share of the scan's algorithmic flops that the split-group kernel runs
-    with tf32 operands: A^T = W1 K^T, Aq0 = W1 Q^T and P^T = W2^T D2'^T."""
-    return 3 * 2 * w.d * w.m / (7 * 2 * w.d * w.m + 2 * w.b * (w.d + w.m))
+    with tf32 operands: A^T = W1 K^T and Aq0 = W1 Q^T (they read the fp32
+    state in tensor memory); every other product takes fp16 operands."""
+    return 2 * 2 * w.d * w.m / (7 * 2 * w.d * w.m + 2 * w.b * (w.d + w.m))
 
 
 def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):

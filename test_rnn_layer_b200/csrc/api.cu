@@ -56,7 +56,7 @@ static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
 // The split-group cluster scan applies the gate in its output group (1) or
 // leaves it to the separate gate kernel (0).
 #ifndef TTT_SPLIT_SCAN_GATES
-#define TTT_SPLIT_SCAN_GATES 0
+#define TTT_SPLIT_SCAN_GATES 1
 #endif
 constexpr bool kSplitScanGates = TTT_SPLIT_SCAN_GATES != 0;
 static std::atomic<int> g_inject_timeout{0};

@@ -58,12 +58,13 @@ __global__ void __launch_bounds__(GT) gemm_kernel(float* C, long long ldc, long 
     float acc[4][4] = {};
     for (long long k0 = k_lo; k0 < k_hi; k0 += GK) {
         __syncthreads();
+        // consecutive threads walk the operand's contiguous dimension (coalesced loads)
         for (int idx = tid; idx < GK * GM; idx += GT) {
-            const int kk = idx / GM, mm = idx % GM;
+            const int kk = A.cs == 1 ? idx % GK : idx / GM, mm = A.cs == 1 ? idx / GK : idx % GM;
             sA[kk][mm] = (m0 + mm < M && k0 + kk < k_hi) ? A.at(bz, m0 + mm, k0 + kk) : 0.f;
         }
         for (int idx = tid; idx < GK * GN; idx += GT) {
-            const int kk = idx / GN, nn = idx % GN;
+            const int kk = B.rs == 1 ? idx % GK : idx / GN, nn = B.rs == 1 ? idx / GK : idx % GN;
             sB[kk][nn] = (n0 + nn < N && k0 + kk < k_hi) ? B.at(bz, k0 + kk, n0 + nn) : 0.f;
         }
         __syncthreads();

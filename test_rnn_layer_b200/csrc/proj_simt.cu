@@ -11,22 +11,22 @@
 namespace ttt {
 namespace {
 
-constexpr int kPhTok = 32;       // tokens per CTA, per-head projection
+constexpr int kPhTok = 256;      // tokens per CTA, per-head projection (theta loaded once per 256 tokens)
 constexpr int kPhThreads = 256;
 
 __global__ void __launch_bounds__(kPhThreads)
 proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk, const void* thv,
                      int th_bf16, float* oq, float* ok, float* ov, int T, int d, int* status) {
     extern __shared__ float sm[];
-    float* th = sm;                     // [3][d][d]
+    float* th = sm;                     // [3][d][d], transposed: th[w][j][e] = theta_w[h][e][j]
     float* xs = sm + 3 * d * d;         // [kPhTok][d]
     const int h = blockIdx.y;
     const int t0 = blockIdx.x * kPhTok;
     const int nt = min(kPhTok, T - t0);
     const void* ths[3] = {thq, thk, thv};
     for (int p = threadIdx.x; p < 3 * d * d; p += blockDim.x) {
-        const int w = p / (d * d), q = p % (d * d);
-        th[p] = load_elem(ths[w], (long long)h * d * d + q, th_bf16);
+        const int w = p / (d * d), q = p % (d * d), e = q / d, j = q % d;
+        th[(w * d + j) * d + e] = load_elem(ths[w], (long long)h * d * d + q, th_bf16);
     }
     for (int p = threadIdx.x; p < nt * d; p += blockDim.x)
         xs[p] = load_elem(X, ((long long)h * T + t0) * d + p, x_bf16);
@@ -36,10 +36,14 @@ proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk
     for (int p = threadIdx.x; p < 3 * nt * d; p += blockDim.x) {
         const int w = p / (nt * d), q = p % (nt * d);
         const int r = q / d, e = q % d;
-        const float* row = th + (w * d + e) * d;
+        const float* col = th + w * d * d + e;   // consecutive threads: consecutive e (no bank conflict)
         const float* x = xs + r * d;
-        float acc = 0.f;
-        for (int j = 0; j < d; ++j) acc = fmaf(row[j], x[j], acc);
+        float acc0 = 0.f, acc1 = 0.f;
+        for (int j = 0; j < d; j += 2) {
+            acc0 = fmaf(col[j * d], x[j], acc0);
+            acc1 = fmaf(col[(j + 1) * d], x[j + 1], acc1);
+        }
+        const float acc = acc0 + acc1;
         outs[w][((long long)h * T + t0 + r) * d + e] = acc;
         bad |= !isfinite(acc);
     }

@@ -135,12 +135,13 @@ __device__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, floa
             float acc[2][4] = {};
             for (int k0 = 0; k0 < Kd; k0 += TK) {
                 __syncthreads();
+                // consecutive threads walk the operand's contiguous dimension (coalesced loads)
                 for (int idx = tid; idx < TK * TM; idx += NT) {
-                    const int kk = idx / TM, mm = idx % TM;
+                    const int kk = A.cs == 1 ? idx % TK : idx / TM, mm = A.cs == 1 ? idx / TK : idx % TM;
                     sA[kk][mm] = (m0 + mm < M && k0 + kk < Kd) ? A.at(m0 + mm, k0 + kk) : 0.f;
                 }
                 for (int idx = tid; idx < TK * TN; idx += NT) {
-                    const int kk = idx / TN, nn = idx % TN;
+                    const int kk = B.rs == 1 ? idx % TK : idx / TN, nn = B.rs == 1 ? idx / TK : idx % TN;
                     sB[kk][nn] = (n0 + nn < N && k0 + kk < Kd) ? B.at(k0 + kk, n0 + nn) : 0.f;
                 }
                 __syncthreads();

@@ -69,14 +69,14 @@ constexpr int BT = 64, DH = 64, MH = 256, MLOC = 128, THREADS = 512, NG = 256;
 constexpr int OFF_W2G = 0;          // [2] x 32 KB, MN-major over K = i: block 0 the W2 copy [i][j], block 1 G [i][t]
 constexpr int OFF_GQ = 65536;       // 16 KB: Gq, MN-major [i][t]
 constexpr int OFF_Q = 81920;        // 16 KB fp32 Q [t][j] (TMA)
-constexpr int OFF_K = 98304;        // 16 KB fp32 K [t][j] (TMA); then D2' [t][j]
+constexpr int OFF_K = 98304;        // 16 KB fp32 K [t][j] (TMA)
 constexpr int OFF_V = 114688;       // 16 KB fp32 V [t][j] (TMA)
 constexpr int OFF_X1 = 131072;      // 8 KB: K fp16, MN-major over K = t: [t][j]
 constexpr int OFF_X2 = 139264;      // 8 KB: M [t][s] fp16 (prefix mask of Q K^T)
 constexpr int OFF_X3 = 147456;      // [2] x 8 KB: D2'^T [j][t] fp16 (a 128-row read of either stays inside X3, X4)
 constexpr int OFF_X4 = 163840;      // 8 KB: -Npost, MN-major over K = s: [s][t] fp16
 constexpr int OFF_RY = 172032;      // [2] x 16 KB: the peer's Y^T partial [j][t] fp32
-constexpr int OFF_RZ = 204800;      // [2] x 8 KB: the peer's z partial for my tokens [j][t_own] fp32
+constexpr int OFF_RZ = 204800;      // [2] x 8 KB: the peer's z partial for my tokens [j][t_own] fp32, then my z
 constexpr int OFF_XS = 221184;      // 8 KB: the gate's x of my 32 tokens [t][j] (bf16 or fp32, by cp.async)
 constexpr int OFF_BAR = 229376;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -128,10 +128,6 @@ struct ScanTc3Args {
     ScanArgs a;
     int full;
 };
-
-__device__ __forceinline__ float tf32r(float x) {   // nearest tf32, ties away (see the two-CTA kernel)
-    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
-}
 
 __device__ __forceinline__ float rcp_approx(float x) {
     float r;
@@ -285,6 +281,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
     auto dW2G = [&](int p) { return tc::smem_desc(s_base + OFF_W2G + p * 32768, 16384, 1024); };
     auto dG = [&](int p) { return tc::smem_desc(s_base + OFF_W2G + p * 32768 + 16384, 16384, 1024); };
     auto dX3 = [&](int p) { return tc::smem_desc(s_base + OFF_X3 + p * 8192, 16, 1024); };
+    auto dX3mn = [&](int p) { return tc::smem_desc(s_base + OFF_X3 + p * 8192, 16384, 1024); };   // read MN-major
+    auto dW2k = [&](int p) { return tc::smem_desc(s_base + OFF_W2G + p * 32768, 16, 1024); };     // W2 copy, K-major
 
     if (a.inject_timeout && warp == 0) {   // tests: a bounded wait that expires (1 ms)
         if (!tc::mbar_wait(bars + B_NEVER, 0, nullptr, 1000000ull) && lane == 0) give_up();
@@ -375,11 +373,15 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
                 if (group_sync()) break;
             }
             tc::tc_fence_after();
+            // A^T first (it is on the chain), then S and Aq0 behind it on the tensor pipe: warp 1
+            // issues only after warp 0 has (a barrier of the two warps orders the issue)
             if (tid == 0) {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ts(tm + TM_R1, tm + TM_W1 + kk * 8, kstep(dK, kk, ST64), ID_TF32, kk > 0);
                 tc::mma_commit(bars + B_A);
-            } else if (tid == 32) {
+            }
+            if (warp < 2) asm volatile("bar.sync 3, 64;" ::: "memory");
+            if (tid == 32) {
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_tf32_ss(tm + TM_R2, kstep(dQ, kk, ST64), kstep(dK, kk, ST64), ID_TF32, kk > 0);
                 for (int kk = 0; kk < 8; ++kk)
@@ -445,10 +447,11 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             wait_bar(B_S, ph_s); ph_s ^= 1;
             if (n >= 1) wait_bar(B_AQ + (1 - p), ((n - 1) >> 1) & 1);
             tc::tc_fence_after();
-            if (tid == 0 && n + 1 < nloc) {   // Q is free: fetch the next chunk's queries
-                int ny0, nbc;
+            if (tid == 0 && n + 1 < nloc) {   // Q and K are free (K was converted before stage B): the next
+                int ny0, nbc;                 // chunk's queries and keys
                 chunk_rows(c + 1, ny0, nbc);
                 load_tile(&P.mapQ, OFF_Q, B_Q, ny0);
+                load_tile(&P.mapK, OFF_K, B_K, ny0);
             }
             if (q < 2) {   // M[t][s] = S[t][s] for s not after t: thread (t, 32 s)
                 const int t = 32 * q + lane;
@@ -476,7 +479,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             tc::tc_fence_after();
             STAMP3(8);
 
-            // ---- D: exchange the Y^T partials; D2' = -2 eta (Y - V) as fp32 [t][j] (into K) and fp16 [j][t] (X3[p])
+            // ---- D: exchange the Y^T partials; D2' = -2 eta (Y - V) as fp16 [j][t] (X3[p])
             if (n >= 2) wait_bar(B_ZD + p, ((n - 2) >> 1) & 1);   // output of chunk c-2 done with X3[p] and RZ[p]
             STAMP3(9);
             if (q < 2) {
@@ -519,9 +522,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
                         }
                     }
 #pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        *reinterpret_cast<float*>(sm + OFF_K + f32_off(tb + k, j, ST64)) = tf32r(d2[k]);
-#pragma unroll
                     for (int c8 = 0; c8 < 2; ++c8)
                         *reinterpret_cast<uint4*>(sm + OFF_X3 + p * 8192 + h_chunk(j, tb + 8 * c8, 0)) =
                             make_uint4(pack_h2(d2[8 * c8], d2[8 * c8 + 1]), pack_h2(d2[8 * c8 + 2], d2[8 * c8 + 3]),
@@ -531,21 +531,20 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             if (group_sync()) break;
             STAMP3(12);
 
-            // ---- E: P^T = W2^T D2'^T (my rows; tf32, the state is fp32)
+            // ---- E: P^T = W2^T D2'^T (my rows), fp16: the W2 copy read K-major (M = i, K = j), D2'^T MN-major
             if (tid == 0) {
-                for (int kk = 0; kk < 8; ++kk)
-                    tc::mma_tf32_ts(tm + TM_R2, tm + TM_W2T + kk * 8, kstep(dK, kk, ST64), ID_TF32, kk > 0);
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16_ss(tm + TM_R2, kstep(dW2k(p), kk, 0), kstep_mn(dX3mn(p), kk), ID_F16_KM, kk > 0);
                 tc::mma_commit(bars + B_P);
+                if (n + 1 < nloc) {   // V is free: fetch the next chunk's values
+                    int ny0, nbc;
+                    chunk_rows(c + 1, ny0, nbc);
+                    load_tile(&P.mapV, OFF_V, B_V, ny0);
+                }
             }
             wait_bar(B_P, ph_p); ph_p ^= 1;
             tc::tc_fence_after();
             STAMP3(13);
-            if (tid == 0 && n + 1 < nloc) {   // K and V are free: fetch the next chunk's tiles
-                int ny0, nbc;
-                chunk_rows(c + 1, ny0, nbc);
-                load_tile(&P.mapK, OFF_K, B_K, ny0);
-                load_tile(&P.mapV, OFF_V, B_V, ny0);
-            }
 
             // ---- F: Dl = P * G' (fp16 pairs into tensor memory as Dl^T)
             {
@@ -624,9 +623,11 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             return ab;
         };
         uint32_t ph_corr = 0;
-        const bool receiver = q < 2 && gh == (int)r_cta;   // finishes z (and the gate) of my 32 tokens, channel j
-        const int jr = 32 * q + lane;
-        const float tan_a = (receiver && a.fuse_gate) ? tanhf(a.alpha[h * DH + jr]) : 0.f;
+        // the gate: thread (token gr of my 32, channels gj .. gj + 7)
+        const int gr = ztid >> 3, gj = 8 * (ztid & 7);
+        float tan_a[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tan_a[e] = a.fuse_gate ? tanhf(a.alpha[h * DH + gj + e]) : 0.f;
         int nonfinite = 0;
         for (int n = 0; n < nloc; ++n) {
             const int c = c_first + n, p = n & 1;
@@ -734,7 +735,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
                     }
                 } else if (tc::mbar_wait_cluster_abort(bars + B_RZ + 2 * p + q, (n >> 1) & 1, abort_flag)) {
                     if (lane == 0) tc::mbar_arrive_expect_tx(bars + B_RZ + 2 * p + q, RZ_WARP_BYTES);   // chunk c+2
-                    const uint8_t* rz = sm + OFF_RZ + p * 8192;
+                    uint8_t* rz = sm + OFF_RZ + p * 8192;
                     const long long base = (long long)h * a.x_hs + (long long)y0 * a.x_ts + j;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
@@ -743,28 +744,21 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int c4 = 0; c4 < 4; ++c4) {
-                            const float4 v4 = *reinterpret_cast<const float4*>(rz + rz_off(j, 16 * half + 4 * c4));
-                            const float zz[4] = {__uint_as_float(r[4 * c4]) + v4.x, __uint_as_float(r[4 * c4 + 1]) + v4.y,
-                                                 __uint_as_float(r[4 * c4 + 2]) + v4.z,
-                                                 __uint_as_float(r[4 * c4 + 3]) + v4.w};
+                            float4* slot = reinterpret_cast<float4*>(rz + rz_off(j, 16 * half + 4 * c4));
+                            const float4 v4 = *slot;
+                            const float4 zz = make_float4(__uint_as_float(r[4 * c4]) + v4.x,
+                                                          __uint_as_float(r[4 * c4 + 1]) + v4.y,
+                                                          __uint_as_float(r[4 * c4 + 2]) + v4.z,
+                                                          __uint_as_float(r[4 * c4 + 3]) + v4.w);
+                            if (a.fuse_gate) {   // my z, for the whole group's gate below
+                                *slot = zz;
+                                continue;
+                            }
+                            const float zv[4] = {zz.x, zz.y, zz.z, zz.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int k = 16 * half + 4 * c4 + e, t = t0 + k;
-                                if (t >= bc) continue;
-                                const long long idx = base + (long long)t * a.x_ts;
-                                if (!a.fuse_gate) {
-                                    a.Zscan[idx] = zz[e];
-                                    continue;
-                                }
-                                // the gate out = x + tanh(alpha) z (paper notes page, "关键设计 / 门控 + 双向机制")
-                                const float dz = tan_a * zz[e];
-                                const float xv = a.xin_bf16
-                                    ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(sm + OFF_XS)[k * DH + j])
-                                    : reinterpret_cast<const float*>(sm + OFF_XS)[k * DH + j];
-                                store_elem(a.Out, idx, a.out_bf16, xv + dz);
-                                if (a.Delta) a.Delta[idx] = __float2bfloat16_rn(dz);
-                                if (a.Zdbg) a.Zdbg[idx] = zz[e];
-                                nonfinite |= !(isfinite(xv) && isfinite(zz[e]));
+                                const int t = t0 + 16 * half + 4 * c4 + e;
+                                if (t < bc) a.Zscan[base + (long long)t * a.x_ts] = zv[e];
                             }
                         }
                     }
@@ -774,6 +768,59 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             }
             STAMP3(23);
             if (group_sync()) break;
+            if (a.fuse_gate && 32 * (int)r_cta + gr < bc) {
+                // the gate out = x + tanh(alpha) z (paper notes page, "关键设计 / 门控 + 双向机制") over my 32
+                // tokens, eight channels per thread with 16-byte loads and stores
+                const uint8_t* rz = sm + OFF_RZ + p * 8192;
+                float zv[8], xv[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    zv[e] = *reinterpret_cast<const float*>(rz + rz_off(gj + e, gr & ~3) + (gr & 3) * 4);
+                if (a.xin_bf16) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(sm + OFF_XS + (gr * DH + gj) * 2);
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                        xv[2 * e] = f.x;
+                        xv[2 * e + 1] = f.y;
+                    }
+                } else {
+                    const float4* src = reinterpret_cast<const float4*>(sm + OFF_XS + (gr * DH + gj) * 4);
+                    const float4 f0 = src[0], f1 = src[1];
+                    xv[0] = f0.x; xv[1] = f0.y; xv[2] = f0.z; xv[3] = f0.w;
+                    xv[4] = f1.x; xv[5] = f1.y; xv[6] = f1.z; xv[7] = f1.w;
+                }
+                float o[8], dz[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    dz[e] = tan_a[e] * zv[e];
+                    o[e] = xv[e] + dz[e];
+                    nonfinite |= !(isfinite(xv[e]) && isfinite(zv[e]));
+                }
+                const long long idx = (long long)h * a.x_hs + (long long)(y0 + 32 * (int)r_cta + gr) * a.x_ts + gj;
+                auto bf2 = [](float lo, float hi) {
+                    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+                    return *reinterpret_cast<const uint32_t*>(&v);
+                };
+                if (a.out_bf16) {
+                    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.Out) + idx) =
+                        make_uint4(bf2(o[0], o[1]), bf2(o[2], o[3]), bf2(o[4], o[5]), bf2(o[6], o[7]));
+                } else {
+                    float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.Out) + idx);
+                    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+                    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+                }
+                if (a.Delta)
+                    *reinterpret_cast<uint4*>(a.Delta + idx) =
+                        make_uint4(bf2(dz[0], dz[1]), bf2(dz[2], dz[3]), bf2(dz[4], dz[5]), bf2(dz[6], dz[7]));
+                if (a.Zdbg) {
+                    float4* dst = reinterpret_cast<float4*>(a.Zdbg + idx);
+                    dst[0] = make_float4(zv[0], zv[1], zv[2], zv[3]);
+                    dst[1] = make_float4(zv[4], zv[5], zv[6], zv[7]);
+                }
+            }
+            if (a.fuse_gate && group_sync()) break;   // RZ[p] and XS are read before they are reused
             if (ztid == 0) tc::mbar_arrive(bars + B_ZD + p);
             STAMP3(24);
         }
