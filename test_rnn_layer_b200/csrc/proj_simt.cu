@@ -14,40 +14,65 @@ namespace {
 constexpr int kPhTok = 256;      // tokens per CTA, per-head projection (theta loaded once per 256 tokens)
 constexpr int kPhThreads = 256;
 
+// One head, 256 tokens: U [tokens x 3d] = X [tokens x d] Theta^T [d x 3d] with
+// Theta = [theta_Q; theta_K; theta_V] of the head, both operands in shared
+// memory (x rows padded to d + 1), 64 x 64 output blocks, 4 x 4 per thread.
+template <int D>
 __global__ void __launch_bounds__(kPhThreads)
 proj_per_head_kernel(const void* X, int x_bf16, const void* thq, const void* thk, const void* thv,
-                     int th_bf16, float* oq, float* ok, float* ov, int T, int d, int* status) {
+                     int th_bf16, float* oq, float* ok, float* ov, int T, int* status) {
+    constexpr int N3 = 3 * D, XP = D + 1;
     extern __shared__ float sm[];
-    float* th = sm;                     // [3][d][d], transposed: th[w][j][e] = theta_w[h][e][j]
-    float* xs = sm + 3 * d * d;         // [kPhTok][d]
+    float* thT = sm;                    // [D][3D]: thT[j][w D + e] = theta_w[h][e][j]
+    float* xs = sm + D * N3;            // [kPhTok][D + 1]
     const int h = blockIdx.y;
     const int t0 = blockIdx.x * kPhTok;
     const int nt = min(kPhTok, T - t0);
     const void* ths[3] = {thq, thk, thv};
-    for (int p = threadIdx.x; p < 3 * d * d; p += blockDim.x) {
-        const int w = p / (d * d), q = p % (d * d), e = q / d, j = q % d;
-        th[(w * d + j) * d + e] = load_elem(ths[w], (long long)h * d * d + q, th_bf16);
+    const int tid = threadIdx.x;
+    for (int p = tid; p < 3 * D * D; p += kPhThreads) {
+        const int w = p / (D * D), q = p % (D * D), e = q / D, j = q % D;
+        thT[j * N3 + w * D + e] = load_elem(ths[w], (long long)h * D * D + q, th_bf16);
     }
-    for (int p = threadIdx.x; p < nt * d; p += blockDim.x)
-        xs[p] = load_elem(X, ((long long)h * T + t0) * d + p, x_bf16);
+    for (int p = tid; p < nt * D; p += kPhThreads)
+        xs[(p / D) * XP + p % D] = load_elem(X, ((long long)h * T + t0) * D + p, x_bf16);
     __syncthreads();
     float* outs[3] = {oq, ok, ov};
+    const int tr = tid / 16, tc = tid % 16;
     int bad = 0;   // a non-finite input reaches every projection of its token
-    for (int p = threadIdx.x; p < 3 * nt * d; p += blockDim.x) {
-        const int w = p / (nt * d), q = p % (nt * d);
-        const int r = q / d, e = q % d;
-        const float* col = th + w * d * d + e;   // consecutive threads: consecutive e (no bank conflict)
-        const float* x = xs + r * d;
-        float acc0 = 0.f, acc1 = 0.f;
-        for (int j = 0; j < d; j += 2) {
-            acc0 = fmaf(col[j * d], x[j], acc0);
-            acc1 = fmaf(col[(j + 1) * d], x[j + 1], acc1);
+    for (int r0 = 0; r0 < nt; r0 += 64) {
+        for (int n0 = 0; n0 < N3; n0 += 64) {
+            float acc[4][4] = {};
+#pragma unroll 4
+            for (int j = 0; j < D; ++j) {
+                float av[4], bv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) av[i] = xs[(r0 + tr + 16 * i) * XP + j];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int n = n0 + tc + 16 * k;
+                    bv[k] = n < N3 ? thT[j * N3 + n] : 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) acc[i][k] = fmaf(av[i], bv[k], acc[i][k]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = r0 + tr + 16 * i;
+                if (r >= nt) continue;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int n = n0 + tc + 16 * k;
+                    if (n >= N3) continue;
+                    outs[n / D][((long long)h * T + t0 + r) * D + n % D] = acc[i][k];
+                    bad |= !isfinite(acc[i][k]);
+                }
+            }
         }
-        const float acc = acc0 + acc1;
-        outs[w][((long long)h * T + t0 + r) * d + e] = acc;
-        bad |= !isfinite(acc);
     }
-    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kStatusNonFinite);
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, kStatusNonFinite);
 }
 
 // C[t, n] (+)= sum_c A[t, c] B[n, c]; 64 x 64 tile, 16-deep k steps, 4 x 4 per thread.
@@ -104,15 +129,22 @@ proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1,
 
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
                                  float* const out[3], int T, int H, int d, int* status, cudaStream_t s) {
-    const size_t smem = sizeof(float) * (3 * (size_t)d * d + (size_t)kPhTok * d);
-    cudaError_t e = cudaFuncSetAttribute(proj_per_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    LaunchScope scope("proj_per_head", s);
-    dim3 grid((T + kPhTok - 1) / kPhTok, H);
-    proj_per_head_kernel<<<grid, kPhThreads, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16,
-                                                        out[0], out[1], out[2], T, d, status);
-    return cudaGetLastError();
+    auto run = [&](auto kernel, int D) -> cudaError_t {
+        const size_t smem = sizeof(float) * (3 * (size_t)D * D + (size_t)kPhTok * (D + 1));
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        LaunchScope scope("proj_per_head", s);
+        dim3 grid((T + kPhTok - 1) / kPhTok, H);
+        kernel<<<grid, kPhThreads, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16, out[0], out[1],
+                                              out[2], T, status);
+        return cudaGetLastError();
+    };
+    switch (d) {
+        case 16: return run(proj_per_head_kernel<16>, 16);
+        case 32: return run(proj_per_head_kernel<32>, 32);
+        case 64: return run(proj_per_head_kernel<64>, 64);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_proj_full_simt(const void* A, int a_bf16, const void* const theta[3], int th_bf16,

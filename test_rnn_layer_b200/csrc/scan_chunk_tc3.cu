@@ -357,7 +357,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             STAMP3(15);
             wait_bar(B_K, ph_k); ph_k ^= 1;
             wait_bar(B_Q, ph_q); ph_q ^= 1;
-            wait_bar(B_V, ph_v); ph_v ^= 1;
             STAMP3(0);
             if (n >= 2) wait_bar(B_ZN + p, ((n - 2) >> 1) & 1);   // output of chunk c-2 read Aq[p], W2G[p]
             STAMP3(1);
@@ -434,7 +433,6 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             }
             STAMP3(5);
             if (group_sync()) break;
-            if (tid == 0 && n >= 1) tc::mbar_arrive(bars + B_W2R + (1 - p));   // output of chunk c-1: W2_c in place
             STAMP3(6);
 
             // ---- C: my Y^T partial = W2_c[:, mine] G[:, mine]^T (rows 64.. of the A operand are G: unused);
@@ -443,6 +441,8 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
                 for (int kk = 0; kk < 8; ++kk)
                     tc::mma_f16_ss(tm + TM_R1, kstep_mn(dW2G(p), kk), kstep_mn(dG(p), kk), ID_F16_MM, kk > 0);
                 tc::mma_commit(bars + B_Y);
+                // the output of chunk c-1 may now read W2_c beside its G: its [Z1; N] MMA queues behind Y^T
+                if (n >= 1) tc::mbar_arrive(bars + B_W2R + (1 - p));
             }
             wait_bar(B_S, ph_s); ph_s ^= 1;
             if (n >= 1) wait_bar(B_AQ + (1 - p), ((n - 1) >> 1) & 1);
@@ -481,6 +481,7 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
 
             // ---- D: exchange the Y^T partials; D2' = -2 eta (Y - V) as fp16 [j][t] (X3[p])
             if (n >= 2) wait_bar(B_ZD + p, ((n - 2) >> 1) & 1);   // output of chunk c-2 done with X3[p] and RZ[p]
+            wait_bar(B_V, ph_v); ph_v ^= 1;                      // V is read here only
             STAMP3(9);
             if (q < 2) {
                 const int j = 32 * q + lane, wx = 2 * gh + q;
@@ -565,13 +566,12 @@ __global__ void __launch_bounds__(THREADS, 1) scan_tc3_kernel(const __grid_const
             if (group_sync()) break;
 
             // ---- G: W1 += Dl^T K, W2^T += G^T D2' (bar U); Aq[p]^T += Dl^T M^T (bar AQ[p], for the output group)
-            if (tid == 0) {
+            if (tid == 0) {   // the state updates first (on the chain), then the output's Aq behind them
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16_ts(tm + TM_W1, tm + TM_DL + kk * 8, kstep_mn(dX1, kk), ID_F16_KM, 1);
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16_ts(tm + TM_W2T, tm + TM_GT + kk * 8, kstep(dX3(p), kk, 0), ID_F16, 1);
                 tc::mma_commit(bars + B_U);
-            } else if (tid == 32) {
                 for (int kk = 0; kk < 4; ++kk)
                     tc::mma_f16_ts(tm + TM_AQ + 64 * p, tm + TM_DL + kk * 8, kstep(dX2, kk, 0), ID_F16, 1);
                 tc::mma_commit(bars + B_AQ + p);
