@@ -266,7 +266,10 @@ std::mutex g_pipe_mu;
 Pipe g_pipes[64];
 
 constexpr int kPipeMinSegChunks = 16;
-constexpr int kPipeSmMargin = 8;
+#ifndef TTT_PIPE_SM_MARGIN
+#define TTT_PIPE_SM_MARGIN 8
+#endif
+constexpr int kPipeSmMargin = TTT_PIPE_SM_MARGIN;
 // When the scan applies the gate itself, the projections of the segments that
 // cover the first kPipeFrontPercent of a direction's chunks run on the whole
 // GPU before that direction's scan starts (a head start: the scan then walks
