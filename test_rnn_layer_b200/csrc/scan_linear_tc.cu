@@ -1,20 +1,25 @@
 // TTT-Linear scan on the tcgen05 tensor cores (d = 64, 2 <= b <= 64), one CTA
 // per head.  The chunk of the linear layer (paper notes page, "实验关键数据 /
 // 消融实验": TTT-Linear; mini-batch reading of "关键设计 / TTT-MLP 层") in
-// matrix form, t, s tokens of the chunk in walking order, W the chunk-start
+// matrix form, t, s tokens of the chunk in walking order, W_c the chunk-start
 // state [i][j]:
-//   E'^T = -2 eta (W K^T - V^T)                      (-eta dl/dz per token, [i][t])
-//   Z^T  = W Q^T + E'^T M^T,  M[t,s] = q_t.k_s for s not after t
-//   W   += E'^T K                                     (the chunk's update)
-// which is token t read with the prefix state W + sum_{s<=t} E'_s k_s^T.
-// W lives in tensor memory as an fp32 accumulator (lanes i) for the whole
-// sequence and is the A operand of W K^T and W Q^T; E'^T (tensor memory) is the
-// A operand of the two products that use it.  Q, K, V arrive by TMA (3-D maps,
-// 128-byte swizzle) a chunk ahead.  Per chunk the dependent chain is one MMA
-// stage (W K^T), one thread stage (E'), one MMA stage (the correction and the
-// update); S = Q K^T and W Q^T run behind the first, the z store of the
-// previous chunk, K^T and the prefix mask overlap the MMAs.  All contractions
-// are kind::tf32 (fp32 accumulate) on K-major operands; every wait is bounded.
+//   E'^T = -2 eta (W_c K^T - V^T)                  (-eta dl/dz per token, [i][t])
+//   W_{c+1} = W_c + E'^T K                         (the chunk's update)
+//   Z^T  = W_{c+1} Q^T - E'^T Npost^T,  Npost[t,s] = q_t.k_s for s after t
+// which is token t read with the prefix state W_c + sum_{s<=t} E'_s k_s^T: the
+// output is read with the state at the chunk's END, less the later tokens'
+// updates.  So W_{c+1} Q_c^T and the next chunk's W_{c+1} K_{c+1}^T share
+// their A operand and run as one N = 128 product over [K_{c+1}; Q_c], and no
+// product that reads W is ever in flight while the update writes it.
+//
+// Per chunk the dependent chain is: [W K^T | W Q_prev^T] (tf32, W the A operand
+// from tensor memory), the E' thread stage (fp16 pairs into tensor memory), the
+// update (kind::f16 on K as fp16).  Off the chain: S = Q K^T (tf32, issued by
+// warp 2), the previous chunk's correction (kind::f16), the mask -Npost as
+// fp16, the z stores, K as fp16, and the tile loads (warp 3) a chunk ahead.
+// fp16 holds the thread-produced operands (E', K, the mask): the same 10-bit
+// mantissa as tf32, rounded rather than truncated.  Every wait is bounded.
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -26,34 +31,51 @@ namespace {
 
 constexpr int BT = 64, DH = 64, THREADS = 512;
 
-// Shared memory (bytes from a 1024-aligned base): 64 x 64 fp32 tiles as
-// 128-byte-swizzled atoms (8 rows x 32 columns; atom rows 1024 B apart, atom
-// columns 8192 B apart).  Q is read as a 128-row A operand: its extra rows fall
-// in K (unused output rows).
-constexpr int OFF_Q = 0;         // Q [t][j] (TMA)
-constexpr int OFF_K = 16384;     // K [t][j] (TMA)
-constexpr int OFF_V = 32768;     // V [t][j] (TMA)
-constexpr int OFF_X1 = 49152;    // K^T [j][t]
-constexpr int OFF_X2 = 65536;    // M [t][s]
-constexpr int OFF_BAR = 81920;
+// Shared memory (bytes from a 1024-aligned base).  fp32 tiles are 128-byte
+// swizzled atoms (8 rows x 32 columns, atom rows 1024 B apart).  K and Q share
+// two 32 KB regions: region r holds K of chunk parity r at +0 (columns 0-31) /
+// +16 KB (columns 32-63) and Q of parity 1-r at +8 KB / +24 KB, so that rows
+// 0-127 of a region are [K_c; Q_{c-1}] with 16 KB between the column halves.
+// A 128-row read of Q as an A operand runs into the next 8 KB (unused rows).
+constexpr int OFF_REG = 0;          // [2] x 32 KB: K / Q regions
+constexpr int REG = 32768;
+constexpr int QSLOT = 8192;         // Q's rows within a region
+constexpr int KQ_HALF = 16384;      // column-half stride of K and Q
+constexpr int OFF_V = 65536;        // [2] x 16 KB: V [t][j], column halves 8 KB apart
+constexpr int V_HALF = 8192;
+constexpr int OFF_X1 = 98304;       // 8 KB: K fp16 [t][j], MN-major (row per K index t)
+constexpr int OFF_X2 = 106496;      // [2] x 8 KB: -Npost fp16 [t][s], K-major (row per t)
+constexpr int OFF_BAR = 122880;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr int ST64 = 8192;
 
-// Tensor memory columns (lanes 0-63 hold the head's 64 rows; 64-127 are unused rows).
-constexpr uint32_t TM_W = 0;     // W [i][j]
-constexpr uint32_t TM_E = 64;    // E^T -> E'^T [i][t]
-constexpr uint32_t TM_S = 128;   // S [t][s]
-constexpr uint32_t TM_Z = 192;   // Z^T [i][t], two buffers (chunk parity) at 192 and 256
+// Tensor memory (128 lanes x 512 columns; lanes 0-63 are the head's rows, 64-127 unused).
+constexpr uint32_t TM_W = 0;        // W [i][j]
+constexpr uint32_t TM_B = 64;       // [2] x 128: [E^T of chunk c | Z^T of chunk c-1], block of parity c
+constexpr uint32_t TM_S = 320;      // S [t][s]
+constexpr uint32_t TM_PK = 384;     // [2] x 32: E'^T [i][t] as fp16 pairs (the A operand)
+
+#ifdef TTT_DEBUG_STAGES
+// Debug builds only: cycles between stage boundaries seen by thread 0 of CTA 0.
+__device__ float* g_dbg_lin = nullptr;
+#define STAMPL(k)                                         \
+    do {                                                  \
+        if (tid == 0 && blockIdx.x == 0) {                \
+            const long long now_ = clock64();             \
+            stamp_acc[k] += now_ - stamp_last;            \
+            stamp_last = now_;                            \
+        }                                                 \
+    } while (0)
+#else
+#define STAMPL(k) \
+    do {          \
+    } while (0)
+#endif
 
 struct LinTcArgs {
     CUtensorMap mapQ, mapK, mapV;
     LinearScanArgs a;
     int full;
 };
-
-__device__ __forceinline__ float tf32r(float x) {   // nearest tf32, ties away (finite inputs)
-    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
-}
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
     asm volatile(
@@ -63,30 +85,42 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-__device__ __forceinline__ uint64_t kstep(uint64_t d0, int kk) {   // K-step kk (8 tf32 = 32 B) of a 64-wide tile
-    return d0 + (uint64_t)(((kk >> 2) * ST64 + (kk & 3) * 32) >> 4);
+// K-step kk (8 tf32 = 32 B) of a 64-wide fp32 tile whose column halves are `half` bytes apart.
+__device__ __forceinline__ uint64_t kstep(uint64_t d0, int kk, int half) {
+    return d0 + (uint64_t)(((kk >> 2) * half + (kk & 3) * 32) >> 4);
+}
+// K-step kk (16 fp16 = 32 B) of a K-major fp16 operand (64 K values per 128-byte row).
+__device__ __forceinline__ uint64_t kstep_h(uint64_t d0, int kk) { return d0 + (uint64_t)((kk * 32) >> 4); }
+// K-step kk (16 K rows = 2 KB) of an MN-major fp16 operand.
+__device__ __forceinline__ uint64_t kstep_mn(uint64_t d0, int kk) { return d0 + (uint64_t)((kk * 2048) >> 4); }
+
+// 16-byte chunk of fp32 columns c..c+3 of row R (column halves `half` bytes apart).
+__device__ __forceinline__ uint32_t row4_off(int R, int c, int half) {
+    return (uint32_t)((c >> 5) * half + (R >> 3) * 1024 + (R & 7) * 128 + ((((c & 31) >> 2) ^ (R & 7)) << 4));
 }
 
-// Column-fixed swizzled addressing: element (R, c) at ph[R & 7] + (R >> 3) * 1024.
-__device__ __forceinline__ void col_phases(int c, uint32_t (&ph)[8]) {
-    const uint32_t base = (uint32_t)((c >> 5) * ST64 + (c & 3) * 4);
-    const uint32_t cq = (uint32_t)((c & 31) >> 2);
-#pragma unroll
-    for (int r = 0; r < 8; ++r) ph[r] = base + r * 128 + ((cq ^ r) << 4);
+// 16-byte chunk of fp16 values c..c+7 (c % 8 == 0, c < 64) of 128-byte row R, 128-byte swizzle.
+__device__ __forceinline__ uint32_t h_chunk(int R, int c) {
+    return (uint32_t)((R >> 3) * 1024 + (R & 7) * 128 + (((c >> 3) ^ (R & 7)) << 4));
 }
 
-__device__ __forceinline__ uint32_t row4_off(int R, int c) {   // 16-byte chunk of columns c..c+3 of row R
-    return (uint32_t)((c >> 5) * ST64 + (R >> 3) * 1024 + (R & 7) * 128 + ((((c & 31) >> 2) ^ (R & 7)) << 4));
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
 }
 
 __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid_constant__ LinTcArgs P) {
     const LinearScanArgs& a = P.a;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bar_mma = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
-    uint64_t* bar_a2 = bar_mma + 1;     // S and W Q^T
-    uint64_t* bar_ld = bar_mma + 2;     // the chunk's Q, K, V tiles
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 3);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+    uint64_t* bar_g = bars + 0;    // [W K^T | W Q_prev^T] of the chunk
+    uint64_t* bar_u = bars + 1;    // the update
+    uint64_t* bar_c = bars + 2;    // the previous chunk's correction (and the last chunk's output products)
+    uint64_t* bar_s = bars + 3;    // S = Q K^T
+    uint64_t* bar_ld = bars + 4;   // [2]: a chunk's Q, K, V tiles, by chunk parity
+    uint64_t* bar_go = bars + 6;   // a chunk has started: its first product is issued, the chunk before is done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -95,12 +129,11 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
     const int T = a.T, b = a.b;
     const int nchunks = (T + b - 1) / b;
     const int c_first = a.c_begin, c_last = a.c_end > 0 ? min(a.c_end, nchunks) : nchunks;
+    const int nloc = c_last - c_first;
     const float m2eta = -2.0f * a.eta;
 
     if (tid == 0) {
-        tc::mbar_init(bar_mma, 1);
-        tc::mbar_init(bar_a2, 1);
-        tc::mbar_init(bar_ld, 1);
+        for (int k = 0; k < 7; ++k) tc::mbar_init(bars + k, 1);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -118,18 +151,32 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
         *abort_flag = 1;
         atomicOr(a.status, kStatusTimeout);
     };
+    auto wait_ok = [&](uint64_t* bar, uint32_t parity) -> bool {
+        if (tc::mbar_wait(bar, parity, abort_flag)) return true;
+        give_up();
+        return false;
+    };
     auto chunk_rows = [&](int c, int& y0, int& bc) {
         bc = min(b, T - c * b);
         y0 = a.reverse ? (T - c * b - bc) : c * b;
     };
-    auto load_tiles = [&](int y0) {   // thread 0
-        tc::mbar_arrive_expect_tx(bar_ld, 3 * BT * DH * 4);
+    // where the tiles of local chunk n live
+    auto k_tile = [&](int n) { return sm + OFF_REG + (n & 1) * REG; };
+    auto q_tile = [&](int n) { return sm + OFF_REG + ((n & 1) ^ 1) * REG + QSLOT; };
+    auto v_tile = [&](int n) { return sm + OFF_V + (n & 1) * 16384; };
+    auto load_tiles = [&](int n) {   // thread 96: local chunk n's Q, K, V
+        int y0, bc;
+        chunk_rows(c_first + n, y0, bc);
+        uint64_t* bl = bar_ld + (n & 1);
+        tc::mbar_arrive_expect_tx(bl, 3 * BT * DH * 4);
         const CUtensorMap* maps[3] = {&P.mapQ, &P.mapK, &P.mapV};
-        const int offs[3] = {OFF_Q, OFF_K, OFF_V};
+        uint8_t* dst[3] = {q_tile(n), k_tile(n), v_tile(n)};
+        const int half[3] = {KQ_HALF, KQ_HALF, V_HALF};
         for (int w = 0; w < 3; ++w)
-            for (int half = 0; half < 2; ++half) {
-                if (P.full) tma_load_3d(sm + offs[w] + half * ST64, maps[w], half * 32, h, y0, bar_ld);
-                else tma_load_3d(sm + offs[w] + half * ST64, maps[w], half * 32, y0, h, bar_ld);
+            for (int hf = 0; hf < 2; ++hf) {
+                uint8_t* d = dst[w] + hf * half[w];
+                if (P.full) tma_load_3d(d, maps[w], hf * 32, h, y0, bl);
+                else tma_load_3d(d, maps[w], hf * 32, y0, h, bl);
             }
     };
 
@@ -148,37 +195,44 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
         tc::tmem_st_32x32b_x16(tm + lane_base + TM_W + j0, r);
         tc::tmem_wait_st();
     }
-    if (tid == 0) {
-        int y0, bc;
-        chunk_rows(c_first, y0, bc);
-        load_tiles(y0);
-    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
 
-    uint32_t ph_mma = 0, ph_a2 = 0, ph_ld = 0;
     constexpr uint32_t ID64 = tc::instr_desc(2, 128, 64, 0, 0);
-    const uint64_t dQ = tc::smem_desc(tc::smem_u32(sm + OFF_Q), 16, 1024);
-    const uint64_t dK = tc::smem_desc(tc::smem_u32(sm + OFF_K), 16, 1024);
-    const uint64_t dX1 = tc::smem_desc(tc::smem_u32(sm + OFF_X1), 16, 1024);
-    const uint64_t dX2 = tc::smem_desc(tc::smem_u32(sm + OFF_X2), 16, 1024);
+    constexpr uint32_t ID128 = tc::instr_desc(2, 128, 128, 0, 0);
+    constexpr uint32_t ID_F16 = tc::instr_desc(0, 128, 64, 0, 0);      // A in tensor memory, B K-major
+    constexpr uint32_t ID_F16_MN = tc::instr_desc(0, 128, 64, 0, 1);   // A in tensor memory, B MN-major
+    auto dsc = [&](const uint8_t* p, uint32_t lbo) { return tc::smem_desc(tc::smem_u32(p), lbo, 1024); };
+    const uint64_t dX1 = dsc(sm + OFF_X1, 16384);   // K fp16 [t][j], MN-major (one 64-wide block)
+    auto dX2 = [&](int n) { return dsc(sm + OFF_X2 + (n & 1) * 8192, 16); };
+    auto tb_of = [](int n) { return TM_B + 128u * (uint32_t)(n & 1); };
+    auto pk_of = [](int n) { return TM_PK + 32u * (uint32_t)(n & 1); };
+#ifdef TTT_DEBUG_STAGES
+    long long stamp_acc[8] = {};
+    long long stamp_last = clock64();
+#endif
 
-    auto wait_mma = [&](uint64_t* bar, uint32_t& ph) {
-        if (!tc::mbar_wait(bar, ph, abort_flag)) give_up();
-        ph ^= 1;
-        tc::tc_fence_after();
-    };
-    auto mma_stage_with = [&](auto issue, auto work) -> bool {
-        tc::fence_proxy_async_smem();
-        tc::tc_fence_before();
-        if (__syncthreads_or(*abort_flag)) return false;
-        tc::tc_fence_after();
-        if (tid == 0) issue();
-        work();
-        wait_mma(bar_mma, ph_mma);
-        return true;
-    };
-    // z of a finished chunk (rows i of quarters 0, 1; 16 tokens per thread) to global memory.
-    auto store_z = [&](uint32_t tz, int y0c, int bcc) {
-        if (q < 2) {
+    if (q < 2) {
+        // =====================================================================================
+        // E warps (0, 1, 4, 5, 8, 9, 12, 13): the chain.  Thread (q, g, lane) owns row i = 32 q + lane of
+        // the [i][t] tiles and tokens 16 g .. 16 g + 15; thread 0 issues the chain's products.
+        // =====================================================================================
+        const int et = (g * 2 + q) * 32 + lane;   // 0 .. 255 over the E warps
+        auto esync = [&]() -> bool {                // the E warps; true if some thread saw an abort
+            tc::fence_proxy_async_smem();
+            tc::tc_fence_before();
+            const bool ab = tc::bar_sync_or(1, 256, *abort_flag != 0);
+            tc::tc_fence_after();
+            return ab;
+        };
+        auto wait_mma = [&](uint64_t* bar, uint32_t& ph) {
+            wait_ok(bar, ph);
+            ph ^= 1;
+            tc::tc_fence_after();
+        };
+        // z of a finished chunk (16 tokens of row i per thread) to global memory
+        auto store_z = [&](uint32_t tz, int y0c, int bcc) {
             const int i = 32 * q + lane, t0 = 16 * g;
             uint32_t r[16];
             tc::tmem_ld_32x32b_x16(tm + lane_base + tz + t0, r);
@@ -187,121 +241,178 @@ __global__ void __launch_bounds__(THREADS, 1) scan_linear_tc_kernel(const __grid
 #pragma unroll
             for (int k = 0; k < 16; ++k)
                 if (t0 + k < bcc) zrow[(long long)(t0 + k) * a.x_ts] = __uint_as_float(r[k]);
-        }
-    };
-    int prev_y0 = 0, prev_bc = 0;
-
-    for (int c = c_first; c < c_last; ++c) {
-        int y0, bc;
-        chunk_rows(c, y0, bc);
-        const uint32_t tz = TM_Z + 64 * (c & 1);
-        if (warp == 0) {
-            if (!tc::mbar_wait(bar_ld, ph_ld, nullptr) && lane == 0) give_up();
-        }
-        ph_ld ^= 1;
-        if (bc < BT) {   // rows beyond the chunk: zero in K and Q (they then add nothing)
-            __syncthreads();
-            float* fK = reinterpret_cast<float*>(sm + OFF_K);
-            float* fQ = reinterpret_cast<float*>(sm + OFF_Q);
-            for (int idx = tid; idx < (BT - bc) * DH; idx += THREADS) {
-                const int rr = bc + idx / DH, j = idx % DH;
-                const uint32_t o = row4_off(rr, j & ~3) + (j & 3) * 4;
-                fK[o / 4] = 0.f;
-                fQ[o / 4] = 0.f;
+        };
+        uint32_t ph_g = 0, ph_u = 0, ph_c = 0, ph_s = 0;
+        int prev_y0 = 0, prev_bc = 0;
+        bool aborted = false;
+        for (int n = 0; n < nloc; ++n) {
+            int y0, bc;
+            chunk_rows(c_first + n, y0, bc);
+            const uint32_t tb = tb_of(n), pk = pk_of(n);
+            STAMPL(0);
+            // ---- 0: the chunk's tiles (rows beyond a short chunk cleared in K and Q), then the first
+            //      product [E^T_c | Z'^T_{c-1}] = W_c [K_c; Q_{c-1}]^T (the B rows 64.. are Q_{c-1})
+            if (tid == 0) wait_ok(bar_ld + (n & 1), (uint32_t)(n >> 1) & 1u);
+            if ((aborted = esync())) break;
+            if (bc < BT) {
+                float* fK = reinterpret_cast<float*>(k_tile(n));
+                float* fQ = reinterpret_cast<float*>(q_tile(n));
+                for (int idx = et; idx < (BT - bc) * DH; idx += 256) {
+                    const int rr = bc + idx / DH, j = idx % DH;
+                    const uint32_t o = row4_off(rr, j & ~3, KQ_HALF) + (j & 3) * 4;
+                    fK[o / 4] = 0.f;
+                    fQ[o / 4] = 0.f;
+                }
+                if ((aborted = esync())) break;
             }
-        }
-
-        // ---- 1: E^T = W K^T (waited for); then S = Q K^T, Z^T = W Q^T (bar_a2).
-        //      Meanwhile: the previous chunk's z out, K^T into X1.
-        if (!mma_stage_with(
-                [&] {
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_E, tm + TM_W + kk * 8, kstep(dK, kk), ID64, kk > 0);
-                    tc::mma_commit(bar_mma);
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ss(tm + TM_S, kstep(dQ, kk), kstep(dK, kk), ID64, kk > 0);
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + tz, tm + TM_W + kk * 8, kstep(dQ, kk), ID64, kk > 0);
-                    tc::mma_commit(bar_a2);
-                },
-                [&] {
-                    if (prev_bc) store_z(TM_Z + 64 * ((c - 1) & 1), prev_y0, prev_bc);
-                    {   // K^T: thread (j, 8 tokens): column reads of K, two 16-byte row writes of K^T
-                        const int j = tid & 63, tb = tid >> 6;
-                        uint32_t ph[8];
-                        col_phases(j, ph);
-                        const uint8_t* src = sm + OFF_K + tb * 1024;
-                        float v[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float*>(src + ph[e]);
-                        *reinterpret_cast<float4*>(sm + OFF_X1 + row4_off(j, 8 * tb)) =
-                            make_float4(v[0], v[1], v[2], v[3]);
-                        *reinterpret_cast<float4*>(sm + OFF_X1 + row4_off(j, 8 * tb + 4)) =
-                            make_float4(v[4], v[5], v[6], v[7]);
-                    }
-                }))
-            break;
-        prev_bc = 0;
-
-        // ---- 2 (threads): E'^T = -2 eta (E^T - V^T) in place (zero beyond the chunk); then the
-        //      prefix mask M from S once bar_a2 is done.  Rows of quarters 0, 1 only.
-        if (q < 2) {
-            const int i = 32 * q + lane, t0 = 16 * g;
-            const uint32_t addr = tm + lane_base + TM_E + t0;
-            uint32_t r[16], ph[8];
-            tc::tmem_ld_32x32b_x16(addr, r);
-            col_phases(i, ph);
-            const uint8_t* vrow = sm + OFF_V + (t0 >> 3) * 1024;
-            float vv[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) vv[k] = *reinterpret_cast<const float*>(vrow + ph[k & 7] + (k >> 3) * 1024);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                r[k] = __float_as_uint((t0 + k < bc) ? tf32r(m2eta * (__uint_as_float(r[k]) - vv[k])) : 0.f);
-            tc::tmem_st_32x32b_x16(addr, r);
-        }
-        wait_mma(bar_a2, ph_a2);
-        if (q < 2) {   // M[t][s] = S[t][s] for s not after t
-            const int t = 32 * q + lane, s0 = 16 * g;
-            uint32_t r[16];
-            tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
-            tc::tmem_wait_ld();
-            float m[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const bool later = a.reverse ? (s0 + k < t) : (s0 + k > t);
-                m[k] = later ? 0.f : tf32r(__uint_as_float(r[k]));
+            if (tid == 0) {
+                const uint64_t d = dsc(k_tile(n), 16);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + tb, tm + TM_W + kk * 8, kstep(d, kk, KQ_HALF), ID128, kk > 0);
+                tc::mma_commit(bar_g);
+                tc::mbar_arrive(bar_go);
             }
+            // ---- 1: K as fp16 [t][j] into X1 (the update of chunk c-1 has read it): thread (t, 16 j)
+            {
+                const int t = et >> 2, j0 = 16 * (et & 3);
+                const uint8_t* kt = k_tile(n);
+                float v[16];
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4)
-                *reinterpret_cast<float4*>(sm + OFF_X2 + row4_off(t, s0 + 4 * c4)) =
-                    make_float4(m[4 * c4], m[4 * c4 + 1], m[4 * c4 + 2], m[4 * c4 + 3]);
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const float4 f = *reinterpret_cast<const float4*>(kt + row4_off(t, j0 + 4 * c4, KQ_HALF));
+                    v[4 * c4] = f.x;
+                    v[4 * c4 + 1] = f.y;
+                    v[4 * c4 + 2] = f.z;
+                    v[4 * c4 + 3] = f.w;
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh)
+                    *reinterpret_cast<uint4*>(sm + OFF_X1 + h_chunk(t, j0 + 8 * hh)) =
+                        make_uint4(pack_h2(v[8 * hh], v[8 * hh + 1]), pack_h2(v[8 * hh + 2], v[8 * hh + 3]),
+                                   pack_h2(v[8 * hh + 4], v[8 * hh + 5]), pack_h2(v[8 * hh + 6], v[8 * hh + 7]));
+            }
+            // ---- 2: E'^T = -2 eta (E^T - V^T) as fp16 pairs (zero beyond the chunk)
+            wait_mma(bar_g, ph_g);
+            STAMPL(1);
+            {
+                const int i = 32 * q + lane, t0 = 16 * g;
+                uint32_t r[16], pr[8];
+                tc::tmem_ld_32x32b_x16(tm + lane_base + tb + t0, r);
+                const uint8_t* vt = v_tile(n);
+                float vv[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    vv[k] = *reinterpret_cast<const float*>(vt + row4_off(t0 + k, i & ~3, V_HALF) + (i & 3) * 4);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    const int k = 2 * k2;
+                    pr[k2] = pack_h2((t0 + k < bc) ? m2eta * (__uint_as_float(r[k]) - vv[k]) : 0.f,
+                                     (t0 + k + 1 < bc) ? m2eta * (__uint_as_float(r[k + 1]) - vv[k + 1]) : 0.f);
+                }
+                tc::tmem_st_32x32b_x8(tm + lane_base + pk + 8 * g, pr);
+                tc::tmem_wait_st();
+            }
+            if ((aborted = esync())) break;
+            STAMPL(2);
+            // ---- 3: W += E'^T K (the chain), then the previous chunk's correction
+            //      Z^T_{c-1} += E'^T_{c-1} (-Npost_{c-1})^T into the Z'_{c-1} the first product left here
+            if (tid == 0) {
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16_ts(tm + TM_W, tm + pk + kk * 8, kstep_mn(dX1, kk), ID_F16_MN, 1);
+                tc::mma_commit(bar_u);
+                if (n > 0) {
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc::mma_f16_ts(tm + tb + 64, tm + pk_of(n - 1) + kk * 8, kstep_h(dX2(n - 1), kk), ID_F16, 1);
+                    tc::mma_commit(bar_c);
+                }
+            }
+            //      meanwhile -Npost of chunk c (fp16, K-major row t) once S is done: thread (t, 16 s)
+            wait_mma(bar_s, ph_s);
+            {
+                const int t = 32 * q + lane, s0 = 16 * g;
+                uint32_t r[16], u[8];
+                tc::tmem_ld_32x32b_x16(tm + lane_base + TM_S + s0, r);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    const int s = s0 + 2 * k2;
+                    const bool l0 = a.reverse ? (s < t) : (s > t), l1 = a.reverse ? (s + 1 < t) : (s + 1 > t);
+                    u[k2] = pack_h2(l0 ? -__uint_as_float(r[2 * k2]) : 0.f, l1 ? -__uint_as_float(r[2 * k2 + 1]) : 0.f);
+                }
+                uint8_t* x2 = sm + OFF_X2 + (n & 1) * 8192;
+                *reinterpret_cast<uint4*>(x2 + h_chunk(t, s0)) = make_uint4(u[0], u[1], u[2], u[3]);
+                *reinterpret_cast<uint4*>(x2 + h_chunk(t, s0 + 8)) = make_uint4(u[4], u[5], u[6], u[7]);
+            }
+            //      and the previous chunk's z once its correction is done
+            if (n > 0) {
+                wait_mma(bar_c, ph_c);
+                store_z(tb + 64, prev_y0, prev_bc);
+            }
+            wait_mma(bar_u, ph_u);
+            STAMPL(3);
+            prev_y0 = y0;
+            prev_bc = bc;
+            if ((aborted = esync())) break;   // the mask, the z and W are done: the next chunk may start
         }
-        tc::tmem_wait_st();
-
-        // ---- 3: Z^T += E'^T M^T;  W += E'^T K.  Q, K, V are free: fetch the next chunk's tiles.
-        if (!mma_stage_with(
-                [&] {
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + tz, tm + TM_E + kk * 8, kstep(dX2, kk), ID64, 1);
-                    for (int kk = 0; kk < 8; ++kk)
-                        tc::mma_tf32_ts(tm + TM_W, tm + TM_E + kk * 8, kstep(dX1, kk), ID64, 1);
-                    tc::mma_commit(bar_mma);
-                    if (c + 1 < c_last) {
-                        int ny0, nbc;
-                        chunk_rows(c + 1, ny0, nbc);
-                        load_tiles(ny0);
-                    }
-                },
-                [] {}))
-            break;
-        prev_y0 = y0;
-        prev_bc = bc;
+        if (!aborted && nloc > 0) {   // the last chunk's output: Z'^T = W_{c+1} Q^T, then its correction
+            const int nl = nloc - 1;
+            const uint32_t tz = tb_of(nl + 1) + 64;
+            if (tid == 0) {
+                const uint64_t d = dsc(q_tile(nl), 16);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ts(tm + tz, tm + TM_W + kk * 8, kstep(d, kk, KQ_HALF), ID64, kk > 0);
+                tc::mma_commit(bar_c);
+            }
+            wait_mma(bar_c, ph_c);
+            if (tid == 0) {
+                for (int kk = 0; kk < 4; ++kk)
+                    tc::mma_f16_ts(tm + tz, tm + pk_of(nl) + kk * 8, kstep_h(dX2(nl), kk), ID_F16, 1);
+                tc::mma_commit(bar_c);
+            }
+            wait_mma(bar_c, ph_c);
+            store_z(tz, prev_y0, prev_bc);
+        }
+    } else if (warp == 2) {
+        // S = Q_c K_c^T once the chunk's first product is issued (A: 128 rows from Q; rows 64.. unused)
+        for (int n = 0; n < nloc; ++n) {
+            int ok = 1;
+            if (lane == 0) {
+                ok = wait_ok(bar_go, (uint32_t)n & 1u);
+                tc::tc_fence_after();
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) {
+                const uint64_t dq = dsc(q_tile(n), 16), dk = dsc(k_tile(n), 16);
+                for (int kk = 0; kk < 8; ++kk)
+                    tc::mma_tf32_ss(tm + TM_S, kstep(dq, kk, KQ_HALF), kstep(dk, kk, KQ_HALF), ID64, kk > 0);
+                tc::mma_commit(bar_s);
+            }
+            __syncwarp();
+        }
+    } else if (warp == 3) {
+        // the tiles, a chunk ahead: chunk n+1's go where chunk n-1's were, once chunk n's first
+        // product (the last reader of Q_{n-1}) is done
+        if (lane == 0 && nloc > 0) load_tiles(0);
+        for (int n = 0; n + 1 < nloc; ++n) {
+            int ok = 1;
+            if (lane == 0) ok = wait_ok(bar_g, (uint32_t)n & 1u);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            if (lane == 0) load_tiles(n + 1);
+            __syncwarp();
+        }
     }
-    if (prev_bc && !*abort_flag) store_z(TM_Z + 64 * ((c_last - 1) & 1), prev_y0, prev_bc);
 
-    if (*abort_flag) {
+#ifdef TTT_DEBUG_STAGES
+    if (tid == 0 && blockIdx.x == 0 && g_dbg_lin) {
+        for (int k = 0; k < 8; ++k) g_dbg_lin[k] = (float)stamp_acc[k];
+        g_dbg_lin[8] = (float)nloc;
+    }
+#endif
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    if (*abort_flag) {   // let copies and MMAs in flight land before the memory goes away
         const uint64_t t0 = tc::globaltimer_ns();
         while (tc::globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
     } else if (a.W_T && q < 2) {
@@ -347,6 +458,12 @@ bool make_map(CUtensorMap* m, const float* base, const LinearScanArgs& a, bool f
 }
 
 }  // namespace
+
+#ifdef TTT_DEBUG_STAGES
+extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump_lin(float* p) {
+    return (int)cudaMemcpyToSymbol(g_dbg_lin, &p, sizeof(p));
+}
+#endif
 
 bool scan_linear_tc_supported(int d, int b) { return d == DH && b >= 2 && b <= BT; }
 
