@@ -190,6 +190,58 @@ TTT_API ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, con
                                     ttt_stream_t stream);
 
 /*
+ * One rank's share of a head-sharded bidirectional layer (full-width input).
+ *
+ * Each head's chain is independent (paper notes page, "关键设计 / TTT-MLP 层":
+ * every head keeps its own hidden state), and the reverse direction reads the
+ * forward direction's output through theta_Q/K/V, which mix all channels
+ * ("关键设计 / 门控 + 双向机制").  So a layer split over R ranks by heads runs
+ * as two phases with one exchange between them:
+ *
+ *   TTT_PHASE_FWD  Q, K, V of heads [h0, h0 + hn) from X; the forward scan of
+ *                  those heads; the gate.  Writes, in the columns of those
+ *                  heads only, X' = X + tanh(alpha_f) z_f (fp32, Xp) and the
+ *                  gate increment bf16(tanh(alpha_f) z_f) (bf16, delta_or_y).
+ *   (exchange)     the caller sums every rank's increment array (the other
+ *                  ranks' columns are zero in each), e.g. an all-reduce.
+ *   TTT_PHASE_REV  Q, K, V of the same heads from theta X + theta delta_all;
+ *                  the reverse scan; the gate on X'.  Writes Y (bf16,
+ *                  delta_or_y) in the columns of those heads only.
+ *
+ * These are the computations of ttt_mlp_forward's bidirectional full-width
+ * layer restricted to the heads: with the same inputs and kernels every
+ * written element equals ttt_mlp_forward's.
+ *
+ *   desc       the WHOLE layer: T, H (all heads), d = 64, m, D = H * d,
+ *              per_head_input = 0, x_dtype = TTT_BF16.
+ *   h0, hn     the heads of this call: 0 <= h0, 1 <= hn, h0 + hn <= H.
+ *   X          [T, D] bf16; theta_q/k/v [D, D] bf16 (all rows; rows h0*d ..
+ *              (h0+hn)*d - 1 are read); W1_0 [H, m, d], W2_0 [H, d, m] fp32
+ *              (heads h0 .. h0+hn-1 read); alpha [D] fp32: alpha_f for the
+ *              forward phase, alpha_r for the reverse phase.
+ *   delta_all  TTT_PHASE_REV: [T, D] bf16, every head's increment; NULL for
+ *              TTT_PHASE_FWD.
+ *   Xp         [T, D] fp32: written by TTT_PHASE_FWD, read by TTT_PHASE_REV.
+ *   delta_or_y [T, D] bf16: the increment (TTT_PHASE_FWD) or Y (TTT_PHASE_REV).
+ *   b          2 <= b <= 64 (the tensor-core scan).
+ *   workspace  ttt_mlp_heads_workspace_size(desc, hn, b) bytes, 256-byte
+ *              aligned; ttt_mlp_status(workspace, stream) reports non-finite
+ *              values and expired waits as for ttt_mlp_forward.
+ * Columns of other heads are neither read (Xp, in the reverse phase) nor
+ * written.  Asynchronous on `stream`; no allocation.  Returns
+ * TTT_ERR_UNSUPPORTED for shapes outside the tensor-core path.
+ */
+typedef enum { TTT_PHASE_FWD = 0, TTT_PHASE_REV = 1 } ttt_phase;
+
+TTT_API size_t ttt_mlp_heads_workspace_size(const ttt_mlp_desc* desc, int hn, int b);
+TTT_API ttt_status ttt_mlp_forward_heads(const ttt_mlp_desc* desc, int h0, int hn, ttt_phase phase,
+                                         const void* X, const void* theta_q, const void* theta_k,
+                                         const void* theta_v, const float* W1_0, const float* W2_0, float eta,
+                                         int b, const float* alpha, const void* delta_all, float* Xp,
+                                         void* delta_or_y, void* workspace, size_t workspace_bytes,
+                                         ttt_stream_t stream);
+
+/*
  * ttt_mlp_forward for callers that cannot allocate device memory.
  *
  * The paper has no counterpart: this is a deployment aid.  Code embedded in a

@@ -935,6 +935,83 @@ ttt_status ttt_mlp_status(void* workspace, ttt_stream_t stream_) {
     return TTT_OK;
 }
 
+// ---------------------------------------------------------------- one rank's heads
+size_t ttt_mlp_heads_workspace_size(const ttt_mlp_desc* desc, int hn, int b) {
+    if (check_desc(desc, b, TTT_BIDIR) != TTT_OK || hn < 1 || hn > desc->H) return 0;
+    const size_t nl = (size_t)desc->T * hn * desc->d;
+    return kAlign + 3 * align_up(nl * sizeof(float));
+}
+
+ttt_status ttt_mlp_forward_heads(const ttt_mlp_desc* desc, int h0, int hn, ttt_phase phase, const void* X,
+                                 const void* theta_q, const void* theta_k, const void* theta_v, const float* W1_0,
+                                 const float* W2_0, float eta, int b, const float* alpha, const void* delta_all,
+                                 float* Xp, void* delta_or_y, void* workspace, size_t workspace_bytes,
+                                 ttt_stream_t stream_) {
+    ttt_status st = check_desc(desc, b, TTT_BIDIR);
+    if (st != TTT_OK) return st;
+    const ttt_mlp_desc& q = *desc;
+    if (q.per_head_input || q.x_dtype != TTT_BF16)
+        return fail(TTT_ERR_UNSUPPORTED, "head phases need a full-width bf16 layer");
+    if (!scan_chunk_tc_supported(q.d, b) || !proj_full_tc_supported(q.d, q.D))
+        return fail(TTT_ERR_UNSUPPORTED, "head phases need d = 64, 2 <= b <= 64 and D %% 64 == 0");
+    if (phase != TTT_PHASE_FWD && phase != TTT_PHASE_REV) return fail(TTT_ERR_INVALID_ARG, "bad phase");
+    if (h0 < 0 || hn < 1 || h0 + hn > q.H)
+        return fail(TTT_ERR_INVALID_ARG, "heads [%d, %d) outside [0, %d)", h0, h0 + hn, q.H);
+    const bool rev = phase == TTT_PHASE_REV;
+    st = check_ptrs(q, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, TTT_FWD, alpha, alpha);
+    if (st != TTT_OK) return st;
+    if (!Xp || !delta_or_y || !workspace || (rev && !delta_all))
+        return fail(TTT_ERR_INVALID_ARG, "Xp, delta_or_y, workspace (and delta_all for the reverse phase) needed");
+    const void* ps[] = {Xp, delta_or_y, delta_all};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+        return fail(TTT_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    const size_t need = ttt_mlp_heads_workspace_size(desc, hn, b);
+    if (workspace_bytes < need)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    char* ws = static_cast<char*>(workspace);
+    int* status = reinterpret_cast<int*>(ws);
+    CUDA_TRY(cudaMemsetAsync(ws, 0, 16, s));
+    const int N = hn * q.d;
+    const size_t nl = (size_t)q.T * N;
+    float* qkv[3];
+    for (int w = 0; w < 3; ++w) qkv[w] = reinterpret_cast<float*>(ws + kAlign + w * align_up(nl * sizeof(float)));
+    // the heads' rows of theta: Q, K, V [T, hn d] from X (and, reverse, the gate increment of every head)
+    const size_t row0 = (size_t)h0 * q.d * q.D;
+    const void* th[3] = {static_cast<const __nv_bfloat16*>(theta_q) + row0,
+                         static_cast<const __nv_bfloat16*>(theta_k) + row0,
+                         static_cast<const __nv_bfloat16*>(theta_v) + row0};
+    CUDA_TRY(launch_proj_full_tc(X, th, qkv, q.T, N, q.D, 0, status, 0, s));
+    if (rev) CUDA_TRY(launch_proj_full_tc(delta_all, th, qkv, q.T, N, q.D, 1, status, 0, s));
+
+    ScanArgs a{};
+    a.Q = qkv[0]; a.K = qkv[1]; a.V = qkv[2];
+    a.qkv_hs = q.d; a.qkv_ts = N;
+    a.x_hs = q.d; a.x_ts = q.D;   // X, X', the increment and Y: [T, D], these heads' columns
+    const size_t col0 = (size_t)h0 * q.d;
+    __nv_bfloat16* dy = static_cast<__nv_bfloat16*>(delta_or_y) + col0;
+    if (rev) {
+        a.Xin = Xp + col0; a.xin_bf16 = 0;
+        a.Out = dy; a.out_bf16 = 1; a.Delta = nullptr;
+    } else {
+        a.Xin = static_cast<const __nv_bfloat16*>(X) + col0; a.xin_bf16 = 1;
+        a.Out = Xp + col0; a.out_bf16 = 0; a.Delta = dy;
+    }
+    a.alpha = alpha + col0;
+    a.W1_0 = W1_0 + (size_t)h0 * q.m * q.d;
+    a.W2_0 = W2_0 + (size_t)h0 * q.d * q.m;
+    a.T = q.T; a.H = hn; a.d = q.d; a.m = q.m; a.b = b; a.reverse = rev ? 1 : 0;
+    a.eta = eta;
+    a.status = status;
+    a.inject_timeout = g_inject_timeout.load();
+    a.fuse_gate = 1;
+    CUDA_TRY(launch_scan_chunk_tc3(a, s));
+    return TTT_OK;
+}
+
 ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, const void* theta_q,
                                 const void* theta_k, const void* theta_v, const float* W1_0, const float* W2_0,
                                 float eta, int b, ttt_direction dir, const float* alpha_f, const float* alpha_r,

@@ -38,6 +38,7 @@ struct ProjTcArgs {
     CUtensorMap mapB[3];
     CUtensorMap mapC[3];
     int K;                 // reduction length (model dim)
+    int N;                 // output columns of each projection (a multiple of 64; the last tile may be partial)
     int m_tiles, n_tiles_per, tiles;
     int accumulate;
     int* status;
@@ -166,8 +167,10 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
                 __syncwarp();
                 if (lane == 0) {
                     const int x = n0 + c * 32, y = mt * BM + 32 * q;
-                    if (p.accumulate) tc::tma_reduce_add_2d(&p.mapC[which], buf, x, y);
-                    else tc::tma_store_2d(&p.mapC[which], buf, x, y);
+                    if (x < p.N) {   // columns of a partial last tile beyond N are zero (theta rows read as fill)
+                        if (p.accumulate) tc::tma_reduce_add_2d(&p.mapC[which], buf, x, y);
+                        else tc::tma_store_2d(&p.mapC[which], buf, x, y);
+                    }
                     tc::bulk_commit_group();
                 }
                 nbuf ^= 1;
@@ -222,7 +225,9 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 
 }  // namespace
 
-bool proj_full_tc_supported(int N, int K) { return N % BN == 0 && K % BK == 0 && N > 0 && K > 0; }
+// N: whole 32-column boxes of the epilogue (64 keeps every box either inside or past N); the B loads of a
+// partial last tile read theta rows beyond N as zero fill.
+bool proj_full_tc_supported(int N, int K) { return N % 64 == 0 && K % BK == 0 && N > 0 && K > 0; }
 
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
                                 int accumulate, int* status, int max_ctas, cudaStream_t s) {
@@ -234,8 +239,9 @@ cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float
     }
     if (!ok) return cudaErrorInvalidValue;
     p.K = K;
+    p.N = N;
     p.m_tiles = (T + BM - 1) / BM;
-    p.n_tiles_per = N / BN;
+    p.n_tiles_per = (N + BN - 1) / BN;
     p.tiles = p.m_tiles * 3 * p.n_tiles_per;
     p.accumulate = accumulate;
     p.status = status;

@@ -20,13 +20,15 @@ STATUS_NAMES = {0: "TTT_OK", 1: "TTT_ERR_INVALID_ARG", 2: "TTT_ERR_UNSUPPORTED",
                 4: "TTT_ERR_NONFINITE", 5: "TTT_ERR_TIMEOUT"}
 TTT_FWD, TTT_REV, TTT_BIDIR = 0, 1, 2
 TTT_F32, TTT_BF16 = 0, 1
+TTT_PHASE_FWD, TTT_PHASE_REV = 0, 1
 DIRS = {"fwd": TTT_FWD, "rev": TTT_REV, "bidir": TTT_BIDIR}
 
 EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_mlp_host_io_workspace_size",
             "ttt_mlp_forward_host", "ttt_mlp_select_kernels", "ttt_last_error", "ttt_launch_count",
             "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_mlp_noalloc_status", "ttt_debug_inject_wait_timeout",
             "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments",
-            "ttt_mlp_backward_workspace_size", "ttt_mlp_backward"]
+            "ttt_mlp_backward_workspace_size", "ttt_mlp_backward", "ttt_mlp_heads_workspace_size",
+            "ttt_mlp_forward_heads"]
 
 
 class TTTError(RuntimeError):
@@ -72,6 +74,10 @@ def lib():
         L.ttt_mlp_backward.restype = i
         L.ttt_mlp_backward.argtypes = [dp, vp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        vp, sz, vp]
+        L.ttt_mlp_heads_workspace_size.restype = sz
+        L.ttt_mlp_heads_workspace_size.argtypes = [dp, i, i]
+        L.ttt_mlp_forward_heads.restype = i
+        L.ttt_mlp_forward_heads.argtypes = [dp, i, i, i, vp, vp, vp, vp, vp, vp, f, i, vp, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_noalloc_status.restype = i
         L.ttt_mlp_noalloc_status.argtypes = [vp]
         L.ttt_linear_workspace_size.restype = sz
@@ -235,6 +241,18 @@ def layer_backward(X, theta_q, theta_k, theta_v, W1_0, W2_0, eta: float, b: int,
         check(ttt_mlp_status(workspace, stream), "ttt_mlp_status")
     out["workspace"] = workspace
     return out
+
+
+def ttt_mlp_heads_workspace_size(desc: ttt_mlp_desc, hn: int, b: int) -> int:
+    return int(lib().ttt_mlp_heads_workspace_size(ctypes.byref(desc), hn, b))
+
+
+def ttt_mlp_forward_heads(desc, h0, hn, phase, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, alpha, delta_all,
+                          Xp, delta_or_y, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_mlp_forward_heads(ctypes.byref(desc), h0, hn, phase, _p(X), _p(theta_q), _p(theta_k),
+                                           _p(theta_v), _p(W1_0), _p(W2_0), float(eta), b, _p(alpha),
+                                           _p(delta_all), _p(Xp), _p(delta_or_y), _p(workspace), workspace_bytes,
+                                           _stream(stream)))
 
 
 def ttt_mlp_noalloc_status(stream=None) -> int:
