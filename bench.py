@@ -732,6 +732,66 @@ def spawn_command(argv, n: int, port: int) -> list:
             "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
 
 
+def run_sharded(args, rank, world, local_rank):
+    """One sequence of the full-width bidirectional layer with its heads split over
+    the ranks (test_rnn_layer_b200/shard.py): per rank the forward phase of its
+    heads, an all-reduce of the gate increment, the reverse phase, an
+    all-reduce of Y.  Strong scaling: `value` is the sequence's tokens per
+    second of the slowest rank."""
+    import torch
+    import torch.distributed as dist
+
+    from test_rnn_layer_b200 import shard
+    from test_rnn_layer_b200 import synth as S
+    from test_rnn_layer_b200 import tttmlp as L
+
+    L.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = _workload(args)
+    if w.per_head or w.dirs != "bidir" or w.dtype != "bf16":
+        raise SystemExit("--shard-heads needs the full-width bidirectional bf16 layer (--workload full63s)")
+    inp = S.make_inputs(w, seed=0, device=dev)   # the same sequence on every rank
+    th = [inp["theta_q"], inp["theta_k"], inp["theta_v"]]
+    desc = L.make_desc(w.T, w.H, w.d, False, True)
+    h0, hn = shard.head_range(w.H, rank, world)
+    ws = shard.heads_workspace(desc, hn, w.b, dev)
+    stream = torch.cuda.current_stream()
+    all_reduce = (lambda t: dist.all_reduce(t)) if world > 1 else (lambda t: None)
+
+    def fwd(X, theta, W1_0, W2_0, eta, b, alpha_f, r, n):
+        return shard.shard_forward(X, theta, W1_0, W2_0, eta, b, alpha_f, r, n, workspace=ws, stream=stream)
+
+    def rev(X, theta, W1_0, W2_0, eta, b, alpha_r, inc, Xp, r, n):
+        return shard.shard_reverse(X, theta, W1_0, W2_0, eta, b, alpha_r, inc, Xp, r, n, workspace=ws,
+                                   stream=stream)
+
+    def step():
+        shard.sharded_layer_forward(inp["X"], th, inp["W1_0"], inp["W2_0"], w.eta_eff, w.b, inp["alpha_f"],
+                                    inp["alpha_r"], rank, world, all_reduce, forward_step=fwd, reverse_step=rev)
+
+    n_launch0 = L.ttt_launch_count()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    time.sleep(0.3)
+    ms = _timed_steps(step, args, world, local_rank, stream, _input_bytes(w) <= 126e6)
+    clocks = sampler.stop()
+    launches = (L.ttt_launch_count() - n_launch0) * args.steps // (args.steps + args.warmup)
+    L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
+    ms_per_step = ms / args.steps
+    if rank == 0:
+        line = {"metric": _metric(w, "mlp"), "value": w.T / (ms_per_step * 1e-3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                "dtype": "bf16-in/tf32+fp16-mma/fp32-state", "data": "synthetic",
+                "config": _config(w, {"parallelism": f"heads split over {world} rank(s), one sequence",
+                                      "heads_per_rank": hn}),
+                "clocks": clocks, "gpu_launches": launches}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -753,6 +813,9 @@ def main():
     ap.add_argument("--cpu-reps", type=int, default=4, help="passes of the oracle's sample for the CPU baseline")
     ap.add_argument("--backward", action="store_true",
                     help="time one training step (forward recomputed + backward) instead of the forward layer")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="one sequence of the full-width layer split by heads over the ranks (strong scaling; "
+                         "an all-reduce of the gate increment between the directions) instead of replicas")
     ap.add_argument("--dry-run-host", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -784,6 +847,8 @@ def main():
             return run_dry_host(args, rank, world)
         if args.backward:
             return run_backward(args, rank, world, local_rank)
+        if args.shard_heads:
+            return run_sharded(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
