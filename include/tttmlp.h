@@ -25,11 +25,13 @@
  * default stream) and the functions return once it is enqueued, except
  * ttt_mlp_status and ttt_mlp_forward_host, which synchronise the stream.
  * The full-width bf16 layer on the tensor-core path runs in chunk segments on
- * the library's own streams (created once per device on first use, shared by
- * all callers, which are ordered among themselves while they enqueue); the
- * call forks from `stream` and joins back into it with events, also when it
- * fails part-way, so `stream` orders everything it launched, and the call can
- * be captured into a CUDA graph (after one call outside the capture).
+ * the library's own streams: one set per device and caller stream, created on
+ * the first call with that stream (calls with the same `stream` take turns
+ * while they enqueue; calls with different streams do not wait on each
+ * other).  The call forks from `stream` and joins back into it with events,
+ * also when it fails part-way, so `stream` orders everything it launched, and
+ * the call can be captured into a CUDA graph (after one call on the capturing
+ * stream outside the capture).
  * "Allocate nothing" means no device memory: those streams and their events
  * are the only resources the library creates.
  */

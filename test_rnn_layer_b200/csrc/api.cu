@@ -9,6 +9,8 @@
 #include <algorithm>
 #include <atomic>
 #include <functional>
+#include <map>
+#include <memory>
 #include <cstdarg>
 #include <cmath>
 #include <cstdio>
@@ -256,14 +258,25 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
 // Only stream order and events connect the two streams (no kernel waits on
 // another).  Projection and gate launches next to a running scan are capped
 // to the free SMs less a margin, so that every CTA pair of the next scan
-// segment finds room; the scan stream has the higher priority.
+// segment finds room; the scan stream has the higher priority.  Each (device,
+// caller stream) pair has its own set of library streams and events, so calls
+// on different caller streams neither wait on each other nor share events;
+// calls on one caller stream take turns while they enqueue.
 struct Pipe {
     cudaStream_t scan = nullptr, side = nullptr, copy = nullptr;
     std::vector<cudaEvent_t> ev;
     int sms = 0;
+    std::mutex mu;
 };
-std::mutex g_pipe_mu;
-Pipe g_pipes[64];
+std::mutex g_pipe_mu;   // guards g_pipes (not the enqueue)
+std::map<std::pair<int, cudaStream_t>, std::unique_ptr<Pipe>> g_pipes;
+
+Pipe& pipe_for(int dev, cudaStream_t caller) {
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    std::unique_ptr<Pipe>& p = g_pipes[{dev, caller}];
+    if (!p) p.reset(new Pipe());
+    return *p;
+}
 
 constexpr int kPipeMinSegChunks = 16;
 #ifndef TTT_PIPE_SM_MARGIN
@@ -346,11 +359,10 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_
                              const void* X, const void* const th[3], float* const qkv[3], int b, ttt_direction dir,
                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, cudaStream_t s,
                              const void* X_host, void* Y_host, bool scan_gates = false) {
-    std::lock_guard<std::mutex> lk(g_pipe_mu);
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= 64) return fail(TTT_ERR_UNSUPPORTED, "device index %d", dev);
-    Pipe& P = g_pipes[dev];
+    Pipe& P = pipe_for(dev, s);
+    std::lock_guard<std::mutex> lk(P.mu);
     if (!P.scan) {
         int lo = 0, hi = 0;
         CUDA_TRY(cudaDeviceGetStreamPriorityRange(&lo, &hi));
