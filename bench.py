@@ -71,6 +71,7 @@ KERNEL_SRC = {
     "scan_chunk_tc2": ("scan_chunk_tc2.cu",),
     "scan_chunk_tc3": ("scan_chunk_tc3.cu",),
     "scan_token": ("scan_token.cu",),
+    "scan_token_cluster": ("scan_token_cluster.cu",),
     "proj_full_simt": ("proj_simt.cu",),
     "proj_full_tc": ("proj_tc.cu",),
     "proj_per_head": ("proj_simt.cu",),
@@ -197,6 +198,7 @@ def _algorithmic(w):
         "scan_chunk_tc3": ("tensor_mixed", scan_flops),
         "scan_chunk_simt": ("alu", scan_flops),
         "scan_token": ("alu", H * T * 7 * 2 * d * m),
+        "scan_token_cluster": ("alu", H * T * 7 * 2 * d * m),
         "proj_full_tc": ("tensor_bf16", proj_flops),
         "proj_full_simt": ("alu", proj_flops),
         "proj_per_head": ("hbm", T * D * (2 + 12)),

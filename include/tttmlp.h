@@ -292,8 +292,10 @@ TTT_API ttt_status ttt_mlp_noalloc_status(ttt_stream_t stream);
  * 2 = the tensor-core kernels (a later ttt_mlp_forward returns
  * TTT_ERR_UNSUPPORTED if the shape is outside them), and for the scan only
  * 3 = the tensor-core scan with one CTA per head instead of a two-CTA
- * cluster, 4 = the two-CTA tensor-core scan whose CTAs each run the state
- * chain and the output of the chunk before on separate warp groups.
+ * cluster (for b = 1: the per-token kernel with one CTA per head instead of
+ * the four-CTA cluster that automatic selection uses for d = 64), 4 = the
+ * two-CTA tensor-core scan whose CTAs each run the state chain and the output
+ * of the chunk before on separate warp groups.
  * scan_impl selects the scan kernel, proj_impl the full-mode
  * projection kernel.
  */

@@ -224,7 +224,11 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
     const int impl = g_scan_impl.load();
     const bool tc_ok = scan_chunk_tc_supported(q.d, b);
     if (impl == 2 && !tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
-    if (impl == 3) {
+    if (impl == 3) {   // one CTA per head
+        if (b == 1) {
+            CUDA_TRY(launch_scan_token(a, s));
+            return TTT_OK;
+        }
         if (!tc_ok) return fail(TTT_ERR_UNSUPPORTED, "tensor-core scan needs d = 64 and 2 <= b <= 64");
         CUDA_TRY(launch_scan_chunk_tc(a, s));
     } else if (impl == 2 || impl == 4 || (impl == 0 && tc_ok && q.x_dtype == TTT_BF16)) {
@@ -240,8 +244,9 @@ ttt_status scan(const ttt_mlp_desc& q, const Layout& L, char* ws, const float* W
             CUDA_TRY(launch_gate(dd.xin, dd.xin_bf16, a.Zscan, dd.alpha, dd.out, dd.out_bf16, dd.delta, a.status,
                                  q.T, q.H, q.d, q.per_head_input, 0, s));
         }
-    } else if (b == 1 && impl != 1) {
-        CUDA_TRY(launch_scan_token(a, s));
+    } else if (b == 1 && impl != 1) {   // per token: a head's state over a four-CTA cluster where it fits
+        if (scan_token_cluster_supported(q.d)) CUDA_TRY(launch_scan_token_cluster(a, s));
+        else CUDA_TRY(launch_scan_token(a, s));
     } else {
         CUDA_TRY(launch_scan_chunk_simt(a, s));
     }

@@ -46,7 +46,10 @@ struct ScanArgs {
 };
 
 // Scan kernels.  Each returns a cudaError_t from the launch.
-cudaError_t launch_scan_token(const ScanArgs& a, cudaStream_t s);        // b == 1
+cudaError_t launch_scan_token(const ScanArgs& a, cudaStream_t s);        // b == 1, one CTA per head
+// b == 1, d = 64: a head's state sharded over a cluster of four CTAs
+bool scan_token_cluster_supported(int d);
+cudaError_t launch_scan_token_cluster(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_scan_chunk_simt(const ScanArgs& a, cudaStream_t s);   // any b
 long long scan_chunk_simt_scratch_floats(int d, int m, int b);
 // tcgen05 chunk scan: d = 64, 2 <= b <= 64, tf32 contractions with fp32 accumulation.

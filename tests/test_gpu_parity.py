@@ -204,3 +204,19 @@ def test_one_cta_tensor_core_scan(w):
         _check(w)
     finally:
         L.ttt_mlp_select_kernels(0, 0)
+
+
+@pytest.mark.parametrize("dirs", ["fwd", "rev", "bidir"])
+@pytest.mark.parametrize("sel", [0, 3], ids=["four-cta-cluster", "one-cta"])
+@pytest.mark.parametrize("per_head", [True, False], ids=["per-head", "full-width"])
+def test_per_token_kernels_d64(sel, dirs, per_head):
+    """b = 1 at d = 64: the per-token scan with each head's state over a cluster of
+    four CTAs (automatic) and with one CTA per head (selector 3), every direction,
+    a token count that is not a multiple of the 32-token staging block."""
+    w = S.Workload("tok-d64", H=3, d=64, T=150, b=1, dirs=dirs, dtype="f32", per_head=per_head, eta=0.05,
+                   D=0 if per_head else 192)
+    L.check(L.ttt_mlp_select_kernels(sel, 0), "select")
+    try:
+        _check(w)
+    finally:
+        L.ttt_mlp_select_kernels(0, 0)
