@@ -13,11 +13,12 @@
 // sums over hidden units (W2 g for the token's y, W2 g_q for the previous
 // token's z) are a shuffle reduce-scatter inside a warp, a sum over the 8
 // warps in shared memory, and a sum over the 4 CTAs whose partials cross
-// distributed shared memory.  The previous token's z is summed together with
+// distributed shared memory as 16-byte asynchronous stores that complete bytes
+// on the receiver's barrier.  The previous token's z is summed together with
 // the current token's y (both read the same state), so each token costs one
-// cluster barrier.  The receive buffers alternate by token parity: a CTA
-// writes buffer p for token n only after every CTA passed the barrier of token
-// n - 1, i.e. after every CTA finished reading buffer p for token n - 2.
+// exchange.  The receive buffers and barriers alternate by token parity: a CTA
+// sends token n + 2's partials only after it received every peer's token n + 1
+// partials, which each peer sends only after it read its buffer for token n.
 #include "common.cuh"
 #include "internal.h"
 #include "tc_prims.cuh"
@@ -82,6 +83,8 @@ __global__ void __launch_bounds__(NT, 1) scan_token_cluster_kernel(ScanArgs a) {
     __shared__ __align__(16) float sY[NT / 32][DT], sZ[NT / 32][DT];
     __shared__ __align__(16) float rcv[2][NCTA][2 * DT];   // [token parity][sender][y partial | z partial]
     __shared__ __align__(16) float sE[DT];   // 16-byte loads of sK, sQ, sE rows
+    __shared__ __align__(8) uint64_t rcvbar[2];   // the peers' partials of a token parity have landed
+    __shared__ int abort_flag;
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int il = tid >> 2, qd = tid & 3;
@@ -107,7 +110,16 @@ __global__ void __launch_bounds__(NT, 1) scan_token_cluster_kernel(ScanArgs a) {
     if (jout >= 0 && jout < DT) tanh_a = tanhf(a.alpha[h * DT + jout]);
     int nonfinite = 0;
     const uint32_t rcv_base = tc::smem_u32(&rcv[0][0][0]);
-    tc::cluster_sync();   // every CTA of the cluster runs before any distributed store
+    constexpr uint32_t kPeerBytes = (NCTA - 1) * 32 * 16;   // three peers x 32 x 16-byte stores per token
+    if (tid == 0) {
+        tc::mbar_init(&rcvbar[0], 1);
+        tc::mbar_init(&rcvbar[1], 1);
+        abort_flag = 0;
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(&rcvbar[0], kPeerBytes);   // tokens 0 and 1
+        tc::mbar_arrive_expect_tx(&rcvbar[1], kPeerBytes);
+    }
+    tc::cluster_sync();   // every CTA of the cluster runs, its barriers armed, before any distributed store
 
 #ifdef TTT_DEBUG_STAGES
     long long stamp_acc[12] = {};
@@ -175,21 +187,41 @@ __global__ void __launch_bounds__(NT, 1) scan_token_cluster_kernel(ScanArgs a) {
         STAMPT(1);
         __syncthreads();
         STAMPT(2);
-        // ---- B: this CTA's partials to every CTA of the cluster (itself included)
+        // ---- B: this CTA's partials (warp 0: 4 consecutive sums per lane) into its own slot of every
+        //      CTA's receive buffer: a plain store here, 16-byte stores that complete bytes on the receive
+        //      barrier of the three peers
         const int par = n & 1;
-        if (tid < 2 * DT) {
-            float v = 0.f;
-            const bool isy = tid < DT;
+        if (w == 0) {
+            const int k0 = 4 * lane;   // y sums 0..63, z sums 64..127
+            const bool isy = k0 < DT;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (isy ? tok : prev) {
 #pragma unroll
-                for (int ww = 0; ww < NT / 32; ++ww) v += isy ? sY[ww][tid] : sZ[ww][tid - DT];
+                for (int ww = 0; ww < NT / 32; ++ww) {
+                    const float4 f = *reinterpret_cast<const float4*>(isy ? &sY[ww][k0] : &sZ[ww][k0 - DT]);
+                    v.x += f.x; v.y += f.y; v.z += f.z; v.w += f.w;
+                }
             }
-            const uint32_t off = (uint32_t)(((par * NCTA + (int)r_cta) * 2 * DT + tid) * 4);
+            *reinterpret_cast<float4*>(&rcv[par][r_cta][k0]) = v;
+            const uint32_t off = (uint32_t)(((par * NCTA + (int)r_cta) * 2 * DT + k0) * 4);
+            const uint32_t bar = tc::smem_u32(&rcvbar[par]);
 #pragma unroll
-            for (int dst = 0; dst < NCTA; ++dst) tc::st_cluster_f32(tc::mapa_shared(rcv_base + off, dst), v);
+            for (int d1 = 1; d1 < NCTA; ++d1) {
+                const uint32_t dst = (r_cta + (uint32_t)d1) % NCTA;
+                tc::st_async_v4(tc::mapa_shared(rcv_base + off, dst), __float_as_uint(v.x), __float_as_uint(v.y),
+                                __float_as_uint(v.z), __float_as_uint(v.w), tc::mapa_shared(bar, dst));
+            }
         }
         STAMPT(3);
-        tc::cluster_sync();
+        __syncthreads();   // my own partials are visible
+        if (tid < 2 * DT) {   // the peers' partials of this token have landed (bounded wait)
+            if (!tc::mbar_wait_cluster_abort(&rcvbar[par], (uint32_t)(n >> 1) & 1u, &abort_flag)) {
+                abort_flag = 1;
+                atomicOr(a.status, kStatusTimeout);
+            }
+            // arm the barrier for token n + 2 (its bytes come only after this CTA's token n + 1 partials)
+            if (tid == 0) tc::mbar_arrive_expect_tx(&rcvbar[par], kPeerBytes);
+        }
         STAMPT(4);
         // ---- C: e' of token n; z and the gate of token n-1 (each CTA stores 16 of the 64 channels)
         if (tid < DT) {
@@ -212,7 +244,7 @@ __global__ void __launch_bounds__(NT, 1) scan_token_cluster_kernel(ScanArgs a) {
             nonfinite |= !isfinite(z);
         }
         STAMPT(5);
-        __syncthreads();
+        if (__syncthreads_or(abort_flag)) break;
         STAMPT(6);
         // ---- D: the update with e' (W2^T e' read before W2 changes)
         if (tok) {
@@ -259,6 +291,10 @@ __global__ void __launch_bounds__(NT, 1) scan_token_cluster_kernel(ScanArgs a) {
         g_dbg_tok[12] = (float)T;
     }
 #endif
+    if (abort_flag) {   // let a peer's stores already in flight land before the memory goes away
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (tc::globaltimer_ns() - t0 < 1000000ull) __nanosleep(1000);
+    }
     tc::cluster_sync();   // no CTA leaves while a peer may still address its shared memory
 }
 
