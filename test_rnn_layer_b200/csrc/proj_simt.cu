@@ -125,6 +125,74 @@ proj_full_simt_kernel(const void* A, int a_bf16, const void* B0, const void* B1,
     if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(status, kStatusNonFinite);
 }
 
+// d = 64: one head, 512 tokens per CTA in tiles of 128.  U [128 x 192] =
+// X [128 x 64] Theta^T [64 x 192] with both operands transposed in shared
+// memory (k-major rows, so that a thread's 8 tokens and its 4-wide output
+// groups are 16-byte loads) and 8 x 12 outputs per thread: 5 shared loads per
+// 96 FMAs.  Thread (ty, tx) computes tokens 8 ty .. 8 ty + 7 and, for each of
+// Q, K, V, channels 4 tx .. 4 tx + 3, so 16 threads store one 256-byte row of
+// an output with float4 stores.
+constexpr int kP64Tile = 128, kP64Tok = 512, kP64XS = kP64Tile + 4, kP64TS = 3 * 64 + 4;
+
+__global__ void __launch_bounds__(256, 2)
+proj_per_head64_kernel(const void* X, int x_bf16, const void* thq, const void* thk, const void* thv, int th_bf16,
+                       float* oq, float* ok, float* ov, int T, int* status) {
+    extern __shared__ __align__(16) float sm64[];
+    float* thT = sm64;                  // [64][kP64TS]: thT[k][w 64 + e] = theta_w[h][e][k]
+    float* xT = sm64 + 64 * kP64TS;     // [64][kP64XS]: xT[k][r] = x[h][t0 + r][k]
+    const int h = blockIdx.y, tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const void* ths[3] = {thq, thk, thv};
+    float* outs[3] = {oq, ok, ov};
+    for (int p = tid; p < 3 * 64 * 64; p += 256) {   // consecutive threads read consecutive k of a row e
+        const int w = p >> 12, e = (p >> 6) & 63, k = p & 63;
+        thT[k * kP64TS + w * 64 + e] = load_elem(ths[w], (long long)h * 4096 + e * 64 + k, th_bf16);
+    }
+    int bad = 0;
+    for (int t0 = blockIdx.x * kP64Tok; t0 < min(T, (int)(blockIdx.x + 1) * kP64Tok); t0 += kP64Tile) {
+        const int nt = min(kP64Tile, T - t0);
+        __syncthreads();   // the previous tile's xT reads are done (and theta is in place)
+        for (int p = tid; p < kP64Tile * 64; p += 256) {
+            const int r = p >> 6, k = p & 63;
+            xT[k * kP64XS + r] = r < nt ? load_elem(X, ((long long)h * T + t0 + r) * 64 + k, x_bf16) : 0.f;
+        }
+        __syncthreads();
+        float acc[8][12];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int c = 0; c < 12; ++c) acc[i][c] = 0.f;
+#pragma unroll 2
+        for (int k = 0; k < 64; ++k) {
+            const float4 x0 = *reinterpret_cast<const float4*>(xT + k * kP64XS + 8 * ty);
+            const float4 x1 = *reinterpret_cast<const float4*>(xT + k * kP64XS + 8 * ty + 4);
+            const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+            float tv[12];
+#pragma unroll
+            for (int g = 0; g < 3; ++g) {
+                const float4 f = *reinterpret_cast<const float4*>(thT + k * kP64TS + 64 * g + 4 * tx);
+                tv[4 * g] = f.x; tv[4 * g + 1] = f.y; tv[4 * g + 2] = f.z; tv[4 * g + 3] = f.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int c = 0; c < 12; ++c) acc[i][c] = fmaf(xv[i], tv[c], acc[i][c]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 8 * ty + i;
+            if (r >= nt) continue;
+#pragma unroll
+            for (int g = 0; g < 3; ++g) {
+                const float4 v = make_float4(acc[i][4 * g], acc[i][4 * g + 1], acc[i][4 * g + 2], acc[i][4 * g + 3]);
+                bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+                *reinterpret_cast<float4*>(outs[g] + ((long long)h * T + t0 + r) * 64 + 4 * tx) = v;
+            }
+        }
+    }
+    if (__syncthreads_or(bad) && tid == 0) atomicOr(status, kStatusNonFinite);
+}
+
 }  // namespace
 
 cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const theta[3], int th_bf16,
@@ -139,10 +207,20 @@ cudaError_t launch_proj_per_head(const void* X, int x_bf16, const void* const th
                                               out[2], T, status);
         return cudaGetLastError();
     };
+    if (d == 64) {   // the register-tiled kernel
+        const size_t smem = sizeof(float) * (64 * (size_t)kP64TS + 64 * (size_t)kP64XS);
+        cudaError_t e = cudaFuncSetAttribute(proj_per_head64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e != cudaSuccess) return e;
+        LaunchScope scope("proj_per_head", s);
+        dim3 grid((T + kP64Tok - 1) / kP64Tok, H);
+        proj_per_head64_kernel<<<grid, 256, smem, s>>>(X, x_bf16, theta[0], theta[1], theta[2], th_bf16, out[0],
+                                                        out[1], out[2], T, status);
+        return cudaGetLastError();
+    }
     switch (d) {
         case 16: return run(proj_per_head_kernel<16>, 16);
         case 32: return run(proj_per_head_kernel<32>, 32);
-        case 64: return run(proj_per_head_kernel<64>, 64);
         default: return cudaErrorInvalidValue;
     }
 }
