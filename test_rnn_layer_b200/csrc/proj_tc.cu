@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
         if (tc::elect_one()) {
             int s = 0;
             uint32_t phase = 0;
+            // theta is read by every M tile: keep it in L2 ahead of the streaming output
+            const uint64_t keep = tc::l2_policy_evict_last();
             for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
                 const int mt = tile / n_tiles, nt = tile % n_tiles;
                 const int which = nt / p.n_tiles_per;
@@ -94,7 +96,7 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
                     uint8_t* st = stage_base + s * STAGE_BYTES;
                     tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
                     tc::tma_load_2d(st, &p.mapA, kb * BK, mt * BM, &full[s]);
-                    tc::tma_load_2d(st + A_BYTES, &p.mapB[which], kb * BK, n0, &full[s]);
+                    tc::tma_load_2d_hint(st + A_BYTES, &p.mapB[which], kb * BK, n0, &full[s], keep);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
             }
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
         const int q = warp % 4;
         uint8_t* bufs = epi_base + (warp - 2) * 2 * EPI_BUF;
         int it = 0, nbuf = 0, nonfinite = 0;
+        const uint64_t stream_out = tc::l2_policy_evict_first();
         for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
@@ -168,8 +171,9 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
                 if (lane == 0) {
                     const int x = n0 + c * 32, y = mt * BM + 32 * q;
                     if (x < p.N) {   // columns of a partial last tile beyond N are zero (theta rows read as fill)
-                        if (p.accumulate) tc::tma_reduce_add_2d(&p.mapC[which], buf, x, y);
-                        else tc::tma_store_2d(&p.mapC[which], buf, x, y);
+                        // the output streams through L2 once: first to be evicted
+                        if (p.accumulate) tc::tma_reduce_add_2d_hint(&p.mapC[which], buf, x, y, stream_out);
+                        else tc::tma_store_2d_hint(&p.mapC[which], buf, x, y, stream_out);
                     }
                     tc::bulk_commit_group();
                 }
