@@ -11,7 +11,9 @@ bench.py times (automatic kernel choice, whole layer in one call).
     Z_f, Z_r, Y and both final states of those heads on six 128-token windows
     spread from the first token to the last.  The forward pass of one head
     (which needs only that head's rows of theta) is also checked over the
-    whole length against the oracle run here.
+    whole length against the oracle run here;
+  * the 3072-wide TTT-Linear layer the same way, from the expected values
+    tests/golden/make_full_linear_golden.py wrote.
 Tolerance: max-normalised error 2e-2 (bf16 inputs, fp32 state).  Every error
 is printed (pytest -s) with the prefix PARITY.
 """
@@ -121,3 +123,44 @@ def test_full_layer_full_length_forward_sampled_head():
     err = maxrel(Zf, ref)
     _report(f"{w.name} forward head={heads} all tokens", {"Z_f": err})
     assert err <= TOL_BF16
+
+
+GOLDEN_LINEAR = os.path.join(GOLDEN_DIR, "full_linear_T313344_seed0.npz")
+
+
+def test_linear_full_layer_full_length_both_directions_with_the_gates():
+    """The 3072-wide TTT-Linear layer at 313,344 tokens, both gates at 0.1, against
+    the expected values tests/golden/make_full_linear_golden.py wrote from the
+    oracle: Z_f, Z_r, Y and both final states of three heads on six windows."""
+    g = np.load(GOLDEN_LINEAR)
+    w = S.FULL63S
+    inp = S.make_linear_inputs(w, seed=0, device="cpu")
+    spec = importlib.util.spec_from_file_location("make_full_linear_golden",
+                                                  os.path.join(GOLDEN_DIR, "make_full_linear_golden.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    assert mod.input_digest(inp) == str(g["digest"]), "inputs differ from those of the stored expected values"
+    assert int(g["T"]) == w.T and int(g["b"]) == w.b and float(g["eta"]) == w.eta_eff
+    dev = torch.device("cuda")
+    d_in = {k: v.to(dev) for k, v in inp.items()}
+    out = L.linear_layer_forward(d_in["X"], d_in["theta_q"], d_in["theta_k"], d_in["theta_v"], d_in["W_0"],
+                                 w.eta_eff, w.b, w.dirs, alpha_f=d_in["alpha_f"], alpha_r=d_in["alpha_r"],
+                                 per_head=False, want_z=True, want_state=True)
+    heads = [int(h) for h in g["heads"]]
+    win = int(g["window"])
+    rows = torch.cat([torch.arange(int(s), int(s) + win) for s in g["starts"]]).to(dev)
+    cols = torch.cat([torch.arange(h * w.d, (h + 1) * w.d) for h in heads]).to(dev)
+    pick = lambda t: to_np(t.index_select(0, rows).index_select(1, cols))
+    Zf, Zr, Y = pick(out["Z"][0]), pick(out["Z"][1]), pick(out["Y"])
+    hidx = torch.tensor(heads, device=dev)
+    Wf, Wr = to_np(out["W_T"][0].index_select(0, hidx)), to_np(out["W_T"][1].index_select(0, hidx))
+    del out, d_in
+    torch.cuda.empty_cache()
+    Xs = inp["X"].double()[rows.cpu()][:, cols.cpu()].numpy()
+    af, ar = to_np(inp["alpha_f"][cols.cpu()]), to_np(inp["alpha_r"][cols.cpu()])
+    Zf_o, Zr_o = g["Z_f"].astype(np.float64), g["Z_r"].astype(np.float64)
+    Y_o = O.gate(O.gate(Xs, Zf_o, af), Zr_o, ar)
+    errs = {"Z_f": maxrel(Zf, Zf_o), "Z_r": maxrel(Zr, Zr_o), "Y": maxrel(Y, Y_o),
+            "W_f": maxrel(Wf, g["W_f"]), "W_r": maxrel(Wr, g["W_r"])}
+    _report(f"linear {w.name} heads={heads} windows={list(map(int, g['starts']))}x{win}", errs)
+    assert all(v <= TOL_BF16 for v in errs.values()), errs
