@@ -244,6 +244,73 @@ TTT_API ttt_status ttt_mlp_forward_heads(const ttt_mlp_desc* desc, int h0, int h
                                          ttt_stream_t stream);
 
 /*
+ * Segment-local attention, the sublayer the TTT layer follows in the pages'
+ * block (paper notes page, "方法详解 / 整体框架": the backbone's self-attention
+ * only spans the tokens of one 3-second segment, the TTT layer the whole
+ * sequence).  For every head h and row t in [row0, row1):
+ *
+ *   Out[t, h*64 + j] = Xres[t, h*64 + j]
+ *                    + sum_{u in seg(t)} softmax_u(q_t . k_u / sqrt(64)) v_u[j]
+ *
+ * where seg(t) = [s L, min((s + 1) L, T)), s = floor(t / L), and q_t, k_u, v_u
+ * are the 64 columns of head h in rows t, u of Q, K, V.  The attention inside
+ * a segment is full, not causal.  Arithmetic: bf16 Q, K, V; Q K^T and P V on
+ * the tensor cores with fp32 accumulation; the softmax weights in fp32, then
+ * rounded to bf16 for P V; the row sum in fp32; the result rounded to bf16.
+ *
+ *   T, H, d, L  tokens, heads (d must be 64), segment length (>= 1).
+ *   Q, K, V     bf16, row t of each at Q + t * ld_qkv (ld_qkv >= H * 64, a
+ *               multiple of 8): three [T, H*64] arrays, or one fused
+ *               [T, 3*H*64] array passed at column offsets 0, H*64, 2*H*64.
+ *   Xres        bf16 [T, ld_out] residual, or NULL for none.
+ *   Out         bf16 [T, ld_out] (ld_out >= H * 64, a multiple of 8); only rows
+ *               [row0, row1) are written, columns past H * 64 never.  Out may
+ *               be Xres itself; it must not overlap Q, K or V.
+ *   row0, row1  0 <= row0 <= row1 <= T.  Each row attends over its whole
+ *               segment whatever the range.
+ *   workspace   ttt_seg_attention_workspace_size() bytes, 256-byte aligned:
+ *               the status word, cleared by the call; ttt_mlp_status(workspace,
+ *               stream) reports non-finite outputs (TTT_ERR_NONFINITE) and
+ *               expired waits (TTT_ERR_TIMEOUT).
+ * All pointers are device pointers, 16-byte aligned.  Asynchronous on
+ * `stream`; no allocation.  TTT_ERR_UNSUPPORTED for d != 64.
+ */
+TTT_API size_t ttt_seg_attention_workspace_size(void);
+TTT_API ttt_status ttt_seg_attention(int T, int H, int d, int L, const void* Q, const void* K,
+                                     const void* V, int ld_qkv, const void* Xres, void* Out, int ld_out,
+                                     int row0, int row1, void* workspace, size_t workspace_bytes,
+                                     ttt_stream_t stream);
+
+/*
+ * The block: segment-local attention, then the bidirectional TTT-MLP layer on
+ * its output, in one schedule.  X = Xres + attention(Qa, Ka, Va) exactly as
+ * ttt_seg_attention with segment length seg_len and ld_out = D, then
+ * Y = ttt_mlp_forward(desc, X, ..., TTT_BIDIR, ...).  The attention of the
+ * rows of each chunk segment of the layer's first direction runs on the side
+ * stream just before that segment's projection, so the first direction's scan
+ * starts as soon as the first rows are ready instead of after the whole
+ * attention.  X and Y hold the same values as the two calls made one after
+ * the other.
+ *
+ *   desc         a full-width bf16 layer (per_head_input = 0, x_dtype =
+ *                TTT_BF16, D = H * d, d = 64).
+ *   seg_len      the attention's segment length L.
+ *   Qa, Ka, Va   bf16, row stride ld_qkv, as for ttt_seg_attention.
+ *   Xres         bf16 [T, D] residual (or NULL).
+ *   X            bf16 [T, D]: written (the layer's input); may be Xres.
+ *   the rest     as for ttt_mlp_forward with dir = TTT_BIDIR and no optional
+ *                outputs; workspace of ttt_block_workspace_size(desc, b)
+ *                bytes, whose status word ttt_mlp_status reads.
+ */
+TTT_API size_t ttt_block_workspace_size(const ttt_mlp_desc* desc, int b);
+TTT_API ttt_status ttt_block_forward(const ttt_mlp_desc* desc, int seg_len, const void* Qa, const void* Ka,
+                                     const void* Va, int ld_qkv, const void* Xres, void* X,
+                                     const void* theta_q, const void* theta_k, const void* theta_v,
+                                     const float* W1_0, const float* W2_0, float eta, int b,
+                                     const float* alpha_f, const float* alpha_r, void* Y, void* workspace,
+                                     size_t workspace_bytes, ttt_stream_t stream);
+
+/*
  * ttt_mlp_forward for callers that cannot allocate device memory.
  *
  * The paper has no counterpart: this is a deployment aid.  Code embedded in a
@@ -344,6 +411,14 @@ TTT_API ttt_status ttt_debug_inject_wait_timeout(int enable);
  * exceed max_segments: only that many are written), or -1 if nchunks < 1.
  */
 TTT_API int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments);
+
+/*
+ * Benchmarks only (process-wide): the head start of ttt_block_forward, i.e.
+ * the percentage of the first direction's chunks whose attention and
+ * projection run on the whole GPU before that direction's scan starts
+ * (0..100; -1 restores the built-in value).  Changes timing, never results.
+ */
+TTT_API ttt_status ttt_debug_set_block_front(int percent);
 
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 TTT_API const char* ttt_last_error(void);

@@ -62,6 +62,13 @@ static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
 #endif
 constexpr bool kSplitScanGates = TTT_SPLIT_SCAN_GATES != 0;
 static std::atomic<int> g_inject_timeout{0};
+// The block's head start: the share of the first direction's chunks whose attention and projection run on the
+// whole GPU before its scan starts (the side SMs then keep ahead of the scan with the rest).
+#ifndef TTT_BLOCK_FRONT_PERCENT
+#define TTT_BLOCK_FRONT_PERCENT 85
+#endif
+constexpr int kBlockFrontPercent = TTT_BLOCK_FRONT_PERCENT;
+static std::atomic<int> g_block_front{-1};
 
 }  // namespace ttt
 
@@ -359,11 +366,15 @@ struct PipeBufs {
 // the segment starts from W_0 / leaves the final state for the caller).
 using SegScan = std::function<cudaError_t(int di, const struct Dir& dd, int c_begin, int c_end, bool first,
                                           bool last, float* zscan, cudaStream_t s)>;
+// Work that produces rows [r0, r1) of X, enqueued on the side stream just before the first direction's
+// projection of those rows (max_ctas: the SM cap of that projection, 0 = whole GPU).
+using RowsHook = std::function<cudaError_t(int r0, int r1, int max_ctas, cudaStream_t s)>;
 
 ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_sms_per_head, const SegScan& seg_scan,
                              const void* X, const void* const th[3], float* const qkv[3], int b, ttt_direction dir,
                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, cudaStream_t s,
-                             const void* X_host, void* Y_host, bool scan_gates = false) {
+                             const void* X_host, void* Y_host, bool scan_gates = false,
+                             const RowsHook* pre_rows = nullptr, int first_front_percent = -1) {
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
     Pipe& P = pipe_for(dev, s);
@@ -439,7 +450,8 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_
             // projections: the first runs alone on the whole GPU (with a gating scan, the segments of the
             // first kPipeFrontPercent of the chunks); the reverse ones after the forward scan wrote X'
             if (prev_dir_done) CUDA_TRY(cudaStreamWaitEvent(P.side, prev_dir_done, 0));
-            const int front_chunks = scan_gates ? nch * kPipeFrontPercent / 100 : 0;
+            const int front_pct = (di == 0 && first_front_percent >= 0) ? first_front_percent : kPipeFrontPercent;
+            const int front_chunks = scan_gates ? (int)((long long)nch * front_pct / 100) : 0;
             int last_front = 0;   // the first scan segment waits for the projections of the head start
             for (int k = 0; k < ns; ++k)
                 if (seg[k].second <= front_chunks) last_front = k;
@@ -450,6 +462,7 @@ ttt_status forward_pipelined(const ttt_mlp_desc& q, const PipeBufs& B, int scan_
                 const void* a = static_cast<const char*>(psrc) + (size_t)r0 * D * 2;
                 float* out[3] = {qkv[0] + (size_t)r0 * D, qkv[1] + (size_t)r0 * D, qkv[2] + (size_t)r0 * D};
                 const bool whole_gpu = k == 0 || seg[k].second <= front_chunks;
+                if (pre_rows && di == 0) CUDA_TRY((*pre_rows)(r0, r1, whole_gpu ? 0 : side_sms, P.side));
                 CUDA_TRY(launch_proj_full_tc(a, th, out, r1 - r0, D, D, pacc, status, whole_gpu ? 0 : side_sms, P.side));
                 CUDA_TRY(cudaEventRecord(ev_proj[k], P.side));
             }
@@ -528,11 +541,35 @@ namespace {
 // The layer on device buffers; with X_host / Y_host (host buffers) X is first
 // copied into the device buffer X and Y copied back out, overlapped with the
 // computation on the pipelined path.
+// Arguments of the segment attention (and of the block's attention step): Out must not overlap Q, K, V
+// (it may be Xres itself: each element is read before the same thread writes it).
+ttt_status check_attention(int T, int H, int d, int L, const void* Q, const void* K, const void* V, int ld_qkv,
+                           const void* Xres, const void* Out, int ld_out) {
+    if (!attn_seg_supported(d)) return fail(TTT_ERR_UNSUPPORTED, "segment attention needs d = 64 (got %d)", d);
+    if (T < 1 || H < 1 || L < 1) return fail(TTT_ERR_INVALID_ARG, "T, H and the segment length must be positive");
+    const long long cols = (long long)H * d;
+    if (ld_qkv < cols || ld_out < cols || ld_qkv % 8 != 0 || ld_out % 8 != 0)
+        return fail(TTT_ERR_INVALID_ARG, "row strides (%d, %d) must hold %lld columns and be multiples of 8", ld_qkv,
+                    ld_out, cols);
+    if (!Q || !K || !V || !Out) return fail(TTT_ERR_INVALID_ARG, "Q, K, V and Out must be non-NULL");
+    const void* ps[] = {Q, K, V, Xres, Out};
+    for (const void* p : ps)
+        if (p && !aligned16(p)) return fail(TTT_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+    const size_t in_bytes = ((size_t)(T - 1) * ld_qkv + cols) * 2, out_bytes = ((size_t)(T - 1) * ld_out + cols) * 2;
+    const char* o = static_cast<const char*>(Out);
+    for (const void* p : {Q, K, V}) {
+        const char* c = static_cast<const char*>(p);
+        if (o < c + in_bytes && c < o + out_bytes) return fail(TTT_ERR_INVALID_ARG, "Out must not overlap Q, K or V");
+    }
+    return TTT_OK;
+}
+
 ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
                         const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
                         ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y, float* Z_out,
                         float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes, ttt_stream_t stream_,
-                        const void* X_host, void* Y_host, bool allow_pipeline = true) {
+                        const void* X_host, void* Y_host, bool allow_pipeline = true,
+                        const RowsHook* pre_rows = nullptr, int first_front_percent = -1) {
     ttt_status st = check_desc(desc, b, dir);
     if (st != TTT_OK) return st;
     const ttt_mlp_desc& q = *desc;
@@ -589,8 +626,9 @@ ttt_status forward_impl(const ttt_mlp_desc* desc, const void* X, const void* the
         const PipeBufs bufs{status, xp, reinterpret_cast<__nv_bfloat16*>(ws + L.delta),
                             reinterpret_cast<float*>(ws + L.zbuf)};
         return forward_pipelined(q, bufs, 2, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, X_host,
-                                 Y_host, split_groups && kSplitScanGates);
+                                 Y_host, split_groups && kSplitScanGates, pre_rows, first_front_percent);
     }
+    if (pre_rows) CUDA_TRY((*pre_rows)(0, q.T, 0, s));   // X's producer, then the layer on one stream
     if (X_host) CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(X), X_host, xbytes, cudaMemcpyHostToDevice, s));
     auto finish = [&]() -> ttt_status {
         if (Y_host) CUDA_TRY(cudaMemcpyAsync(Y_host, Y, xbytes, cudaMemcpyDeviceToHost, s));
@@ -1029,6 +1067,52 @@ ttt_status ttt_mlp_forward_heads(const ttt_mlp_desc* desc, int h0, int hn, ttt_p
     return TTT_OK;
 }
 
+// ---------------------------------------------------------------- segment-local attention, the block
+size_t ttt_seg_attention_workspace_size(void) { return kAlign; }
+
+ttt_status ttt_seg_attention(int T, int H, int d, int L, const void* Q, const void* K, const void* V, int ld_qkv,
+                             const void* Xres, void* Out, int ld_out, int row0, int row1, void* workspace,
+                             size_t workspace_bytes, ttt_stream_t stream_) {
+    ttt_status st = check_attention(T, H, d, L, Q, K, V, ld_qkv, Xres, Out, ld_out);
+    if (st != TTT_OK) return st;
+    if (row0 < 0 || row1 < row0 || row1 > T)
+        return fail(TTT_ERR_INVALID_ARG, "rows [%d, %d) outside [0, %d]", row0, row1, T);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || workspace_bytes < kAlign)
+        return fail(TTT_ERR_INVALID_ARG, "workspace must be %zu bytes, 256-byte aligned", kAlign);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream_);
+    int* status = static_cast<int*>(workspace);
+    CUDA_TRY(cudaMemsetAsync(status, 0, 16, s));
+    CUDA_TRY(launch_attn_seg(Q, K, V, ld_qkv, Xres, ld_out, Out, ld_out, T, H, L, row0, row1, status, 0, s));
+    return TTT_OK;
+}
+
+size_t ttt_block_workspace_size(const ttt_mlp_desc* desc, int b) { return ttt_mlp_workspace_size(desc, b, TTT_BIDIR); }
+
+ttt_status ttt_block_forward(const ttt_mlp_desc* desc, int seg_len, const void* Qa, const void* Ka, const void* Va,
+                             int ld_qkv, const void* Xres, void* X, const void* theta_q, const void* theta_k,
+                             const void* theta_v, const float* W1_0, const float* W2_0, float eta, int b,
+                             const float* alpha_f, const float* alpha_r, void* Y, void* workspace,
+                             size_t workspace_bytes, ttt_stream_t stream) {
+    ttt_status st = check_desc(desc, b, TTT_BIDIR);
+    if (st != TTT_OK) return st;
+    const ttt_mlp_desc& q = *desc;
+    if (q.per_head_input || q.x_dtype != TTT_BF16 || q.D != q.H * q.d)
+        return fail(TTT_ERR_UNSUPPORTED, "the block needs a full-width bf16 layer with D = H * d");
+    st = check_attention(q.T, q.H, q.d, seg_len, Qa, Ka, Va, ld_qkv, Xres, X, q.D);
+    if (st != TTT_OK) return st;
+    if (workspace_bytes < ttt_block_workspace_size(desc, b) || !workspace)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small");
+    int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan(q, b, TTT_BIDIR).status);
+    const RowsHook attention = [&](int r0, int r1, int max_ctas, cudaStream_t ss) {
+        return launch_attn_seg(Qa, Ka, Va, ld_qkv, Xres, q.D, X, q.D, q.T, q.H, seg_len, r0, r1, status, max_ctas,
+                               ss);
+    };
+    const int front = g_block_front.load();
+    return forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, TTT_BIDIR, alpha_f, alpha_r, Y,
+                        nullptr, nullptr, nullptr, workspace, workspace_bytes, stream, nullptr, nullptr, true,
+                        &attention, front >= 0 ? front : kBlockFrontPercent);
+}
+
 ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, const void* theta_q,
                                 const void* theta_k, const void* theta_v, const float* W1_0, const float* W2_0,
                                 float eta, int b, ttt_direction dir, const float* alpha_f, const float* alpha_r,
@@ -1109,6 +1193,12 @@ int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments) {
         out[2 * k + 1] = seg[k].second;
     }
     return (int)seg.size();
+}
+
+ttt_status ttt_debug_set_block_front(int percent) {
+    if (percent < -1 || percent > 100) return fail(TTT_ERR_INVALID_ARG, "percent must be -1 (default) or 0..100");
+    g_block_front.store(percent);
+    return TTT_OK;
 }
 
 ttt_status ttt_debug_inject_wait_timeout(int enable) {

@@ -98,6 +98,16 @@ bool proj_full_tc_supported(int N, int K);
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
                                 int accumulate, int* status, int max_ctas, cudaStream_t s);
 
+// Segment-local attention (d = 64, bf16) with a residual add, tcgen05:
+// rows [row0, row1) of Out = Xres + softmax(Q K^T / 8) V inside segments of L
+// tokens.  Q, K, V share the row stride ld_qkv; Xres (optional) and Out share
+// ld_out / ld_res.  max_ctas > 0 caps the persistent grid.
+bool attn_seg_supported(int d);
+long long attn_seg_items(int T, int H, int L, int row0, int row1);
+cudaError_t launch_attn_seg(const void* Q, const void* K, const void* V, long long ld_qkv, const void* Xres,
+                            long long ld_res, void* Out, long long ld_out, int T, int H, int L, int row0, int row1,
+                            int* status, int max_ctas, cudaStream_t s);
+
 // out = x + tanh(alpha) z (+ bf16 increment, + non-finite check) over one direction.
 cudaError_t launch_gate(const void* X, int x_bf16, const float* Z, const float* alpha, void* Out, int out_bf16,
                         __nv_bfloat16* Delta, int* status, int T, int H, int d, int per_head, int max_blocks,

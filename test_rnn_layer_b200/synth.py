@@ -119,3 +119,32 @@ def make_linear_inputs(w: Workload, seed: int = 0, device: str | torch.device = 
     inp["W_0"] = torch.randn((w.H, w.d, w.d), generator=g, device=dev, dtype=torch.float32).mul_(
         math.sqrt(1.0 / w.d))
     return inp
+
+
+# The segment-local attention before the layer: 63 s of video in 3-s segments.
+SEGMENTS_63S = 21
+
+
+def segment_length(T: int, n_segments: int = SEGMENTS_63S) -> int:
+    """Tokens per segment when T tokens cover ``n_segments`` equal segments
+    (ceil(T / n); the last one is shorter when n does not divide T)."""
+    return -(-T // n_segments)
+
+
+def make_attention_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu",
+                          qk_std: float = 1.0) -> dict:
+    """Q_a, K_a, V_a [T, D] bf16 for the attention sublayer: Q_a and K_a
+    N(0, qk_std^2), V_a N(0, 1), drawn in that order from a generator seeded
+    ``seed + 2_000_003`` (independent of make_inputs' draws, whose X is the
+    sublayer's residual)."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 2_000_003)
+    T, D = w.T, w.model_dim
+    out = {}
+    for k, std in (("Q_a", qk_std), ("K_a", qk_std), ("V_a", 1.0)):
+        t = torch.randn((T, D), generator=g, device=dev, dtype=torch.float32)
+        if std != 1.0:
+            t.mul_(std)
+        out[k] = t.to(torch.bfloat16)
+    return out

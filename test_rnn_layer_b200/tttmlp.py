@@ -28,7 +28,8 @@ EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_
             "ttt_kernel_timing", "ttt_kernel_times", "ttt_mlp_forward_noalloc", "ttt_mlp_noalloc_status", "ttt_debug_inject_wait_timeout",
             "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments",
             "ttt_mlp_backward_workspace_size", "ttt_mlp_backward", "ttt_mlp_heads_workspace_size",
-            "ttt_mlp_forward_heads"]
+            "ttt_mlp_forward_heads", "ttt_seg_attention_workspace_size", "ttt_seg_attention",
+            "ttt_block_workspace_size", "ttt_block_forward", "ttt_debug_set_block_front"]
 
 
 class TTTError(RuntimeError):
@@ -78,6 +79,16 @@ def lib():
         L.ttt_mlp_heads_workspace_size.argtypes = [dp, i, i]
         L.ttt_mlp_forward_heads.restype = i
         L.ttt_mlp_forward_heads.argtypes = [dp, i, i, i, vp, vp, vp, vp, vp, vp, f, i, vp, vp, vp, vp, vp, sz, vp]
+        L.ttt_seg_attention_workspace_size.restype = sz
+        L.ttt_seg_attention_workspace_size.argtypes = []
+        L.ttt_seg_attention.restype = i
+        L.ttt_seg_attention.argtypes = [i, i, i, i, vp, vp, vp, i, vp, vp, i, i, i, vp, sz, vp]
+        L.ttt_block_workspace_size.restype = sz
+        L.ttt_block_workspace_size.argtypes = [dp, i]
+        L.ttt_block_forward.restype = i
+        L.ttt_block_forward.argtypes = [dp, i, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, f, i, vp, vp, vp, vp, sz, vp]
+        L.ttt_debug_set_block_front.restype = i
+        L.ttt_debug_set_block_front.argtypes = [i]
         L.ttt_mlp_noalloc_status.restype = i
         L.ttt_mlp_noalloc_status.argtypes = [vp]
         L.ttt_linear_workspace_size.restype = sz
@@ -253,6 +264,32 @@ def ttt_mlp_forward_heads(desc, h0, hn, phase, X, theta_q, theta_k, theta_v, W1_
                                            _p(theta_v), _p(W1_0), _p(W2_0), float(eta), b, _p(alpha),
                                            _p(delta_all), _p(Xp), _p(delta_or_y), _p(workspace), workspace_bytes,
                                            _stream(stream)))
+
+
+def ttt_seg_attention_workspace_size() -> int:
+    return int(lib().ttt_seg_attention_workspace_size())
+
+
+def ttt_seg_attention(T, H, d, L, Q, K, V, ld_qkv, Xres, Out, ld_out, row0, row1, workspace, workspace_bytes,
+                      stream=None) -> int:
+    return int(lib().ttt_seg_attention(T, H, d, L, _p(Q), _p(K), _p(V), ld_qkv, _p(Xres), _p(Out), ld_out, row0,
+                                       row1, _p(workspace), workspace_bytes, _stream(stream)))
+
+
+def ttt_block_workspace_size(desc: ttt_mlp_desc, b: int) -> int:
+    return int(lib().ttt_block_workspace_size(ctypes.byref(desc), b))
+
+
+def ttt_block_forward(desc, seg_len, Qa, Ka, Va, ld_qkv, Xres, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b,
+                      alpha_f, alpha_r, Y, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_block_forward(ctypes.byref(desc), seg_len, _p(Qa), _p(Ka), _p(Va), ld_qkv, _p(Xres), _p(X),
+                                       _p(theta_q), _p(theta_k), _p(theta_v), _p(W1_0), _p(W2_0), float(eta), b,
+                                       _p(alpha_f), _p(alpha_r), _p(Y), _p(workspace), workspace_bytes,
+                                       _stream(stream)))
+
+
+def ttt_debug_set_block_front(percent: int) -> int:
+    return int(lib().ttt_debug_set_block_front(percent))
 
 
 def ttt_mlp_noalloc_status(stream=None) -> int:

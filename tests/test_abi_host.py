@@ -179,3 +179,43 @@ def test_pipeline_segments_of_the_benchmark_layer():
     assert sizes[:4] == [16, 24, 36, 54] and sizes[-4:] == [54, 36, 24, 16]
     middle = sizes[9:-9]   # between the two ramps (9 segments each, capped at 408 = 4896 / 12)
     assert max(middle) - min(middle) <= 1 and max(middle) <= 408
+
+
+def test_attention_argument_errors_before_any_cuda_call():
+    """ttt_seg_attention and ttt_block_forward reject bad arguments before any
+    CUDA call (fake device addresses; skipped where a GPU exists)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake device addresses are only used where no GPU exists")
+    T, H = 1000, 2
+    Q, K, V, O, W = 0x10000000, 0x20000000, 0x30000000, 0x40000000, 0x50000000
+
+    def att(**kw):
+        a = dict(T=T, H=H, d=64, L=300, Q=Q, K=K, V=V, ld=128, X=None, O=O, ldo=128, r0=0, r1=T, ws=W, wsb=256)
+        a.update(kw)
+        return L.ttt_seg_attention(a["T"], a["H"], a["d"], a["L"], a["Q"], a["K"], a["V"], a["ld"], a["X"], a["O"],
+                                   a["ldo"], a["r0"], a["r1"], a["ws"], a["wsb"], 0)
+
+    assert L.ttt_seg_attention_workspace_size() == 256
+    assert att(d=32) == L.TTT_ERR_UNSUPPORTED
+    assert att(L=0) == L.TTT_ERR_INVALID_ARG
+    assert att(ld=120) == L.TTT_ERR_INVALID_ARG and "strides" in L.ttt_last_error()
+    assert att(ldo=132) == L.TTT_ERR_INVALID_ARG
+    assert att(V=None) == L.TTT_ERR_INVALID_ARG
+    assert att(Q=Q + 8) == L.TTT_ERR_INVALID_ARG and "aligned" in L.ttt_last_error()
+    assert att(O=K + 4096) == L.TTT_ERR_INVALID_ARG and "overlap" in L.ttt_last_error()
+    assert att(r0=10, r1=5) == L.TTT_ERR_INVALID_ARG
+    assert att(r1=T + 1) == L.TTT_ERR_INVALID_ARG
+    assert att(ws=None) == L.TTT_ERR_INVALID_ARG
+    assert att(wsb=16) == L.TTT_ERR_INVALID_ARG
+    d = L.make_desc(T, H, 64, False, True)
+    assert L.ttt_block_workspace_size(d, 64) == L.ttt_mlp_workspace_size(d, 64, L.TTT_BIDIR) > 0
+    ph = L.make_desc(T, H, 64, True, True)
+    blk = lambda desc, **kw: L.ttt_block_forward(desc, kw.get("L", 300), Q, K, V, 128, None, kw.get("X", O), 0x60000000,
+                                                 0x61000000, 0x62000000, 0x63000000, 0x64000000, 0.01, 64,
+                                                 0x65000000, 0x66000000, 0x67000000, W, 1 << 40, 0)
+    assert blk(ph) == L.TTT_ERR_UNSUPPORTED
+    assert blk(d, L=0) == L.TTT_ERR_INVALID_ARG
+    assert blk(d, X=Q) == L.TTT_ERR_INVALID_ARG and "overlap" in L.ttt_last_error()
+    assert L.ttt_debug_set_block_front(101) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_debug_set_block_front(-1) == L.TTT_OK
