@@ -78,6 +78,7 @@ KERNEL_SRC = {
     "gate": ("gate.cu",),
     "scan_linear": ("scan_linear.cu",),
     "scan_linear_tc": ("scan_linear_tc.cu",),
+    "attn_seg_tc": ("attn_seg_tc.cu",),
 }
 
 
@@ -568,6 +569,188 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+METRIC_BLOCK = ("block tokens/s (segment-local attention in 21 segments + bidirectional TTT-MLP layer, 48 heads) "
+                "at T≈313k; % of roofline")
+
+
+def _attention_flops(T: int, D: int, L: int) -> float:
+    """Q K^T and P V over every segment and head: 2 x 2 L_s^2 D flops per segment."""
+    return sum(4.0 * (min(s0 + L, T) - s0) ** 2 * D for s0 in range(0, T, L))
+
+
+def cpu_baseline_block(w, L_seg, args) -> dict:
+    """The oracles on a bounded sample: the attention of the first 256 query
+    rows of a segment for every head (each against the segment's keys), and
+    the layer's own sample (cpu_baseline); block tokens/s = 1 / (attention
+    seconds per token + layer seconds per token)."""
+    from oracle import seg_attention as A
+    from test_rnn_layer_b200 import synth as S
+
+    rows = 256
+    a = S.make_attention_inputs(w.with_T(L_seg), seed=0, device="cpu")
+    Q, K, V = (a[k].double().numpy() for k in ("Q_a", "K_a", "V_a"))
+
+    def att():
+        t0 = time.perf_counter()
+        for h in range(w.H):
+            c = slice(h * w.d, (h + 1) * w.d)
+            A.attention_segment(Q[:rows, c], K[:, c], V[:, c])
+        return time.perf_counter() - t0
+
+    t_att = min(att() for _ in range(2)) / rows
+    layer = cpu_baseline(w, args)
+    value = 1.0 / (t_att + 1.0 / layer["value"])
+    return {"value": value, "unit": UNIT, "cores": max(layer["cores"], os.cpu_count() or 1), "kind": "oracle",
+            "sample": (f"attention: {rows} query rows of a {L_seg}-token segment, all {w.H} heads (fp64, numpy); "
+                       f"layer: {layer['sample']}; combined as seconds per token"),
+            "attention_s_per_token": t_att, "layer_tokens_per_s": layer["value"], "cpu_model": cpu_model()}
+
+
+def run_block(args, rank, world, local_rank):
+    """One step = the block: segment-local attention (21 segments) feeding the
+    bidirectional layer, through ttt_block_forward; besides it, the attention
+    and the layer timed alone, the two calls one after the other, and the
+    interleaved schedule (each segment's attention beside the scan)."""
+    import torch
+    import torch.distributed as dist
+
+    from test_rnn_layer_b200 import synth as S
+    from test_rnn_layer_b200 import tttmlp as L
+
+    L.lib()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = _workload(args)
+    if w.per_head or w.dirs != "bidir" or w.dtype != "bf16":
+        raise SystemExit("--block needs the full-width bidirectional bf16 layer (--workload full63s)")
+    L_seg = S.segment_length(w.T)
+    inp = S.make_inputs(w, seed=rank_seed(rank), device=dev)
+    inp.update(S.make_attention_inputs(w, seed=rank_seed(rank), device=dev))
+    desc = L.make_desc(w.T, w.H, w.d, False, True)
+    nws = L.ttt_block_workspace_size(desc, w.b)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    aws = torch.empty(L.ttt_seg_attention_workspace_size(), dtype=torch.uint8, device=dev)
+    X = torch.empty_like(inp["X"])
+    Y = torch.empty_like(inp["X"])
+    stream = torch.cuda.current_stream()
+    th = (inp["theta_q"], inp["theta_k"], inp["theta_v"])
+
+    def block(Qa=None, Ka=None, Va=None, Xr=None):
+        L.check(L.ttt_block_forward(desc, L_seg, inp["Q_a"] if Qa is None else Qa, inp["K_a"] if Ka is None else Ka,
+                                    inp["V_a"] if Va is None else Va, w.D, inp["X"] if Xr is None else Xr, X, *th,
+                                    inp["W1_0"], inp["W2_0"], w.eta_eff, w.b, inp["alpha_f"], inp["alpha_r"], Y, ws,
+                                    nws, stream), "ttt_block_forward")
+
+    def attention():
+        L.check(L.ttt_seg_attention(w.T, w.H, w.d, L_seg, inp["Q_a"], inp["K_a"], inp["V_a"], w.D, inp["X"], X, w.D,
+                                    0, w.T, aws, aws.numel(), stream), "ttt_seg_attention")
+
+    def layer():
+        L.check(L.ttt_mlp_forward(desc, X, *th, inp["W1_0"], inp["W2_0"], w.eta_eff, w.b, L.TTT_BIDIR,
+                                  inp["alpha_f"], inp["alpha_r"], Y, None, None, None, ws, nws, stream),
+                "ttt_mlp_forward")
+
+    for _ in range(args.warmup):
+        block()
+    torch.cuda.synchronize()
+    L.check(L.ttt_mlp_status(ws, stream), "warm-up status")
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    sampler.start()
+    time.sleep(0.3)
+    n_launch0 = L.ttt_launch_count()
+    ms = _timed_steps(block, argparse.Namespace(warmup=0, steps=args.steps), world, local_rank, stream, False)
+    launches = L.ttt_launch_count() - n_launch0
+    clocks = sampler.stop()
+    L.check(L.ttt_mlp_status(ws, stream), "timed-run status")
+    ms_per_step = ms / args.steps
+    value = whole_job_tokens_per_s(world, w.T, ms_per_step)
+
+    def alone(fn, n=3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    # per-kernel device times of the block (events on each launch's stream)
+    L.ttt_kernel_timing(True)
+    kpass = 2
+    for _ in range(kpass):
+        block()
+    torch.cuda.synchronize()
+    ktimes = L.ttt_kernel_times()
+    L.ttt_kernel_timing(False)
+    total = sum(v[0] for v in ktimes.values()) or 1.0
+    kernels = {k: {"ms_per_step": round(v[0] / kpass, 3), "launches_per_step": v[1] // kpass,
+                   "share": round(v[0] / total, 4)} for k, v in ktimes.items()}
+    att_ms = alone(attention)
+    layer_ms = alone(layer)
+    two_calls_ms = alone(lambda: (attention(), layer()))
+    L.check(L.ttt_debug_set_block_front(95), "ttt_debug_set_block_front")
+    interleaved_ms = alone(block)
+    L.check(L.ttt_debug_set_block_front(-1), "ttt_debug_set_block_front")
+    L.check(L.ttt_mlp_status(ws, stream), "comparison status")
+
+    peaks = _peaks()
+    src = "of " + peaks["_source"]
+    flops = _attention_flops(w.T, w.D, L_seg)
+    k_att = ktimes["attn_seg_tc"]
+    att_launch_ms = k_att[0] / k_att[1]
+    achieved = flops * kpass / k_att[1] / (att_launch_ms * 1e-3) / 1e12
+    roof = {"kernel": "attn_seg_tc", "bound": "tensor", "achieved": round(achieved, 2),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "traffic": _traffic("attn_seg_tc", w.T / 1024.0), "peak_note": f"bf16 dense burst {src} (kernel timed "
+            "alone, one launch of the whole sequence)", "ms_per_launch": round(att_launch_ms, 3),
+            "work_per_launch": flops, "work": "4 L_s^2 D flops per segment (Q K^T and P V, all heads)",
+            "share": round(k_att[0] / total, 4)}
+
+    e2e = None
+    if not args.no_e2e:
+        host = {k: inp[k].cpu().pin_memory() for k in ("Q_a", "K_a", "V_a", "X")}
+        dev_in = {k: torch.empty_like(inp[k]) for k in host}
+        Yh = torch.empty_like(host["X"]).pin_memory()
+        ns = max(1, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            for k in host:
+                dev_in[k].copy_(host[k], non_blocking=True)
+            block(dev_in["Q_a"], dev_in["K_a"], dev_in["V_a"], dev_in["X"])
+            Yh.copy_(Y, non_blocking=True)
+            L.check(L.ttt_mlp_status(ws, stream), "status")
+
+        e2e_step()
+        t0 = time.perf_counter()
+        for _ in range(ns):
+            e2e_step()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev) / ns
+        nb = host["X"].numel() * 2
+        e2e = {"value": whole_job_tokens_per_s(world, w.T, e2e_s * 1e3), "unit": UNIT, "h2d_bytes_per_step": 4 * nb,
+               "d2h_bytes_per_step": nb, "ms_per_step": e2e_s * 1e3, "steps": ns}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline_block(w, L_seg, args)
+    if rank == 0:
+        cfg = _config(w, {"workload": "block-" + w.name, "attention": f"segment-local, {S.SEGMENTS_63S} segments of "
+                          f"{L_seg} tokens (the last {w.T - (S.SEGMENTS_63S - 1) * L_seg}), full inside a segment, "
+                          "Q/K/V ~N(0,1) bf16, residual X", "schedule": "attention of every row, then the layer"})
+        line = {"metric": METRIC_BLOCK, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16-in/bf16-mma-attention/tf32+fp16-mma-scan/fp32-state",
+                "data": "synthetic", "config": cfg, "gpu_launches": launches, "clocks": clocks, "roofline": roof,
+                "kernels": kernels, "schedules_ms": {"block": round(ms_per_step, 2), "attention_alone":
+                round(att_ms, 2), "layer_alone": round(layer_ms, 2), "attention_then_layer_two_calls":
+                round(two_calls_ms, 2), "interleaved_front95": round(interleaved_ms, 2)},
+                "e2e": e2e, "cpu_baseline": cpu, "impl": "ours"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_backward(args, rank, world, local_rank):
     """One training step of the layer: ttt_mlp_backward (the forward pass
     recomputed inside, then the gradients of every input) for a seeded
@@ -818,6 +1001,9 @@ def main():
     ap.add_argument("--shard-heads", action="store_true",
                     help="one sequence of the full-width layer split by heads over the ranks (strong scaling; "
                          "an all-reduce of the gate increment between the directions) instead of replicas")
+    ap.add_argument("--block", action="store_true",
+                    help="time the block (segment-local attention feeding the layer, ttt_block_forward) instead "
+                         "of the layer alone")
     ap.add_argument("--dry-run-host", action="store_true", help=argparse.SUPPRESS)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -851,6 +1037,8 @@ def main():
             return run_backward(args, rank, world, local_rank)
         if args.shard_heads:
             return run_sharded(args, rank, world, local_rank)
+        if args.block:
+            return run_block(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

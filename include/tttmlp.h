@@ -285,12 +285,14 @@ TTT_API ttt_status ttt_seg_attention(int T, int H, int d, int L, const void* Q, 
  * The block: segment-local attention, then the bidirectional TTT-MLP layer on
  * its output, in one schedule.  X = Xres + attention(Qa, Ka, Va) exactly as
  * ttt_seg_attention with segment length seg_len and ld_out = D, then
- * Y = ttt_mlp_forward(desc, X, ..., TTT_BIDIR, ...).  The attention of the
- * rows of each chunk segment of the layer's first direction runs on the side
- * stream just before that segment's projection, so the first direction's scan
- * starts as soon as the first rows are ready instead of after the whole
- * attention.  X and Y hold the same values as the two calls made one after
- * the other.
+ * Y = ttt_mlp_forward(desc, X, ..., TTT_BIDIR, ...), enqueued as one schedule
+ * on the layer's streams: the attention of every row as one launch on the
+ * whole GPU ahead of the first projection, then the layer's segments.  (The
+ * layer's scan and projections already occupy every SM, so running each
+ * segment's attention beside the scan, just before that segment's projection,
+ * measured slower; ttt_debug_set_block_front selects that schedule for
+ * comparison.)  X and Y hold the same values as the two calls made one after
+ * the other, in either schedule.
  *
  *   desc         a full-width bf16 layer (per_head_input = 0, x_dtype =
  *                TTT_BF16, D = H * d, d = 64).
@@ -413,10 +415,11 @@ TTT_API ttt_status ttt_debug_inject_wait_timeout(int enable);
 TTT_API int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments);
 
 /*
- * Benchmarks only (process-wide): the head start of ttt_block_forward, i.e.
- * the percentage of the first direction's chunks whose attention and
- * projection run on the whole GPU before that direction's scan starts
- * (0..100; -1 restores the built-in value).  Changes timing, never results.
+ * Benchmarks only (process-wide): the schedule of ttt_block_forward.  -1 (the
+ * default): the whole attention first.  0..100: the attention of each chunk
+ * segment's rows just before that segment's projection, and the attention and
+ * projection of the first `percent`% of the first direction's chunks on the
+ * whole GPU before that direction's scan starts.  Changes timing, never results.
  */
 TTT_API ttt_status ttt_debug_set_block_front(int percent);
 

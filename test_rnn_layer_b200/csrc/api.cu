@@ -62,12 +62,8 @@ static std::atomic<int> g_scan_impl{0}, g_proj_impl{0};
 #endif
 constexpr bool kSplitScanGates = TTT_SPLIT_SCAN_GATES != 0;
 static std::atomic<int> g_inject_timeout{0};
-// The block's head start: the share of the first direction's chunks whose attention and projection run on the
-// whole GPU before its scan starts (the side SMs then keep ahead of the scan with the rest).
-#ifndef TTT_BLOCK_FRONT_PERCENT
-#define TTT_BLOCK_FRONT_PERCENT 85
-#endif
-constexpr int kBlockFrontPercent = TTT_BLOCK_FRONT_PERCENT;
+// The block's schedule: -1 = the whole attention first; p >= 0 = each segment's attention just before its
+// projection, with the first p% of the first direction's chunks on the whole GPU before its scan starts.
 static std::atomic<int> g_block_front{-1};
 
 }  // namespace ttt
@@ -1103,14 +1099,25 @@ ttt_status ttt_block_forward(const ttt_mlp_desc* desc, int seg_len, const void* 
     if (workspace_bytes < ttt_block_workspace_size(desc, b) || !workspace)
         return fail(TTT_ERR_INVALID_ARG, "workspace too small");
     int* status = reinterpret_cast<int*>(static_cast<char*>(workspace) + plan(q, b, TTT_BIDIR).status);
-    const RowsHook attention = [&](int r0, int r1, int max_ctas, cudaStream_t ss) {
+    // Default: the attention of every row as one launch on the whole GPU, ahead of the first projection, then
+    // the layer's own schedule.  The layer's projections and scan already occupy every SM (the scan's CTA
+    // pairs, the projections the rest), so attention beside them only takes SMs from the projections; with a
+    // head start p >= 0 set (ttt_debug_set_block_front), each segment's rows are attended to just before
+    // that segment's projection instead.
+    const int front = g_block_front.load();
+    const bool interleave = front >= 0;
+    const RowsHook attention = [&](int r0, int r1, int max_ctas, cudaStream_t ss) -> cudaError_t {
+        if (!interleave) {
+            if (r0 != 0) return cudaSuccess;
+            r1 = q.T;
+            max_ctas = 0;
+        }
         return launch_attn_seg(Qa, Ka, Va, ld_qkv, Xres, q.D, X, q.D, q.T, q.H, seg_len, r0, r1, status, max_ctas,
                                ss);
     };
-    const int front = g_block_front.load();
     return forward_impl(desc, X, theta_q, theta_k, theta_v, W1_0, W2_0, eta, b, TTT_BIDIR, alpha_f, alpha_r, Y,
                         nullptr, nullptr, nullptr, workspace, workspace_bytes, stream, nullptr, nullptr, true,
-                        &attention, front >= 0 ? front : kBlockFrontPercent);
+                        &attention, interleave ? front : -1);
 }
 
 ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_host, const void* theta_q,

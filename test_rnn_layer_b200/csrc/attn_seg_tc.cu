@@ -21,10 +21,11 @@
 // online softmax with a lazily raised maximum: the quotient O_X / l_X is the
 // same for any reference value, only overflow has to be excluded.
 //
-// Roles (320 threads): warps 0-3 the softmax of tile A, warps 4-7 that of
+// Roles (352 threads): warps 0-3 the softmax of tile A, warps 4-7 that of
 // tile B (a thread per query row, i.e. per tensor-memory lane), warp 8 the TMA
-// producer, warp 9 the MMA issuer.  While one softmax group works on the
-// exponential unit, the tensor cores run the other group's products.
+// producer, warps 9 and 10 the MMA issuers of tiles A and B (one each, so that
+// neither tile's products queue behind the other's waits).  While one softmax
+// group works on the exponential unit, the tensor cores run the other's products.
 //
 // Tensor memory (512 columns): S_A 0, S_B 128 (fp32 128 x 128); O_A 256,
 // O_B 320 (fp32 128 x 64); P_A 384, P_B 448 (128 x 128 bf16, two per column).
@@ -46,7 +47,10 @@
 namespace ttt {
 namespace {
 
-constexpr int DH = 64, BQ = 128, BKV = 128, ROWS = 2 * BQ, NST = 4, THREADS = 320;
+#ifndef TTT_ATTN_NST
+#define TTT_ATTN_NST 4
+#endif
+constexpr int DH = 64, BQ = 128, BKV = 128, ROWS = 2 * BQ, NST = TTT_ATTN_NST, THREADS = 352;
 constexpr int TILE = BQ * DH * 2;                 // 16 KB: a 128 x 64 bf16 tile
 constexpr int OFF_Q = 0;                          // Q_A, Q_B
 constexpr int OFF_KV = 2 * TILE;                  // stage s: K at OFF_KV + 2 s TILE, V after it
@@ -54,14 +58,23 @@ constexpr int OFF_BAR = OFF_KV + NST * 2 * TILE;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr uint32_t TM_S = 0, TM_O = 256, TM_P = 384;   // + 128 X (S), + 64 X (O, P) for tile X
 constexpr float kLazy = 8.0f;                     // log2 of the largest unscaled exponential
+// Pairs of every 8 whose exponentials run as a polynomial on the FMA pipe
+// (the exponential unit, 16 results per cycle per SM, is the softmax's bound).
+#ifndef TTT_ATTN_EMU
+#define TTT_ATTN_EMU 2
+#endif
+constexpr int EMU = TTT_ATTN_EMU;
+// 2^f on [-1/2, 1/2], f^0 .. f^3 (see ex2_poly).
+constexpr float kExp2C0 = 0.9999281764030457f, kExp2C1 = 0.6932609677314758f, kExp2C2 = 0.24260970950126648f,
+                kExp2C3 = 0.05517097935080528f;
 
 // Barrier slots (8 bytes each) from OFF_BAR.
 enum : int {
     B_QF = 0,              // Q_A, Q_B landed (TMA bytes)
-    B_QE = 1,              // the item's last S products are done: Q may be reloaded (MMA commit)
+    B_QE = 1,              // the item's last S products of both tiles are done: Q may be reloaded (2 MMA commits)
     B_KF = 2,              // [NST] K tile landed
     B_VF = 2 + NST,        // [NST] V tile landed
-    B_KVE = 2 + 2 * NST,   // [NST] the stage's last P V product is done (MMA commit)
+    B_KVE = 2 + 2 * NST,   // [NST] both tiles' P V products of the stage are done (2 MMA commits)
     B_SF = 2 + 3 * NST,    // [2] S_X is in tensor memory (MMA commit)
     B_SR = B_SF + 2,       // [2] the softmax group has read S_X (4 warp arrivals)
     B_PF = B_SR + 2,       // [2] P_X written, O_X rescaled (4 warp arrivals)
@@ -69,6 +82,7 @@ enum : int {
     B_SLOT = B_PV + 2      // tensor memory address (u32) and the abort flag (int)
 };
 static_assert(B_SLOT * 8 + 8 <= 256, "barrier area");
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 
 // Rows [q0, q1) of one segment whose keys are [kv0, kv1); `pairs` items of
 // 256 rows per head, items item0 .. item0 + H pairs - 1 (head-major).
@@ -89,6 +103,25 @@ struct AttnArgs {
     AttnGroup g[kMaxGroups];
 };
 
+#ifdef TTT_DEBUG_STAGES
+// Debug builds only: cycles between stage boundaries seen in CTA 0 by thread 0
+// (tile A's softmax, slots 0-7), thread 128 (tile B's, 8-15) and the MMA
+// issuer (16-23).
+__device__ long long* g_dbg_attn = nullptr;   // 40 slots
+#define STAMPA(k)                                                   \
+    do {                                                            \
+        if (stamper) {                                              \
+            const long long now_ = clock64();                       \
+            stamp_acc[k] += now_ - stamp_last;                      \
+            stamp_last = now_;                                      \
+        }                                                           \
+    } while (0)
+#else
+#define STAMPA(k) \
+    do {          \
+    } while (0)
+#endif
+
 __device__ __forceinline__ void item_of(const AttnArgs& p, int w, int& gi, int& h, int& pr) {
     gi = 0;
     while (gi + 1 < p.n_groups && p.g[gi + 1].item0 <= w) ++gi;
@@ -101,6 +134,68 @@ __device__ __forceinline__ float ex2(float x) {
     float r;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
     return r;
+}
+
+// max that returns NaN if an operand is NaN (fmaxf would drop it); two- and three-input forms
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Pairs of fp32 values in one 64-bit register pair, for the packed f32x2 arithmetic of sm_100
+// (one instruction for two elements).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// 2^x0, 2^x1 on the FMA pipe, for x <= 8 (below -125 it returns 2^-125, which
+// next to a row maximum of at least 2^-8 is far below fp32 resolution).
+// x = n + f with n = rint(x), read from the low mantissa bits of x + 1.5 * 2^23,
+// and f in [-1/2, 1/2]; 2^f from a cubic whose coefficients are a least-squares
+// fit weighted for equal relative error (Lawson's iteration), relative error at
+// most 7.6e-5 in fp32 -- 25 times below the bf16 rounding P gets; then 2^n is
+// added to the exponent field (n << 23: the shift drops the bits of 1.5 * 2^23).
+__device__ __forceinline__ void ex2_poly2(uint64_t x, float& p0, float& p1) {
+    float x0, x1;
+    f2_split(x, x0, x1);
+    x = f2(max_nan(x0, -125.0f), max_nan(x1, -125.0f));   // NaN stays NaN
+    const uint64_t shift = f2(12582912.0f, 12582912.0f);
+    const uint64_t t = f2_add(x, shift);
+    const uint64_t f = f2_sub(x, f2_sub(t, shift));
+    uint64_t p = f2_fma(f2(kExp2C3, kExp2C3), f, f2(kExp2C2, kExp2C2));
+    p = f2_fma(p, f, f2(kExp2C1, kExp2C1));
+    p = f2_fma(p, f, f2(kExp2C0, kExp2C0));
+    float t0, t1, q0, q1;
+    f2_split(t, t0, t1);
+    f2_split(p, q0, q1);
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -122,11 +217,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
 
     if (tid == 0) {
         tc::mbar_init(bars + B_QF, 1);
-        tc::mbar_init(bars + B_QE, 1);
+        tc::mbar_init(bars + B_QE, 2);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(bars + B_KF + s, 1);
             tc::mbar_init(bars + B_VF + s, 1);
-            tc::mbar_init(bars + B_KVE + s, 1);
+            tc::mbar_init(bars + B_KVE + s, 2);
         }
         for (int x = 0; x < 2; ++x) {
             tc::mbar_init(bars + B_SF + x, 1);
@@ -153,6 +248,11 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
         *abort_flag = 1;
         atomicOr(p.status, kStatusTimeout);
     };
+#ifdef TTT_DEBUG_STAGES
+    const bool stamper = blockIdx.x == 0 && (tid == 0 || tid == 128 || tid == 288 || tid == 320 || tid == 256);
+    long long stamp_acc[8] = {};
+    long long stamp_last = clock64();
+#endif
 
     if (warp == 8) {
         // ---------------- TMA producer: the item's Q tiles, then its K and V tiles through the ring
@@ -165,30 +265,38 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
                 const AttnGroup& G = p.g[gi];
                 const int q_lo = G.q0 + ROWS * pr, x = h * DH;
                 const int nkv = (G.kv1 - G.kv0 + BKV - 1) / BKV;
+                STAMPA(3);
                 if (it > 0 && !tc::mbar_wait(bars + B_QE, (it - 1) & 1, abort_flag)) { ok = false; break; }
+                STAMPA(2);
                 tc::mbar_arrive_expect_tx(bars + B_QF, 2 * TILE);
                 tc::tma_load_2d(sm + OFF_Q, &p.mapQ, x, q_lo, bars + B_QF);
                 // tile B past the last token: load tile A's rows again (its rows are never stored)
                 tc::tma_load_2d(sm + OFF_Q + TILE, &p.mapQ, x, q_lo + BQ < p.T ? q_lo + BQ : q_lo, bars + B_QF);
                 for (int j = 0; j < nkv; ++j, ++gkv) {
                     const int s = gkv % NST, use = gkv / NST;
+                    STAMPA(3);
                     if (use > 0 && !tc::mbar_wait(bars + B_KVE + s, (use - 1) & 1, abort_flag)) { ok = false; break; }
+                    STAMPA(0);
                     uint8_t* kt = sm + OFF_KV + s * 2 * TILE;
                     tc::mbar_arrive_expect_tx(bars + B_KF + s, TILE);
                     tc::tma_load_2d(kt, &p.mapK, x, G.kv0 + BKV * j, bars + B_KF + s);
                     tc::mbar_arrive_expect_tx(bars + B_VF + s, TILE);
                     tc::tma_load_2d(kt + TILE, &p.mapV, x, G.kv0 + BKV * j, bars + B_VF + s);
+                    STAMPA(1);
                 }
             }
             if (!ok) give_up();
         }
-    } else if (warp == 9) {
-        // ---------------- MMA issuer.  Step n = (item, key tile j) in the CTA's order; at iteration j it
-        // issues S of step j (once the group has read S of the step before) and then P V of step j - 1.
+    } else if (warp >= 9) {
+        // ---------------- MMA issuers, one per tile (warp 9: A, warp 10: B), so that neither tile's products
+        // wait behind the other's.  Step n = (item, key tile j) in the CTA's order; at iteration j the issuer
+        // of tile X issues S_X of step j (once its group has read S_X of the step before), then P_X V of
+        // step j - 1.  A stage of the ring and the Q tiles are released when both issuers' products are done.
+        const int X = warp - 9;
         if (tc::elect_one()) {
             constexpr uint32_t ID_S = tc::instr_desc(1, BQ, BKV, 0, 0);   // bf16, both K-major
             constexpr uint32_t ID_PV = tc::instr_desc(1, BQ, DH, 0, 1);   // bf16, A in tensor memory, V MN-major
-            const uint64_t dQ[2] = {kmajor_desc(sm + OFF_Q), kmajor_desc(sm + OFF_Q + TILE)};
+            const uint64_t dQ = kmajor_desc(sm + OFF_Q + X * TILE);
             int gkv = 0, gs = 0, it = 0;
             bool ok = true;
             for (int w = blockIdx.x; w < p.n_items && ok && !*abort_flag; w += gridDim.x, ++it) {
@@ -197,37 +305,39 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
                 const int nkv = (p.g[gi].kv1 - p.g[gi].kv0 + BKV - 1) / BKV;
                 if (!tc::mbar_wait(bars + B_QF, it & 1, abort_flag)) { ok = false; break; }
                 tc::tc_fence_after();
+                STAMPA(5);
                 for (int j = 0; j <= nkv && ok; ++j) {
                     if (j < nkv) {
                         const int n = gs + j, s = (gkv + j) % NST, use = (gkv + j) / NST;
+#ifdef TTT_DEBUG_STAGES
+                        if (stamper && tc::mbar_try_wait(bars + B_KF + s, use & 1)) stamp_acc[6] += 1;
+#endif
                         if (!tc::mbar_wait(bars + B_KF + s, use & 1, abort_flag)) { ok = false; break; }
+                        STAMPA(0);
+                        if (n > 0 && !tc::mbar_wait(bars + B_SR + X, (n - 1) & 1, abort_flag)) { ok = false; break; }
+                        tc::tc_fence_after();
                         const uint64_t dK = kmajor_desc(sm + OFF_KV + s * 2 * TILE);
-                        for (int X = 0; X < 2 && ok; ++X) {
-                            if (n > 0 && !tc::mbar_wait(bars + B_SR + X, (n - 1) & 1, abort_flag)) { ok = false; break; }
-                            tc::tc_fence_after();
 #pragma unroll
-                            for (int kk = 0; kk < DH / 16; ++kk)
-                                tc::mma_f16_ss(tm + TM_S + 128 * X, dQ[X] + 2 * kk, dK + 2 * kk, ID_S, kk > 0);
-                            tc::mma_commit(bars + B_SF + X);
-                        }
-                        if (!ok) break;
+                        for (int kk = 0; kk < DH / 16; ++kk)
+                            tc::mma_f16_ss(tm + TM_S + 128 * X, dQ + 2 * kk, dK + 2 * kk, ID_S, kk > 0);
+                        tc::mma_commit(bars + B_SF + X);
                         if (j == nkv - 1) tc::mma_commit(bars + B_QE);
+                        STAMPA(1);
                     }
                     if (j > 0) {
                         const int n = gs + j - 1, s = (gkv + j - 1) % NST, use = (gkv + j - 1) / NST;
                         if (!tc::mbar_wait(bars + B_VF + s, use & 1, abort_flag)) { ok = false; break; }
+                        if (!tc::mbar_wait(bars + B_PF + X, n & 1, abort_flag)) { ok = false; break; }
+                        tc::tc_fence_after();
+                        STAMPA(2);
                         const uint64_t dV = mnmajor_desc(sm + OFF_KV + s * 2 * TILE + TILE);
-                        for (int X = 0; X < 2 && ok; ++X) {
-                            if (!tc::mbar_wait(bars + B_PF + X, n & 1, abort_flag)) { ok = false; break; }
-                            tc::tc_fence_after();
 #pragma unroll
-                            for (int kk = 0; kk < BKV / 16; ++kk)
-                                tc::mma_f16_ts(tm + TM_O + 64 * X, tm + TM_P + 64 * X + 8 * kk, dV + (uint64_t)(kk * 128),
-                                               ID_PV, (j > 1 || kk > 0) ? 1u : 0u);
-                            tc::mma_commit(bars + B_PV + X);
-                        }
-                        if (!ok) break;
+                        for (int kk = 0; kk < BKV / 16; ++kk)
+                            tc::mma_f16_ts(tm + TM_O + 64 * X, tm + TM_P + 64 * X + 8 * kk, dV + (uint64_t)(kk * 128),
+                                           ID_PV, (j > 1 || kk > 0) ? 1u : 0u);
+                        tc::mma_commit(bars + B_PV + X);
                         tc::mma_commit(bars + B_KVE + s);
+                        STAMPA(3);
                     }
                 }
                 gs += nkv;
@@ -258,6 +368,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
             for (int j = 0; j < nkv; ++j, ++gs) {
                 if (!wait_all(bars + B_SF + X, gs & 1)) { ok = false; break; }
                 tc::tc_fence_after();
+                STAMPA(0);
                 uint32_t s[BKV];
                 tc::tmem_ld_32x32b_x32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(s + 0));
                 tc::tmem_ld_32x32b_x32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(s + 32));
@@ -267,16 +378,27 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars + B_SR + X);   // S_X may be overwritten
+                STAMPA(1);
                 const int valid = G.kv1 - (G.kv0 + BKV * j);
                 if (valid < BKV) {   // the segment's last key tile: keys past its end do not take part
 #pragma unroll
                     for (int k = 0; k < BKV; ++k)
                         if (k >= valid) s[k] = 0xff800000u;   // -inf
                 }
-                float mt = __uint_as_float(s[0]);
+                // the tile's row maximum in eight independent chains of three-input maxima (a NaN anywhere
+                // makes it NaN, so a non-finite input spoils the whole row and reaches the output check)
+                float m8[8];
 #pragma unroll
-                for (int k = 1; k < BKV; ++k) mt = fmaxf(mt, __uint_as_float(s[k]));
+                for (int i = 0; i < 8; ++i) m8[i] = max_nan(__uint_as_float(s[2 * i]), __uint_as_float(s[2 * i + 1]));
+#pragma unroll
+                for (int k = 16; k < BKV; k += 16) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        m8[i] = max3_nan(m8[i], __uint_as_float(s[k + 2 * i]), __uint_as_float(s[k + 2 * i + 1]));
+                }
+                float mt = max3_nan(max3_nan(m8[0], m8[1], m8[2]), max3_nan(m8[3], m8[4], m8[5]), max_nan(m8[6], m8[7]));
                 mt *= c;
+                STAMPA(2);
                 float f = 1.f;
                 bool rescale = false;
                 if (mt > m_run + kLazy) {   // raise the reference maximum (always on the item's first tile)
@@ -286,20 +408,40 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
                     l *= f;
                 }
                 // P as bf16 pairs, packed into the front of s (pair k2 lands in s[k2] after s[2 k2], s[2 k2 + 1] are read)
-                float lsum = 0.f;
+                // x = s c - m two at a time; EMU of every 8 pairs take 2^x on the FMA pipe, the rest on the
+                // exponential unit; row sums in four packed partial sums
+                const uint64_t c2 = f2(c, c), nm2 = f2(-m_run, -m_run);
+                uint64_t ls[4] = {0, 0, 0, 0};
 #pragma unroll
                 for (int k2 = 0; k2 < BKV / 2; ++k2) {
-                    const float p0 = ex2(fmaf(__uint_as_float(s[2 * k2]), c, -m_run));
-                    const float p1 = ex2(fmaf(__uint_as_float(s[2 * k2 + 1]), c, -m_run));
-                    lsum += p0 + p1;
+                    const uint64_t x = f2_fma(f2(__uint_as_float(s[2 * k2]), __uint_as_float(s[2 * k2 + 1])), c2, nm2);
+                    float p0, p1;
+                    if ((k2 & 7) >= 8 - EMU) {
+                        ex2_poly2(x, p0, p1);
+                    } else {
+                        float x0, x1;
+                        f2_split(x, x0, x1);
+                        p0 = ex2(x0);
+                        p1 = ex2(x1);
+                    }
+                    const uint64_t pp = f2(p0, p1);
+                    ls[k2 & 3] = f2_add(ls[k2 & 3], pp);
                     s[k2] = pack_bf16(p0, p1);
                 }
-                l += lsum;
+                {
+                    float a0, a1, b0, b1;
+                    f2_split(f2_add(f2_add(ls[0], ls[1]), f2_add(ls[2], ls[3])), a0, a1);
+                    (void)b0;
+                    (void)b1;
+                    l += a0 + a1;
+                }
+                STAMPA(3);
                 // the previous step's P V is done: P_X may be rewritten and O_X is stable
                 if (gs > 0) {
                     if (!wait_all(bars + B_PV + X, (gs - 1) & 1)) { ok = false; break; }
                     tc::tc_fence_after();
                 }
+                STAMPA(4);
                 if (__any_sync(0xffffffffu, rescale)) {
                     const float g = rescale ? f : 1.f;
                     uint32_t o[32];
@@ -318,6 +460,7 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars + B_PF + X);
+                STAMPA(5);
             }
             if (!ok) break;
             // ---- epilogue: O_X / l (+ residual) as bf16, row q_lo + 128 X + r if it belongs to the item
@@ -361,6 +504,12 @@ __global__ void __launch_bounds__(THREADS, 1) attn_seg_kernel(const __grid_const
         if (__any_sync(0xffffffffu, nonfinite) && lane == 0) atomicOr(p.status, kStatusNonFinite);
     }
 
+#ifdef TTT_DEBUG_STAGES
+    if (stamper && g_dbg_attn) {
+        const int role = tid == 0 ? 0 : tid == 128 ? 1 : tid == 288 ? 2 : tid == 320 ? 3 : 4;
+        for (int k = 0; k < 8; ++k) g_dbg_attn[8 * role + k] = stamp_acc[k];
+    }
+#endif
     if (*abort_flag) {
         // let copies and products already in flight land before the CTA's memory goes away
         const uint64_t t0 = tc::globaltimer_ns();
@@ -402,6 +551,12 @@ bool make_map(CUtensorMap* m, const void* base, int T, int cols, long long ld) {
 }
 
 }  // namespace
+
+#ifdef TTT_DEBUG_STAGES
+extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump_attn(long long* p) {
+    return (int)cudaMemcpyToSymbol(g_dbg_attn, &p, sizeof(p));
+}
+#endif
 
 bool attn_seg_supported(int d) { return d == DH; }
 

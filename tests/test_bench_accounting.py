@@ -60,3 +60,9 @@ def test_traffic_record_scales_with_the_tokens_of_a_launch(tmp_path, monkeypatch
     rec["scan_chunk_tc2"]["src_hash"] = "stale"
     path.write_text(json.dumps(rec))
     assert bench._roofline("scan_chunk_tc2", 1.0, 50, w, PEAKS, CLOCKS)["traffic"] is None
+
+
+def test_attention_flops_count_every_segment():
+    """4 L_s^2 D per segment, the last segment ragged."""
+    assert bench._attention_flops(10, 8, 4) == 4.0 * (16 + 16 + 4) * 8
+    assert bench._attention_flops(313344, 3072, 14922) == 4.0 * 3072 * (20 * 14922 ** 2 + 14904 ** 2)
