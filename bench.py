@@ -623,7 +623,7 @@ def run_block(args, rank, world, local_rank):
     w = _workload(args)
     if w.per_head or w.dirs != "bidir" or w.dtype != "bf16":
         raise SystemExit("--block needs the full-width bidirectional bf16 layer (--workload full63s)")
-    L_seg = S.segment_length(w.T)
+    L_seg = S.segment_length(S.FULL63S.T)   # the tokens of one 3-s segment of the 63-s video, whatever --T is
     inp = S.make_inputs(w, seed=rank_seed(rank), device=dev)
     inp.update(S.make_attention_inputs(w, seed=rank_seed(rank), device=dev))
     desc = L.make_desc(w.T, w.H, w.d, False, True)
@@ -736,9 +736,10 @@ def run_block(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline_block(w, L_seg, args)
     if rank == 0:
-        cfg = _config(w, {"workload": "block-" + w.name, "attention": f"segment-local, {S.SEGMENTS_63S} segments of "
-                          f"{L_seg} tokens (the last {w.T - (S.SEGMENTS_63S - 1) * L_seg}), full inside a segment, "
-                          "Q/K/V ~N(0,1) bf16, residual X", "schedule": "attention of every row, then the layer"})
+        nseg = -(-w.T // L_seg)
+        cfg = _config(w, {"workload": "block-" + w.name, "attention": f"segment-local, {nseg} segments of {L_seg} "
+                          f"tokens (the last {w.T - (nseg - 1) * L_seg}), full inside a segment, Q/K/V ~N(0,1) bf16, "
+                          "residual X", "schedule": "attention of every row, then the layer"})
         line = {"metric": METRIC_BLOCK, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16-in/bf16-mma-attention/tf32+fp16-mma-scan/fp32-state",
