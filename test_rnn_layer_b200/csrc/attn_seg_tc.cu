@@ -41,6 +41,7 @@
 #include <mutex>
 #include <vector>
 
+#include "fma_exp2.cuh"
 #include "internal.h"
 #include "tc_prims.cuh"
 
@@ -64,9 +65,7 @@ constexpr float kLazy = 8.0f;                     // log2 of the largest unscale
 #define TTT_ATTN_EMU 2
 #endif
 constexpr int EMU = TTT_ATTN_EMU;
-// 2^f on [-1/2, 1/2], f^0 .. f^3 (see ex2_poly).
-constexpr float kExp2C0 = 0.9999281764030457f, kExp2C1 = 0.6932609677314758f, kExp2C2 = 0.24260970950126648f,
-                kExp2C3 = 0.05517097935080528f;
+
 
 // Barrier slots (8 bytes each) from OFF_BAR.
 enum : int {
@@ -174,28 +173,25 @@ __device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
     return r;
 }
 
-// 2^x0, 2^x1 on the FMA pipe, for x <= 8 (below -125 it returns 2^-125, which
-// next to a row maximum of at least 2^-8 is far below fp32 resolution).
-// x = n + f with n = rint(x), read from the low mantissa bits of x + 1.5 * 2^23,
-// and f in [-1/2, 1/2]; 2^f from a cubic whose coefficients are a least-squares
-// fit weighted for equal relative error (Lawson's iteration), relative error at
-// most 7.6e-5 in fp32 -- 25 times below the bf16 rounding P gets; then 2^n is
-// added to the exponent field (n << 23: the shift drops the bits of 1.5 * 2^23).
+// 2^x0, 2^x1 on the FMA pipe: fma_exp2.cuh's cubic (relative error 7.6e-5, 25 times below the bf16
+// rounding P gets) on a pair, with the packed f32x2 arithmetic.  x <= 8 here; below -125 it returns about
+// 2^-125, which next to a row maximum of at least 2^-8 is far below fp32 resolution.
 __device__ __forceinline__ void ex2_poly2(uint64_t x, float& p0, float& p1) {
     float x0, x1;
     f2_split(x, x0, x1);
-    x = f2(max_nan(x0, -125.0f), max_nan(x1, -125.0f));   // NaN stays NaN
-    const uint64_t shift = f2(12582912.0f, 12582912.0f);
+    x = f2(max_nan(x0, -125.0f), max_nan(x1, -125.0f));   // as fexp::clamp_low; NaN stays NaN
+    using namespace fexp;
+    const uint64_t shift = f2(kShift, kShift);
     const uint64_t t = f2_add(x, shift);
     const uint64_t f = f2_sub(x, f2_sub(t, shift));
-    uint64_t p = f2_fma(f2(kExp2C3, kExp2C3), f, f2(kExp2C2, kExp2C2));
-    p = f2_fma(p, f, f2(kExp2C1, kExp2C1));
-    p = f2_fma(p, f, f2(kExp2C0, kExp2C0));
+    uint64_t p = f2_fma(f2(kC3_3, kC3_3), f, f2(kC3_2, kC3_2));
+    p = f2_fma(p, f, f2(kC3_1, kC3_1));
+    p = f2_fma(p, f, f2(kC3_0, kC3_0));
     float t0, t1, q0, q1;
     f2_split(t, t0, t1);
     f2_split(p, q0, q1);
-    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
-    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+    p0 = scale_by_rint(q0, t0);
+    p1 = scale_by_rint(q1, t1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
