@@ -62,7 +62,7 @@ constexpr float kLazy = 8.0f;                     // log2 of the largest unscale
 // Pairs of every 8 whose exponentials run as a polynomial on the FMA pipe
 // (the exponential unit, 16 results per cycle per SM, is the softmax's bound).
 #ifndef TTT_ATTN_EMU
-#define TTT_ATTN_EMU 2
+#define TTT_ATTN_EMU 1
 #endif
 constexpr int EMU = TTT_ATTN_EMU;
 

@@ -32,6 +32,14 @@ constexpr int EPI_BUF = 32 * 32 * 4;          // one 32 x 32 fp32 box
 constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_WARPS * 2 * EPI_BUF + 256;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
+// Tile order: groups of GROUP_M row tiles, and within a group every column tile over the group's row
+// tiles before the next column tile.  A theta panel (256 rows, the whole reduction) is then read by
+// GROUP_M row tiles in a row while the group's X tiles (GROUP_M x 768 KB) stay in L2, instead of
+// cycling through all of theta for every row tile next to the scan's streams.
+#ifndef TTT_PROJ_GROUP_M
+#define TTT_PROJ_GROUP_M 32
+#endif
+constexpr int GROUP_M = TTT_PROJ_GROUP_M;
 
 struct ProjTcArgs {
     CUtensorMap mapA;
@@ -43,6 +51,15 @@ struct ProjTcArgs {
     int accumulate;
     int* status;
 };
+
+// Row tile and column tile of linear tile index `tile` (see GROUP_M).
+__device__ __forceinline__ void tile_of(int tile, int m_tiles, int n_tiles, int& mt, int& nt) {
+    const int per_group = GROUP_M * n_tiles;
+    const int g = tile / per_group, local = tile - g * per_group;
+    const int gm = min(GROUP_M, m_tiles - g * GROUP_M);   // row tiles in this (possibly last, short) group
+    nt = local / gm;
+    mt = g * GROUP_M + (local - nt * gm);
+}
 
 __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_constant__ ProjTcArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -88,7 +105,8 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
             // theta is read by every M tile: keep it in L2 ahead of the streaming output
             const uint64_t keep = tc::l2_policy_evict_last();
             for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
-                const int mt = tile / n_tiles, nt = tile % n_tiles;
+                int mt, nt;
+                tile_of(tile, p.m_tiles, n_tiles, mt, nt);
                 const int which = nt / p.n_tiles_per;
                 const int n0 = (nt % p.n_tiles_per) * BN;
                 for (int kb = 0; kb < KB; ++kb) {
@@ -142,7 +160,8 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
         for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
-            const int mt = tile / n_tiles, nt = tile % n_tiles;
+            int mt, nt;
+            tile_of(tile, p.m_tiles, n_tiles, mt, nt);
             const int which = nt / p.n_tiles_per;
             const int n0 = (nt % p.n_tiles_per) * BN;
             // the whole warp leaves together (it meets __syncwarp below and __any_sync after the loop)
