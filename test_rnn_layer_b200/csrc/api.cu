@@ -296,7 +296,7 @@ constexpr int kPipeSmMargin = TTT_PIPE_SM_MARGIN;
 // GPU before that direction's scan starts (a head start: the scan then walks
 // faster than the projection can follow on the SMs the scan leaves free).
 #ifndef TTT_PIPE_FRONT_PERCENT
-#define TTT_PIPE_FRONT_PERCENT 30
+#define TTT_PIPE_FRONT_PERCENT 15
 #endif
 constexpr int kPipeFrontPercent = TTT_PIPE_FRONT_PERCENT;
 
