@@ -705,6 +705,73 @@ BwdLayout plan_backward(const ttt_mlp_desc& q, int b, ttt_direction dir) {
 }
 
 // dX += dU theta (X layout) and dtheta += dU^T src, for one projection.
+// Full-width bf16 layer: the projections' gradients on the tensor cores (the projection kernel as a
+// general GEMM).  Each fp32 dU_w is split into bf16 halves hi + lo (stored in U_w, free once the scan's
+// backward has read it), so every product keeps about 16 significand bits of dU; theta and the sources
+// are bf16 already.
+//   dX (in G):  G[t, c] += sum_w sum_j (hi_w + lo_w)[t, j] theta_w[j, c]     (theta read MN-major)
+//   dtheta_w:   dtheta_w[j, c] += sum_t (hi_w + lo_w)[t, j] src[t, c]        (both read MN-major)
+// with src = X, and for the reverse pass of the bidirectional layer src = X + bf16 increment, the two
+// bf16 arrays the forward pass projected.
+ttt_status projection_grads_tc(const ttt_mlp_desc& q, float* const dU[3], const void* const th[3], const void* X,
+                               const __nv_bfloat16* delta, float* const U[3], float* G, float* const dth[3],
+                               int* status, cudaStream_t s) {
+    const long long T = q.T, D = q.D, n = T * D;
+    __nv_bfloat16* hi[3];
+    __nv_bfloat16* lo[3];
+    for (int w = 0; w < 3; ++w) {
+        hi[w] = reinterpret_cast<__nv_bfloat16*>(U[w]);
+        lo[w] = hi[w] + n;
+        CUDA_TRY(launch_split_bf16(dU[w], hi[w], lo[w], n, s));
+    }
+    for (int part = 0; part < 2; ++part) {   // dX from the high halves, then the low halves
+        GemmTc g{};
+        g.nw = 1;
+        g.nseg = 3;
+        g.a_mn = 0;
+        g.b_mn = 1;
+        g.M = (int)T;
+        g.N = (int)D;
+        g.K = (int)D;
+        for (int w = 0; w < 3; ++w) {
+            g.A[0][w] = {part ? lo[w] : hi[w], D};
+            g.B[0][w] = {th[w], D};
+        }
+        g.C[0] = G;
+        g.ldc = D;
+        g.accumulate = 1;
+        g.status = status;
+        g.name = "grad_gemm_tc";
+        CUDA_TRY(launch_gemm_tc(g, s));
+    }
+    const void* srcs[2] = {X, delta};
+    const int nsrc = delta ? 2 : 1;
+    GemmTc g{};
+    g.nw = 3;
+    g.nseg = 2 * nsrc;
+    g.a_mn = 1;
+    g.b_mn = 1;
+    g.M = (int)D;
+    g.N = (int)D;
+    g.K = (int)T;
+    for (int w = 0; w < 3; ++w) {
+        int sg = 0;
+        for (int k = 0; k < nsrc; ++k)
+            for (int part = 0; part < 2; ++part) {
+                g.A[w][sg] = {part ? lo[w] : hi[w], D};
+                g.B[w][sg] = {srcs[k], D};
+                ++sg;
+            }
+        g.C[w] = dth[w];
+    }
+    g.ldc = D;
+    g.accumulate = 1;
+    g.status = status;
+    g.name = "grad_gemm_tc";
+    CUDA_TRY(launch_gemm_tc(g, s));
+    return TTT_OK;
+}
+
 ttt_status projection_grads(const ttt_mlp_desc& q, const float* dU, const void* theta, int th_bf16, const void* src,
                             int src_bf16, float* G, float* dtheta, cudaStream_t s) {
     const long long T = q.T, D = q.D, d = q.d;
@@ -940,8 +1007,12 @@ ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, const void*
     float* G = reinterpret_cast<float*>(ws + B.g);   // gradient with respect to the current gate's output
     CUDA_TRY(cudaMemcpyAsync(G, dY, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
     float* xp = reinterpret_cast<float*>(ws + B.xp);
+    // the full-width bf16 layer takes its projection gradients on the tensor cores, and (as its forward pass
+    // does) projects the reverse direction's input as X plus the bf16 gate increment, kept where Y was
+    const bool tc_grads = !q.per_head_input && x_bf16 && proj_full_tc_supported(q.D, q.D) && g_proj_impl.load() != 1;
+    __nv_bfloat16* delta = tc_grads && dir == TTT_BIDIR ? reinterpret_cast<__nv_bfloat16*>(ws + B.y) : nullptr;
     if (dir == TTT_BIDIR)   // X' = X + tanh(alpha_f) z_f, the reverse direction's input
-        CUDA_TRY(launch_gate(X, x_bf16, zs, alpha_f, xp, 0, nullptr, status, q.T, q.H, q.d, q.per_head_input, 0, s));
+        CUDA_TRY(launch_gate(X, x_bf16, zs, alpha_f, xp, 0, delta, status, q.T, q.H, q.d, q.per_head_input, 0, s));
     const void* th[3] = {theta_q, theta_k, theta_v};
     float* U[3] = {reinterpret_cast<float*>(ws + B.u[0]), reinterpret_cast<float*>(ws + B.u[1]),
                    reinterpret_cast<float*>(ws + B.u[2])};
@@ -959,14 +1030,24 @@ ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, const void*
         const int src_bf16 = on_xp ? 0 : x_bf16;
         CUDA_TRY(launch_gate_backward(G, zs + k * n, reverse ? alpha_r : alpha_f, dz, reverse ? dalpha_r : dalpha_f,
                                       q.T, q.H, q.d, q.per_head_input, s));
-        st = project(q, src, src_bf16, th, U, 0, status, s);
+        if (on_xp && delta) {
+            st = project(q, X, 1, th, U, 0, status, s);
+            if (st == TTT_OK) st = project(q, delta, 1, th, U, 1, status, s);
+        } else {
+            st = project(q, src, src_bf16, th, U, 0, status, s);
+        }
         if (st != TTT_OK) return st;
         CUDA_TRY(launch_scan_backward(U[0], U[1], U[2], qkv_hs, qkv_ts, dz, qkv_hs, qkv_ts, W1_0, W2_0, dU[0], dU[1],
                                       dU[2], dW1_0, dW2_0, reinterpret_cast<float*>(ws + B.scratch), q.T, q.H, q.d, b,
                                       reverse ? 1 : 0, eta, s));
-        for (int w = 0; w < 3; ++w) {   // the gate's x path keeps G; the projections add theta's share
-            st = projection_grads(q, dU[w], th[w], x_bf16, src, src_bf16, G, dth[w], s);
+        if (tc_grads) {   // the gate's x path keeps G; the projections add theta's share
+            st = projection_grads_tc(q, dU, th, X, on_xp ? delta : nullptr, U, G, dth, status, s);
             if (st != TTT_OK) return st;
+        } else {
+            for (int w = 0; w < 3; ++w) {
+                st = projection_grads(q, dU[w], th[w], x_bf16, src, src_bf16, G, dth[w], s);
+                if (st != TTT_OK) return st;
+            }
         }
     }
     CUDA_TRY(cudaMemcpyAsync(dX, G, n * sizeof(float), cudaMemcpyDeviceToDevice, s));

@@ -93,7 +93,35 @@ __global__ void __launch_bounds__(GT) gemm_kernel(float* C, long long ldc, long 
         }
 }
 
+// hi = bf16(x) (nearest), lo = bf16(x - hi): the pair carries 16 bits of x's 24-bit significand, so a
+// product with a bf16 operand formed as hi b + lo b keeps about 2^-16 relative; four elements per thread.
+__global__ void __launch_bounds__(256) split_bf16_kernel(const float4* x, uint2* hi, uint2* lo, long long n4) {
+    for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n4; i += (long long)gridDim.x * 256) {
+        const float4 v = x[i];
+        const __nv_bfloat162 h01 = __floats2bfloat162_rn(v.x, v.y), h23 = __floats2bfloat162_rn(v.z, v.w);
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(v.x - __low2float(h01), v.y - __high2float(h01));
+        const __nv_bfloat162 l23 = __floats2bfloat162_rn(v.z - __low2float(h23), v.w - __high2float(h23));
+        hi[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+        lo[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_split_bf16(const float* x, __nv_bfloat16* hi, __nv_bfloat16* lo, long long n, cudaStream_t s) {
+    if (n % 4 != 0) return cudaErrorInvalidValue;
+    const long long n4 = n / 4;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (n4 + 255) / 256;
+    const int grid = (int)(want < 8LL * sms ? want : 8LL * sms);
+    LaunchScope scope("split_bf16", s);
+    split_bf16_kernel<<<grid > 0 ? grid : 1, 256, 0, s>>>(reinterpret_cast<const float4*>(x),
+                                                           reinterpret_cast<uint2*>(hi), reinterpret_cast<uint2*>(lo),
+                                                           n4);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_gate_backward(const float* g, const float* z, const float* alpha, float* dz, float* dalpha, int T,
                                  int H, int d, int per_head, cudaStream_t s) {

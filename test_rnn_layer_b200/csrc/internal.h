@@ -98,6 +98,31 @@ bool proj_full_tc_supported(int N, int K);
 cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
                                 int accumulate, int* status, int max_ctas, cudaStream_t s);
 
+// The same tcgen05 kernel as a general bf16 GEMM: up to 3 outputs
+//   C_w[M x N] (+)= sum_{s < nseg} A_{w,s} B_{w,s}^T   (fp32 accumulate, fp32 C, row stride ldc)
+// with every operand bf16 and row-major in memory: K-major (a_mn / b_mn = 0) means A is [M x K] and B is
+// [N x K]; MN-major (= 1) means A is [K x M] and B is [K x N], K the row index.  N must be a multiple
+// of 64; operand rows or columns past M, N or K read as zero.  ld: the operand's row stride (elements,
+// a multiple of 8).
+struct GemmTcOperand {
+    const void* ptr;
+    long long ld;
+};
+struct GemmTc {
+    int nw, nseg, a_mn, b_mn;
+    int M, N, K;   // K: the reduction length of every segment
+    GemmTcOperand A[3][4], B[3][4];
+    float* C[3];
+    long long ldc;
+    int accumulate;
+    int* status;
+    int max_ctas;      // 0: one CTA per SM
+    const char* name;  // for the launch timing ("gemm_tc" if null)
+};
+cudaError_t launch_gemm_tc(const GemmTc& g, cudaStream_t s);
+// hi = bf16(x), lo = bf16(x - hi): x = hi + lo to about 2^-16 relative (n elements, 16-byte aligned).
+cudaError_t launch_split_bf16(const float* x, __nv_bfloat16* hi, __nv_bfloat16* lo, long long n, cudaStream_t s);
+
 // Segment-local attention (d = 64, bf16) with a residual add, tcgen05:
 // rows [row0, row1) of Out = Xres + softmax(Q K^T / 8) V inside segments of L
 // tokens.  Q, K, V share the row stride ld_qkv; Xres (optional) and Out share

@@ -41,13 +41,19 @@ constexpr uint32_t TMEM_COLS = 512;
 #endif
 constexpr int GROUP_M = TTT_PROJ_GROUP_M;
 
+// Up to 3 outputs C_w (+)= sum over segments s of A_{w,s} B_{w,s}^T, every segment the same reduction
+// length K: the projections pass one A for all three outputs and one segment; the projection gradients
+// pass several (the high and low bf16 halves of an fp32 operand, two sources).
+constexpr int kMaxSeg = 4;
 struct ProjTcArgs {
-    CUtensorMap mapA;
-    CUtensorMap mapB[3];
+    CUtensorMap mapA[3][kMaxSeg];
+    CUtensorMap mapB[3][kMaxSeg];
     CUtensorMap mapC[3];
-    int K;                 // reduction length (model dim)
-    int N;                 // output columns of each projection (a multiple of 64; the last tile may be partial)
-    int m_tiles, n_tiles_per, tiles;
+    int K;                 // reduction length of one segment
+    int nseg;              // segments along the reduction
+    int a_mn, b_mn;        // 1: that operand is MN-major in memory (rows = K), 0: K-major (rows = M or N)
+    int N;                 // output columns of each output (a multiple of 64; the last tile may be partial)
+    int m_tiles, n_tiles_per, nw, tiles;
     int accumulate;
     int* status;
 };
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
         for (int a = 0; a < 2; ++a) { tc::mbar_init(&tmem_full[a], 1); tc::mbar_init(&tmem_empty[a], EPI_WARPS); }
         *abort_flag = 0;
         tc::fence_mbar_init();
-        tc::tma_prefetch_desc(&p.mapA);
+        tc::tma_prefetch_desc(&p.mapA[0][0]);
     }
     if (warp == 1) {
         tc::tmem_alloc(tmem_base_slot, TMEM_COLS);
@@ -89,8 +95,8 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_slot;
-    const int KB = p.K / BK;
-    const int n_tiles = 3 * p.n_tiles_per;
+    const int KB = (p.K + BK - 1) / BK;   // per segment; operand columns or rows past K read as zero
+    const int n_tiles = p.nw * p.n_tiles_per;
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -109,12 +115,21 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
                 tile_of(tile, p.m_tiles, n_tiles, mt, nt);
                 const int which = nt / p.n_tiles_per;
                 const int n0 = (nt % p.n_tiles_per) * BN;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = 0; kb < KB * p.nseg; ++kb) {
                     if (!tc::mbar_wait(&empty[s], phase ^ 1, abort_flag)) { give_up(); break; }
                     uint8_t* st = stage_base + s * STAGE_BYTES;
+                    const int seg = kb / KB, k0 = (kb - seg * KB) * BK;
+                    const CUtensorMap* ma = &p.mapA[which][seg];
+                    const CUtensorMap* mb = &p.mapB[which][seg];
                     tc::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                    tc::tma_load_2d(st, &p.mapA, kb * BK, mt * BM, &full[s]);
-                    tc::tma_load_2d_hint(st + A_BYTES, &p.mapB[which], kb * BK, n0, &full[s], keep);
+                    // K-major: one box of BK columns; MN-major: boxes of 64 M/N columns x BK rows, 8 KB apart
+                    if (!p.a_mn) tc::tma_load_2d(st, ma, k0, mt * BM, &full[s]);
+                    else
+                        for (int i = 0; i < BM / 64; ++i) tc::tma_load_2d(st + i * 8192, ma, mt * BM + 64 * i, k0, &full[s]);
+                    if (!p.b_mn) tc::tma_load_2d_hint(st + A_BYTES, mb, k0, n0, &full[s], keep);
+                    else
+                        for (int i = 0; i < BN / 64; ++i)
+                            tc::tma_load_2d_hint(st + A_BYTES + i * 8192, mb, n0 + 64 * i, k0, &full[s], keep);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
             }
@@ -122,7 +137,11 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (tc::elect_one()) {
-            constexpr uint32_t idesc = tc::instr_desc(1, BM, BN, 0, 0);
+            const uint32_t idesc = tc::instr_desc(1, BM, BN, p.a_mn, p.b_mn);
+            // K step of 16: K-major +32 bytes inside the 128-byte row; MN-major +16 rows (2 KB), the 64-wide
+            // M/N blocks 8 KB apart (leading offset), 8-row groups 1 KB apart (stride offset)
+            const uint32_t a_step = p.a_mn ? 2048 : 32, b_step = p.b_mn ? 2048 : 32;
+            const uint32_t a_lbo = p.a_mn ? 8192 : 16, b_lbo = p.b_mn ? 8192 : 16;
             int s = 0;
             uint32_t phase = 0;
             int it = 0;
@@ -133,15 +152,15 @@ __global__ void __launch_bounds__(THREADS, 1) proj_tc_kernel(const __grid_consta
                 tc::tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * BN;
                 bool ok = true;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = 0; kb < KB * p.nseg; ++kb) {
                     if (!tc::mbar_wait(&full[s], phase, abort_flag)) { ok = false; break; }
                     tc::tc_fence_after();
                     const uint32_t a_addr = tc::smem_u32(stage_base + s * STAGE_BYTES);
                     const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = tc::smem_desc(a_addr + k * 32, 16, 1024);
-                        const uint64_t bd = tc::smem_desc(b_addr + k * 32, 16, 1024);
+                        const uint64_t ad = tc::smem_desc(a_addr + k * a_step, a_lbo, 1024);
+                        const uint64_t bd = tc::smem_desc(b_addr + k * b_step, b_lbo, 1024);
                         tc::mma_f16_ss(d_tmem, ad, bd, idesc, (kb | k) != 0);
                     }
                     tc::mma_commit(&empty[s]);
@@ -252,32 +271,65 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 // partial last tile read theta rows beyond N as zero fill.
 bool proj_full_tc_supported(int N, int K) { return N % 64 == 0 && K % BK == 0 && N > 0 && K > 0; }
 
-cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
-                                int accumulate, int* status, int max_ctas, cudaStream_t s) {
+cudaError_t launch_gemm_tc(const GemmTc& g, cudaStream_t s) {
+    if (g.nw < 1 || g.nw > 3 || g.nseg < 1 || g.nseg > kMaxSeg || g.M < 1 || g.N < 1 || g.K < 1 || g.N % 64 != 0)
+        return cudaErrorInvalidValue;
     ProjTcArgs p{};
-    bool ok = make_map(&p.mapA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, T, (uint64_t)K * 2, BK, BM);
-    for (int w = 0; w < 3 && ok; ++w) {
-        ok = make_map(&p.mapB[w], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, theta[w], K, N, (uint64_t)K * 2, BK, BN) &&
-             make_map(&p.mapC[w], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out[w], N, T, (uint64_t)N * 4, 32, 32);
+    bool ok = true;
+    for (int w = 0; w < g.nw && ok; ++w) {
+        for (int sg = 0; sg < g.nseg && ok; ++sg) {
+            const GemmTcOperand& a = g.A[w][sg];
+            const GemmTcOperand& b = g.B[w][sg];
+            ok = (g.a_mn ? make_map(&p.mapA[w][sg], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.ptr, g.M, g.K, a.ld * 2, 64, BK)
+                         : make_map(&p.mapA[w][sg], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.ptr, g.K, g.M, a.ld * 2, BK, BM)) &&
+                 (g.b_mn ? make_map(&p.mapB[w][sg], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b.ptr, g.N, g.K, b.ld * 2, 64, BK)
+                         : make_map(&p.mapB[w][sg], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b.ptr, g.K, g.N, b.ld * 2, BK, BN));
+        }
+        ok = ok && make_map(&p.mapC[w], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.C[w], g.N, g.M, (uint64_t)g.ldc * 4, 32, 32);
     }
     if (!ok) return cudaErrorInvalidValue;
-    p.K = K;
-    p.N = N;
-    p.m_tiles = (T + BM - 1) / BM;
-    p.n_tiles_per = (N + BN - 1) / BN;
-    p.tiles = p.m_tiles * 3 * p.n_tiles_per;
-    p.accumulate = accumulate;
-    p.status = status;
+    p.K = g.K;
+    p.nseg = g.nseg;
+    p.a_mn = g.a_mn;
+    p.b_mn = g.b_mn;
+    p.N = g.N;
+    p.m_tiles = (g.M + BM - 1) / BM;
+    p.n_tiles_per = (g.N + BN - 1) / BN;
+    p.nw = g.nw;
+    p.tiles = p.m_tiles * g.nw * p.n_tiles_per;
+    p.accumulate = g.accumulate;
+    p.status = g.status;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    LaunchScope scope("proj_full_tc", s);
+    LaunchScope scope(g.name ? g.name : "gemm_tc", s);
     int grid = p.tiles < sms ? p.tiles : sms;
-    if (max_ctas > 0 && grid > max_ctas) grid = max_ctas;
+    if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
     proj_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_proj_full_tc(const void* A, const void* const theta[3], float* const out[3], int T, int N, int K,
+                                int accumulate, int* status, int max_ctas, cudaStream_t s) {
+    GemmTc g{};
+    g.nw = 3;
+    g.nseg = 1;
+    g.M = T;
+    g.N = N;
+    g.K = K;
+    for (int w = 0; w < 3; ++w) {
+        g.A[w][0] = {A, K};
+        g.B[w][0] = {theta[w], K};
+        g.C[w] = out[w];
+    }
+    g.ldc = N;
+    g.accumulate = accumulate;
+    g.status = status;
+    g.max_ctas = max_ctas;
+    g.name = "proj_full_tc";
+    return launch_gemm_tc(g, s);
 }
 
 }  // namespace ttt

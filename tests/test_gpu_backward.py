@@ -54,3 +54,4 @@ def test_backward_rejects_chunks_above_64():
     desc = L.make_desc(w.T, w.H, w.d, w.per_head, True)
     assert L.ttt_mlp_backward_workspace_size(desc, 100, L.TTT_BIDIR) == 0
     assert "64" in L.ttt_last_error()
+
