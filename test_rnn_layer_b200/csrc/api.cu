@@ -288,7 +288,7 @@ Pipe& pipe_for(int dev, cudaStream_t caller) {
 
 constexpr int kPipeMinSegChunks = 16;
 #ifndef TTT_PIPE_SM_MARGIN
-#define TTT_PIPE_SM_MARGIN 8
+#define TTT_PIPE_SM_MARGIN 4
 #endif
 constexpr int kPipeSmMargin = TTT_PIPE_SM_MARGIN;
 // When the scan applies the gate itself, the projections of the segments that
@@ -303,9 +303,12 @@ constexpr int kPipeFrontPercent = TTT_PIPE_FRONT_PERCENT;
 // Chunk ranges [begin, end) of a walk over `nchunks` chunks: segments grow
 // by 3/2 from 16 chunks at both ends (short exposed head and tail: 16, 24,
 // 36, ... and ..., 36, 24, 16), with equal pieces of at most
-// max(16, ceil(nchunks / 12)) chunks in between.
+// max(16, ceil(nchunks / TTT_PIPE_SEG_DIV)) chunks in between.
+#ifndef TTT_PIPE_SEG_DIV
+#define TTT_PIPE_SEG_DIV 16
+#endif
 std::vector<std::pair<int, int>> pipe_segments(int nchunks) {
-    const int cap = std::max(kPipeMinSegChunks, (nchunks + 11) / 12);
+    const int cap = std::max(kPipeMinSegChunks, (nchunks + TTT_PIPE_SEG_DIV - 1) / TTT_PIPE_SEG_DIV);
     std::vector<int> front, back;
     int rem = nchunks;
     for (int sz = kPipeMinSegChunks; sz < cap && rem > 0; sz = sz * 3 / 2) {

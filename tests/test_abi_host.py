@@ -158,14 +158,14 @@ def test_pipeline_segments_tile_the_walk(nchunks):
     """The pipelined full-width layer splits a direction's walk into chunk
     segments: contiguous, non-empty, covering [0, nchunks) exactly; the first
     and last segments are the shortest (their projection or gate is not
-    overlapped), no segment exceeds max(16, ceil(nchunks / 12))."""
+    overlapped), no segment exceeds max(16, ceil(nchunks / 16))."""
     seg = L.ttt_debug_pipe_segments(nchunks)
     assert seg[0][0] == 0 and seg[-1][1] == nchunks
     for (a0, a1), (b0, _) in zip(seg, seg[1:]):
         assert a1 == b0
     sizes = [e - b for b, e in seg]
     assert min(sizes) >= 1
-    cap = max(16, -(-nchunks // 12))
+    cap = max(16, -(-nchunks // 16))
     assert max(sizes) <= cap
     if len(seg) > 2:
         assert sizes[0] <= min(sizes[1:-1]) and sizes[-1] <= min(sizes[1:-1])
@@ -177,8 +177,8 @@ def test_pipeline_segments_of_the_benchmark_layer():
     from 16 at both ends and the middle is split into equal pieces."""
     sizes = [e - b for b, e in L.ttt_debug_pipe_segments(4896)]
     assert sizes[:4] == [16, 24, 36, 54] and sizes[-4:] == [54, 36, 24, 16]
-    middle = sizes[9:-9]   # between the two ramps (9 segments each, capped at 408 = 4896 / 12)
-    assert max(middle) - min(middle) <= 1 and max(middle) <= 408
+    middle = sizes[8:-8]   # between the two ramps (8 segments each: 16 ... 271), at most 306 = 4896 / 16
+    assert max(middle) - min(middle) <= 1 and max(middle) <= 306
 
 
 def test_attention_argument_errors_before_any_cuda_call():
