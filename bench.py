@@ -454,7 +454,7 @@ def run_ours(args, rank, world, local_rank):
     direction = L.DIRS[w.dirs]
     if linear:
         ws_dev_bytes = L.ttt_linear_workspace_size(desc, w.b, direction)
-        ws = torch.empty(ws_dev_bytes, dtype=torch.uint8, device=dev)
+        ws = torch.empty(L.ttt_linear_host_io_workspace_size(desc, w.b, direction), dtype=torch.uint8, device=dev)
     else:
         ws = L.alloc_workspace(desc, w.b, direction, dev, host_io=True)
         ws_dev_bytes = L.ttt_mlp_workspace_size(desc, w.b, direction)
@@ -516,15 +516,14 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_e2e:
         Xh = inp["X"].cpu().pin_memory()
         Yh = torch.empty_like(Xh).pin_memory()
-        Xd = torch.empty_like(inp["X"])
         ns = max(1, min(args.steps, args.e2e_steps))
 
         def e2e_step():
-            if linear:   # the TTT-Linear layer has no host-buffer entry point: copies around the device call
-                Xd.copy_(Xh, non_blocking=True)
-                step(Xd, Y)
-                Yh.copy_(Y, non_blocking=True)
-                L.check(L.ttt_mlp_status(ws, stream), "status")
+            if linear:
+                st = L.ttt_linear_forward_host(desc, Xh, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W_0"],
+                                               w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"], Yh, ws,
+                                               ws.numel(), stream)
+                L.check(st, "ttt_linear_forward_host")
             else:
                 st = L.ttt_mlp_forward_host(desc, Xh, inp["theta_q"], inp["theta_k"], inp["theta_v"], inp["W1_0"],
                                             inp["W2_0"], w.eta_eff, w.b, direction, inp["alpha_f"], inp["alpha_r"],

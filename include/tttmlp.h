@@ -396,6 +396,22 @@ TTT_API ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, c
                               ttt_stream_t stream);
 
 /*
+ * TTT-Linear with HOST buffers, as ttt_mlp_forward_host is for the MLP layer:
+ * X_host in, Y_host out (pinned for full copy speed), everything else device
+ * memory as in ttt_linear_forward; the workspace of
+ * ttt_linear_host_io_workspace_size bytes adds device staging for X and Y.
+ * On the segmented full-width bf16 path X crosses segment by segment ahead of
+ * its projection and Y comes back segment by segment behind its gate.
+ * Synchronises `stream` and returns the status as ttt_mlp_status would.
+ */
+TTT_API size_t ttt_linear_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
+TTT_API ttt_status ttt_linear_forward_host(const ttt_mlp_desc* desc, const void* X_host,
+                                           const void* theta_q, const void* theta_k, const void* theta_v,
+                                           const float* W_0, float eta, int b, ttt_direction dir,
+                                           const float* alpha_f, const float* alpha_r, void* Y_host,
+                                           void* workspace, size_t workspace_bytes, ttt_stream_t stream);
+
+/*
  * Fault injection for tests (process-wide).  While enabled, the two-CTA
  * tensor-core scan kernel (the default for bf16 inputs) first waits on an
  * mbarrier that nothing arrives on, with a 1 ms limit; the wait expires, the

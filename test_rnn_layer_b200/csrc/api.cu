@@ -884,10 +884,16 @@ size_t ttt_linear_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction 
     return plan_linear(*desc, dir).total;
 }
 
-ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
-                              const void* theta_v, const float* W_0, float eta, int b, ttt_direction dir,
-                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, float* W_T,
-                              void* workspace, size_t workspace_bytes, ttt_stream_t stream_) {
+}  // extern "C"
+
+namespace {
+// ttt_linear_forward; with X_host / Y_host set, X is copied in from X_host and Y out to Y_host (segment by
+// segment on the pipelined path, whole otherwise) and X, Y are the device staging arrays.
+ttt_status linear_impl(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                       const void* theta_v, const float* W_0, float eta, int b, ttt_direction dir,
+                       const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, float* W_T,
+                       void* workspace, size_t workspace_bytes, ttt_stream_t stream_, const void* X_host,
+                       void* Y_host) {
     ttt_status st = check_desc_linear(desc, b, dir);
     if (st != TTT_OK) return st;
     const ttt_mlp_desc& q = *desc;
@@ -940,19 +946,64 @@ ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const voi
             return launch_scan_linear_tc(a, ss);
         };
         const PipeBufs bufs{status, xp, delta, reinterpret_cast<float*>(ws + L.zbuf)};
-        return forward_pipelined(q, bufs, 1, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, nullptr,
-                                 nullptr);
+        return forward_pipelined(q, bufs, 1, seg_scan, X, th, qkv, b, dir, alpha_f, alpha_r, Y, Z_out, s, X_host,
+                                 Y_host);
     }
-    if (dir != TTT_BIDIR)
-        return linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, dir == TTT_REV,
-                                dir == TTT_REV ? alpha_r : alpha_f, Y, x_bf16, nullptr, Z_out, W_T, s);
-    st = linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, 0, alpha_f, xp, 0, delta, Z_out, W_T,
-                          s);
+    if (X_host) CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(X), X_host, xbytes, cudaMemcpyHostToDevice, s));
+    if (dir != TTT_BIDIR) {
+        st = linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, dir == TTT_REV,
+                              dir == TTT_REV ? alpha_r : alpha_f, Y, x_bf16, nullptr, Z_out, W_T, s);
+    } else {
+        st = linear_direction(q, L, ws, X, x_bf16, X, x_bf16, 0, th, W_0, eta, b, 0, alpha_f, xp, 0, delta, Z_out,
+                              W_T, s);
+        if (st != TTT_OK) return st;
+        // reverse on X' = X + tanh(alpha_f) z_f; theta X' = theta X + theta bf16(X' - X) where X is bf16 and full
+        // width
+        st = linear_direction(q, L, ws, xp, 0, L.split_reverse ? static_cast<const void*>(delta) : xp,
+                              L.split_reverse ? 1 : 0, L.split_reverse ? 1 : 0, th, W_0, eta, b, 1, alpha_r, Y,
+                              x_bf16, nullptr, Z_out ? Z_out + n : nullptr, W_T ? W_T + nW : nullptr, s);
+    }
     if (st != TTT_OK) return st;
-    // reverse on X' = X + tanh(alpha_f) z_f; theta X' = theta X + theta bf16(X' - X) where X is bf16 and full width
-    return linear_direction(q, L, ws, xp, 0, L.split_reverse ? static_cast<const void*>(delta) : xp,
-                            L.split_reverse ? 1 : 0, L.split_reverse ? 1 : 0, th, W_0, eta, b, 1, alpha_r, Y,
-                            x_bf16, nullptr, Z_out ? Z_out + n : nullptr, W_T ? W_T + nW : nullptr, s);
+    if (Y_host) CUDA_TRY(cudaMemcpyAsync(Y_host, Y, xbytes, cudaMemcpyDeviceToHost, s));
+    return TTT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ttt_status ttt_linear_forward(const ttt_mlp_desc* desc, const void* X, const void* theta_q, const void* theta_k,
+                              const void* theta_v, const float* W_0, float eta, int b, ttt_direction dir,
+                              const float* alpha_f, const float* alpha_r, void* Y, float* Z_out, float* W_T,
+                              void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+    return linear_impl(desc, X, theta_q, theta_k, theta_v, W_0, eta, b, dir, alpha_f, alpha_r, Y, Z_out, W_T,
+                       workspace, workspace_bytes, stream, nullptr, nullptr);
+}
+
+size_t ttt_linear_host_io_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {
+    if (check_desc_linear(desc, b, dir) != TTT_OK) return 0;
+    const size_t io = align_up((size_t)desc->T * desc->D * elem_size(desc->x_dtype));
+    return plan_linear(*desc, dir).total + 2 * io;
+}
+
+ttt_status ttt_linear_forward_host(const ttt_mlp_desc* desc, const void* X_host, const void* theta_q,
+                                   const void* theta_k, const void* theta_v, const float* W_0, float eta, int b,
+                                   ttt_direction dir, const float* alpha_f, const float* alpha_r, void* Y_host,
+                                   void* workspace, size_t workspace_bytes, ttt_stream_t stream) {
+    ttt_status st = check_desc_linear(desc, b, dir);
+    if (st != TTT_OK) return st;
+    if (!X_host || !Y_host || !workspace) return fail(TTT_ERR_INVALID_ARG, "X_host, Y_host, workspace must be non-NULL");
+    const size_t need = ttt_linear_host_io_workspace_size(desc, b, dir);
+    if (workspace_bytes < need)
+        return fail(TTT_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    const LinearLayout L = plan_linear(*desc, dir);
+    const size_t xbytes = (size_t)desc->T * desc->D * elem_size(desc->x_dtype);
+    char* ws = static_cast<char*>(workspace);
+    void* Xd = ws + L.total;
+    void* Yd = ws + L.total + align_up(xbytes);
+    st = linear_impl(desc, Xd, theta_q, theta_k, theta_v, W_0, eta, b, dir, alpha_f, alpha_r, Yd, nullptr, nullptr,
+                     workspace, L.total, stream, X_host, Y_host);
+    if (st != TTT_OK) return st;
+    return ttt_mlp_status(workspace, stream);
 }
 
 size_t ttt_mlp_backward_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir) {

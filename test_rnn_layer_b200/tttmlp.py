@@ -29,7 +29,8 @@ EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_
             "ttt_linear_workspace_size", "ttt_linear_forward", "ttt_debug_pipe_segments",
             "ttt_mlp_backward_workspace_size", "ttt_mlp_backward", "ttt_mlp_heads_workspace_size",
             "ttt_mlp_forward_heads", "ttt_seg_attention_workspace_size", "ttt_seg_attention",
-            "ttt_block_workspace_size", "ttt_block_forward", "ttt_debug_set_block_front"]
+            "ttt_block_workspace_size", "ttt_block_forward", "ttt_debug_set_block_front",
+            "ttt_linear_host_io_workspace_size", "ttt_linear_forward_host"]
 
 
 class TTTError(RuntimeError):
@@ -93,6 +94,10 @@ def lib():
         L.ttt_mlp_noalloc_status.argtypes = [vp]
         L.ttt_linear_workspace_size.restype = sz
         L.ttt_linear_workspace_size.argtypes = [dp, i, i]
+        L.ttt_linear_host_io_workspace_size.restype = sz
+        L.ttt_linear_host_io_workspace_size.argtypes = [dp, i, i]
+        L.ttt_linear_forward_host.restype = i
+        L.ttt_linear_forward_host.argtypes = [dp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, sz, vp]
         L.ttt_linear_forward.restype = i
         L.ttt_linear_forward.argtypes = [dp, vp, vp, vp, vp, vp, f, i, i, vp, vp, vp, vp, vp, vp, sz, vp]
         L.ttt_mlp_status.restype = i
@@ -300,6 +305,17 @@ def ttt_mlp_noalloc_status(stream=None) -> int:
 
 def ttt_linear_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
     return int(lib().ttt_linear_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_linear_host_io_workspace_size(desc: ttt_mlp_desc, b: int, direction: int) -> int:
+    return int(lib().ttt_linear_host_io_workspace_size(ctypes.byref(desc), b, direction))
+
+
+def ttt_linear_forward_host(desc, X_host, theta_q, theta_k, theta_v, W_0, eta, b, direction, alpha_f, alpha_r,
+                            Y_host, workspace, workspace_bytes, stream=None) -> int:
+    return int(lib().ttt_linear_forward_host(ctypes.byref(desc), _p(X_host), _p(theta_q), _p(theta_k), _p(theta_v),
+                                             _p(W_0), float(eta), b, direction, _p(alpha_f), _p(alpha_r),
+                                             _p(Y_host), _p(workspace), workspace_bytes, _stream(stream)))
 
 
 def ttt_linear_forward(desc, X, theta_q, theta_k, theta_v, W_0, eta, b, direction, alpha_f, alpha_r, Y, Z_out,

@@ -82,3 +82,26 @@ def test_linear_nonfinite_state_is_reported():
                                  w.dirs, alpha_f=g["alpha_f"], alpha_r=g["alpha_r"], per_head=True,
                                  check_status=False)
     assert L.ttt_mlp_status(out["workspace"]) == L.TTT_ERR_NONFINITE
+
+
+@pytest.mark.parametrize("w", [S.FULL63S.with_(T=3000, H=4, D=256), S.MINIBATCH.with_(T=500, H=3),
+                               S.FULL63S.with_(T=3000, H=4, D=256, dirs="rev")],
+                         ids=["full-bidir-segmented", "per-head-bidir", "full-rev"])
+def test_linear_host_buffers_equal_device_call(w):
+    """ttt_linear_forward_host (X in from pinned host memory, Y back to it; on the segmented path the copies
+    go segment by segment) runs the same kernels on the same values as ttt_linear_forward: the same bits."""
+    inp = S.make_linear_inputs(w, seed=2)
+    dev = torch.device("cuda")
+    g = {k: v.to(dev) for k, v in inp.items()}
+    out = L.linear_layer_forward(g["X"], g["theta_q"], g["theta_k"], g["theta_v"], g["W_0"], w.eta_eff, w.b, w.dirs,
+                                 alpha_f=g["alpha_f"], alpha_r=g["alpha_r"], per_head=w.per_head)
+    desc = L.make_desc(w.T, w.H, w.d, w.per_head, w.dtype == "bf16")
+    direction = L.DIRS[w.dirs]
+    n = L.ttt_linear_host_io_workspace_size(desc, w.b, direction)
+    assert n > L.ttt_linear_workspace_size(desc, w.b, direction)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    Xh = inp["X"].contiguous().pin_memory()
+    Yh = torch.empty_like(Xh).pin_memory()
+    L.check(L.ttt_linear_forward_host(desc, Xh, g["theta_q"], g["theta_k"], g["theta_v"], g["W_0"], w.eta_eff, w.b,
+                                      direction, g["alpha_f"], g["alpha_r"], Yh, ws, n), "ttt_linear_forward_host")
+    assert torch.equal(Yh, out["Y"].cpu())
