@@ -35,7 +35,6 @@ namespace {
 constexpr int NT = 512;          // threads per CTA
 constexpr int BMAX = 64;         // largest chunk
 constexpr int kCkpt = 32;        // chunks between two checkpoints
-constexpr int TM = 64, TN = 64, TK = 16;   // GEMM tile
 
 struct BwdArgs {
     const float* Q;
@@ -125,42 +124,88 @@ __device__ __forceinline__ Mat T_(const float* p, int ld) { return Mat{p, 1, ld}
 // C[M x N] (+)= alpha * A[M x Kd] B[Kd x N], C row-major with leading dimension ldc.
 // mask: 0 none, 1 keep C[r][c] only for c <= r (lower triangle incl. diagonal).
 // All threads of the CTA call it; it ends with a barrier.
-__device__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha, bool accumulate,
-                     int mask = 0) {
-    __shared__ float sA[TK][TM + 1], sB[TK][TN + 1];
-    const int tid = threadIdx.x;
-    const int tr = tid / 16, tc = tid % 16;          // 32 x 16 threads, 2 x 4 outputs each
-    for (int m0 = 0; m0 < M; m0 += TM) {
-        for (int n0 = 0; n0 < N; n0 += TN) {
-            float acc[2][4] = {};
-            for (int k0 = 0; k0 < Kd; k0 += TK) {
-                __syncthreads();
-                // consecutive threads walk the operand's contiguous dimension (coalesced loads)
-                for (int idx = tid; idx < TK * TM; idx += NT) {
-                    const int kk = A.cs == 1 ? idx % TK : idx / TM, mm = A.cs == 1 ? idx / TK : idx % TM;
-                    sA[kk][mm] = (m0 + mm < M && k0 + kk < Kd) ? A.at(m0 + mm, k0 + kk) : 0.f;
-                }
-                for (int idx = tid; idx < TK * TN; idx += NT) {
-                    const int kk = B.rs == 1 ? idx % TK : idx / TN, nn = B.rs == 1 ? idx / TK : idx % TN;
-                    sB[kk][nn] = (n0 + nn < N && k0 + kk < Kd) ? B.at(k0 + kk, n0 + nn) : 0.f;
-                }
-                __syncthreads();
+//
+// CTA tiles of BM x BN outputs (a thread RM x RN of them), the reduction in blocks of KB: the block
+// after the current one is fetched into registers while the current one is multiplied out of shared
+// memory, so each block costs one L2 round trip hidden behind the previous block's arithmetic.
+constexpr int KB = 32;
+constexpr int SM_FLOATS = KB * (256 + 1) + KB * (64 + 1);   // the larger of the two staging shapes
+
+template <int BM, int BN, int RM, int RN>
+__device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd, float alpha,
+                           bool accumulate, int mask, float* smem) {
+    static_assert((BM / RM) * (BN / RN) == NT, "thread tile");
+    constexpr int TC = BN / RN;                                  // threads along the columns
+    constexpr int LA = BM * KB / NT, LB = BN * KB / NT;          // staged elements per thread and block
+    float* sA = smem;                                            // [KB][BM + 1]
+    float* sB = smem + KB * (BM + 1);                            // [KB][BN + 1]
+    const int tid = threadIdx.x, tr = tid / TC, tc = tid % TC;
+    // element e of the staging: consecutive threads walk the operand's contiguous dimension
+    auto a_pos = [&](int e, int& kk, int& mm) {
+        const int idx = tid + e * NT;
+        if (A.cs == 1) { kk = idx % KB; mm = idx / KB; } else { kk = idx / BM; mm = idx % BM; }
+    };
+    auto b_pos = [&](int e, int& kk, int& nn) {
+        const int idx = tid + e * NT;
+        if (B.rs == 1) { kk = idx % KB; nn = idx / KB; } else { kk = idx / BN; nn = idx % BN; }
+    };
+    for (int m0 = 0; m0 < M; m0 += BM) {
+        for (int n0 = 0; n0 < N; n0 += BN) {
+            float acc[RM][RN];
 #pragma unroll
-                for (int kk = 0; kk < TK; ++kk) {
-                    const float a0 = sA[kk][2 * tr], a1 = sA[kk][2 * tr + 1];
+            for (int i = 0; i < RM; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const float bv = sB[kk][tc + 16 * j];
-                        acc[0][j] = fmaf(a0, bv, acc[0][j]);
-                        acc[1][j] = fmaf(a1, bv, acc[1][j]);
-                    }
+                for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
+            float ra[LA], rb[LB];
+            auto fetch = [&](int k0) {
+#pragma unroll
+                for (int e = 0; e < LA; ++e) {
+                    int kk, mm;
+                    a_pos(e, kk, mm);
+                    ra[e] = (m0 + mm < M && k0 + kk < Kd) ? A.at(m0 + mm, k0 + kk) : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < LB; ++e) {
+                    int kk, nn;
+                    b_pos(e, kk, nn);
+                    rb[e] = (n0 + nn < N && k0 + kk < Kd) ? B.at(k0 + kk, n0 + nn) : 0.f;
+                }
+            };
+            fetch(0);
+            for (int k0 = 0; k0 < Kd; k0 += KB) {
+                __syncthreads();   // the previous block's products are done with the staging
+#pragma unroll
+                for (int e = 0; e < LA; ++e) {
+                    int kk, mm;
+                    a_pos(e, kk, mm);
+                    sA[kk * (BM + 1) + mm] = ra[e];
+                }
+#pragma unroll
+                for (int e = 0; e < LB; ++e) {
+                    int kk, nn;
+                    b_pos(e, kk, nn);
+                    sB[kk * (BN + 1) + nn] = rb[e];
+                }
+                __syncthreads();
+                if (k0 + KB < Kd) fetch(k0 + KB);
+                const int kend = min(KB, Kd - k0);
+                for (int kk = 0; kk < kend; ++kk) {
+                    float a[RM], bv[RN];
+#pragma unroll
+                    for (int i = 0; i < RM; ++i) a[i] = sA[kk * (BM + 1) + tr * RM + i];
+#pragma unroll
+                    for (int j = 0; j < RN; ++j) bv[j] = sB[kk * (BN + 1) + tc + TC * j];
+#pragma unroll
+                    for (int i = 0; i < RM; ++i)
+#pragma unroll
+                        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], bv[j], acc[i][j]);
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < RM; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = m0 + 2 * tr + i, c = n0 + tc + 16 * j;
+                for (int j = 0; j < RN; ++j) {
+                    const int r = m0 + tr * RM + i, c = n0 + tc + TC * j;
                     if (r < M && c < N) {
                         float v = alpha * acc[i][j];
                         if (mask == 1 && c > r) v = 0.f;
@@ -171,6 +216,17 @@ __device__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, floa
         }
     }
     __syncthreads();
+}
+
+__device__ __noinline__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha, bool accumulate,
+                     int mask = 0) {
+    __shared__ float smem[SM_FLOATS];
+    if (N > 64 && M <= 64)
+        gemm_tiles<64, 256, 4, 8>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
+    else if (M > 64 && N <= 64)
+        gemm_tiles<256, 64, 8, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
+    else
+        gemm_tiles<64, 64, 2, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
 }
 
 __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
