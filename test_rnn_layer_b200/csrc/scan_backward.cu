@@ -201,17 +201,26 @@ __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M,
                         for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], bv[j], acc[i][j]);
                 }
             }
+            // accumulating: every old value is loaded before any is stored (one memory round trip)
+            if (accumulate) {
+#pragma unroll
+                for (int i = 0; i < RM; ++i)
+#pragma unroll
+                    for (int j = 0; j < RN; ++j) {
+                        const int r = m0 + tr * RM + i, c = n0 + tc + TC * j;
+                        if (r < M && c < N)
+                            acc[i][j] = (mask == 1 && c > r ? 0.f : alpha * acc[i][j]) + C[(long long)r * ldc + c];
+                        else
+                            acc[i][j] = 0.f;
+                    }
+            }
 #pragma unroll
             for (int i = 0; i < RM; ++i)
 #pragma unroll
                 for (int j = 0; j < RN; ++j) {
                     const int r = m0 + tr * RM + i, c = n0 + tc + TC * j;
-                    if (r < M && c < N) {
-                        float v = alpha * acc[i][j];
-                        if (mask == 1 && c > r) v = 0.f;
-                        float* dst = C + (long long)r * ldc + c;
-                        *dst = accumulate ? *dst + v : v;
-                    }
+                    if (r < M && c < N)
+                        C[(long long)r * ldc + c] = accumulate ? acc[i][j] : (mask == 1 && c > r ? 0.f : alpha * acc[i][j]);
                 }
         }
     }
@@ -233,6 +242,23 @@ __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 -
     return 0.39894228040143268f * expf(-0.5f * a * a) * (2.0f - a * a);
 }
 
+#ifdef TTT_DEBUG_STAGES
+// Debug builds only: cycles between stage boundaries seen by thread 0 of CTA 0 (16 slots).
+__device__ long long* g_dbg_bwd = nullptr;
+#define STAMPB(k)                                           \
+    do {                                                    \
+        if (tid == 0 && blockIdx.x == 0) {                  \
+            const long long now_ = clock64();               \
+            stamp_acc[k] += now_ - stamp_last;              \
+            stamp_last = now_;                              \
+        }                                                   \
+    } while (0)
+#else
+#define STAMPB(k) \
+    do {          \
+    } while (0)
+#endif
+
 template <int D>
 __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     constexpr int M = 4 * D;
@@ -243,31 +269,60 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     Scratch s = carve(a.scratch + (long long)h * a.scratch_per_head, D, nck);
     const float eta = a.eta;
 
+#ifdef TTT_DEBUG_STAGES
+    long long stamp_acc[16] = {};
+    long long stamp_last = clock64();
+#endif
     auto token = [&](int c, int r) { return a.reverse ? T - 1 - (c * b + r) : c * b + r; };
     auto load_chunk = [&](int c, int n, bool with_q, bool with_dz) {
+        const float* __restrict__ gK = a.K;
+        const float* __restrict__ gV = a.V;
+        const float* __restrict__ gQ = a.Q;
+        const float* __restrict__ gdZ = a.dZ;
+        float* __restrict__ Kc = s.Kc;
+        float* __restrict__ Vc = s.Vc;
+        float* __restrict__ Qc = s.Qc;
+        float* __restrict__ dZc = s.dZc;
+#pragma unroll 4
         for (int idx = tid; idx < n * D; idx += NT) {
             const int r = idx / D, j = idx % D;
             const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
-            s.Kc[idx] = a.K[off];
-            s.Vc[idx] = a.V[off];
-            if (with_q) s.Qc[idx] = a.Q[off];
-            if (with_dz) s.dZc[idx] = a.dZ[(long long)h * a.x_hs + (long long)token(c, r) * a.x_ts + j];
+            Kc[idx] = gK[off];
+            Vc[idx] = gV[off];
+            if (with_q) Qc[idx] = gQ[off];
+            if (with_dz) dZc[idx] = gdZ[(long long)h * a.x_hs + (long long)token(c, r) * a.x_ts + j];
         }
         __syncthreads();
     };
     // A = K W1^T, G = GELU(A), D2 = -2 eta (G W2^T - V), P = D2 W2, Dl = P GELU'(A)
     auto chunk_core = [&](int n) {
         gemm(s.A, M, N_(s.Kc, D), T_(s.W1, D), n, M, D, 1.f, false);
-        for (int idx = tid; idx < n * M; idx += NT) s.G[idx] = gelu(s.A[idx]);
+        {   // (restrict views scoped to each loop: several iterations' loads may be in flight)
+            const float* __restrict__ A_ = s.A;
+            float* __restrict__ G_ = s.G;
+#pragma unroll 4
+            for (int idx = tid; idx < n * M; idx += NT) G_[idx] = gelu(A_[idx]);
+        }
         __syncthreads();
         gemm(s.D2, D, N_(s.G, M), T_(s.W2, M), n, D, M, 1.f, false);
-        for (int idx = tid; idx < n * D; idx += NT) s.D2[idx] = -2.0f * eta * (s.D2[idx] - s.Vc[idx]);
+        {
+            float* __restrict__ D2_ = s.D2;
+            const float* __restrict__ V_ = s.Vc;
+#pragma unroll 4
+            for (int idx = tid; idx < n * D; idx += NT) D2_[idx] = -2.0f * eta * (D2_[idx] - V_[idx]);
+        }
         __syncthreads();
         gemm(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
-        for (int idx = tid; idx < n * M; idx += NT) {
-            float g, gp;
-            gelu_and_prime(s.A[idx], g, gp);
-            s.Dl[idx] = s.P[idx] * gp;
+        {
+            const float* __restrict__ A_ = s.A;
+            const float* __restrict__ P_ = s.P;
+            float* __restrict__ Dl_ = s.Dl;
+#pragma unroll 4
+            for (int idx = tid; idx < n * M; idx += NT) {
+                float g, gp;
+                gelu_and_prime(A_[idx], g, gp);
+                Dl_[idx] = P_[idx] * gp;
+            }
         }
         __syncthreads();
     };
@@ -276,8 +331,20 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         gemm(s.W1, D, T_(s.Dl, M), N_(s.Kc, D), M, D, n, 1.f, true);
         gemm(s.W2, M, T_(s.D2, D), N_(s.G, M), D, M, n, 1.f, true);
     };
+    // cnt a multiple of 4, both 16-byte aligned: four 16-byte loads in flight per thread before their stores
     auto copy = [&](float* dst, const float* src, long long cnt) {
-        for (long long i = tid; i < cnt; i += NT) dst[i] = src[i];
+        const float4* __restrict__ s4 = reinterpret_cast<const float4*>(src);
+        float4* __restrict__ d4 = reinterpret_cast<float4*>(dst);
+        const long long n4 = cnt / 4;
+        for (long long i = tid; i < n4; i += 4 * NT) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i + u * NT < n4) v[u] = s4[i + u * NT];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (i + u * NT < n4) d4[i + u * NT] = v[u];
+        }
         __syncthreads();
     };
 
@@ -290,9 +357,13 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             copy(s.ck + (long long)(c / kCkpt) * 2 * MD, s.W1, MD);
             copy(s.ck + (long long)(c / kCkpt) * 2 * MD + MD, s.W2, MD);
         }
+        STAMPB(0);
         load_chunk(c, n, false, false);
+        STAMPB(1);
         chunk_core(n);
+        STAMPB(2);
         chunk_update(n);
+        STAMPB(3);
     }
 
     // ---- backward, segment by segment from the end
@@ -302,39 +373,56 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         const int c0 = sg * kCkpt, c1 = min(nch, c0 + kCkpt);
         copy(s.W1, s.ck + (long long)sg * 2 * MD, MD);
         copy(s.W2, s.ck + (long long)sg * 2 * MD + MD, MD);
+        STAMPB(4);
         for (int c = c0; c < c1; ++c) {   // chunk-start states of the segment
             copy(s.seg + (long long)(c - c0) * 2 * MD, s.W1, MD);
             copy(s.seg + (long long)(c - c0) * 2 * MD + MD, s.W2, MD);
+            STAMPB(4);
             if (c + 1 < c1) {
                 const int n = min(b, T - c * b);
                 load_chunk(c, n, false, false);
                 chunk_core(n);
                 chunk_update(n);
             }
+            STAMPB(5);
         }
         for (int c = c1 - 1; c >= c0; --c) {
             const int n = min(b, T - c * b);
             copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
             copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
+            STAMPB(6);
             load_chunk(c, n, true, true);
+            STAMPB(7);
             // forward intermediates
             chunk_core(n);
+            STAMPB(8);
             gemm(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
             gemm(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
             gemm(s.Aq, M, N_(s.Mk, BMAX), N_(s.Dl, M), n, M, n, 1.f, true);
-            for (int idx = tid; idx < n * M; idx += NT) s.Gq[idx] = gelu(s.Aq[idx]);
+            {
+                const float* __restrict__ Aq_ = s.Aq;
+                float* __restrict__ Gq_ = s.Gq;
+#pragma unroll 4
+                for (int idx = tid; idx < n * M; idx += NT) Gq_[idx] = gelu(Aq_[idx]);
+            }
             __syncthreads();
             gemm(s.Ng, BMAX, N_(s.Gq, M), T_(s.G, M), n, n, M, 1.f, false, 1);
+            STAMPB(9);
             // output branch
             gemm(s.dGq, M, N_(s.dZc, D), N_(s.W2, M), n, M, D, 1.f, false);                 // dZ W2
             gemm(s.dNg, BMAX, N_(s.dZc, D), T_(s.D2, D), n, n, D, 1.f, false, 1);            // tril(dZ D2^T)
             gemm(s.dD2, D, T_(s.Ng, BMAX), N_(s.dZc, D), n, D, n, 1.f, false);               // Ng^T dZ
             gemm(s.dGq, M, N_(s.dNg, BMAX), N_(s.G, M), n, M, n, 1.f, true);                 // + dNg G
             gemm(s.dG, M, T_(s.dNg, BMAX), N_(s.Gq, M), n, M, n, 1.f, false);                // dNg^T Gq
-            for (int idx = tid; idx < n * M; idx += NT) {                                    // dAq (in dGq)
-                float g, gp;
-                gelu_and_prime(s.Aq[idx], g, gp);
-                s.dGq[idx] *= gp;
+            {                                                                                // dAq (in dGq)
+                const float* __restrict__ Aq_ = s.Aq;
+                float* __restrict__ dGq_ = s.dGq;
+#pragma unroll 4
+                for (int idx = tid; idx < n * M; idx += NT) {
+                    float g, gp;
+                    gelu_and_prime(Aq_[idx], g, gp);
+                    dGq_[idx] *= gp;
+                }
             }
             __syncthreads();
             gemm(s.dQc, D, N_(s.dGq, M), N_(s.W1, D), n, D, M, 1.f, false);                 // dAq W1
@@ -342,48 +430,85 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             gemm(s.dDl, M, T_(s.Mk, BMAX), N_(s.dGq, M), n, M, n, 1.f, false);               // Mk^T dAq
             gemm(s.dQc, D, N_(s.dMk, BMAX), N_(s.Kc, D), n, D, n, 1.f, true);                // + dMk K
             gemm(s.dKc, D, T_(s.dMk, BMAX), N_(s.Qc, D), n, D, n, 1.f, false);               // dMk^T Q
+            STAMPB(10);
             // the chunk-end state gradient
             gemm(s.dDl, M, N_(s.Kc, D), T_(s.dW1, D), n, M, D, 1.f, true);                  // + K dW1'^T
             gemm(s.dKc, D, N_(s.Dl, M), N_(s.dW1, D), n, D, M, 1.f, true);                  // + Dl dW1'
             gemm(s.dD2, D, N_(s.G, M), T_(s.dW2, M), n, D, M, 1.f, true);                   // + G dW2'^T
             gemm(s.dG, M, N_(s.D2, D), N_(s.dW2, M), n, M, D, 1.f, true);                   // + D2 dW2'
             // dP (in dDl), dA
-            for (int idx = tid; idx < n * M; idx += NT) {
-                float g, gp;
-                gelu_and_prime(s.A[idx], g, gp);
-                const float ddl = s.dDl[idx];
-                s.dA[idx] = ddl * s.P[idx] * gelu_pp(s.A[idx]);
-                s.dDl[idx] = ddl * gp;
+            {
+                const float* __restrict__ A_ = s.A;
+                const float* __restrict__ P_ = s.P;
+                float* __restrict__ dDl_ = s.dDl;
+                float* __restrict__ dA_ = s.dA;
+#pragma unroll 4
+                for (int idx = tid; idx < n * M; idx += NT) {
+                    float g, gp;
+                    const float av = A_[idx];
+                    gelu_and_prime(av, g, gp);
+                    const float ddl = dDl_[idx];
+                    dA_[idx] = ddl * P_[idx] * gelu_pp(av);
+                    dDl_[idx] = ddl * gp;
+                }
             }
             __syncthreads();
             gemm(s.dD2, D, N_(s.dDl, M), T_(s.W2, M), n, D, M, 1.f, true);                  // + dP W2^T
-            for (int idx = tid; idx < n * D; idx += NT) s.dD2[idx] *= -2.0f * eta;            // dE (in dD2)
+            {                                                                                // dE (in dD2)
+                float* __restrict__ dD2_ = s.dD2;
+#pragma unroll 4
+                for (int idx = tid; idx < n * D; idx += NT) dD2_[idx] *= -2.0f * eta;
+            }
             __syncthreads();
             gemm(s.dG, M, N_(s.dD2, D), N_(s.W2, M), n, M, D, 1.f, true);                   // + dE W2
-            for (int idx = tid; idx < n * M; idx += NT) {                                    // dA += dG GELU'(A)
-                float g, gp;
-                gelu_and_prime(s.A[idx], g, gp);
-                s.dA[idx] += s.dG[idx] * gp;
+            {                                                                                // dA += dG GELU'(A)
+                const float* __restrict__ A_ = s.A;
+                const float* __restrict__ dG_ = s.dG;
+                float* __restrict__ dA_ = s.dA;
+#pragma unroll 4
+                for (int idx = tid; idx < n * M; idx += NT) {
+                    float g, gp;
+                    gelu_and_prime(A_[idx], g, gp);
+                    dA_[idx] += dG_[idx] * gp;
+                }
             }
             __syncthreads();
             gemm(s.dKc, D, N_(s.dA, M), N_(s.W1, D), n, D, M, 1.f, true);                   // + dA W1
+            STAMPB(11);
             // the chunk-start state gradient (accumulated onto the chunk-end one)
             gemm(s.dW2, M, T_(s.dZc, D), N_(s.Gq, M), D, M, n, 1.f, true);                  // dZ^T Gq
             gemm(s.dW2, M, T_(s.D2, D), N_(s.dDl, M), D, M, n, 1.f, true);                  // D2^T dP
             gemm(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, 1.f, true);                   // dE^T G
             gemm(s.dW1, D, T_(s.dGq, M), N_(s.Qc, D), M, D, n, 1.f, true);                  // dAq^T Q
             gemm(s.dW1, D, T_(s.dA, M), N_(s.Kc, D), M, D, n, 1.f, true);                   // dA^T K
+            STAMPB(12);
             // dQ, dK, dV of the chunk's tokens
-            for (int idx = tid; idx < n * D; idx += NT) {
-                const int r = idx / D, j = idx % D;
-                const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
-                a.dQ[off] = s.dQc[idx];
-                a.dK[off] = s.dKc[idx];
-                a.dV[off] = -s.dD2[idx];   // dV = -dE
+            {
+                const float* __restrict__ dQc_ = s.dQc;
+                const float* __restrict__ dKc_ = s.dKc;
+                const float* __restrict__ dD2_ = s.dD2;
+                float* __restrict__ gdQ = a.dQ;
+                float* __restrict__ gdK = a.dK;
+                float* __restrict__ gdV = a.dV;
+#pragma unroll 4
+                for (int idx = tid; idx < n * D; idx += NT) {
+                    const int r = idx / D, j = idx % D;
+                    const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
+                    gdQ[off] = dQc_[idx];
+                    gdK[off] = dKc_[idx];
+                    gdV[off] = -dD2_[idx];   // dV = -dE
+                }
             }
             __syncthreads();
+            STAMPB(13);
         }
     }
+#ifdef TTT_DEBUG_STAGES
+    if (tid == 0 && blockIdx.x == 0 && g_dbg_bwd) {
+        for (int k = 0; k < 16; ++k) g_dbg_bwd[k] = stamp_acc[k];
+        g_dbg_bwd[15] = nch;
+    }
+#endif
     for (long long i = tid; i < MD; i += NT) {
         a.dW1[(long long)h * MD + i] += s.dW1[i];
         a.dW2[(long long)h * MD + i] += s.dW2[i];
@@ -391,6 +516,12 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
 }
 
 }  // namespace
+
+#ifdef TTT_DEBUG_STAGES
+extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump_bwd(long long* p) {
+    return (int)cudaMemcpyToSymbol(g_dbg_bwd, &p, sizeof(p));
+}
+#endif
 
 long long scan_backward_scratch_floats(int d, int b, int T) { return scratch_floats_for(d, b, T); }
 
