@@ -188,8 +188,10 @@ __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M,
                 }
                 __syncthreads();
                 if (k0 + KB < Kd) fetch(k0 + KB);
-                const int kend = min(KB, Kd - k0);
-                for (int kk = 0; kk < kend; ++kk) {
+                // the whole block every time (past Kd the staged values are zero): a fixed trip count the
+                // compiler unrolls, so the shared loads of later steps are issued ahead of their FMAs
+#pragma unroll 8
+                for (int kk = 0; kk < KB; ++kk) {
                     float a[RM], bv[RN];
 #pragma unroll
                     for (int i = 0; i < RM; ++i) a[i] = sA[kk * (BM + 1) + tr * RM + i];
