@@ -19,9 +19,10 @@
 //   dE = -2 eta dD2,  dV = -dE,  dG += dE W2,  dA += dG * GELU'(A),  dK += dA W1,
 //   dW1 = dW1' + dAq^T Q + dA^T K,  dW2 = dW2' + dZ^T Gq + D2^T dP + dE^T G.
 // The chunk-start states come from checkpoints: the kernel first walks the
-// sequence forward (state updates only) keeping the state every kCkpt chunks,
-// then, segment by segment from the end, rebuilds the segment's chunk-start
-// states from its checkpoint and runs the chunks' backward steps in reverse.
+// sequence forward (state updates only) keeping the state every kCkpt chunks
+// (by default every chunk), then, from the end, runs the chunks' backward steps
+// in reverse, each segment's chunk-start states rebuilt from its checkpoint
+// first when kCkpt > 1.
 //
 // One CTA of 512 threads per head; the matrices of a chunk live in a per-head
 // scratch area in global memory (it stays in L2); every product is a block
@@ -34,7 +35,12 @@ namespace {
 
 constexpr int NT = 512;          // threads per CTA
 constexpr int BMAX = 64;         // largest chunk
-constexpr int kCkpt = 32;        // chunks between two checkpoints
+// Chunks between two checkpoints.  1: every chunk-start state is kept (128 KB per chunk and head at
+// d = 64), so nothing is rebuilt; larger spacings trade that memory for a rebuild of each segment.
+#ifndef TTT_BWD_CKPT
+#define TTT_BWD_CKPT 1
+#endif
+constexpr int kCkpt = TTT_BWD_CKPT;
 
 struct BwdArgs {
     const float* Q;
@@ -373,6 +379,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     __syncthreads();
     for (int sg = nck - 1; sg >= 0; --sg) {
         const int c0 = sg * kCkpt, c1 = min(nch, c0 + kCkpt);
+        if constexpr (kCkpt > 1) {
         copy(s.W1, s.ck + (long long)sg * 2 * MD, MD);
         copy(s.W2, s.ck + (long long)sg * 2 * MD + MD, MD);
         STAMPB(4);
@@ -388,10 +395,16 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             }
             STAMPB(5);
         }
+        }
         for (int c = c1 - 1; c >= c0; --c) {
             const int n = min(b, T - c * b);
-            copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
-            copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
+            if constexpr (kCkpt > 1) {
+                copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
+                copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
+            } else {   // every chunk-start state is a checkpoint: read it in place
+                s.W1 = s.ck + (long long)c * 2 * MD;
+                s.W2 = s.W1 + MD;
+            }
             STAMPB(6);
             load_chunk(c, n, true, true);
             STAMPB(7);
