@@ -23,7 +23,8 @@ CASES = [
                D=128),
     S.Workload("bwd-full-f32-b8", H=2, d=16, T=45, b=8, dirs="bidir", dtype="f32", per_head=False, eta=0.1, D=32),
     S.Workload("bwd-head-T1", H=2, d=64, T=1, b=16, dirs="bidir", dtype="bf16", per_head=True, eta=0.05),
-    # several 32-chunk checkpoint segments: 128 chunks of 16, and 65 chunks of 64 with a ragged last one
+    # long runs: 128 chunks of 16, and 65 chunks of 64 with a ragged last one (several segments when the
+    # backward is built with sparser checkpoints)
     S.Workload("bwd-head-bf16-b16-128chunks", H=2, d=64, T=2048, b=16, dirs="bidir", dtype="bf16", per_head=True,
                eta=0.05),
     S.Workload("bwd-full-bf16-b64-65chunks", H=4, d=64, T=4131, b=64, dirs="bidir", dtype="bf16", per_head=False,
