@@ -442,6 +442,17 @@ TTT_API int ttt_debug_pipe_segments(int nchunks, int* out, int max_segments);
  */
 TTT_API ttt_status ttt_debug_set_block_front(int percent);
 
+/*
+ * Tests and benchmarks only (process-wide): how many CTAs of one cluster walk
+ * one head in the backward scan of ttt_mlp_backward.  0 (the default): two
+ * while twice the head count fits on the GPU's SMs, else one; 1 or 2 forces
+ * that number.  The products' output tiles and the elementwise passes are
+ * dealt out over the cluster; every value is computed by the same operations
+ * in the same order either way, so this changes timing, never results.
+ * TTT_ERR_INVALID_ARG for any other value.
+ */
+TTT_API ttt_status ttt_debug_set_backward_ctas(int ctas);
+
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 TTT_API const char* ttt_last_error(void);
 

@@ -1343,6 +1343,12 @@ ttt_status ttt_debug_set_block_front(int percent) {
     return TTT_OK;
 }
 
+ttt_status ttt_debug_set_backward_ctas(int ctas) {
+    if (ctas < 0 || ctas > 2) return fail(TTT_ERR_INVALID_ARG, "ctas must be 0 (automatic), 1 or 2");
+    set_scan_backward_ctas(ctas);
+    return TTT_OK;
+}
+
 ttt_status ttt_debug_inject_wait_timeout(int enable) {
     g_inject_timeout.store(enable ? 1 : 0);
     return TTT_OK;

@@ -155,6 +155,8 @@ cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V,
                                  const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
                                  const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
                                  float* scratch, int T, int H, int d, int b, int reverse, float eta, cudaStream_t s);
+// CTAs per head of launch_scan_backward (process-wide): 0 automatic, 1 or 2.
+void set_scan_backward_ctas(int ctas);
 // Gate backward: dz = tanh(alpha) g, dalpha += (1 - tanh^2 alpha) sum_t g z (per channel).
 cudaError_t launch_gate_backward(const float* g, const float* z, const float* alpha, float* dz, float* dalpha, int T,
                                  int H, int d, int per_head, cudaStream_t s);

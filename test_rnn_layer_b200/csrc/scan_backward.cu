@@ -24,9 +24,15 @@
 // in reverse, each segment's chunk-start states rebuilt from its checkpoint
 // first when kCkpt > 1.
 //
-// One CTA of 512 threads per head; the matrices of a chunk live in a per-head
-// scratch area in global memory (it stays in L2); every product is a block
-// GEMM tiled through shared memory.
+// One cluster of CS CTAs of 512 threads per head (CS = 1 or 2); the matrices of
+// a chunk live in a per-head scratch area in global memory (it stays in L2);
+// every product is a block GEMM tiled through shared memory whose output tiles
+// are dealt out over the cluster's CTAs, and every elementwise pass strides over
+// all of the cluster's threads, with a cluster barrier (release / acquire) where
+// the CTAs' results meet.  Each output element is computed by the same sequence
+// of operations whatever CS is, so the results do not depend on it.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -118,6 +124,16 @@ __device__ Scratch carve(float* base, int d, int nck) {
     return s;
 }
 
+// The barrier between the stages of a head: the CTA's own with one CTA per head, else the cluster's
+// (release / acquire at cluster scope, so the other CTAs' global-memory results are visible after it).
+// Every thread of every CTA of the cluster reaches the same sequence of these.
+__device__ __forceinline__ void head_sync(int ncta) {
+    if (ncta == 1)
+        __syncthreads();
+    else
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // A matrix operand: element (r, c) of op(X) at X[r * rs + c * cs].
 struct Mat {
     const float* p;
@@ -139,7 +155,7 @@ constexpr int SM_FLOATS = KB * (256 + 1) + KB * (64 + 1);   // the larger of the
 
 template <int BM, int BN, int RM, int RN>
 __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd, float alpha,
-                           bool accumulate, int mask, float* smem) {
+                           bool accumulate, int mask, int rank, int ncta, float* smem) {
     static_assert((BM / RM) * (BN / RN) == NT, "thread tile");
     constexpr int TC = BN / RN;                                  // threads along the columns
     constexpr int LA = BM * KB / NT, LB = BN * KB / NT;          // staged elements per thread and block
@@ -155,8 +171,10 @@ __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M,
         const int idx = tid + e * NT;
         if (B.rs == 1) { kk = idx % KB; nn = idx / KB; } else { kk = idx / BN; nn = idx % BN; }
     };
+    int tile = 0;
     for (int m0 = 0; m0 < M; m0 += BM) {
         for (int n0 = 0; n0 < N; n0 += BN) {
+            if (tile++ % ncta != rank) continue;   // another CTA of the cluster owns this tile
             float acc[RM][RN];
 #pragma unroll
             for (int i = 0; i < RM; ++i)
@@ -232,18 +250,29 @@ __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M,
                 }
         }
     }
-    __syncthreads();
+    head_sync(ncta);
 }
 
-__device__ __noinline__ void gemm(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha, bool accumulate,
-                     int mask = 0) {
+// Tile shapes: one CTA tile covers a whole b x m (or m x d) product when the head has one CTA, half of
+// it per CTA with two; the b x b and b x d products take 64 x 64 tiles (32 x 64 with two CTAs).
+__device__ __noinline__ void gemm_cs(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha,
+                                     bool accumulate, int mask, int rank, int ncta) {
     __shared__ float smem[SM_FLOATS];
-    if (N > 64 && M <= 64)
-        gemm_tiles<64, 256, 4, 8>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
-    else if (M > 64 && N <= 64)
-        gemm_tiles<256, 64, 8, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
-    else
-        gemm_tiles<64, 64, 2, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, smem);
+    if (ncta == 1) {
+        if (N > 64 && M <= 64)
+            gemm_tiles<64, 256, 4, 8>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+        else if (M > 64 && N <= 64)
+            gemm_tiles<256, 64, 8, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+        else
+            gemm_tiles<64, 64, 2, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+    } else {
+        if (N > 64 && M <= 64)
+            gemm_tiles<64, 128, 4, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+        else if (M > 64 && N <= 64)
+            gemm_tiles<128, 64, 4, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+        else
+            gemm_tiles<32, 64, 2, 2>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+    }
 }
 
 __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
@@ -267,11 +296,18 @@ __device__ long long* g_dbg_bwd = nullptr;
     } while (0)
 #endif
 
-template <int D>
+template <int D, int CS>
 __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     constexpr int M = 4 * D;
     constexpr long long MD = (long long)M * D;
-    const int h = blockIdx.x, tid = threadIdx.x;
+    constexpr int GNT = CS * NT;   // threads of the head's cluster
+    int rank = 0;
+    if constexpr (CS > 1) asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    const int h = blockIdx.x / CS, tid = threadIdx.x, gtid = rank * NT + tid;
+    // a product of the head, its output tiles dealt out over the cluster (ends with the head's barrier)
+    auto gemm = [&](float* C, int ldc, Mat A_, Mat B_, int M_, int N_, int Kd, float alpha, bool accumulate,
+                    int mask = 0) { gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, mask, rank, CS); };
+    auto sync = [&]() { head_sync(CS); };
     const int T = a.T, b = a.b;
     const int nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
     Scratch s = carve(a.scratch + (long long)h * a.scratch_per_head, D, nck);
@@ -292,7 +328,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         float* __restrict__ Qc = s.Qc;
         float* __restrict__ dZc = s.dZc;
 #pragma unroll 4
-        for (int idx = tid; idx < n * D; idx += NT) {
+        for (int idx = gtid; idx < n * D; idx += GNT) {
             const int r = idx / D, j = idx % D;
             const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
             Kc[idx] = gK[off];
@@ -300,7 +336,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             if (with_q) Qc[idx] = gQ[off];
             if (with_dz) dZc[idx] = gdZ[(long long)h * a.x_hs + (long long)token(c, r) * a.x_ts + j];
         }
-        __syncthreads();
+        sync();
     };
     // A = K W1^T, G = GELU(A), D2 = -2 eta (G W2^T - V), P = D2 W2, Dl = P GELU'(A)
     auto chunk_core = [&](int n) {
@@ -309,30 +345,30 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             const float* __restrict__ A_ = s.A;
             float* __restrict__ G_ = s.G;
 #pragma unroll 4
-            for (int idx = tid; idx < n * M; idx += NT) G_[idx] = gelu(A_[idx]);
+            for (int idx = gtid; idx < n * M; idx += GNT) G_[idx] = gelu(A_[idx]);
         }
-        __syncthreads();
+        sync();
         gemm(s.D2, D, N_(s.G, M), T_(s.W2, M), n, D, M, 1.f, false);
         {
             float* __restrict__ D2_ = s.D2;
             const float* __restrict__ V_ = s.Vc;
 #pragma unroll 4
-            for (int idx = tid; idx < n * D; idx += NT) D2_[idx] = -2.0f * eta * (D2_[idx] - V_[idx]);
+            for (int idx = gtid; idx < n * D; idx += GNT) D2_[idx] = -2.0f * eta * (D2_[idx] - V_[idx]);
         }
-        __syncthreads();
+        sync();
         gemm(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
         {
             const float* __restrict__ A_ = s.A;
             const float* __restrict__ P_ = s.P;
             float* __restrict__ Dl_ = s.Dl;
 #pragma unroll 4
-            for (int idx = tid; idx < n * M; idx += NT) {
+            for (int idx = gtid; idx < n * M; idx += GNT) {
                 float g, gp;
                 gelu_and_prime(A_[idx], g, gp);
                 Dl_[idx] = P_[idx] * gp;
             }
         }
-        __syncthreads();
+        sync();
     };
     // W1 += Dl^T K, W2 += D2^T G
     auto chunk_update = [&](int n) {
@@ -344,16 +380,16 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         const float4* __restrict__ s4 = reinterpret_cast<const float4*>(src);
         float4* __restrict__ d4 = reinterpret_cast<float4*>(dst);
         const long long n4 = cnt / 4;
-        for (long long i = tid; i < n4; i += 4 * NT) {
+        for (long long i = gtid; i < n4; i += 4 * GNT) {
             float4 v[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (i + u * NT < n4) v[u] = s4[i + u * NT];
+                if (i + u * GNT < n4) v[u] = s4[i + u * GNT];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (i + u * NT < n4) d4[i + u * NT] = v[u];
+                if (i + u * GNT < n4) d4[i + u * GNT] = v[u];
         }
-        __syncthreads();
+        sync();
     };
 
     // ---- forward walk: checkpoints of the state every kCkpt chunks
@@ -375,8 +411,8 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     }
 
     // ---- backward, segment by segment from the end
-    for (long long i = tid; i < MD; i += NT) { s.dW1[i] = 0.f; s.dW2[i] = 0.f; }
-    __syncthreads();
+    for (long long i = gtid; i < MD; i += GNT) { s.dW1[i] = 0.f; s.dW2[i] = 0.f; }
+    sync();
     for (int sg = nck - 1; sg >= 0; --sg) {
         const int c0 = sg * kCkpt, c1 = min(nch, c0 + kCkpt);
         if constexpr (kCkpt > 1) {
@@ -418,9 +454,9 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                 const float* __restrict__ Aq_ = s.Aq;
                 float* __restrict__ Gq_ = s.Gq;
 #pragma unroll 4
-                for (int idx = tid; idx < n * M; idx += NT) Gq_[idx] = gelu(Aq_[idx]);
+                for (int idx = gtid; idx < n * M; idx += GNT) Gq_[idx] = gelu(Aq_[idx]);
             }
-            __syncthreads();
+            sync();
             gemm(s.Ng, BMAX, N_(s.Gq, M), T_(s.G, M), n, n, M, 1.f, false, 1);
             STAMPB(9);
             // output branch
@@ -433,13 +469,13 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                 const float* __restrict__ Aq_ = s.Aq;
                 float* __restrict__ dGq_ = s.dGq;
 #pragma unroll 4
-                for (int idx = tid; idx < n * M; idx += NT) {
+                for (int idx = gtid; idx < n * M; idx += GNT) {
                     float g, gp;
                     gelu_and_prime(Aq_[idx], g, gp);
                     dGq_[idx] *= gp;
                 }
             }
-            __syncthreads();
+            sync();
             gemm(s.dQc, D, N_(s.dGq, M), N_(s.W1, D), n, D, M, 1.f, false);                 // dAq W1
             gemm(s.dMk, BMAX, N_(s.dGq, M), T_(s.Dl, M), n, n, M, 1.f, false, 1);            // tril(dAq Dl^T)
             gemm(s.dDl, M, T_(s.Mk, BMAX), N_(s.dGq, M), n, M, n, 1.f, false);               // Mk^T dAq
@@ -458,7 +494,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                 float* __restrict__ dDl_ = s.dDl;
                 float* __restrict__ dA_ = s.dA;
 #pragma unroll 4
-                for (int idx = tid; idx < n * M; idx += NT) {
+                for (int idx = gtid; idx < n * M; idx += GNT) {
                     float g, gp;
                     const float av = A_[idx];
                     gelu_and_prime(av, g, gp);
@@ -467,27 +503,27 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                     dDl_[idx] = ddl * gp;
                 }
             }
-            __syncthreads();
+            sync();
             gemm(s.dD2, D, N_(s.dDl, M), T_(s.W2, M), n, D, M, 1.f, true);                  // + dP W2^T
             {                                                                                // dE (in dD2)
                 float* __restrict__ dD2_ = s.dD2;
 #pragma unroll 4
-                for (int idx = tid; idx < n * D; idx += NT) dD2_[idx] *= -2.0f * eta;
+                for (int idx = gtid; idx < n * D; idx += GNT) dD2_[idx] *= -2.0f * eta;
             }
-            __syncthreads();
+            sync();
             gemm(s.dG, M, N_(s.dD2, D), N_(s.W2, M), n, M, D, 1.f, true);                   // + dE W2
             {                                                                                // dA += dG GELU'(A)
                 const float* __restrict__ A_ = s.A;
                 const float* __restrict__ dG_ = s.dG;
                 float* __restrict__ dA_ = s.dA;
 #pragma unroll 4
-                for (int idx = tid; idx < n * M; idx += NT) {
+                for (int idx = gtid; idx < n * M; idx += GNT) {
                     float g, gp;
                     gelu_and_prime(A_[idx], g, gp);
                     dA_[idx] += dG_[idx] * gp;
                 }
             }
-            __syncthreads();
+            sync();
             gemm(s.dKc, D, N_(s.dA, M), N_(s.W1, D), n, D, M, 1.f, true);                   // + dA W1
             STAMPB(11);
             // the chunk-start state gradient (accumulated onto the chunk-end one)
@@ -506,7 +542,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                 float* __restrict__ gdK = a.dK;
                 float* __restrict__ gdV = a.dV;
 #pragma unroll 4
-                for (int idx = tid; idx < n * D; idx += NT) {
+                for (int idx = gtid; idx < n * D; idx += GNT) {
                     const int r = idx / D, j = idx % D;
                     const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
                     gdQ[off] = dQc_[idx];
@@ -514,7 +550,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                     gdV[off] = -dD2_[idx];   // dV = -dE
                 }
             }
-            __syncthreads();
+            sync();
             STAMPB(13);
         }
     }
@@ -524,7 +560,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         g_dbg_bwd[15] = nch;
     }
 #endif
-    for (long long i = tid; i < MD; i += NT) {
+    for (long long i = gtid; i < MD; i += GNT) {
         a.dW1[(long long)h * MD + i] += s.dW1[i];
         a.dW2[(long long)h * MD + i] += s.dW2[i];
     }
@@ -540,6 +576,11 @@ extern "C" __attribute__((visibility("default"))) int ttt_debug_set_dump_bwd(lon
 
 long long scan_backward_scratch_floats(int d, int b, int T) { return scratch_floats_for(d, b, T); }
 
+// CTAs per head of the backward scan: 0 picks (2 while 2 H CTAs fit on the GPU's SMs, else 1); 1 or 2 forces.
+static std::atomic<int> g_bwd_cluster{0};
+
+void set_scan_backward_ctas(int ctas) { g_bwd_cluster.store(ctas); }
+
 cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V, long long qkv_hs, long long qkv_ts,
                                  const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
                                  const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
@@ -553,13 +594,41 @@ cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V,
     a.dQ = dQ; a.dK = dK; a.dV = dV; a.dW1 = dW1; a.dW2 = dW2;
     a.scratch = scratch; a.scratch_per_head = scratch_floats_for(d, b, T);
     a.T = T; a.H = H; a.d = d; a.b = b; a.reverse = reverse; a.eta = eta;
-    LaunchScope scope("scan_backward", s);
-    switch (d) {
-        case 16: scan_bwd_kernel<16><<<H, NT, 0, s>>>(a); break;
-        case 32: scan_bwd_kernel<32><<<H, NT, 0, s>>>(a); break;
-        case 64: scan_bwd_kernel<64><<<H, NT, 0, s>>>(a); break;
+    // two CTAs per head while the heads' pairs fit on the GPU at once, else one
+    int cs = g_bwd_cluster.load();
+    if (cs == 0) {
+        int dev = 0, sms = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        cs = 2 * H <= sms ? 2 : 1;
+    }
+    if (cs != 1 && cs != 2) return cudaErrorInvalidValue;
+    void (*kern)(BwdArgs) = nullptr;
+    switch (d * 4 + cs) {
+        case 16 * 4 + 1: kern = scan_bwd_kernel<16, 1>; break;
+        case 32 * 4 + 1: kern = scan_bwd_kernel<32, 1>; break;
+        case 64 * 4 + 1: kern = scan_bwd_kernel<64, 1>; break;
+        case 16 * 4 + 2: kern = scan_bwd_kernel<16, 2>; break;
+        case 32 * 4 + 2: kern = scan_bwd_kernel<32, 2>; break;
+        case 64 * 4 + 2: kern = scan_bwd_kernel<64, 2>; break;
         default: return cudaErrorInvalidValue;
     }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(H * cs);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope scope("scan_backward", s);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -30,7 +30,7 @@ EXPORTED = ["ttt_mlp_workspace_size", "ttt_mlp_forward", "ttt_mlp_status", "ttt_
             "ttt_mlp_backward_workspace_size", "ttt_mlp_backward", "ttt_mlp_heads_workspace_size",
             "ttt_mlp_forward_heads", "ttt_seg_attention_workspace_size", "ttt_seg_attention",
             "ttt_block_workspace_size", "ttt_block_forward", "ttt_debug_set_block_front",
-            "ttt_linear_host_io_workspace_size", "ttt_linear_forward_host"]
+            "ttt_linear_host_io_workspace_size", "ttt_linear_forward_host", "ttt_debug_set_backward_ctas"]
 
 
 class TTTError(RuntimeError):
@@ -90,6 +90,8 @@ def lib():
         L.ttt_block_forward.argtypes = [dp, i, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, f, i, vp, vp, vp, vp, sz, vp]
         L.ttt_debug_set_block_front.restype = i
         L.ttt_debug_set_block_front.argtypes = [i]
+        L.ttt_debug_set_backward_ctas.restype = i
+        L.ttt_debug_set_backward_ctas.argtypes = [i]
         L.ttt_mlp_noalloc_status.restype = i
         L.ttt_mlp_noalloc_status.argtypes = [vp]
         L.ttt_linear_workspace_size.restype = sz
@@ -295,6 +297,10 @@ def ttt_block_forward(desc, seg_len, Qa, Ka, Va, ld_qkv, Xres, X, theta_q, theta
 
 def ttt_debug_set_block_front(percent: int) -> int:
     return int(lib().ttt_debug_set_block_front(percent))
+
+
+def ttt_debug_set_backward_ctas(ctas: int) -> int:
+    return int(lib().ttt_debug_set_backward_ctas(ctas))
 
 
 def ttt_mlp_noalloc_status(stream=None) -> int:

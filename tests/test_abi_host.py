@@ -219,3 +219,6 @@ def test_attention_argument_errors_before_any_cuda_call():
     assert blk(d, X=Q) == L.TTT_ERR_INVALID_ARG and "overlap" in L.ttt_last_error()
     assert L.ttt_debug_set_block_front(101) == L.TTT_ERR_INVALID_ARG
     assert L.ttt_debug_set_block_front(-1) == L.TTT_OK
+    assert L.ttt_debug_set_backward_ctas(3) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_debug_set_backward_ctas(-1) == L.TTT_ERR_INVALID_ARG
+    assert L.ttt_debug_set_backward_ctas(0) == L.TTT_OK

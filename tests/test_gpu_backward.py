@@ -50,6 +50,30 @@ def test_backward_matches_the_oracle(w):
     assert all(v <= tol for v in errs.values()), errs
 
 
+@pytest.mark.parametrize("w", [CASES[2], CASES[7]], ids=lambda w: w.name)
+def test_backward_cluster_of_two_ctas_equals_one_cta(w):
+    # a head's backward scan on one CTA or on a cluster of two: the same operations for every value
+    inp = S.make_inputs(w, seed=3)
+    gen = torch.Generator().manual_seed(5)
+    dY = torch.randn(inp["X"].shape, generator=gen, dtype=torch.float32).cuda()
+    g = {k: v.cuda() for k, v in inp.items()}
+    outs = []
+    try:
+        for ctas in (1, 2):
+            L.check(L.ttt_debug_set_backward_ctas(ctas), "ttt_debug_set_backward_ctas")
+            outs.append(L.layer_backward(g["X"], g["theta_q"], g["theta_k"], g["theta_v"], g["W1_0"], g["W2_0"],
+                                         w.eta_eff, w.b, w.dirs, g["alpha_f"], g["alpha_r"], dY,
+                                         per_head=w.per_head))
+            torch.cuda.synchronize()
+    finally:
+        L.ttt_debug_set_backward_ctas(0)
+    for k in ("dX", "dtheta_q", "dtheta_k", "dtheta_v", "dW1_0", "dW2_0"):
+        assert torch.equal(outs[0][k], outs[1][k]), k
+    # dalpha sums over tokens with atomic adds, in an order that varies from run to run
+    for k in ("dalpha_f", "dalpha_r"):
+        assert torch.allclose(outs[0][k], outs[1][k], rtol=1e-5, atol=1e-5 * float(outs[0][k].abs().max())), k
+
+
 def test_backward_rejects_chunks_above_64():
     w = S.SCALE18S.with_(T=300, b=100, H=2)
     desc = L.make_desc(w.T, w.H, w.d, w.per_head, True)
