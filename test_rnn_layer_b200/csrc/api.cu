@@ -1093,7 +1093,7 @@ ttt_status ttt_mlp_backward(const ttt_mlp_desc* desc, const void* X, const void*
         if (st != TTT_OK) return st;
         CUDA_TRY(launch_scan_backward(U[0], U[1], U[2], qkv_hs, qkv_ts, dz, qkv_hs, qkv_ts, W1_0, W2_0, dU[0], dU[1],
                                       dU[2], dW1_0, dW2_0, reinterpret_cast<float*>(ws + B.scratch), q.T, q.H, q.d, b,
-                                      reverse ? 1 : 0, eta, s));
+                                      reverse ? 1 : 0, eta, x_bf16 ? 0 : 1, s));
         if (tc_grads) {   // the gate's x path keeps G; the projections add theta's share
             st = projection_grads_tc(q, dU, th, X, on_xp ? delta : nullptr, U, G, dth, status, s);
             if (st != TTT_OK) return st;

@@ -147,14 +147,17 @@ ttt_status forward_single_stream(const ttt_mlp_desc* desc, const void* X, const 
                                  float* W1_T, float* W2_T, void* workspace, size_t workspace_bytes,
                                  ttt_stream_t stream);
 
-// Backward pass of one direction of the scan (fp32, b <= 64, d = 16/32/64):
+// Backward pass of one direction of the scan (fp32 state, b <= 64, d = 16/32/64):
 // dQ, dK, dV (qkv layout) from dZ (X layout); dW1, dW2 [H, m, d] / [H, d, m]
 // accumulated; scratch of H * scan_backward_scratch_floats(d, b, T) floats.
+// split_tf32: products on tf32 tensor cores in the split form (fp32-accurate);
+// 0: single tf32 products (the precision of the bf16 layer's forward products).
 long long scan_backward_scratch_floats(int d, int b, int T);
 cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V, long long qkv_hs, long long qkv_ts,
                                  const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
                                  const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
-                                 float* scratch, int T, int H, int d, int b, int reverse, float eta, cudaStream_t s);
+                                 float* scratch, int T, int H, int d, int b, int reverse, float eta, int split_tf32,
+                                 cudaStream_t s);
 // CTAs per head of launch_scan_backward (process-wide): 0 automatic, 1 or 2.
 void set_scan_backward_ctas(int ctas);
 // Gate backward: dz = tanh(alpha) g, dalpha += (1 - tanh^2 alpha) sum_t g z (per channel).

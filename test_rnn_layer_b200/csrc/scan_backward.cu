@@ -66,6 +66,7 @@ struct BwdArgs {
     long long scratch_per_head;
     int T, H, d, b, reverse;
     float eta;
+    int split_tf32;              // products in the split (fp32-accurate) form; else single tf32
 };
 
 // Per-head scratch layout (floats).
@@ -138,116 +139,195 @@ __device__ __forceinline__ void head_sync(int ncta) {
 struct Mat {
     const float* p;
     int rs, cs;
-    __device__ float at(int r, int c) const { return p[(long long)r * rs + (long long)c * cs]; }
 };
 __device__ __forceinline__ Mat N_(const float* p, int ld) { return Mat{p, ld, 1}; }   // row-major as is
 __device__ __forceinline__ Mat T_(const float* p, int ld) { return Mat{p, 1, ld}; }   // transposed view
 
 // C[M x N] (+)= alpha * A[M x Kd] B[Kd x N], C row-major with leading dimension ldc.
 // mask: 0 none, 1 keep C[r][c] only for c <= r (lower triangle incl. diagonal).
-// All threads of the CTA call it; it ends with a barrier.
+// All threads of the head's CTAs call it; it ends with the head's barrier.
 //
-// CTA tiles of BM x BN outputs (a thread RM x RN of them), the reduction in blocks of KB: the block
-// after the current one is fetched into registers while the current one is multiplied out of shared
-// memory, so each block costs one L2 round trip hidden behind the previous block's arithmetic.
+// The products are small (at most 64 x 256 outputs, a reduction of at most 256) and each waits on the
+// previous one, so what sets their time is the number of dependent memory round trips, not arithmetic:
+// the operands' reduction blocks (KB deep) are copied into shared memory by cp.async (16-byte copies
+// that bypass L1 and zero-fill past the matrices' edges), NSTAGE blocks in flight at once, and an
+// accumulating product loads its old C before the reduction starts, so a product with a reduction of
+// at most 96 costs one round trip for its inputs and one for its stores.
+//
+// Arithmetic: mma.sync m16n8k8 on tf32 operands in the split form ("3xTF32"): each operand
+// x = hi + lo with hi = tf32(x) and lo = tf32(x - hi), and a b is taken as a_hi b_hi + a_hi b_lo +
+// a_lo b_hi, the small terms first; the dropped a_lo b_lo and the rounding of lo leave about 2^-21 of
+// |a b|, fp32 accuracy for these sums.  16 warps in a grid of WM x WN warp tiles.  Staging: an operand
+// whose reduction index is contiguous in memory is kept as [row][KB + 4] in shared memory, otherwise as
+// [k][rows + 8]; either way the fragment loads (lanes g = lane / 4 along rows, t = lane % 4 along k)
+// fall in 32 distinct banks and the 16-byte copies run along the contiguous index.
 constexpr int KB = 32;
-constexpr int SM_FLOATS = KB * (256 + 1) + KB * (64 + 1);   // the larger of the two staging shapes
+constexpr int NSTAGE = 4;
+constexpr int PADK = 4, PADR = 8;
+__host__ __device__ constexpr int stage_floats(int rows) {
+    return rows * (KB + PADK) > KB * (rows + PADR) ? rows * (KB + PADK) : KB * (rows + PADR);
+}
+// dynamic shared memory of the kernel: the largest tile pair of the head's CTA count, NSTAGE times
+__host__ __device__ constexpr int gemm_smem_floats(int ncta) {
+    return NSTAGE * (ncta == 1 ? stage_floats(64) + stage_floats(256) : stage_floats(64) + stage_floats(128));
+}
 
-template <int BM, int BN, int RM, int RN>
-__device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd, float alpha,
-                           bool accumulate, int mask, int rank, int ncta, float* smem) {
-    static_assert((BM / RM) * (BN / RN) == NT, "thread tile");
-    constexpr int TC = BN / RN;                                  // threads along the columns
-    constexpr int LA = BM * KB / NT, LB = BN * KB / NT;          // staged elements per thread and block
-    float* sA = smem;                                            // [KB][BM + 1]
-    float* sB = smem + KB * (BM + 1);                            // [KB][BN + 1]
-    const int tid = threadIdx.x, tr = tid / TC, tc = tid % TC;
-    // element e of the staging: consecutive threads walk the operand's contiguous dimension
-    auto a_pos = [&](int e, int& kk, int& mm) {
-        const int idx = tid + e * NT;
-        if (A.cs == 1) { kk = idx % KB; mm = idx / KB; } else { kk = idx / BM; mm = idx % BM; }
+__device__ __forceinline__ void cp_async16(float* dst, const float* src, int bytes) {
+    const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ int clamp4(int x) { return x < 0 ? 0 : (x > 4 ? 4 : x); }
+
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+    const float r = x - __uint_as_float(hi);   // exact: x and hi agree in their leading bits
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(lo) : "f"(r));
+}
+
+// SPLIT: hi and lo as above; else hi = tf32(x) alone (lo unused)
+template <bool SPLIT>
+__device__ __forceinline__ void to_tf32(float x, uint32_t& hi, uint32_t& lo) {
+    if constexpr (SPLIT) {
+        split_tf32(x, hi, lo);
+    } else {
+        asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(hi) : "f"(x));
+        lo = 0;
+    }
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Copies reduction block [k0, k0 + KB) of a ROWS-row operand X (element (r, k) of the operand at
+// X.at(r, k) when X is A; at X.at(k, r) when X is B, i.e. B's columns are its rows here) into stage
+// buffer st.  kmaj: the reduction index is contiguous in memory.
+template <int ROWS>
+__device__ __forceinline__ void stage_operand(float* st, const float* p, long long rstride, long long kstride,
+                                              bool kmaj, int r0, int R, int k0, int Kd, int tid) {
+    if (kmaj) {   // 16 bytes = 4 consecutive k of one row; layout [row][KB + PADK]
+        for (int e = tid; e < ROWS * (KB / 4); e += NT) {
+            const int rr = e / (KB / 4), kq = (e % (KB / 4)) * 4;
+            const int gr = r0 + rr, gk = k0 + kq;
+            const int bytes = gr < R ? 4 * clamp4(Kd - gk) : 0;
+            cp_async16(st + rr * (KB + PADK) + kq, bytes ? p + gr * rstride + gk : p, bytes);
+        }
+    } else {      // 16 bytes = 4 consecutive rows at one k; layout [k][ROWS + PADR]
+        for (int e = tid; e < KB * (ROWS / 4); e += NT) {
+            const int kk = e / (ROWS / 4), rq = (e % (ROWS / 4)) * 4;
+            const int gr = r0 + rq, gk = k0 + kk;
+            const int bytes = gk < Kd ? 4 * clamp4(R - gr) : 0;
+            cp_async16(st + kk * (ROWS + PADR) + rq, bytes ? p + gr + gk * kstride : p, bytes);
+        }
+    }
+}
+
+template <int BM, int BN, int WM, int WN, bool SPLIT>
+__device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
+                                        float alpha, bool accumulate, int mask, int rank, int ncta, float* smem) {
+    constexpr int WGN = BN / WN;
+    static_assert((BM / WM) * WGN == NT / 32, "warp grid");
+    static_assert(WM % 16 == 0 && WN % 8 == 0 && BM % 4 == 0 && BN % 4 == 0, "warp tile");
+    constexpr int MT = WM / 16, NTL = WN / 8;
+    constexpr int SA = stage_floats(BM), STAGE = SA + stage_floats(BN);
+    static_assert(STAGE * NSTAGE <= gemm_smem_floats(BM + BN > 192 ? 1 : 2), "staging");
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    const int g = lane / 4, t = lane % 4;
+    const int wr = (warp / WGN) * WM, wc = (warp % WGN) * WN;
+    const bool a_k = A.cs == 1, b_k = B.rs == 1;   // reduction index contiguous in memory
+    // A (r, k) = A.p[r rs + k cs]; B's column n at k: B.p[k rs + n cs]
+    const long long a_rstr = a_k ? A.rs : 1, a_kstr = a_k ? 1 : A.cs;
+    const long long b_rstr = b_k ? B.cs : 1, b_kstr = b_k ? 1 : B.rs;
+    auto sa = [&](const float* st, int mm, int kk) {
+        return a_k ? st[mm * (KB + PADK) + kk] : st[kk * (BM + PADR) + mm];
     };
-    auto b_pos = [&](int e, int& kk, int& nn) {
-        const int idx = tid + e * NT;
-        if (B.rs == 1) { kk = idx % KB; nn = idx / KB; } else { kk = idx / BN; nn = idx % BN; }
+    auto sb = [&](const float* st, int nn, int kk) {
+        return b_k ? st[SA + nn * (KB + PADK) + kk] : st[SA + kk * (BN + PADR) + nn];
     };
+    const int nkb = (Kd + KB - 1) / KB;
     int tile = 0;
     for (int m0 = 0; m0 < M; m0 += BM) {
         for (int n0 = 0; n0 < N; n0 += BN) {
             if (tile++ % ncta != rank) continue;   // another CTA of the cluster owns this tile
-            float acc[RM][RN];
-#pragma unroll
-            for (int i = 0; i < RM; ++i)
-#pragma unroll
-                for (int j = 0; j < RN; ++j) acc[i][j] = 0.f;
-            float ra[LA], rb[LB];
-            auto fetch = [&](int k0) {
-#pragma unroll
-                for (int e = 0; e < LA; ++e) {
-                    int kk, mm;
-                    a_pos(e, kk, mm);
-                    ra[e] = (m0 + mm < M && k0 + kk < Kd) ? A.at(m0 + mm, k0 + kk) : 0.f;
-                }
-#pragma unroll
-                for (int e = 0; e < LB; ++e) {
-                    int kk, nn;
-                    b_pos(e, kk, nn);
-                    rb[e] = (n0 + nn < N && k0 + kk < Kd) ? B.at(k0 + kk, n0 + nn) : 0.f;
-                }
+            __syncthreads();                       // the previous tile's reads of the staging are done
+            auto row_of = [&](int i, int q) { return m0 + wr + i * 16 + g + (q >= 2 ? 8 : 0); };
+            auto col_of = [&](int j, int q) { return n0 + wc + j * 8 + 2 * t + (q & 1); };
+            auto issue = [&](int kb) {
+                float* st = smem + (kb % NSTAGE) * STAGE;
+                stage_operand<BM>(st, A.p, a_rstr, a_kstr, a_k, m0, M, kb * KB, Kd, tid);
+                stage_operand<BN>(st + SA, B.p, b_rstr, b_kstr, b_k, n0, N, kb * KB, Kd, tid);
             };
-            fetch(0);
-            for (int k0 = 0; k0 < Kd; k0 += KB) {
-                __syncthreads();   // the previous block's products are done with the staging
 #pragma unroll
-                for (int e = 0; e < LA; ++e) {
-                    int kk, mm;
-                    a_pos(e, kk, mm);
-                    sA[kk * (BM + 1) + mm] = ra[e];
-                }
-#pragma unroll
-                for (int e = 0; e < LB; ++e) {
-                    int kk, nn;
-                    b_pos(e, kk, nn);
-                    sB[kk * (BN + 1) + nn] = rb[e];
-                }
-                __syncthreads();
-                if (k0 + KB < Kd) fetch(k0 + KB);
-                // the whole block every time (past Kd the staged values are zero): a fixed trip count the
-                // compiler unrolls, so the shared loads of later steps are issued ahead of their FMAs
-#pragma unroll 8
-                for (int kk = 0; kk < KB; ++kk) {
-                    float a[RM], bv[RN];
-#pragma unroll
-                    for (int i = 0; i < RM; ++i) a[i] = sA[kk * (BM + 1) + tr * RM + i];
-#pragma unroll
-                    for (int j = 0; j < RN; ++j) bv[j] = sB[kk * (BN + 1) + tc + TC * j];
-#pragma unroll
-                    for (int i = 0; i < RM; ++i)
-#pragma unroll
-                        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(a[i], bv[j], acc[i][j]);
-                }
+            for (int sidx = 0; sidx < NSTAGE - 1; ++sidx) {
+                if (sidx < nkb) issue(sidx);
+                cp_async_commit();
             }
-            // accumulating: every old value is loaded before any is stored (one memory round trip)
-            if (accumulate) {
+            float acc[MT][NTL][4], cold[MT][NTL][4];
 #pragma unroll
-                for (int i = 0; i < RM; ++i)
+            for (int i = 0; i < MT; ++i)
 #pragma unroll
-                    for (int j = 0; j < RN; ++j) {
-                        const int r = m0 + tr * RM + i, c = n0 + tc + TC * j;
-                        if (r < M && c < N)
-                            acc[i][j] = (mask == 1 && c > r ? 0.f : alpha * acc[i][j]) + C[(long long)r * ldc + c];
-                        else
-                            acc[i][j] = 0.f;
+                for (int j = 0; j < NTL; ++j)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc[i][j][q] = 0.f;
+                        const int r = row_of(i, q), c = col_of(j, q);
+                        cold[i][j][q] = accumulate && r < M && c < N ? __ldcg(C + (long long)r * ldc + c) : 0.f;
                     }
-            }
+            for (int kb = 0; kb < nkb; ++kb) {
+                cp_async_wait<NSTAGE - 2>();   // block kb has landed (this thread's copies)
+                __syncthreads();               // everyone's copies, and block kb - 1's products are done
+                if (kb + NSTAGE - 1 < nkb) issue(kb + NSTAGE - 1);
+                cp_async_commit();
+                const float* st = smem + (kb % NSTAGE) * STAGE;
 #pragma unroll
-            for (int i = 0; i < RM; ++i)
+                for (int k8 = 0; k8 < KB; k8 += 8) {
+                    uint32_t ah[MT][4], al[MT][4];
 #pragma unroll
-                for (int j = 0; j < RN; ++j) {
-                    const int r = m0 + tr * RM + i, c = n0 + tc + TC * j;
-                    if (r < M && c < N)
-                        C[(long long)r * ldc + c] = accumulate ? acc[i][j] : (mask == 1 && c > r ? 0.f : alpha * acc[i][j]);
+                    for (int i = 0; i < MT; ++i) {
+                        const int r = wr + i * 16 + g;
+                        to_tf32<SPLIT>(sa(st, r, k8 + t), ah[i][0], al[i][0]);
+                        to_tf32<SPLIT>(sa(st, r + 8, k8 + t), ah[i][1], al[i][1]);
+                        to_tf32<SPLIT>(sa(st, r, k8 + t + 4), ah[i][2], al[i][2]);
+                        to_tf32<SPLIT>(sa(st, r + 8, k8 + t + 4), ah[i][3], al[i][3]);
+                    }
+#pragma unroll
+                    for (int j = 0; j < NTL; ++j) {
+                        const int c = wc + j * 8 + g;
+                        uint32_t bh0, bl0, bh1, bl1;
+                        to_tf32<SPLIT>(sb(st, c, k8 + t), bh0, bl0);
+                        to_tf32<SPLIT>(sb(st, c, k8 + t + 4), bh1, bl1);
+#pragma unroll
+                        for (int i = 0; i < MT; ++i) {
+                            if constexpr (SPLIT) {
+                                mma_tf32(acc[i][j], al[i], bh0, bh1);
+                                mma_tf32(acc[i][j], ah[i], bl0, bl1);
+                            }
+                            mma_tf32(acc[i][j], ah[i], bh0, bh1);
+                        }
+                    }
                 }
+            }
+            cp_async_wait<0>();
+            // accumulator q of warp tile (i, j): row wr + 16 i + g (+ 8 for q >= 2), column wc + 8 j + 2 t (+ 1 if q odd)
+#pragma unroll
+            for (int i = 0; i < MT; ++i)
+#pragma unroll
+                for (int j = 0; j < NTL; ++j)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = row_of(i, q), c = col_of(j, q);
+                        if (r < M && c < N)
+                            C[(long long)r * ldc + c] = (mask == 1 && c > r ? 0.f : alpha * acc[i][j][q]) + cold[i][j][q];
+                    }
         }
     }
     head_sync(ncta);
@@ -255,24 +335,34 @@ __device__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M,
 
 // Tile shapes: one CTA tile covers a whole b x m (or m x d) product when the head has one CTA, half of
 // it per CTA with two; the b x b and b x d products take 64 x 64 tiles (32 x 64 with two CTAs).
-__device__ __noinline__ void gemm_cs(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha,
-                                     bool accumulate, int mask, int rank, int ncta) {
-    __shared__ float smem[SM_FLOATS];
+template <bool SPLIT>
+__device__ __forceinline__ void gemm_shapes(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
+                                            float alpha, bool accumulate, int mask, int rank, int ncta, float* sm) {
     if (ncta == 1) {
         if (N > 64 && M <= 64)
-            gemm_tiles<64, 256, 4, 8>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+            gemm_tiles<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
         else if (M > 64 && N <= 64)
-            gemm_tiles<256, 64, 8, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+            gemm_tiles<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
         else
-            gemm_tiles<64, 64, 2, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, smem);
+            gemm_tiles<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
     } else {
         if (N > 64 && M <= 64)
-            gemm_tiles<64, 128, 4, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+            gemm_tiles<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
         else if (M > 64 && N <= 64)
-            gemm_tiles<128, 64, 4, 4>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+            gemm_tiles<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
         else
-            gemm_tiles<32, 64, 2, 2>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, smem);
+            gemm_tiles<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
     }
+}
+
+// split: the split ("3xTF32", fp32-accurate) products; else single tf32 products (one MMA instead of three)
+__device__ __noinline__ void gemm_cs(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha,
+                                     bool accumulate, int mask, int rank, int ncta, bool split) {
+    extern __shared__ __align__(16) float dyn_smem[];
+    if (split)
+        gemm_shapes<true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, dyn_smem);
+    else
+        gemm_shapes<false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, dyn_smem);
 }
 
 __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
@@ -306,7 +396,9 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     const int h = blockIdx.x / CS, tid = threadIdx.x, gtid = rank * NT + tid;
     // a product of the head, its output tiles dealt out over the cluster (ends with the head's barrier)
     auto gemm = [&](float* C, int ldc, Mat A_, Mat B_, int M_, int N_, int Kd, float alpha, bool accumulate,
-                    int mask = 0) { gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, mask, rank, CS); };
+                    int mask = 0) {
+        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, mask, rank, CS, a.split_tf32 != 0);
+    };
     auto sync = [&]() { head_sync(CS); };
     const int T = a.T, b = a.b;
     const int nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
@@ -585,7 +677,7 @@ cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V,
                                  const float* dZ, long long x_hs, long long x_ts, const float* W1_0,
                                  const float* W2_0, float* dQ, float* dK, float* dV, float* dW1, float* dW2,
                                  float* scratch, int T, int H, int d, int b, int reverse, float eta,
-                                 cudaStream_t s) {
+                                 int split_tf32, cudaStream_t s) {
     if (b < 1 || b > BMAX) return cudaErrorInvalidValue;
     BwdArgs a{};
     a.Q = Q; a.K = K; a.V = V; a.qkv_hs = qkv_hs; a.qkv_ts = qkv_ts;
@@ -593,7 +685,7 @@ cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V,
     a.W1_0 = W1_0; a.W2_0 = W2_0;
     a.dQ = dQ; a.dK = dK; a.dV = dV; a.dW1 = dW1; a.dW2 = dW2;
     a.scratch = scratch; a.scratch_per_head = scratch_floats_for(d, b, T);
-    a.T = T; a.H = H; a.d = d; a.b = b; a.reverse = reverse; a.eta = eta;
+    a.T = T; a.H = H; a.d = d; a.b = b; a.reverse = reverse; a.eta = eta; a.split_tf32 = split_tf32;
     // two CTAs per head while the heads' pairs fit on the GPU at once, else one
     int cs = g_bwd_cluster.load();
     if (cs == 0) {
@@ -617,8 +709,13 @@ cudaError_t launch_scan_backward(const float* Q, const float* K, const float* V,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(H * cs);
     cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = (size_t)gemm_smem_floats(cs) * sizeof(float);
     cfg.stream = s;
+    {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)cfg.dynamicSmemBytes);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = cs;
