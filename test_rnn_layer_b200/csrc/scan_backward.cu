@@ -255,10 +255,12 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
     };
     const int nkb = (Kd + KB - 1) / KB;
     int tile = 0;
+    bool first = true;   // the call starts behind the head's barrier: the staging is free
     for (int m0 = 0; m0 < M; m0 += BM) {
         for (int n0 = 0; n0 < N; n0 += BN) {
             if (tile++ % ncta != rank) continue;   // another CTA of the cluster owns this tile
-            __syncthreads();                       // the previous tile's reads of the staging are done
+            if (!first) __syncthreads();           // the previous tile's reads of the staging are done
+            first = false;
             auto row_of = [&](int i, int q) { return m0 + wr + i * 16 + g + (q >= 2 ? 8 : 0); };
             auto col_of = [&](int j, int q) { return n0 + wc + j * 8 + 2 * t + (q & 1); };
             auto issue = [&](int kb) {
@@ -271,16 +273,27 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
                 if (sidx < nkb) issue(sidx);
                 cp_async_commit();
             }
+            // accumulators q and q + 1 (q even) are neighbours in a row of C: one 8-byte access (ldc and the
+            // column are even) unless the pair straddles the last column
             float acc[MT][NTL][4], cold[MT][NTL][4];
 #pragma unroll
             for (int i = 0; i < MT; ++i)
 #pragma unroll
                 for (int j = 0; j < NTL; ++j)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        acc[i][j][q] = 0.f;
+                    for (int q = 0; q < 4; q += 2) {
+                        acc[i][j][q] = acc[i][j][q + 1] = 0.f;
+                        cold[i][j][q] = cold[i][j][q + 1] = 0.f;
                         const int r = row_of(i, q), c = col_of(j, q);
-                        cold[i][j][q] = accumulate && r < M && c < N ? __ldcg(C + (long long)r * ldc + c) : 0.f;
+                        if (!accumulate || r >= M || c >= N) continue;
+                        const float* src = C + (long long)r * ldc + c;
+                        if (c + 1 < N) {
+                            const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+                            cold[i][j][q] = v.x;
+                            cold[i][j][q + 1] = v.y;
+                        } else {
+                            cold[i][j][q] = __ldcg(src);
+                        }
                     }
             for (int kb = 0; kb < nkb; ++kb) {
                 cp_async_wait<NSTAGE - 2>();   // block kb has landed (this thread's copies)
@@ -323,10 +336,16 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
 #pragma unroll
                 for (int j = 0; j < NTL; ++j)
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                    for (int q = 0; q < 4; q += 2) {
                         const int r = row_of(i, q), c = col_of(j, q);
-                        if (r < M && c < N)
-                            C[(long long)r * ldc + c] = (mask == 1 && c > r ? 0.f : alpha * acc[i][j][q]) + cold[i][j][q];
+                        if (r >= M || c >= N) continue;
+                        const float v0 = (mask == 1 && c > r ? 0.f : alpha * acc[i][j][q]) + cold[i][j][q];
+                        const float v1 = (mask == 1 && c + 1 > r ? 0.f : alpha * acc[i][j][q + 1]) + cold[i][j][q + 1];
+                        float* dst = C + (long long)r * ldc + c;
+                        if (c + 1 < N)
+                            *reinterpret_cast<float2*>(dst) = make_float2(v0, v1);
+                        else
+                            *dst = v0;
                     }
         }
     }
@@ -344,14 +363,18 @@ __device__ __forceinline__ void gemm_shapes(float* C, int ldc, const Mat& A, con
         else if (M > 64 && N <= 64)
             gemm_tiles<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
         else
-            gemm_tiles<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_tiles<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1,
+                                                             sm);
     } else {
         if (N > 64 && M <= 64)
-            gemm_tiles<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
+                                                            ncta, sm);
         else if (M > 64 && N <= 64)
-            gemm_tiles<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
+                                                            ncta, sm);
         else
-            gemm_tiles<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
+                                                            ncta, sm);
     }
 }
 
