@@ -210,11 +210,11 @@ __device__ __forceinline__ void mma_tf32(float (&c)[4], const uint32_t (&a)[4], 
 
 // Copies reduction block [k0, k0 + KB) of a ROWS-row operand X (element (r, k) of the operand at
 // X.at(r, k) when X is A; at X.at(k, r) when X is B, i.e. B's columns are its rows here) into stage
-// buffer st.  kmaj: the reduction index is contiguous in memory.
-template <int ROWS>
+// buffer st.  KMAJ: the reduction index is contiguous in memory.
+template <int ROWS, bool KMAJ>
 __device__ __forceinline__ void stage_operand(float* st, const float* p, long long rstride, long long kstride,
-                                              bool kmaj, int r0, int R, int k0, int Kd, int tid) {
-    if (kmaj) {   // 16 bytes = 4 consecutive k of one row; layout [row][KB + PADK]
+                                              int r0, int R, int k0, int Kd, int tid) {
+    if constexpr (KMAJ) {   // 16 bytes = 4 consecutive k of one row; layout [row][KB + PADK]
         for (int e = tid; e < ROWS * (KB / 4); e += NT) {
             const int rr = e / (KB / 4), kq = (e % (KB / 4)) * 4;
             const int gr = r0 + rr, gk = k0 + kq;
@@ -231,7 +231,10 @@ __device__ __forceinline__ void stage_operand(float* st, const float* p, long lo
     }
 }
 
-template <int BM, int BN, int WM, int WN, bool SPLIT>
+// A_K / B_K: the operand's reduction index is contiguous in memory (A.cs == 1 / B.rs == 1), which fixes
+// its staging layout at compile time, so that every fragment load is one shared load at a constant
+// offset from a per-thread base.
+template <int BM, int BN, int WM, int WN, bool SPLIT, bool A_K, bool B_K>
 __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
                                         float alpha, bool accumulate, int mask, int rank, int ncta, float* smem) {
     constexpr int WGN = BN / WN;
@@ -243,16 +246,15 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     const int g = lane / 4, t = lane % 4;
     const int wr = (warp / WGN) * WM, wc = (warp % WGN) * WN;
-    const bool a_k = A.cs == 1, b_k = B.rs == 1;   // reduction index contiguous in memory
     // A (r, k) = A.p[r rs + k cs]; B's column n at k: B.p[k rs + n cs]
-    const long long a_rstr = a_k ? A.rs : 1, a_kstr = a_k ? 1 : A.cs;
-    const long long b_rstr = b_k ? B.cs : 1, b_kstr = b_k ? 1 : B.rs;
-    auto sa = [&](const float* st, int mm, int kk) {
-        return a_k ? st[mm * (KB + PADK) + kk] : st[kk * (BM + PADR) + mm];
-    };
-    auto sb = [&](const float* st, int nn, int kk) {
-        return b_k ? st[SA + nn * (KB + PADK) + kk] : st[SA + kk * (BN + PADR) + nn];
-    };
+    const long long a_rstr = A_K ? A.rs : 1, a_kstr = A_K ? 1 : A.cs;
+    const long long b_rstr = B_K ? B.cs : 1, b_kstr = B_K ? 1 : B.rs;
+    // staged element (row, k) of A at a_base + row * A_RS + k * A_KS (B likewise), relative to this
+    // thread's first fragment element (row wr + g or wc + g, k = t)
+    constexpr int A_RS = A_K ? KB + PADK : 1, A_KS = A_K ? 1 : BM + PADR;
+    constexpr int B_RS = B_K ? KB + PADK : 1, B_KS = B_K ? 1 : BN + PADR;
+    const int a_base = (wr + g) * A_RS + t * A_KS;
+    const int b_base = SA + (wc + g) * B_RS + t * B_KS;
     const int nkb = (Kd + KB - 1) / KB;
     int tile = 0;
     bool first = true;   // the call starts behind the head's barrier: the staging is free
@@ -265,8 +267,8 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
             auto col_of = [&](int j, int q) { return n0 + wc + j * 8 + 2 * t + (q & 1); };
             auto issue = [&](int kb) {
                 float* st = smem + (kb % NSTAGE) * STAGE;
-                stage_operand<BM>(st, A.p, a_rstr, a_kstr, a_k, m0, M, kb * KB, Kd, tid);
-                stage_operand<BN>(st + SA, B.p, b_rstr, b_kstr, b_k, n0, N, kb * KB, Kd, tid);
+                stage_operand<BM, A_K>(st, A.p, a_rstr, a_kstr, m0, M, kb * KB, Kd, tid);
+                stage_operand<BN, B_K>(st + SA, B.p, b_rstr, b_kstr, n0, N, kb * KB, Kd, tid);
             };
 #pragma unroll
             for (int sidx = 0; sidx < NSTAGE - 1; ++sidx) {
@@ -300,24 +302,25 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
                 __syncthreads();               // everyone's copies, and block kb - 1's products are done
                 if (kb + NSTAGE - 1 < nkb) issue(kb + NSTAGE - 1);
                 cp_async_commit();
-                const float* st = smem + (kb % NSTAGE) * STAGE;
+                const float* sta = smem + (kb % NSTAGE) * STAGE + a_base;
+                const float* stb = smem + (kb % NSTAGE) * STAGE + b_base;
 #pragma unroll
                 for (int k8 = 0; k8 < KB; k8 += 8) {
                     uint32_t ah[MT][4], al[MT][4];
 #pragma unroll
                     for (int i = 0; i < MT; ++i) {
-                        const int r = wr + i * 16 + g;
-                        to_tf32<SPLIT>(sa(st, r, k8 + t), ah[i][0], al[i][0]);
-                        to_tf32<SPLIT>(sa(st, r + 8, k8 + t), ah[i][1], al[i][1]);
-                        to_tf32<SPLIT>(sa(st, r, k8 + t + 4), ah[i][2], al[i][2]);
-                        to_tf32<SPLIT>(sa(st, r + 8, k8 + t + 4), ah[i][3], al[i][3]);
+                        const float* pa = sta + i * 16 * A_RS + k8 * A_KS;
+                        to_tf32<SPLIT>(pa[0], ah[i][0], al[i][0]);
+                        to_tf32<SPLIT>(pa[8 * A_RS], ah[i][1], al[i][1]);
+                        to_tf32<SPLIT>(pa[4 * A_KS], ah[i][2], al[i][2]);
+                        to_tf32<SPLIT>(pa[8 * A_RS + 4 * A_KS], ah[i][3], al[i][3]);
                     }
 #pragma unroll
                     for (int j = 0; j < NTL; ++j) {
-                        const int c = wc + j * 8 + g;
+                        const float* pb = stb + j * 8 * B_RS + k8 * B_KS;
                         uint32_t bh0, bl0, bh1, bl1;
-                        to_tf32<SPLIT>(sb(st, c, k8 + t), bh0, bl0);
-                        to_tf32<SPLIT>(sb(st, c, k8 + t + 4), bh1, bl1);
+                        to_tf32<SPLIT>(pb[0], bh0, bl0);
+                        to_tf32<SPLIT>(pb[4 * B_KS], bh1, bl1);
 #pragma unroll
                         for (int i = 0; i < MT; ++i) {
                             if constexpr (SPLIT) {
@@ -354,27 +357,40 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
 
 // Tile shapes: one CTA tile covers a whole b x m (or m x d) product when the head has one CTA, half of
 // it per CTA with two; the b x b and b x d products take 64 x 64 tiles (32 x 64 with two CTAs).
+template <int BM, int BN, int WM, int WN, bool SPLIT>
+__device__ __forceinline__ void gemm_major(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
+                                           float alpha, bool accumulate, int mask, int rank, int ncta, float* sm) {
+    if (A.cs == 1) {
+        if (B.rs == 1)
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+        else
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+    } else {
+        if (B.rs == 1)
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+        else
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta,
+                                                              sm);
+    }
+}
+
 template <bool SPLIT>
 __device__ __forceinline__ void gemm_shapes(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
                                             float alpha, bool accumulate, int mask, int rank, int ncta, float* sm) {
     if (ncta == 1) {
         if (N > 64 && M <= 64)
-            gemm_tiles<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_major<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
         else if (M > 64 && N <= 64)
-            gemm_tiles<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_major<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
         else
-            gemm_tiles<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1,
-                                                             sm);
+            gemm_major<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
     } else {
         if (N > 64 && M <= 64)
-            gemm_tiles<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
-                                                            ncta, sm);
+            gemm_major<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
         else if (M > 64 && N <= 64)
-            gemm_tiles<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
-                                                            ncta, sm);
+            gemm_major<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
         else
-            gemm_tiles<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank,
-                                                            ncta, sm);
+            gemm_major<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
     }
 }
 
