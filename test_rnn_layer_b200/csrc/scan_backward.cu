@@ -19,10 +19,13 @@
 //   dE = -2 eta dD2,  dV = -dE,  dG += dE W2,  dA += dG * GELU'(A),  dK += dA W1,
 //   dW1 = dW1' + dAq^T Q + dA^T K,  dW2 = dW2' + dZ^T Gq + D2^T dP + dE^T G.
 // The chunk-start states come from checkpoints: the kernel first walks the
-// sequence forward (state updates only) keeping the state every kCkpt chunks
-// (by default every chunk), then, from the end, runs the chunks' backward steps
-// in reverse, each segment's chunk-start states rebuilt from its checkpoint
-// first when kCkpt > 1.
+// sequence forward (state updates only) keeping the state every kCkpt chunks,
+// then, from the end, runs the chunks' backward steps in reverse, each
+// segment's chunk-start states rebuilt from its checkpoint first when kCkpt > 1.
+// By default (kCkpt = 1) the walk keeps every chunk-start state and every
+// chunk's A, G, P and D2 as well (T (3m + d) + (T / b) 2 m d floats per head),
+// writes each state update straight into the next chunk's slot, and the
+// backward steps read all of it in place (only Dl = P GELU'(A) is recomputed).
 //
 // One cluster of CS CTAs of 512 threads per head (CS = 1 or 2); the matrices of
 // a chunk live in a per-head scratch area in global memory (it stays in L2);
@@ -75,6 +78,7 @@ struct Scratch {
     float *dW1, *dW2;            // carried state gradient
     float *ck;                   // checkpoints: [nck][2 m d]
     float *seg;                  // chunk-start states of one segment: [kCkpt][2 m d]
+    float *fw;                   // kCkpt = 1: each chunk's A, G, P [b x m] and D2 [b x d]: [nch][b (3m + d)]
     // chunk matrices
     float *Qc, *Kc, *Vc, *dZc;                 // [n x d]
     float *A, *G, *P, *Dl, *Aq, *Gq;           // [n x m]
@@ -86,8 +90,9 @@ struct Scratch {
 __host__ __device__ inline long long scratch_floats_for(int d, int b, int T) {
     const long long m = 4LL * d, md = m * d;
     const long long nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
+    const long long fw = kCkpt == 1 ? nch * b * (3 * m + d) : 0;
     return 4 * md + nck * 2 * md + kCkpt * 2 * md + 4LL * BMAX * d + 10LL * BMAX * m + 4LL * BMAX * d +
-           4LL * BMAX * BMAX + 64;
+           4LL * BMAX * BMAX + 64 + fw;
 }
 
 __device__ Scratch carve(float* base, int d, int nck) {
@@ -122,6 +127,7 @@ __device__ Scratch carve(float* base, int d, int nck) {
     s.Ng = p; p += BMAX * BMAX;
     s.dNg = p; p += BMAX * BMAX;
     s.dMk = p; p += BMAX * BMAX;
+    s.fw = p;
     return s;
 }
 
@@ -236,7 +242,8 @@ __device__ __forceinline__ void stage_operand(float* st, const float* p, long lo
 // offset from a per-thread base.
 template <int BM, int BN, int WM, int WN, bool SPLIT, bool A_K, bool B_K>
 __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                        float alpha, bool accumulate, int mask, int rank, int ncta, float* smem) {
+                                        float alpha, bool accumulate, const float* Cin, int mask, int rank, int ncta,
+                                        float* smem) {
     constexpr int WGN = BN / WN;
     static_assert((BM / WM) * WGN == NT / 32, "warp grid");
     static_assert(WM % 16 == 0 && WN % 8 == 0 && BM % 4 == 0 && BN % 4 == 0, "warp tile");
@@ -288,7 +295,7 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
                         cold[i][j][q] = cold[i][j][q + 1] = 0.f;
                         const int r = row_of(i, q), c = col_of(j, q);
                         if (!accumulate || r >= M || c >= N) continue;
-                        const float* src = C + (long long)r * ldc + c;
+                        const float* src = Cin + (long long)r * ldc + c;
                         if (c + 1 < N) {
                             const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
                             cold[i][j][q] = v.x;
@@ -359,49 +366,52 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
 // it per CTA with two; the b x b and b x d products take 64 x 64 tiles (32 x 64 with two CTAs).
 template <int BM, int BN, int WM, int WN, bool SPLIT>
 __device__ __forceinline__ void gemm_major(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                           float alpha, bool accumulate, int mask, int rank, int ncta, float* sm) {
+                                           float alpha, bool accumulate, const float* Cin, int mask, int rank, int ncta,
+                                           float* sm) {
     if (A.cs == 1) {
         if (B.rs == 1)
-            gemm_tiles<BM, BN, WM, WN, SPLIT, true, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
         else
-            gemm_tiles<BM, BN, WM, WN, SPLIT, true, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
     } else {
         if (B.rs == 1)
-            gemm_tiles<BM, BN, WM, WN, SPLIT, false, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
         else
-            gemm_tiles<BM, BN, WM, WN, SPLIT, false, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta,
-                                                              sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank,
+                                                              ncta, sm);
     }
 }
 
 template <bool SPLIT>
 __device__ __forceinline__ void gemm_shapes(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                            float alpha, bool accumulate, int mask, int rank, int ncta, float* sm) {
+                                            float alpha, bool accumulate, const float* Cin, int mask, int rank,
+                                            int ncta, float* sm) {
     if (ncta == 1) {
         if (N > 64 && M <= 64)
-            gemm_major<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_major<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
         else if (M > 64 && N <= 64)
-            gemm_major<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_major<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
         else
-            gemm_major<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, 0, 1, sm);
+            gemm_major<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
     } else {
         if (N > 64 && M <= 64)
-            gemm_major<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_major<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
         else if (M > 64 && N <= 64)
-            gemm_major<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_major<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
         else
-            gemm_major<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, sm);
+            gemm_major<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
     }
 }
 
 // split: the split ("3xTF32", fp32-accurate) products; else single tf32 products (one MMA instead of three)
+// Cin: where an accumulating product reads its old C (null: C itself).
 __device__ __noinline__ void gemm_cs(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha,
-                                     bool accumulate, int mask, int rank, int ncta, bool split) {
+                                     bool accumulate, const float* Cin, int mask, int rank, int ncta, bool split) {
     extern __shared__ __align__(16) float dyn_smem[];
     if (split)
-        gemm_shapes<true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, dyn_smem);
+        gemm_shapes<true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, rank, ncta, dyn_smem);
     else
-        gemm_shapes<false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, mask, rank, ncta, dyn_smem);
+        gemm_shapes<false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, rank, ncta, dyn_smem);
 }
 
 __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
@@ -435,8 +445,8 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     const int h = blockIdx.x / CS, tid = threadIdx.x, gtid = rank * NT + tid;
     // a product of the head, its output tiles dealt out over the cluster (ends with the head's barrier)
     auto gemm = [&](float* C, int ldc, Mat A_, Mat B_, int M_, int N_, int Kd, float alpha, bool accumulate,
-                    int mask = 0) {
-        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, mask, rank, CS, a.split_tf32 != 0);
+                    int mask = 0, const float* Cin = nullptr) {
+        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, Cin, mask, rank, CS, a.split_tf32 != 0);
     };
     auto sync = [&]() { head_sync(CS); };
     const int T = a.T, b = a.b;
@@ -523,12 +533,28 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         sync();
     };
 
+    // kCkpt = 1: chunk c's state and forward intermediates, in place
+    float* const fw0 = s.fw;
+    auto point_at_chunk = [&](int c) {
+        s.W1 = s.ck + (long long)c * 2 * MD;
+        s.W2 = s.W1 + MD;
+        float* f = fw0 + (long long)c * b * (3 * M + D);
+        s.A = f; s.G = f + b * M; s.P = f + 2 * b * M; s.D2 = f + 3 * b * M;
+    };
+
     // ---- forward walk: checkpoints of the state every kCkpt chunks
-    copy(s.W1, a.W1_0 + (long long)h * MD, MD);
-    copy(s.W2, a.W2_0 + (long long)h * MD, MD);
+    if constexpr (kCkpt == 1) {
+        copy(s.ck, a.W1_0 + (long long)h * MD, MD);
+        copy(s.ck + MD, a.W2_0 + (long long)h * MD, MD);
+    } else {
+        copy(s.W1, a.W1_0 + (long long)h * MD, MD);
+        copy(s.W2, a.W2_0 + (long long)h * MD, MD);
+    }
     for (int c = 0; c < nch; ++c) {
         const int n = min(b, T - c * b);
-        if (c % kCkpt == 0) {
+        if constexpr (kCkpt == 1) {
+            point_at_chunk(c);
+        } else if (c % kCkpt == 0) {
             copy(s.ck + (long long)(c / kCkpt) * 2 * MD, s.W1, MD);
             copy(s.ck + (long long)(c / kCkpt) * 2 * MD + MD, s.W2, MD);
         }
@@ -537,7 +563,15 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         STAMPB(1);
         chunk_core(n);
         STAMPB(2);
-        chunk_update(n);
+        if constexpr (kCkpt == 1) {   // the next chunk's state = this one's + the update (the last is not needed)
+            if (c + 1 < nch) {
+                float* W1n = s.ck + (long long)(c + 1) * 2 * MD;
+                gemm(W1n, D, T_(s.Dl, M), N_(s.Kc, D), M, D, n, 1.f, true, 0, s.W1);
+                gemm(W1n + MD, M, T_(s.D2, D), N_(s.G, M), D, M, n, 1.f, true, 0, s.W2);
+            }
+        } else {
+            chunk_update(n);
+        }
         STAMPB(3);
     }
 
@@ -568,15 +602,27 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             if constexpr (kCkpt > 1) {
                 copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
                 copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
-            } else {   // every chunk-start state is a checkpoint: read it in place
-                s.W1 = s.ck + (long long)c * 2 * MD;
-                s.W2 = s.W1 + MD;
+            } else {   // the chunk's state and forward intermediates, kept by the walk: read in place
+                point_at_chunk(c);
             }
             STAMPB(6);
             load_chunk(c, n, true, true);
             STAMPB(7);
             // forward intermediates
-            chunk_core(n);
+            if constexpr (kCkpt > 1) {
+                chunk_core(n);
+            } else {   // Dl = P GELU'(A) (A, G, P, D2 kept by the walk)
+                const float* __restrict__ A_ = s.A;
+                const float* __restrict__ P_ = s.P;
+                float* __restrict__ Dl_ = s.Dl;
+#pragma unroll 4
+                for (int idx = gtid; idx < n * M; idx += GNT) {
+                    float g, gp;
+                    gelu_and_prime(A_[idx], g, gp);
+                    Dl_[idx] = P_[idx] * gp;
+                }
+                sync();
+            }
             STAMPB(8);
             gemm(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
             gemm(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
