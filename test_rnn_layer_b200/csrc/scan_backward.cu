@@ -22,10 +22,11 @@
 // sequence forward (state updates only) keeping the state every kCkpt chunks,
 // then, from the end, runs the chunks' backward steps in reverse, each
 // segment's chunk-start states rebuilt from its checkpoint first when kCkpt > 1.
-// By default (kCkpt = 1) the walk keeps every chunk-start state and every
-// chunk's A, G, P and D2 as well (T (3m + d) + (T / b) 2 m d floats per head),
-// writes each state update straight into the next chunk's slot, and the
-// backward steps read all of it in place (only Dl = P GELU'(A) is recomputed).
+// By default (kCkpt = 1) the walk keeps every chunk-start state ((T / b) 2 m d
+// floats per head), writing each state update straight into the next chunk's
+// slot, and the backward steps read the states in place.  (Keeping each
+// chunk's A, G, P and D2 too, 50 GB more at 313,344 tokens, measured no
+// faster: the reads from HBM cost what the recomputation did.)
 //
 // One cluster of CS CTAs of 512 threads per head (CS = 1 or 2); the matrices of
 // a chunk live in a per-head scratch area in global memory (it stays in L2);
@@ -78,7 +79,6 @@ struct Scratch {
     float *dW1, *dW2;            // carried state gradient
     float *ck;                   // checkpoints: [nck][2 m d]
     float *seg;                  // chunk-start states of one segment: [kCkpt][2 m d]
-    float *fw;                   // kCkpt = 1: each chunk's A, G, P [b x m] and D2 [b x d]: [nch][b (3m + d)]
     // chunk matrices
     float *Qc, *Kc, *Vc, *dZc;                 // [n x d]
     float *A, *G, *P, *Dl, *Aq, *Gq;           // [n x m]
@@ -90,9 +90,8 @@ struct Scratch {
 __host__ __device__ inline long long scratch_floats_for(int d, int b, int T) {
     const long long m = 4LL * d, md = m * d;
     const long long nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
-    const long long fw = kCkpt == 1 ? nch * b * (3 * m + d) : 0;
     return 4 * md + nck * 2 * md + kCkpt * 2 * md + 4LL * BMAX * d + 10LL * BMAX * m + 4LL * BMAX * d +
-           4LL * BMAX * BMAX + 64 + fw;
+           4LL * BMAX * BMAX + 64;
 }
 
 __device__ Scratch carve(float* base, int d, int nck) {
@@ -127,7 +126,6 @@ __device__ Scratch carve(float* base, int d, int nck) {
     s.Ng = p; p += BMAX * BMAX;
     s.dNg = p; p += BMAX * BMAX;
     s.dMk = p; p += BMAX * BMAX;
-    s.fw = p;
     return s;
 }
 
@@ -533,13 +531,10 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         sync();
     };
 
-    // kCkpt = 1: chunk c's state and forward intermediates, in place
-    float* const fw0 = s.fw;
+    // kCkpt = 1: chunk c's state, in place
     auto point_at_chunk = [&](int c) {
         s.W1 = s.ck + (long long)c * 2 * MD;
         s.W2 = s.W1 + MD;
-        float* f = fw0 + (long long)c * b * (3 * M + D);
-        s.A = f; s.G = f + b * M; s.P = f + 2 * b * M; s.D2 = f + 3 * b * M;
     };
 
     // ---- forward walk: checkpoints of the state every kCkpt chunks
@@ -602,27 +597,14 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             if constexpr (kCkpt > 1) {
                 copy(s.W1, s.seg + (long long)(c - c0) * 2 * MD, MD);
                 copy(s.W2, s.seg + (long long)(c - c0) * 2 * MD + MD, MD);
-            } else {   // the chunk's state and forward intermediates, kept by the walk: read in place
+            } else {   // the chunk's state, kept by the walk: read in place
                 point_at_chunk(c);
             }
             STAMPB(6);
             load_chunk(c, n, true, true);
             STAMPB(7);
             // forward intermediates
-            if constexpr (kCkpt > 1) {
-                chunk_core(n);
-            } else {   // Dl = P GELU'(A) (A, G, P, D2 kept by the walk)
-                const float* __restrict__ A_ = s.A;
-                const float* __restrict__ P_ = s.P;
-                float* __restrict__ Dl_ = s.Dl;
-#pragma unroll 4
-                for (int idx = gtid; idx < n * M; idx += GNT) {
-                    float g, gp;
-                    gelu_and_prime(A_[idx], g, gp);
-                    Dl_[idx] = P_[idx] * gp;
-                }
-                sync();
-            }
+            chunk_core(n);
             STAMPB(8);
             gemm(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
             gemm(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
