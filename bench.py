@@ -848,7 +848,10 @@ def run_backward(args, rank, world, local_rank):
         line = {"metric": "TTT-MLP training step (forward + backward) " + _metric(w, "mlp"),
                 "value": whole_job_tokens_per_s(world, w.T, ms_per_step), "unit": UNIT, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "fp32-backward", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": ("bf16-in/tf32-mma/fp32-state-backward" if w.dtype == "bf16"
+                          else "fp32-in/3xtf32-mma/fp32-state-backward"),
+                "data": "synthetic",
                 "config": _config(w, {"step": "forward recomputed + backward of every input"}),
                 "gpu_launches": launches, "clocks": clocks, "roofline": roof, "kernels": kernels, "e2e": e2e,
                 "cpu_baseline": cpu, "impl": "ours"}

@@ -177,12 +177,17 @@ TTT_API ttt_status ttt_mlp_forward_host(const ttt_mlp_desc* desc, const void* X_
  *   workspace ttt_mlp_backward_workspace_size(desc, b, dir) bytes, 256-byte
  *             aligned; ttt_mlp_status(workspace, stream) reports non-finite
  *             values and expired waits as for ttt_mlp_forward.
- * Every gradient output is overwritten.  The scan's backward runs in fp32 on
- * the SIMT cores (one CTA per head); its forward walk keeps every chunk-start
- * state, 2 m d fp32 values per chunk and head (128 KB at d = 64: about 30 GB
- * of the workspace for 48 heads and 313,344 tokens in chunks of 64).  The
- * projections' gradients run on the tensor cores for a full-width bf16 layer
- * (fp32 dU split into two bf16 halves), as fp32 GEMMs otherwise.
+ * Every gradient output is overwritten.  The scan's backward keeps its state
+ * and gradients in fp32 and runs its products on tf32 tensor cores: in the
+ * split form (three products, fp32-accurate) for fp32 layers, as single tf32
+ * products for bf16 layers (the precision of their forward pass).  It walks
+ * each head on a cluster of two CTAs while twice the head count fits on the
+ * SMs (else one CTA; ttt_debug_set_backward_ctas), with the same results
+ * either way.  Its forward walk keeps every chunk-start state, 2 m d fp32
+ * values per chunk and head (128 KB at d = 64: about 30 GB of the workspace
+ * for 48 heads and 313,344 tokens in chunks of 64).  The projections'
+ * gradients run on the tensor cores for a full-width bf16 layer (fp32 dU split
+ * into two bf16 halves), as fp32 GEMMs otherwise.
  * Returns TTT_ERR_UNSUPPORTED for b > 64.
  */
 TTT_API size_t ttt_mlp_backward_workspace_size(const ttt_mlp_desc* desc, int b, ttt_direction dir);
