@@ -240,8 +240,8 @@ __device__ __forceinline__ void stage_operand(float* st, const float* p, long lo
 // offset from a per-thread base.
 template <int BM, int BN, int WM, int WN, bool SPLIT, bool A_K, bool B_K>
 __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                        float alpha, bool accumulate, const float* Cin, int mask, int rank, int ncta,
-                                        float* smem) {
+                                        float alpha, bool accumulate, const float* Cin, int mask, bool bar, int rank,
+                                        int ncta, float* smem) {
     constexpr int WGN = BN / WN;
     static_assert((BM / WM) * WGN == NT / 32, "warp grid");
     static_assert(WM % 16 == 0 && WN % 8 == 0 && BM % 4 == 0 && BN % 4 == 0, "warp tile");
@@ -357,59 +357,66 @@ __device__ __noinline__ void gemm_tiles(float* C, int ldc, const Mat& A, const M
                     }
         }
     }
-    head_sync(ncta);
+    if (bar)
+        head_sync(ncta);
+    else
+        __syncthreads();   // only the staging is reused by the CTA's next product
 }
 
 // Tile shapes: one CTA tile covers a whole b x m (or m x d) product when the head has one CTA, half of
 // it per CTA with two; the b x b and b x d products take 64 x 64 tiles (32 x 64 with two CTAs).
 template <int BM, int BN, int WM, int WN, bool SPLIT>
 __device__ __forceinline__ void gemm_major(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                           float alpha, bool accumulate, const float* Cin, int mask, int rank, int ncta,
-                                           float* sm) {
+                                           float alpha, bool accumulate, const float* Cin, int mask, bool bar,
+                                           int rank, int ncta, float* sm) {
     if (A.cs == 1) {
         if (B.rs == 1)
-            gemm_tiles<BM, BN, WM, WN, SPLIT, true, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
         else
-            gemm_tiles<BM, BN, WM, WN, SPLIT, true, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, true, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
     } else {
         if (B.rs == 1)
-            gemm_tiles<BM, BN, WM, WN, SPLIT, false, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
         else
-            gemm_tiles<BM, BN, WM, WN, SPLIT, false, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank,
-                                                              ncta, sm);
+            gemm_tiles<BM, BN, WM, WN, SPLIT, false, false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar,
+                                                              rank, ncta, sm);
     }
 }
 
 template <bool SPLIT>
 __device__ __forceinline__ void gemm_shapes(float* C, int ldc, const Mat& A, const Mat& B, int M, int N, int Kd,
-                                            float alpha, bool accumulate, const float* Cin, int mask, int rank,
-                                            int ncta, float* sm) {
+                                            float alpha, bool accumulate, const float* Cin, int mask, bool bar,
+                                            int rank, int ncta, float* sm) {
     if (ncta == 1) {
         if (N > 64 && M <= 64)
-            gemm_major<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
+            gemm_major<64, 256, 16, 64, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, 0, 1, sm);
         else if (M > 64 && N <= 64)
-            gemm_major<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
+            gemm_major<256, 64, 32, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, 0, 1, sm);
         else
-            gemm_major<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, 0, 1, sm);
+            gemm_major<64, 64, 16, 16, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, 0, 1, sm);
     } else {
         if (N > 64 && M <= 64)
-            gemm_major<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_major<64, 128, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
         else if (M > 64 && N <= 64)
-            gemm_major<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_major<128, 64, 16, 32, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
         else
-            gemm_major<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, rank, ncta, sm);
+            gemm_major<32, 64, 16, 8, SPLIT>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin, mask, bar, rank, ncta, sm);
     }
 }
 
 // split: the split ("3xTF32", fp32-accurate) products; else single tf32 products (one MMA instead of three)
-// Cin: where an accumulating product reads its old C (null: C itself).
+// Cin: where an accumulating product reads its old C (null: C itself).  bar: end with the head's barrier;
+// false only where the next products of the head read nothing this one writes and write nothing it reads
+// (a later accumulation into the same C by a product of the same shape is fine: the same threads own the
+// same elements of C).
 __device__ __noinline__ void gemm_cs(float* C, int ldc, Mat A, Mat B, int M, int N, int Kd, float alpha,
-                                     bool accumulate, const float* Cin, int mask, int rank, int ncta, bool split) {
+                                     bool accumulate, const float* Cin, int mask, bool bar, int rank, int ncta,
+                                     bool split) {
     extern __shared__ __align__(16) float dyn_smem[];
     if (split)
-        gemm_shapes<true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, rank, ncta, dyn_smem);
+        gemm_shapes<true>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, bar, rank, ncta, dyn_smem);
     else
-        gemm_shapes<false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, rank, ncta, dyn_smem);
+        gemm_shapes<false>(C, ldc, A, B, M, N, Kd, alpha, accumulate, Cin ? Cin : C, mask, bar, rank, ncta, dyn_smem);
 }
 
 __device__ __forceinline__ float gelu_pp(float a) {   // GELU''(a) = phi(a) (2 - a^2)
@@ -444,7 +451,13 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
     // a product of the head, its output tiles dealt out over the cluster (ends with the head's barrier)
     auto gemm = [&](float* C, int ldc, Mat A_, Mat B_, int M_, int N_, int Kd, float alpha, bool accumulate,
                     int mask = 0, const float* Cin = nullptr) {
-        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, Cin, mask, rank, CS, a.split_tf32 != 0);
+        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, Cin, mask, true, rank, CS, a.split_tf32 != 0);
+    };
+    // the same, without the head's barrier: for a product whose successors up to the next barrier are
+    // independent of it
+    auto gemm_nb = [&](float* C, int ldc, Mat A_, Mat B_, int M_, int N_, int Kd, float alpha, bool accumulate,
+                       int mask = 0, const float* Cin = nullptr) {
+        gemm_cs(C, ldc, A_, B_, M_, N_, Kd, alpha, accumulate, Cin, mask, false, rank, CS, a.split_tf32 != 0);
     };
     auto sync = [&]() { head_sync(CS); };
     const int T = a.T, b = a.b;
@@ -478,8 +491,17 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         sync();
     };
     // A = K W1^T, G = GELU(A), D2 = -2 eta (G W2^T - V), P = D2 W2, Dl = P GELU'(A)
-    auto chunk_core = [&](int n) {
-        gemm(s.A, M, N_(s.Kc, D), T_(s.W1, D), n, M, D, 1.f, false);
+    // bwd: the backward step's first products that need only the loaded chunk and the state (Mk, Q W1^T,
+    // dZ W2) go beside A, and tril(dZ D2^T) beside P
+    auto chunk_core = [&](int n, bool bwd) {
+        if (bwd) {
+            gemm_nb(s.A, M, N_(s.Kc, D), T_(s.W1, D), n, M, D, 1.f, false);
+            gemm_nb(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
+            gemm_nb(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
+            gemm(s.dGq, M, N_(s.dZc, D), N_(s.W2, M), n, M, D, 1.f, false);                 // dZ W2
+        } else {
+            gemm(s.A, M, N_(s.Kc, D), T_(s.W1, D), n, M, D, 1.f, false);
+        }
         {   // (restrict views scoped to each loop: several iterations' loads may be in flight)
             const float* __restrict__ A_ = s.A;
             float* __restrict__ G_ = s.G;
@@ -495,7 +517,12 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             for (int idx = gtid; idx < n * D; idx += GNT) D2_[idx] = -2.0f * eta * (D2_[idx] - V_[idx]);
         }
         sync();
-        gemm(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
+        if (bwd) {
+            gemm_nb(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
+            gemm(s.dNg, BMAX, N_(s.dZc, D), T_(s.D2, D), n, n, D, 1.f, false, 1);            // tril(dZ D2^T)
+        } else {
+            gemm(s.P, M, N_(s.D2, D), N_(s.W2, M), n, M, D, 1.f, false);
+        }
         {
             const float* __restrict__ A_ = s.A;
             const float* __restrict__ P_ = s.P;
@@ -556,12 +583,12 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
         STAMPB(0);
         load_chunk(c, n, false, false);
         STAMPB(1);
-        chunk_core(n);
+        chunk_core(n, false);
         STAMPB(2);
         if constexpr (kCkpt == 1) {   // the next chunk's state = this one's + the update (the last is not needed)
             if (c + 1 < nch) {
                 float* W1n = s.ck + (long long)(c + 1) * 2 * MD;
-                gemm(W1n, D, T_(s.Dl, M), N_(s.Kc, D), M, D, n, 1.f, true, 0, s.W1);
+                gemm_nb(W1n, D, T_(s.Dl, M), N_(s.Kc, D), M, D, n, 1.f, true, 0, s.W1);
                 gemm(W1n + MD, M, T_(s.D2, D), N_(s.G, M), D, M, n, 1.f, true, 0, s.W2);
             }
         } else {
@@ -586,7 +613,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             if (c + 1 < c1) {
                 const int n = min(b, T - c * b);
                 load_chunk(c, n, false, false);
-                chunk_core(n);
+                chunk_core(n, false);
                 chunk_update(n);
             }
             STAMPB(5);
@@ -603,48 +630,40 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             STAMPB(6);
             load_chunk(c, n, true, true);
             STAMPB(7);
-            // forward intermediates
-            chunk_core(n);
+            // forward intermediates (and the first products of the output branch)
+            chunk_core(n, true);
             STAMPB(8);
-            gemm(s.Mk, BMAX, N_(s.Qc, D), T_(s.Kc, D), n, n, D, 1.f, false, 1);
-            gemm(s.Aq, M, N_(s.Qc, D), T_(s.W1, D), n, M, D, 1.f, false);
-            gemm(s.Aq, M, N_(s.Mk, BMAX), N_(s.Dl, M), n, M, n, 1.f, true);
-            {
+            gemm_nb(s.Aq, M, N_(s.Mk, BMAX), N_(s.Dl, M), n, M, n, 1.f, true);              // Aq += Mk Dl
+            gemm(s.dGq, M, N_(s.dNg, BMAX), N_(s.G, M), n, M, n, 1.f, true);                 // + dNg G
+            {   // Gq = GELU(Aq), dAq = dGq GELU'(Aq) (in dGq)
                 const float* __restrict__ Aq_ = s.Aq;
                 float* __restrict__ Gq_ = s.Gq;
-#pragma unroll 4
-                for (int idx = gtid; idx < n * M; idx += GNT) Gq_[idx] = gelu(Aq_[idx]);
-            }
-            sync();
-            gemm(s.Ng, BMAX, N_(s.Gq, M), T_(s.G, M), n, n, M, 1.f, false, 1);
-            STAMPB(9);
-            // output branch
-            gemm(s.dGq, M, N_(s.dZc, D), N_(s.W2, M), n, M, D, 1.f, false);                 // dZ W2
-            gemm(s.dNg, BMAX, N_(s.dZc, D), T_(s.D2, D), n, n, D, 1.f, false, 1);            // tril(dZ D2^T)
-            gemm(s.dD2, D, T_(s.Ng, BMAX), N_(s.dZc, D), n, D, n, 1.f, false);               // Ng^T dZ
-            gemm(s.dGq, M, N_(s.dNg, BMAX), N_(s.G, M), n, M, n, 1.f, true);                 // + dNg G
-            gemm(s.dG, M, T_(s.dNg, BMAX), N_(s.Gq, M), n, M, n, 1.f, false);                // dNg^T Gq
-            {                                                                                // dAq (in dGq)
-                const float* __restrict__ Aq_ = s.Aq;
                 float* __restrict__ dGq_ = s.dGq;
 #pragma unroll 4
                 for (int idx = gtid; idx < n * M; idx += GNT) {
+                    const float aq = Aq_[idx];
                     float g, gp;
-                    gelu_and_prime(Aq_[idx], g, gp);
+                    gelu_and_prime(aq, g, gp);
+                    Gq_[idx] = gelu(aq);
                     dGq_[idx] *= gp;
                 }
             }
             sync();
-            gemm(s.dQc, D, N_(s.dGq, M), N_(s.W1, D), n, D, M, 1.f, false);                 // dAq W1
-            gemm(s.dMk, BMAX, N_(s.dGq, M), T_(s.Dl, M), n, n, M, 1.f, false, 1);            // tril(dAq Dl^T)
+            STAMPB(9);
+            // output branch
+            gemm_nb(s.Ng, BMAX, N_(s.Gq, M), T_(s.G, M), n, n, M, 1.f, false, 1);            // tril(Gq G^T)
+            gemm_nb(s.dG, M, T_(s.dNg, BMAX), N_(s.Gq, M), n, M, n, 1.f, false);             // dNg^T Gq
+            gemm_nb(s.dQc, D, N_(s.dGq, M), N_(s.W1, D), n, D, M, 1.f, false);               // dAq W1
+            gemm_nb(s.dMk, BMAX, N_(s.dGq, M), T_(s.Dl, M), n, n, M, 1.f, false, 1);         // tril(dAq Dl^T)
             gemm(s.dDl, M, T_(s.Mk, BMAX), N_(s.dGq, M), n, M, n, 1.f, false);               // Mk^T dAq
-            gemm(s.dQc, D, N_(s.dMk, BMAX), N_(s.Kc, D), n, D, n, 1.f, true);                // + dMk K
-            gemm(s.dKc, D, T_(s.dMk, BMAX), N_(s.Qc, D), n, D, n, 1.f, false);               // dMk^T Q
             STAMPB(10);
+            gemm_nb(s.dD2, D, T_(s.Ng, BMAX), N_(s.dZc, D), n, D, n, 1.f, false);            // Ng^T dZ
+            gemm_nb(s.dQc, D, N_(s.dMk, BMAX), N_(s.Kc, D), n, D, n, 1.f, true);             // + dMk K
+            gemm_nb(s.dKc, D, T_(s.dMk, BMAX), N_(s.Qc, D), n, D, n, 1.f, false);            // dMk^T Q
             // the chunk-end state gradient
-            gemm(s.dDl, M, N_(s.Kc, D), T_(s.dW1, D), n, M, D, 1.f, true);                  // + K dW1'^T
-            gemm(s.dKc, D, N_(s.Dl, M), N_(s.dW1, D), n, D, M, 1.f, true);                  // + Dl dW1'
-            gemm(s.dD2, D, N_(s.G, M), T_(s.dW2, M), n, D, M, 1.f, true);                   // + G dW2'^T
+            gemm_nb(s.dDl, M, N_(s.Kc, D), T_(s.dW1, D), n, M, D, 1.f, true);               // + K dW1'^T
+            gemm_nb(s.dKc, D, N_(s.Dl, M), N_(s.dW1, D), n, D, M, 1.f, true);               // + Dl dW1'
+            gemm_nb(s.dD2, D, N_(s.G, M), T_(s.dW2, M), n, D, M, 1.f, true);                // + G dW2'^T
             gemm(s.dG, M, N_(s.D2, D), N_(s.dW2, M), n, M, D, 1.f, true);                   // + D2 dW2'
             // dP (in dDl), dA
             {
@@ -683,13 +702,13 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                 }
             }
             sync();
-            gemm(s.dKc, D, N_(s.dA, M), N_(s.W1, D), n, D, M, 1.f, true);                   // + dA W1
             STAMPB(11);
+            gemm_nb(s.dKc, D, N_(s.dA, M), N_(s.W1, D), n, D, M, 1.f, true);                // + dA W1
             // the chunk-start state gradient (accumulated onto the chunk-end one)
-            gemm(s.dW2, M, T_(s.dZc, D), N_(s.Gq, M), D, M, n, 1.f, true);                  // dZ^T Gq
-            gemm(s.dW2, M, T_(s.D2, D), N_(s.dDl, M), D, M, n, 1.f, true);                  // D2^T dP
-            gemm(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, 1.f, true);                   // dE^T G
-            gemm(s.dW1, D, T_(s.dGq, M), N_(s.Qc, D), M, D, n, 1.f, true);                  // dAq^T Q
+            gemm_nb(s.dW2, M, T_(s.dZc, D), N_(s.Gq, M), D, M, n, 1.f, true);               // dZ^T Gq
+            gemm_nb(s.dW2, M, T_(s.D2, D), N_(s.dDl, M), D, M, n, 1.f, true);               // D2^T dP
+            gemm_nb(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, 1.f, true);                // dE^T G
+            gemm_nb(s.dW1, D, T_(s.dGq, M), N_(s.Qc, D), M, D, n, 1.f, true);               // dAq^T Q
             gemm(s.dW1, D, T_(s.dA, M), N_(s.Kc, D), M, D, n, 1.f, true);                   // dA^T K
             STAMPB(12);
             // dQ, dK, dV of the chunk's tokens
