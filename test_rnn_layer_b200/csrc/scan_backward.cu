@@ -83,6 +83,7 @@ struct Scratch {
     float *Qc, *Kc, *Vc, *dZc;                 // [n x d]
     float *A, *G, *P, *Dl, *Aq, *Gq;           // [n x m]
     float *dA, *dG, *dGq, *dDl;                // [n x m]
+    float *GpA;                                // GELU'(A) [n x m]
     float *D2, *dD2, *dQc, *dKc;               // [n x d]
     float *Mk, *Ng, *dNg, *dMk;                // [n x n]
 };
@@ -90,7 +91,7 @@ struct Scratch {
 __host__ __device__ inline long long scratch_floats_for(int d, int b, int T) {
     const long long m = 4LL * d, md = m * d;
     const long long nch = (T + b - 1) / b, nck = (nch + kCkpt - 1) / kCkpt;
-    return 4 * md + nck * 2 * md + kCkpt * 2 * md + 4LL * BMAX * d + 10LL * BMAX * m + 4LL * BMAX * d +
+    return 4 * md + nck * 2 * md + kCkpt * 2 * md + 4LL * BMAX * d + 11LL * BMAX * m + 4LL * BMAX * d +
            4LL * BMAX * BMAX + 64;
 }
 
@@ -118,6 +119,7 @@ __device__ Scratch carve(float* base, int d, int nck) {
     s.dG = p; p += BMAX * m;
     s.dGq = p; p += BMAX * m;
     s.dDl = p; p += BMAX * m;
+    s.GpA = p; p += BMAX * m;
     s.D2 = p; p += BMAX * d;
     s.dD2 = p; p += BMAX * d;
     s.dQc = p; p += BMAX * d;
@@ -527,11 +529,13 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             const float* __restrict__ A_ = s.A;
             const float* __restrict__ P_ = s.P;
             float* __restrict__ Dl_ = s.Dl;
+            float* __restrict__ Gp_ = s.GpA;
 #pragma unroll 4
             for (int idx = gtid; idx < n * M; idx += GNT) {
                 float g, gp;
                 gelu_and_prime(A_[idx], g, gp);
                 Dl_[idx] = P_[idx] * gp;
+                if (bwd) Gp_[idx] = gp;   // for the backward step's passes
             }
         }
         sync();
@@ -669,37 +673,26 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             {
                 const float* __restrict__ A_ = s.A;
                 const float* __restrict__ P_ = s.P;
+                const float* __restrict__ Gp_ = s.GpA;
                 float* __restrict__ dDl_ = s.dDl;
                 float* __restrict__ dA_ = s.dA;
 #pragma unroll 4
                 for (int idx = gtid; idx < n * M; idx += GNT) {
-                    float g, gp;
-                    const float av = A_[idx];
-                    gelu_and_prime(av, g, gp);
                     const float ddl = dDl_[idx];
-                    dA_[idx] = ddl * P_[idx] * gelu_pp(av);
-                    dDl_[idx] = ddl * gp;
+                    dA_[idx] = ddl * P_[idx] * gelu_pp(A_[idx]);
+                    dDl_[idx] = ddl * Gp_[idx];
                 }
             }
             sync();
+            // dE = -2 eta dD2 is applied as the products' alpha (dD2 itself is kept)
             gemm(s.dD2, D, N_(s.dDl, M), T_(s.W2, M), n, D, M, 1.f, true);                  // + dP W2^T
-            {                                                                                // dE (in dD2)
-                float* __restrict__ dD2_ = s.dD2;
-#pragma unroll 4
-                for (int idx = gtid; idx < n * D; idx += GNT) dD2_[idx] *= -2.0f * eta;
-            }
-            sync();
-            gemm(s.dG, M, N_(s.dD2, D), N_(s.W2, M), n, M, D, 1.f, true);                   // + dE W2
+            gemm(s.dG, M, N_(s.dD2, D), N_(s.W2, M), n, M, D, -2.0f * eta, true);           // + dE W2
             {                                                                                // dA += dG GELU'(A)
-                const float* __restrict__ A_ = s.A;
+                const float* __restrict__ Gp_ = s.GpA;
                 const float* __restrict__ dG_ = s.dG;
                 float* __restrict__ dA_ = s.dA;
 #pragma unroll 4
-                for (int idx = gtid; idx < n * M; idx += GNT) {
-                    float g, gp;
-                    gelu_and_prime(A_[idx], g, gp);
-                    dA_[idx] += dG_[idx] * gp;
-                }
+                for (int idx = gtid; idx < n * M; idx += GNT) dA_[idx] += dG_[idx] * Gp_[idx];
             }
             sync();
             STAMPB(11);
@@ -707,7 +700,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
             // the chunk-start state gradient (accumulated onto the chunk-end one)
             gemm_nb(s.dW2, M, T_(s.dZc, D), N_(s.Gq, M), D, M, n, 1.f, true);               // dZ^T Gq
             gemm_nb(s.dW2, M, T_(s.D2, D), N_(s.dDl, M), D, M, n, 1.f, true);               // D2^T dP
-            gemm_nb(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, 1.f, true);                // dE^T G
+            gemm_nb(s.dW2, M, T_(s.dD2, D), N_(s.G, M), D, M, n, -2.0f * eta, true);        // dE^T G
             gemm_nb(s.dW1, D, T_(s.dGq, M), N_(s.Qc, D), M, D, n, 1.f, true);               // dAq^T Q
             gemm(s.dW1, D, T_(s.dA, M), N_(s.Kc, D), M, D, n, 1.f, true);                   // dA^T K
             STAMPB(12);
@@ -725,7 +718,7 @@ __global__ void __launch_bounds__(NT, 1) scan_bwd_kernel(BwdArgs a) {
                     const long long off = (long long)h * a.qkv_hs + (long long)token(c, r) * a.qkv_ts + j;
                     gdQ[off] = dQc_[idx];
                     gdK[off] = dKc_[idx];
-                    gdV[off] = -dD2_[idx];   // dV = -dE
+                    gdV[off] = dD2_[idx] * (2.0f * eta);   // dV = -dE = 2 eta dD2
                 }
             }
             sync();
