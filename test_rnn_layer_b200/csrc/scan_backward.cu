@@ -1,6 +1,7 @@
-// Backward pass of one direction of the TTT-MLP scan (fp32 SIMT, any b <= 64,
-// d = 16, 32 or 64): given dZ = dLoss/dz for every token, the gradients with
-// respect to the token streams Q, K, V and the initial state W1_0, W2_0.
+// Backward pass of one direction of the TTT-MLP scan (fp32 state and
+// gradients, tf32 tensor-core products; any b <= 64, d = 16, 32 or 64): given
+// dZ = dLoss/dz for every token, the gradients with respect to the token
+// streams Q, K, V and the initial state W1_0, W2_0.
 //
 // The forward chunk (paper notes page, "关键设计 / TTT-MLP 层"; n tokens in
 // walking order, state W1 [m x d], W2 [d x m] at the chunk start, rows of the
@@ -33,8 +34,11 @@
 // every product is a block GEMM tiled through shared memory whose output tiles
 // are dealt out over the cluster's CTAs, and every elementwise pass strides over
 // all of the cluster's threads, with a cluster barrier (release / acquire) where
-// the CTAs' results meet.  Each output element is computed by the same sequence
-// of operations whatever CS is, so the results do not depend on it.
+// the CTAs' results meet: after each group of products that do not depend on
+// one another, and after each pass.  dE = -2 eta dD2 is never formed: the
+// products that read it take -2 eta as their alpha.  Each output element is
+// computed by the same sequence of operations whatever CS is, so the results
+// do not depend on it.
 #include <atomic>
 
 #include "common.cuh"
