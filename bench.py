@@ -212,9 +212,11 @@ def _algorithmic(w):
         # correction (2 x 2 b d over the causal half)
         "scan_linear_tc": ("tensor_tf32", H * T * (6 * d * d + 2 * b * d)),
         # backward of the scan: the forward chunk recomputed plus its reverse-mode derivative, counted
-        # as three forward passes (the kernel does more: the state walk for the checkpoints and the
-        # rebuild of each segment's chunk-start states)
-        "scan_backward": ("alu", 3 * H * T * (7 * 2 * d * m + 2 * b * (d + m))),
+        # as three forward passes (the kernel does more: the state walk that keeps the chunk-start
+        # states); its products run on tf32 tensor cores, in the split form (three products each) for
+        # fp32 layers
+        "scan_backward": ("tensor_tf32" if w.dtype == "bf16" else "tensor_3xtf32",
+                          3 * H * T * (7 * 2 * d * m + 2 * b * (d + m))),
         # projections' gradients: dX += dU theta and dtheta += dU^T X for the three projections
         "grad_gemm": ("alu", 2 * 3 * 2.0 * T * D * (d if w.per_head else D)),
         "gate_backward": ("hbm", T * D * 16),
@@ -250,6 +252,10 @@ def _roofline(name, ms_per_launch, launches_per_step, w, peaks, clocks):
     elif bound == "tensor_tf32":
         peak, unit, kind = sus * TF32_PER_BF16, "TFLOP/s", "tensor"
         note = f"tf32 dense = bf16 sustained {src} x 1.1/2.25 (nominal ratio)"
+        achieved = work / (ms_per_launch * 1e-3) / 1e12
+    elif bound == "tensor_3xtf32":   # every product taken as three tf32 products
+        peak, unit, kind = sus * TF32_PER_BF16 / 3, "TFLOP/s", "tensor"
+        note = f"tf32 dense = bf16 sustained {src} x 1.1/2.25 (nominal ratio), / 3 for the split products"
         achieved = work / (ms_per_launch * 1e-3) / 1e12
     elif bound == "alu":
         mhz = peaks.get("sm_max_mhz", 1965.0)

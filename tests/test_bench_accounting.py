@@ -46,6 +46,12 @@ def test_gate_and_alu_bounds():
     assert g["work_per_launch"] == w.T * w.model_dim * 11
     s = bench._roofline("scan_linear", 100.0, 2, w, PEAKS, CLOCKS)
     assert s["bound"] == "alu" and s["peak"] == pytest.approx(148 * 128 * 2 * 1965e6 / 1e12, rel=1e-3)
+    # the scan backward's products: tf32 for a bf16 layer, three tf32 products each for an fp32 one
+    tf32 = PEAKS["bf16_tflops_sustained"] * 1.1 / 2.25
+    b16 = bench._roofline("scan_backward", 100.0, 2, w, PEAKS, CLOCKS)
+    b32 = bench._roofline("scan_backward", 100.0, 2, w.with_(dtype="f32"), PEAKS, CLOCKS)
+    assert b16["bound"] == b32["bound"] == "tensor"
+    assert b16["peak"] == pytest.approx(tf32, rel=1e-3) and b32["peak"] == pytest.approx(tf32 / 3, rel=1e-3)
 
 
 def test_traffic_record_scales_with_the_tokens_of_a_launch(tmp_path, monkeypatch):
