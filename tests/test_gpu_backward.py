@@ -2,8 +2,10 @@
 fp64 backward oracle (oracle/ttt_backward.py: autograd of the primal chunk
 form, pinned to the C oracle and to finite differences), gradient by gradient:
 dX, dtheta_Q/K/V, dW1_0, dW2_0, dalpha_f, dalpha_r for a seeded upstream
-gradient dY.  Tolerances: 1e-3 max-normalised for fp32 inputs, 2e-2 for bf16
-inputs (the forward pass recomputed inside runs on the tensor cores there)."""
+gradient dY.  Tolerances: 1e-3 max-normalised for fp32 inputs (the scan
+backward's products in the split, fp32-accurate tf32 form), 2e-2 for bf16
+inputs (the forward pass recomputed inside and the scan backward's products
+run on single tf32 / fp16 / bf16 tensor-core products there)."""
 import numpy as np
 import pytest
 import torch
